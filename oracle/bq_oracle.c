@@ -1,0 +1,334 @@
+/*
+ * bq_oracle.c -- plain, slow CPU oracle for linear layers on packed binary-g128 and
+ * ternary-g128 weights.
+ *
+ * TEST INFRASTRUCTURE ONLY. It is called by the test suite, by the smoke check and by
+ * the CPU-baseline leg of the benchmark. The product library (libbq) never links,
+ * loads or calls it, and the two share no code: not a header, not a helper, not a table.
+ *
+ * Every floating-point result is computed in IEEE binary64 ("fp64"), summing k in
+ * ascending order; there is no blocking, fusion or reordering.
+ *
+ * What it follows
+ *   [card]    "prism-ml/Bonsai-27B-mlx-1bit - Hugging Face" model card.
+ *             Section "Weight representation: Binary g128": each weight is one sign
+ *             bit, 0 maps to -scale and 1 maps to +scale, and every 128 weights share
+ *             one FP16 scale (1 + 16/128 = 1.125 bits per weight).
+ *             Section "MLX packaging": scale-only groups are stored in MLX's
+ *             scale+bias form with s_mlx = 2*s_g and bias = -s_g, which reproduces
+ *             +-s_g exactly at 1.25 bits per weight.
+ *             Section "CUDA (NVIDIA GPUs)": the fused kernel unpacks the sign codes
+ *             inside the matrix product and applies the group scale; the model is
+ *             never expanded to a dense FP16 tensor.
+ *   [tern]    "Ternary Bonsai 27B vs ..." article (wmrh.cn), section
+ *             "三元量化技术突破" and "局限性与未来发展": ternary weights in {-1, 0, +1}
+ *             with the same FP16 scale per 128 weights, currently kept in 2-bit storage.
+ *   [agent]   "Bonsai 27B 将 270 亿参数 AI 带到手机" (agentlenshq), section
+ *             "两种硬件对应的运行点": ternary (-1, 0, +1) and binary (-1, +1) share the
+ *             same group scaling.
+ *
+ * Readings taken where the pages are silent (each is a choice, not a page fact):
+ *   - The group of 128 runs along K, the reduction axis of y = x W^T; weights are
+ *     row-major over the N output rows with K inner.
+ *   - Binary bits are LSB-first: bit (k % 32) of word (k / 32) of a row holds weight k,
+ *     so one group is 4 consecutive uint32 words.
+ *   - Ternary codes are 2-bit fields, LSB-first: bits 2*(k % 16)..2*(k % 16)+1 of word
+ *     (k / 16) hold code c with value c - 1 (0 -> -1, 1 -> 0, 2 -> +1); c = 3 is invalid.
+ *   - Scales are IEEE binary16 [N, K/128]; x is binary16 or bfloat16 [M, K].
+ *   - The tolerance bound of an output is 2e-3 * sum_k |x[m,k] * s[n, k/128]|; for
+ *     ternary weights the scale counts even where the code is 0.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "bq_oracle.h"
+
+/* ---------------------------------------------------------------------------------------
+ * Number formats.  Written from the IEEE 754-2008 binary16 definition and from bfloat16
+ * being the upper 16 bits of a binary32.
+ * ------------------------------------------------------------------------------------- */
+
+double bqo_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);                 /* subnormal: f * 2^-24 */
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25);     /* (1 + f/1024) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+double bqo_bf16_to_f64(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a double to a binary format with `p` significant bits, minimum normal exponent
+ * `emin` (value 2^emin) and largest finite value `maxv`; ties to even. Returns the
+ * rounded value as a double (inf on overflow). */
+static double round_to_format(double v, int p, int emin, double maxv)
+{
+    if (isnan(v) || isinf(v) || v == 0.0)
+        return v;
+    int e;
+    frexp(v, &e);                 /* v = m * 2^e, 0.5 <= |m| < 1 */
+    int exp_unbiased = e - 1;     /* v = 1.xxx * 2^(e-1) */
+    if (exp_unbiased < emin)
+        exp_unbiased = emin;      /* subnormal range: fixed quantum */
+    int quantum_exp = exp_unbiased - (p - 1);
+    double q = nearbyint(ldexp(v, -quantum_exp));   /* default rounding mode: ties-to-even */
+    double r = ldexp(q, quantum_exp);
+    if (fabs(r) > maxv)
+        return v > 0 ? INFINITY : -INFINITY;
+    return r;
+}
+
+uint16_t bqo_f64_to_bf16(double v)
+{
+    if (isnan(v))
+        return 0x7fc0;
+    double r = round_to_format(v, 8, -126, 3.38953138925153547590470800371487866880e+38);
+    float f = (float)r;           /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+void bqo_f64_to_bf16_array(const double *v, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = bqo_f64_to_bf16(v[i]);
+}
+
+uint16_t bqo_f64_to_f16(double v)
+{
+    if (isnan(v))
+        return 0x7e00;
+    double r = round_to_format(v, 11, -14, 65504.0);
+    uint16_t sign = signbit(r) ? 0x8000 : 0;
+    double a = fabs(r);
+    if (isinf(a))
+        return sign | 0x7c00;
+    if (a == 0.0)
+        return sign;
+    if (a < ldexp(1.0, -14))                           /* subnormal */
+        return sign | (uint16_t)ldexp(a, 24);
+    int e;
+    double m = frexp(a, &e);                           /* a = m * 2^e */
+    int biased = (e - 1) + 15;
+    uint16_t frac = (uint16_t)(ldexp(m, 11) - 1024.0);
+    return sign | (uint16_t)(biased << 10) | frac;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Sizes.
+ * ------------------------------------------------------------------------------------- */
+
+int64_t bqo_words_per_row(int fmt, int64_t K)
+{
+    if (K <= 0 || K % 128)
+        return -1;
+    if (fmt == BQO_BINARY)
+        return K / 32;            /* one bit per weight */
+    if (fmt == BQO_TERNARY)
+        return K / 16;            /* two bits per weight */
+    return -1;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Pack / unpack: loop over every k and set or read its bit (binary) or 2-bit field
+ * (ternary). [card] "Weight representation: Binary g128"; [tern] 2-bit storage.
+ * ------------------------------------------------------------------------------------- */
+
+int bqo_pack_binary_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                         uint32_t *words, uint16_t *s_out)
+{
+    int64_t W = bqo_words_per_row(BQO_BINARY, K);
+    if (W < 0 || N < 0)
+        return BQO_ERR_SHAPE;
+    for (int64_t i = 0; i < N * W; i++)
+        words[i] = 0;
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t k = 0; k < K; k++) {
+            int8_t v = q[n * K + k];
+            if (v == 1)
+                words[n * W + k / 32] |= (uint32_t)1 << (k % 32);   /* 1 -> +scale */
+            else if (v != -1)
+                return BQO_ERR_CODE;                                 /* 0 -> -scale */
+        }
+    }
+    for (int64_t i = 0; i < N * (K / 128); i++)
+        s_out[i] = s_in[i];
+    return BQO_OK;
+}
+
+int bqo_pack_ternary_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                          uint32_t *words, uint16_t *s_out)
+{
+    int64_t W = bqo_words_per_row(BQO_TERNARY, K);
+    if (W < 0 || N < 0)
+        return BQO_ERR_SHAPE;
+    for (int64_t i = 0; i < N * W; i++)
+        words[i] = 0;
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t k = 0; k < K; k++) {
+            int8_t v = q[n * K + k];
+            if (v < -1 || v > 1)
+                return BQO_ERR_CODE;
+            uint32_t code = (uint32_t)(v + 1);                       /* -1->0, 0->1, +1->2 */
+            words[n * W + k / 16] |= code << (2 * (k % 16));
+        }
+    }
+    for (int64_t i = 0; i < N * (K / 128); i++)
+        s_out[i] = s_in[i];
+    return BQO_OK;
+}
+
+int64_t bqo_unpack_binary_g128(const uint32_t *words, int64_t N, int64_t K, int8_t *q)
+{
+    int64_t W = bqo_words_per_row(BQO_BINARY, K);
+    if (W < 0 || N < 0)
+        return -1;
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) {
+            uint32_t bit = (words[n * W + k / 32] >> (k % 32)) & 1u;
+            q[n * K + k] = bit ? 1 : -1;
+        }
+    return 0;
+}
+
+/* Returns the number of invalid (code 3) fields; their q is set to 0. */
+int64_t bqo_unpack_ternary_g128(const uint32_t *words, int64_t N, int64_t K, int8_t *q)
+{
+    int64_t W = bqo_words_per_row(BQO_TERNARY, K);
+    if (W < 0 || N < 0)
+        return -1;
+    int64_t bad = 0;
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) {
+            uint32_t code = (words[n * W + k / 16] >> (2 * (k % 16))) & 3u;
+            if (code == 3) {
+                bad++;
+                q[n * K + k] = 0;
+            } else {
+                q[n * K + k] = (int8_t)((int)code - 1);
+            }
+        }
+    return bad;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Dequantised weight W[n, k] = s[n, k/128] * (2b - 1)   (binary, [card])
+ *                            = s[n, k/128] * (c - 1)    (ternary, [tern])
+ * ------------------------------------------------------------------------------------- */
+
+double bqo_weight(int fmt, const uint32_t *words, const uint16_t *scales, int64_t K,
+                  int64_t n, int64_t k)
+{
+    double s = bqo_f16_to_f64(scales[n * (K / 128) + k / 128]);
+    if (fmt == BQO_BINARY) {
+        uint32_t bit = (words[n * (K / 32) + k / 32] >> (k % 32)) & 1u;
+        return bit ? s : -s;
+    }
+    uint32_t code = (words[n * (K / 16) + k / 16] >> (2 * (k % 16))) & 3u;
+    if (code == 3)
+        return NAN;
+    return s * (double)((int)code - 1);
+}
+
+int bqo_dequant(int fmt, const uint32_t *words, const uint16_t *scales, int64_t N, int64_t K,
+                double *Wd)
+{
+    if (bqo_words_per_row(fmt, K) < 0 || N < 0)
+        return BQO_ERR_SHAPE;
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++)
+            Wd[n * K + k] = bqo_weight(fmt, words, scales, K, n, k);
+    return BQO_OK;
+}
+
+static double x_value(const uint16_t *x, int xt, int64_t i)
+{
+    return xt == BQO_X_F16 ? bqo_f16_to_f64(x[i]) : bqo_bf16_to_f64(x[i]);
+}
+
+/* ---------------------------------------------------------------------------------------
+ * y[m, r] = sum_k x[m, k] * W[rows[r], k]   in fp64, k ascending, and the tolerance bound
+ * bound[m, r] = 2e-3 * sum_k |x[m, k] * s[rows[r], k/128]|.
+ * The same function serves the decode GEMV (M <= 8) and the prefill GEMM (any M): a GEMM
+ * is the GEMV for every row of x. Outputs are [M, R] row-major.
+ * ------------------------------------------------------------------------------------- */
+
+int bqo_gemv_rows(int fmt, const uint16_t *x, int xt, int64_t M, int64_t K,
+                  const uint32_t *words, const uint16_t *scales, int64_t N,
+                  const int64_t *rows, int64_t R, double *y, double *bound)
+{
+    if (bqo_words_per_row(fmt, K) < 0 || M < 0 || N < 0 || R < 0)
+        return BQO_ERR_SHAPE;
+    for (int64_t r = 0; r < R; r++) {
+        int64_t n = rows[r];
+        if (n < 0 || n >= N)
+            return BQO_ERR_SHAPE;
+        for (int64_t m = 0; m < M; m++) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                double xv = x_value(x, xt, m * K + k);
+                acc += xv * bqo_weight(fmt, words, scales, K, n, k);
+                mag += fabs(xv * bqo_f16_to_f64(scales[n * (K / 128) + k / 128]));
+            }
+            y[m * R + r] = acc;
+            if (bound)
+                bound[m * R + r] = 2e-3 * mag;
+        }
+    }
+    return BQO_OK;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Embedding lookup: out[t, k] = W[ids[t], k]. [card] "Highlights": the embedding is one
+ * of the binary layers. Ids outside [0, N) give a row of zeros and are counted.
+ * ------------------------------------------------------------------------------------- */
+
+int64_t bqo_embed(int fmt, const int32_t *ids, int64_t T, const uint32_t *words,
+                  const uint16_t *scales, int64_t N, int64_t K, double *out)
+{
+    if (bqo_words_per_row(fmt, K) < 0 || T < 0 || N < 0)
+        return -1;
+    int64_t bad = 0;
+    for (int64_t t = 0; t < T; t++) {
+        int64_t id = ids[t];
+        for (int64_t k = 0; k < K; k++) {
+            if (id < 0 || id >= N)
+                out[t * K + k] = 0.0;
+            else
+                out[t * K + k] = bqo_weight(fmt, words, scales, K, id, k);
+        }
+        if (id < 0 || id >= N)
+            bad++;
+    }
+    return bad;
+}
+
+/* ---------------------------------------------------------------------------------------
+ * MLX affine form ([card] "MLX packaging"): w = s_mlx * q + bias with q in {0, 1},
+ * s_mlx = 2 * s and bias = -s, each stored and each operation rounded in binary16.
+ * Returns the binary16 bits of w.
+ * ------------------------------------------------------------------------------------- */
+
+uint16_t bqo_mlx_affine_dequant(uint16_t s_f16, int q01)
+{
+    double s = bqo_f16_to_f64(s_f16);
+    uint16_t s_mlx = bqo_f64_to_f16(2.0 * s);
+    uint16_t bias = bqo_f64_to_f16(-s);
+    double prod = bqo_f16_to_f64(bqo_f64_to_f16(bqo_f16_to_f64(s_mlx) * (double)q01));
+    return bqo_f64_to_f16(prod + bqo_f16_to_f64(bias));
+}

@@ -1,0 +1,383 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself -- a figure
+the pages print, a hand-derived layout example, a closed form, an invariant, a library
+routine (numpy / torch) on a special case, or brute force on tiny inputs.
+
+Every check is a ``pin_*`` function taking an oracle instance, so that
+``test_oracle_mutants.py`` can run the same checks against deliberately broken copies
+of the oracle (built on the CPU) and show that each plausible mistake fails one of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+from ternary_g128_weight_bq_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+B, T = oracle.BINARY, oracle.TERNARY
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _exact_x(M, K, seed):
+    """x with small dyadic values (multiples of 1/8 in [-4, 4]); products with fp16 scales
+    that are powers of two and all partial sums are exact in fp64, so any summation order
+    gives the same bits."""
+    rng = np.random.default_rng(seed)
+    return (rng.integers(-32, 33, size=(M, K)) / 8.0).astype(np.float16)
+
+
+def _pow2_scales(N, G, seed):
+    rng = np.random.default_rng(seed)
+    return (2.0 ** rng.integers(-6, 3, size=(N, G))).astype(np.float16)
+
+
+# --------------------------------------------------------------------------------------
+# Number formats (library routines: numpy float16, torch bfloat16)
+# --------------------------------------------------------------------------------------
+
+def pin_f16_decode(o):
+    bits = np.arange(65536, dtype=np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([o.f16_value(int(b)) for b in bits])
+    finite = np.isfinite(ref)
+    assert np.array_equal(got[finite], ref[finite])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[np.isinf(ref)], ref[np.isinf(ref)])
+
+
+def pin_bf16_decode(o):
+    bits = torch.arange(0, 65536, 7, dtype=torch.int32).to(torch.int16)
+    ref = bits.view(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([o.bf16_value(int(b) & 0xFFFF) for b in bits.tolist()])
+    finite = np.isfinite(ref)
+    assert np.array_equal(got[finite], ref[finite])
+
+
+def pin_bf16_round(o):
+    rng = np.random.default_rng(1)
+    # fp32-exact inputs so torch's float->bf16 conversion rounds once (ties to even)
+    v = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-39).astype(np.float32),          # bf16 subnormals
+        np.array([1.00390625, 1.01171875, -1.00390625, 3.0e38, -3.4e38, 0.0], np.float32),
+    ]).astype(np.float64)
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = o.to_bf16_bits(v)
+    assert np.array_equal(got, ref)
+
+
+def pin_f16_round(o):
+    rng = np.random.default_rng(2)
+    v = np.concatenate([
+        rng.standard_normal(5000) * 100.0,
+        rng.standard_normal(2000) * 1e-6,                                  # fp16 subnormals
+        np.array([65504.0, 65519.0, 65520.0, -70000.0, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11]),
+    ])
+    with np.errstate(over="ignore"):
+        ref = v.astype(np.float16).view(np.uint16)
+    got = o.to_f16_bits(v)
+    assert np.array_equal(got, ref)
+
+
+# --------------------------------------------------------------------------------------
+# Layout: hand-derived examples
+# --------------------------------------------------------------------------------------
+
+def pin_layout_examples(o):
+    g = _golden("layout_examples.json")
+    for ex in g["binary"]:
+        K = ex["K"]
+        q = -np.ones((1, K), np.int8)
+        q[0, ex["plus_one_at"]] = 1
+        st, words, _ = o.pack(B, q, np.ones((1, K // 128), np.float16))
+        assert st == oracle.OK
+        assert [f"{w:08x}" for w in words[0]] == ex["words_hex"]
+        back, bad = o.unpack(B, words, K)
+        assert bad == 0 and np.array_equal(back, q)
+    for ex in g["ternary"]:
+        K = ex["K"]
+        q = np.full((1, K), ex["default"], np.int8)
+        for k, v in ex["values_at"].items():
+            q[0, int(k)] = v
+        st, words, _ = o.pack(T, q, np.ones((1, K // 128), np.float16))
+        assert st == oracle.OK
+        assert [f"{w:08x}" for w in words[0]] == ex["words_hex"]
+        back, bad = o.unpack(T, words, K)
+        assert bad == 0 and np.array_equal(back, q)
+
+
+def pin_scale_index(o):
+    """Weight (n, k) takes the scale of row n, group k // 128."""
+    N, K = 3, 384
+    s = np.array([[1, 2, 4], [8, 16, 32], [0.5, 0.25, 0.125]], np.float16)
+    q = np.ones((N, K), np.int8)
+    _, words, s_out = o.pack(B, q, s)
+    W = o.dequant(B, words, s_out, K)
+    for n in range(N):
+        for k in (0, 127, 128, 255, 256, 383):
+            assert W[n, k] == float(s[n, k // 128])
+
+
+# --------------------------------------------------------------------------------------
+# Round trips
+# --------------------------------------------------------------------------------------
+
+def pin_roundtrip_binary(o):
+    N, K = 7, 640
+    words = synth.binary_words(3, N, K).numpy().view(np.uint32)
+    q, bad = o.unpack(B, words, K)
+    assert bad == 0 and set(np.unique(q)) <= {-1, 1}
+    st, words2, _ = o.pack(B, q, np.ones((N, K // 128), np.float16))
+    assert st == oracle.OK and np.array_equal(words2, words)
+
+
+def pin_roundtrip_ternary(o):
+    N, K = 5, 512
+    q = synth.random_ternary(4, synth.TID_TERNARY, (N, K)).numpy()
+    st, words, _ = o.pack(T, q, np.ones((N, K // 128), np.float16))
+    assert st == oracle.OK
+    back, bad = o.unpack(T, words, K)
+    assert bad == 0 and np.array_equal(back, q)
+    st, words2, _ = o.pack(T, back, np.ones((N, K // 128), np.float16))
+    assert np.array_equal(words2, words)
+
+
+def pin_invalid_codes(o):
+    K = 128
+    for fmt, badv in ((B, 0), (B, 2), (B, -2), (T, 2), (T, -2)):
+        q = np.ones((1, K), np.int8) if fmt == B else np.zeros((1, K), np.int8)
+        q[0, 77] = badv
+        st, _, _ = o.pack(fmt, q, np.ones((1, 1), np.float16))
+        assert st == oracle.ERR_CODE
+    # ternary code 3 in a packed word is reported by unpack
+    words = np.zeros((1, 8), np.uint32)
+    words[0, 2] = 0x3 << 6                       # field 3 of word 2 = k = 35
+    q, bad = o.unpack(T, words, K)
+    assert bad == 1 and q[0, 35] == 0
+    assert np.isnan(o.dequant(T, words, np.ones((1, 1), np.float16), K)[0, 35])
+    assert o.words_per_row(B, 100) == -1 and o.words_per_row(T, 0) == -1
+
+
+# --------------------------------------------------------------------------------------
+# Mapping and closed forms
+# --------------------------------------------------------------------------------------
+
+def pin_mapping_closed_form(o):
+    """All-ones group -> s * sum(x); all-zeros -> -s * sum(x)."""
+    K = 256
+    x = _exact_x(2, K, 5)
+    s = np.array([[0.5, 4.0], [0.5, 4.0]], np.float16)
+    words = np.zeros((2, K // 32), np.uint32)
+    words[0, :] = 0xFFFFFFFF                     # row 0: every bit 1
+    y, _ = o.gemv(B, x, oracle.X_F16, words, s, K)
+    xs = x.astype(np.float64)
+    for m in range(2):
+        expect1 = 0.5 * math.fsum(xs[m, :128]) + 4.0 * math.fsum(xs[m, 128:])
+        assert y[m, 0] == expect1
+        assert y[m, 1] == -expect1
+
+
+def pin_bound_closed_form(o):
+    K = 128
+    x = np.array([[1.0, -2.0] + [0.0] * 126], np.float16)
+    words = np.zeros((1, 4), np.uint32)
+    _, b = o.gemv(B, x, oracle.X_F16, words, np.array([[0.25]], np.float16), K)
+    assert b[0, 0] == 2e-3 * (0.25 + 0.5)
+    tw = np.full((1, 8), 0x55555555, np.uint32)   # ternary all-zero codes: scale still counts
+    _, bt = o.gemv(T, x, oracle.X_F16, tw, np.array([[0.25]], np.float16), K)
+    assert bt[0, 0] == 2e-3 * (0.25 + 0.5)
+
+
+# --------------------------------------------------------------------------------------
+# Brute force: dense fp64 matmul (numpy) of W = q * s built directly from the inputs
+# --------------------------------------------------------------------------------------
+
+def _dense(q, s):
+    return q.astype(np.float64) * np.repeat(s.astype(np.float64), 128, axis=1)
+
+
+def pin_bruteforce_exact(o):
+    for fmt, N, K, M in ((B, 9, 256, 3), (T, 6, 384, 8), (B, 1, 128, 1)):
+        q = (synth.random_signs(6, 1, (N, K)) if fmt == B
+             else synth.random_ternary(6, 2, (N, K))).numpy()
+        s = _pow2_scales(N, K // 128, 7)
+        x = _exact_x(M, K, 8)
+        st, words, s_out = o.pack(fmt, q, s)
+        assert st == oracle.OK
+        y, _ = o.gemv(fmt, x, oracle.X_F16, words, s_out, K)
+        ref = x.astype(np.float64) @ _dense(q, s).T
+        assert np.array_equal(y, ref)
+
+
+def pin_bruteforce_random(o):
+    N, K, M = 33, 512, 4
+    q = synth.random_signs(9, 1, (N, K)).numpy()
+    s = synth.scales(9, N, K // 128).numpy()
+    xb = synth.activations(9, M, K, dtype=torch.bfloat16)
+    st, words, s_out = o.pack(B, q, s)
+    y, b = o.gemv(B, xb, oracle.X_BF16, words, s_out, K)
+    ref = xb.to(torch.float64).numpy() @ _dense(q, s).T
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+    # the bound by brute force: 2e-3 * |x| @ |W|^T
+    bref = 2e-3 * (np.abs(xb.to(torch.float64).numpy()) @ np.abs(_dense(q, s)).T)
+    assert np.allclose(b, bref, rtol=1e-12, atol=0)
+
+
+def pin_dequant_vs_dense(o):
+    N, K = 4, 256
+    for fmt in (B, T):
+        q = (synth.random_signs(10, 1, (N, K)) if fmt == B
+             else synth.random_ternary(10, 2, (N, K))).numpy()
+        s = synth.scales(10, N, K // 128).numpy()
+        _, words, s_out = o.pack(fmt, q, s)
+        assert np.array_equal(o.dequant(fmt, words, s_out, K), _dense(q, s))
+
+
+# --------------------------------------------------------------------------------------
+# Invariants
+# --------------------------------------------------------------------------------------
+
+def pin_invariants(o):
+    N, K, M = 5, 256, 2
+    x = _exact_x(M, K, 11)
+    s = _pow2_scales(N, K // 128, 12)
+    words = synth.binary_words(13, N, K).numpy().view(np.uint32)
+    y, _ = o.gemv(B, x, oracle.X_F16, words, s, K)
+    # flipping every bit negates y
+    yn, _ = o.gemv(B, x, oracle.X_F16, ~words, s, K)
+    assert np.array_equal(yn, -y)
+    # scaling every scale by 2^j scales y by 2^j
+    y4, _ = o.gemv(B, x, oracle.X_F16, words, (s.astype(np.float64) * 4).astype(np.float16), K)
+    assert np.array_equal(y4, 4 * y)
+    # ternary with codes in {0, 2} equals binary with bit = code / 2
+    q, _ = o.unpack(B, words, K)
+    _, tw, _ = o.pack(T, q, s)
+    yt, _ = o.gemv(T, x, oracle.X_F16, tw, s, K)
+    assert np.array_equal(yt, y)
+    # ternary with every code 1 (value 0) gives exactly 0
+    z, _ = o.gemv(T, x, oracle.X_F16, np.full((N, K // 16), 0x55555555, np.uint32), s, K)
+    assert np.all(z == 0.0)
+    # linearity in x (exact values)
+    x2 = _exact_x(M, K, 14)
+    ya, _ = o.gemv(B, x2, oracle.X_F16, words, s, K)
+    yab, _ = o.gemv(B, (x.astype(np.float64) + x2.astype(np.float64)).astype(np.float16),
+                    oracle.X_F16, words, s, K)
+    assert np.array_equal(yab, y + ya)
+
+
+def pin_bf16_x(o):
+    """bf16 and fp16 encodings of the same values give the same y."""
+    K = 128
+    x16 = _exact_x(1, K, 15)
+    xbf = torch.from_numpy(x16.astype(np.float32)).to(torch.bfloat16)
+    words = synth.binary_words(16, 3, K).numpy().view(np.uint32)
+    s = _pow2_scales(3, 1, 17)
+    y1, _ = o.gemv(B, x16, oracle.X_F16, words, s, K)
+    y2, _ = o.gemv(B, xbf, oracle.X_BF16, words, s, K)
+    assert np.array_equal(y1, y2)
+
+
+# --------------------------------------------------------------------------------------
+# Embedding
+# --------------------------------------------------------------------------------------
+
+def pin_embed(o):
+    N, K = 50, 256
+    q = synth.random_signs(18, 1, (N, K)).numpy()
+    s = synth.scales(18, N, K // 128).numpy()
+    _, words, s_out = o.pack(B, q, s)
+    ids = np.array([3, 0, 49, 3, 17], np.int32)
+    out, bad = o.embed(B, ids, words, s_out, K)
+    assert bad == 0 and np.array_equal(out, _dense(q, s)[ids])
+    # bf16 rounding of the gathered rows equals torch's (fp16 values are fp32-exact)
+    ref = torch.from_numpy(out.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(o.to_bf16_bits(out), ref)
+    out2, bad2 = o.embed(B, np.array([-1, 50, 2], np.int32), words, s_out, K)
+    assert bad2 == 2 and np.all(out2[:2] == 0) and np.array_equal(out2[2], _dense(q, s)[2])
+
+
+# --------------------------------------------------------------------------------------
+# Sizes and the pages' printed figures
+# --------------------------------------------------------------------------------------
+
+def _stored_bpw(o, fmt, N=4, K=1280):
+    """Stored bits per weight from the sizes of the oracle's packed buffers."""
+    q = np.ones((N, K), np.int8)
+    st, words, s_out = o.pack(fmt, q, np.ones((N, K // 128), np.float16))
+    assert st == oracle.OK
+    return (words.nbytes + s_out.nbytes) * 8 / (N * K)
+
+
+def pin_bits_per_weight(o):
+    g = _golden("pages_figures.json")
+    bpw_b = _stored_bpw(o, B)
+    bpw_t = _stored_bpw(o, T)
+    assert bpw_b == g["bits_per_weight_binary"]["value"]
+    assert bpw_t == 2.125                           # 2-bit codes + the same 16-bit scale per 128
+    assert round(g["fp16_bits_per_weight"]["value"] / bpw_b, 1) == g["reduction_vs_fp16"]["value"]
+    # MLX scale+bias form: two fp16 values per group
+    mlx = (1 + 2 * 16 / 128)
+    assert mlx == g["mlx_bits_per_weight"]["value"]
+    P = g["language_params_billion"]["value"] * 1e9
+    assert abs(P * bpw_b / 8 / 1e9 - g["binary_deploy_gb"]["value"]) <= g["binary_deploy_gb"]["tol"]
+    assert abs(P * 16 / 8 / 1e9 - g["fp16_gb"]["value"]) <= g["fp16_gb"]["tol"]
+    assert abs(P * bpw_t / 8 / 1e9 - g["ternary_deploy_gb_2bit_storage"]["value"]) <= \
+        g["ternary_deploy_gb_2bit_storage"]["tol"]
+    true_t = math.log2(3) + 16 / 128
+    assert round(true_t, 2) == g["ternary_true_bits_per_weight"]["value"]
+    assert abs(P * true_t / 8 / 1e9 - g["ternary_theoretical_gb"]["value"]) <= g["ternary_theoretical_gb"]["tol"]
+    assert round(bpw_t / bpw_b, 1) == g["ternary_over_binary_bytes_per_step"]["value"]
+    # untied embedding + LM head: 2 * vocab * hidden ~ 2.5B
+    eh = 2 * g["vocab_size"]["value"] * g["hidden_size"]["value"] / 1e9
+    assert round(eh, 1) == g["embed_lmhead_params_billion"]["value"]
+    assert g["hidden_size"]["value"] % g["group_size"]["value"] == 0
+
+
+def pin_mlx_identity(o):
+    """s_mlx = 2 s, bias = -s reproduces +-s bit-exactly for every finite non-zero fp16 s
+    with |2s| finite (for s = +-0 the sum s + (-s) is +0, equal in value)."""
+    checked = 0
+    for sb in range(65536):
+        s = o.f16_value(sb)
+        if not math.isfinite(s) or abs(2 * s) > 65504:
+            continue
+        if s == 0.0:
+            assert o.f16_value(o.mlx_affine_dequant(sb, 0)) == 0.0
+            assert o.f16_value(o.mlx_affine_dequant(sb, 1)) == 0.0
+            continue
+        assert o.mlx_affine_dequant(sb, 1) == sb
+        assert o.mlx_affine_dequant(sb, 0) == sb ^ 0x8000
+        checked += 1
+    assert checked > 60000
+
+
+PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
+
+
+def test_f16_decode(orc): pin_f16_decode(orc)
+def test_bf16_decode(orc): pin_bf16_decode(orc)
+def test_bf16_round(orc): pin_bf16_round(orc)
+def test_f16_round(orc): pin_f16_round(orc)
+def test_layout_examples(orc): pin_layout_examples(orc)
+def test_scale_index(orc): pin_scale_index(orc)
+def test_roundtrip_binary(orc): pin_roundtrip_binary(orc)
+def test_roundtrip_ternary(orc): pin_roundtrip_ternary(orc)
+def test_invalid_codes(orc): pin_invalid_codes(orc)
+def test_mapping_closed_form(orc): pin_mapping_closed_form(orc)
+def test_bound_closed_form(orc): pin_bound_closed_form(orc)
+def test_bruteforce_exact(orc): pin_bruteforce_exact(orc)
+def test_bruteforce_random(orc): pin_bruteforce_random(orc)
+def test_dequant_vs_dense(orc): pin_dequant_vs_dense(orc)
+def test_invariants(orc): pin_invariants(orc)
+def test_bf16_x(orc): pin_bf16_x(orc)
+def test_embed(orc): pin_embed(orc)
+def test_bits_per_weight(orc): pin_bits_per_weight(orc)
+def test_mlx_identity(orc): pin_mlx_identity(orc)
