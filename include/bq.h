@@ -1,0 +1,184 @@
+/*
+ * bq.h -- C ABI of libbq: linear layers run directly on packed binary-g128 and
+ * ternary-g128 weights on an NVIDIA B200 (sm_100a). The weights are never expanded to a
+ * dense FP16/BF16 tensor in device memory.
+ *
+ * The operations follow these pages:
+ *   "prism-ml/Bonsai-27B-mlx-1bit - Hugging Face" model card
+ *     - section "Weight representation: Binary g128": one sign bit per weight, bit 0 is
+ *       -scale and bit 1 is +scale; 128 weights share one FP16 scale (1.125 bits/weight).
+ *     - section "Highlights" / "Model overview": embedding, attention and MLP projections
+ *       and the LM head are all binary-g128 layers.
+ *     - section "CUDA (NVIDIA GPUs)": the matrix product unpacks the sign codes inside
+ *       the kernel and applies the group scale; no dense FP16 copy is made.
+ *     - section "Cross-platform throughput": tg128 (batch-1 decode) is bound by memory
+ *       bandwidth, pp512 (512-token prompt) by compute.
+ *   "Ternary Bonsai 27B vs ..." article (wmrh.cn), sections "三元量化技术突破" and
+ *     "局限性与未来发展": ternary weights {-1, 0, +1} with the same FP16 scale per 128
+ *     weights, kept in 2-bit storage.
+ *
+ * Packed layout (this library's fixed format; the pages give only the meaning of a
+ * bit and the group size):
+ *   - A weight matrix has N output rows and K inputs, K a multiple of 128; groups of 128
+ *     run along K. Row-major over N with K inner.
+ *   - Binary: uint32 words[N][K/32]; weight k of a row is bit (k % 32) of word (k / 32)
+ *     (LSB first), so one group is 4 consecutive words (16 bytes).
+ *   - Ternary: uint32 words[N][K/16]; weight k is the 2-bit field at bits
+ *     2*(k % 16) .. 2*(k % 16)+1 of word (k / 16); code 0 -> -1, 1 -> 0, 2 -> +1, and code 3
+ *     is invalid (never written by the pack calls; results of the compute calls are
+ *     undefined where it occurs; bq_unpack_g128 reports it). One group is 8 words.
+ *   - Scales: IEEE binary16 scales[N][K/128].
+ *   - Activations x[M][K] and outputs y[M][N] are dense row-major.
+ *
+ * Conventions for every call:
+ *   - All data pointers are DEVICE pointers on the current CUDA device, owned by the
+ *     caller; the library keeps no reference after the call returns. Pointers to words,
+ *     scales, x, y, q and workspace must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` unless stated otherwise. The returned status
+ *     covers argument validation and the kernel launch; BQ_OK means "enqueued".
+ *   - On any status other than BQ_OK nothing has been launched, and bq_last_error()
+ *     returns a message for the calling thread.
+ *   - Device-side conditions (an out-of-range token id, a bounded wait that gave up) set
+ *     a per-device error word that bq_get_device_error() reads and clears.
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BQ_OK = 0,
+    BQ_ERR_INVALID_ARG = 1,   /* null pointer, negative size or unknown enum value */
+    BQ_ERR_SHAPE = 2,         /* K not a multiple of 128, M or N out of the supported range */
+    BQ_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+    BQ_ERR_DTYPE = 4,         /* unsupported dtype for this argument */
+    BQ_ERR_INVALID_CODE = 5,  /* a weight value outside the format's value set */
+    BQ_ERR_CUDA = 6,          /* a CUDA runtime call or a launch failed */
+    BQ_ERR_TIMEOUT = 7,       /* a bounded device-side wait gave up */
+    BQ_ERR_UNSUPPORTED = 8,   /* the current device is not sm_100 */
+    BQ_ERR_WORKSPACE = 9      /* workspace pointer null or smaller than required */
+} bq_status;
+
+typedef enum { BQ_F16 = 0, BQ_BF16 = 1, BQ_F32 = 2 } bq_dtype;
+
+typedef enum { BQ_BINARY_G128 = 0, BQ_TERNARY_G128 = 1 } bq_format;
+
+/* Non-owning view of a packed weight matrix (device memory). */
+typedef struct {
+    bq_format fmt;
+    int64_t N;                /* output rows, >= 1 */
+    int64_t K;                /* inputs per row, a positive multiple of 128 */
+    const uint32_t *words;    /* [N][K/32] (binary) or [N][K/16] (ternary) */
+    const uint16_t *scales;   /* fp16 [N][K/128] */
+} bq_weight;
+
+/* Library version string, e.g. "bq 0.1.0 sm_100a". */
+const char *bq_version(void);
+
+/* Name of a status code. */
+const char *bq_status_string(bq_status st);
+
+/* Message describing the last non-OK status returned to the calling thread. */
+const char *bq_last_error(void);
+
+/* Number of uint32 words in a packed matrix: N*K/32 (binary) or N*K/16 (ternary);
+ * 0 if the arguments are invalid. Scales always take N*K/128 fp16 values. */
+size_t bq_packed_words(bq_format fmt, int64_t N, int64_t K);
+
+/*
+ * Pack already-quantised weights into the binary-g128 format.
+ *   q      int8 [N][K], values in {-1, +1} (-1 -> bit 0 -> -scale, +1 -> bit 1 -> +scale)
+ *   s_in   fp16 [N][K/128] group scales; copied to s_out (s_out may equal s_in)
+ *   words  out, uint32 [N][K/32]
+ * Model card "prism-ml/Bonsai-27B-mlx-1bit", section "Weight representation: Binary g128".
+ * SYNCHRONOUS: validates every q on the device, then waits for `stream`.
+ * Returns BQ_ERR_INVALID_CODE if any q is outside {-1, +1} (words then hold garbage).
+ */
+bq_status bq_pack_binary_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                              uint32_t *words, uint16_t *s_out, cudaStream_t stream);
+
+/*
+ * Pack already-quantised ternary weights (q in {-1, 0, +1}) into 2-bit codes
+ * (code = q + 1), uint32 [N][K/16]. Ternary Bonsai 27B article (wmrh.cn), section
+ * "局限性与未来发展" (2-bit storage). Synchronous, like the binary call; returns
+ * BQ_ERR_INVALID_CODE if any q is outside {-1, 0, +1}.
+ */
+bq_status bq_pack_ternary_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                               uint32_t *words, uint16_t *s_out, cudaStream_t stream);
+
+/*
+ * Inverse of the pack calls: q int8 [N][K] and, if s_out is not NULL, a copy of the
+ * scales. SYNCHRONOUS. Returns BQ_ERR_INVALID_CODE if a ternary code 3 is found (its q is
+ * written as 0).
+ */
+bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStream_t stream);
+
+/*
+ * Decode GEMV: y[m][n] = sum_g s[n][g] * sum_{k in group g} v[n][k] * x[m][k], with
+ * v = 2b - 1 (binary) or c - 1 (ternary), for M <= 8 token rows.
+ * Model card "prism-ml/Bonsai-27B-mlx-1bit", sections "Weight representation: Binary g128"
+ * and "CUDA (NVIDIA GPUs)"; the decode (tg128) workload of section "Cross-platform
+ * throughput".
+ *   x          [M][K], xt = BQ_F16 or BQ_BF16
+ *   M          1..8
+ *   y          [M][N], yt = BQ_F32, BQ_BF16 or BQ_F16 (fp32 accumulation, rounded once)
+ *   workspace  device scratch of at least bq_gemv_workspace_bytes(M, w) bytes (may be
+ *              NULL when that size is 0); its contents need not be initialised and are
+ *              left undefined. Calls that share a workspace must be ordered on one stream.
+ */
+bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w,
+                  void *y, bq_dtype yt, void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes bq_gemv needs for this shape (0 if none). */
+size_t bq_gemv_workspace_bytes(int64_t M, const bq_weight *w);
+
+/*
+ * Prefill GEMM: the same product for M up to 512 token rows (larger M is accepted),
+ * Y[M][N] = X[M][K] * W^T with W the dequantised +-s (binary) or {-s, 0, +s} (ternary)
+ * matrix. The packed tiles are unpacked into shared memory next to the tensor cores
+ * (tcgen05, accumulation in fp32 in tensor memory); no expanded copy is written to device
+ * memory. The pp512 (512-token prompt, compute-bound) workload of the model card's section
+ * "Cross-platform throughput" and of the Ternary Bonsai 27B article's throughput table.
+ *   x  [M][K], xt = BQ_F16 or BQ_BF16. The scale is applied inside the operand, rounded to
+ *      x's type (exact for BQ_F16; bf16 keeps 8 of the scale's 11 significant bits).
+ *   y  [M][N], yt = BQ_F32, BQ_BF16 or BQ_F16.
+ *   workspace: at least bq_gemm_prefill_workspace_bytes(M, w) bytes (currently 0).
+ */
+bq_status bq_gemm_prefill(const void *x, bq_dtype xt, int64_t M, const bq_weight *w,
+                          void *y, bq_dtype yt, void *workspace, size_t ws_bytes,
+                          cudaStream_t stream);
+
+size_t bq_gemm_prefill_workspace_bytes(int64_t M, const bq_weight *w);
+
+/*
+ * Embedding lookup on a packed matrix: out[t][k] = s[id][k/128] * v[id][k] for
+ * id = ids[t]. Model card section "Highlights": the embedding is one of the binary layers.
+ *   ids  int32 [T] device array
+ *   out  [T][K], ot = BQ_BF16 (the +-s value rounded to nearest even), BQ_F16 (exact) or
+ *        BQ_F32 (exact)
+ * An id outside [0, N) is not read: its row is written as zeros and the device error
+ * word records BQ_ERR_INVALID_ARG (see bq_get_device_error).
+ */
+bq_status bq_embed_gather(const int32_t *ids, int64_t T, const bq_weight *w, void *out,
+                          bq_dtype ot, cudaStream_t stream);
+
+/*
+ * Wait for `stream`, then read and clear the current device's error word. Returns BQ_OK,
+ * BQ_ERR_INVALID_ARG (an out-of-range embedding id was seen) or BQ_ERR_TIMEOUT (a bounded
+ * device wait gave up; that kernel's outputs are undefined). Kernels on any stream of
+ * the device share the word.
+ */
+bq_status bq_get_device_error(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H */

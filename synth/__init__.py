@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for the packed g128 linear layers.
+"""Seeded synthetic inputs for the packed g128 linear layers (a module of its own).
 
 This module is the one piece of code that both the CUDA path's tests/benchmark and
 the CPU oracle's tests use: it only draws random numbers. It holds none of the

@@ -1,0 +1,233 @@
+"""Python binding of libbq: linear layers on packed binary-g128 / ternary-g128 weights for
+NVIDIA B200 (sm_100a).
+
+This module only marshals arguments: it passes device pointers of torch tensors and the
+current CUDA stream to the C ABI declared in ``include/bq.h``. Every step of the
+computation runs in libbq's CUDA kernels. If the compiled library is missing the import
+fails loudly; there is no fallback.
+
+Build the library with ``python -m ternary_g128_weight_bq_b200.build``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbq.so")
+
+BINARY_G128 = 0
+TERNARY_G128 = 1
+
+_DTYPE = {torch.float16: 0, torch.bfloat16: 1, torch.float32: 2}
+
+STATUS = {
+    0: "BQ_OK", 1: "BQ_ERR_INVALID_ARG", 2: "BQ_ERR_SHAPE", 3: "BQ_ERR_ALIGNMENT",
+    4: "BQ_ERR_DTYPE", 5: "BQ_ERR_INVALID_CODE", 6: "BQ_ERR_CUDA", 7: "BQ_ERR_TIMEOUT",
+    8: "BQ_ERR_UNSUPPORTED", 9: "BQ_ERR_WORKSPACE",
+}
+
+
+class BQError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+        self.status_name = STATUS.get(status, str(status))
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("words", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libbq (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libbq.so not found at {LIB_PATH}; build it with "
+                              "`python -m ternary_g128_weight_bq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        W = ctypes.POINTER(_Weight)
+        sig = {
+            "bq_version": ([], ctypes.c_char_p),
+            "bq_status_string": ([I], ctypes.c_char_p),
+            "bq_last_error": ([], ctypes.c_char_p),
+            "bq_packed_words": ([I, I64, I64], ctypes.c_size_t),
+            "bq_pack_binary_g128": ([P, P, I64, I64, P, P, P], I),
+            "bq_pack_ternary_g128": ([P, P, I64, I64, P, P, P], I),
+            "bq_unpack_g128": ([W, P, P, P], I),
+            "bq_gemv": ([P, I, I64, W, P, I, P, ctypes.c_size_t, P], I),
+            "bq_gemv_workspace_bytes": ([I64, W], ctypes.c_size_t),
+            "bq_gemm_prefill": ([P, I, I64, W, P, I, P, ctypes.c_size_t, P], I),
+            "bq_gemm_prefill_workspace_bytes": ([I64, W], ctypes.c_size_t),
+            "bq_embed_gather": ([P, I64, W, P, I, P], I),
+            "bq_get_device_error": ([P], I),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise BQError(status, lib().bq_last_error().decode())
+
+
+def _stream(device=None) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclass
+class BQWeight:
+    """A packed weight matrix held in device memory.
+
+    words: int32 [N, K/32] (binary) or [N, K/16] (ternary), the uint32 bit patterns.
+    scales: float16 [N, K/128].
+    """
+    fmt: int
+    N: int
+    K: int
+    words: torch.Tensor
+    scales: torch.Tensor
+
+    def __post_init__(self):
+        _dev(self.words, "words")
+        _dev(self.scales, "scales")
+        wpr = self.K // (32 if self.fmt == BINARY_G128 else 16)
+        if tuple(self.words.shape) != (self.N, wpr) or self.words.dtype != torch.int32:
+            raise ValueError(f"words must be int32 [{self.N}, {wpr}]")
+        if tuple(self.scales.shape) != (self.N, self.K // 128) or self.scales.dtype != torch.float16:
+            raise ValueError(f"scales must be float16 [{self.N}, {self.K // 128}]")
+        self._c = _Weight(self.fmt, self.N, self.K, self.words.data_ptr(), self.scales.data_ptr())
+
+    @property
+    def c(self):
+        return ctypes.byref(self._c)
+
+    @property
+    def nbytes(self) -> int:
+        return self.words.numel() * 4 + self.scales.numel() * 2
+
+
+def version() -> str:
+    return lib().bq_version().decode()
+
+
+def packed_words(fmt: int, N: int, K: int) -> int:
+    return int(lib().bq_packed_words(fmt, N, K))
+
+
+def _pack(fn, fmt, q, s):
+    _dev(q, "q")
+    _dev(s, "s")
+    if q.dtype != torch.int8 or q.dim() != 2:
+        raise ValueError("q must be int8 [N, K]")
+    N, K = q.shape
+    if s.dtype != torch.float16:
+        raise ValueError("s must be float16 [N, K/128]")
+    wpr = max(K // (32 if fmt == BINARY_G128 else 16), 1)
+    words = torch.empty((N, wpr), dtype=torch.int32, device=q.device)
+    s_out = torch.empty((N, max(K // 128, 1)), dtype=torch.float16, device=q.device)
+    _check(fn(q.data_ptr(), s.data_ptr(), N, K, words.data_ptr(), s_out.data_ptr(),
+              _stream(q.device)))
+    return BQWeight(fmt, N, K, words, s_out)
+
+
+def pack_binary_g128(q: torch.Tensor, s: torch.Tensor) -> BQWeight:
+    """Pack int8 q in {-1, +1} [N, K] and fp16 scales [N, K/128] (synchronous; validates q)."""
+    return _pack(lib().bq_pack_binary_g128, BINARY_G128, q, s)
+
+
+def pack_ternary_g128(q: torch.Tensor, s: torch.Tensor) -> BQWeight:
+    """Pack int8 q in {-1, 0, +1} [N, K] and fp16 scales (synchronous; validates q)."""
+    return _pack(lib().bq_pack_ternary_g128, TERNARY_G128, q, s)
+
+
+def unpack_g128(w: BQWeight):
+    """(q int8 [N, K], scales fp16 [N, K/128]) of a packed matrix (synchronous)."""
+    q = torch.empty((w.N, w.K), dtype=torch.int8, device=w.words.device)
+    s = torch.empty_like(w.scales)
+    _check(lib().bq_unpack_g128(w.c, q.data_ptr(), s.data_ptr(), _stream(q.device)))
+    return q, s
+
+
+def gemv_workspace_bytes(M: int, w: BQWeight) -> int:
+    return int(lib().bq_gemv_workspace_bytes(M, w.c))
+
+
+def gemv(x: torch.Tensor, w: BQWeight, out_dtype=torch.float32, out: torch.Tensor = None,
+         workspace: torch.Tensor = None) -> torch.Tensor:
+    """Decode GEMV: y[M, N] = x[M, K] @ W^T for M <= 8 (fp32 accumulation)."""
+    _dev(x, "x")
+    if x.dim() != 2 or x.shape[1] != w.K:
+        raise ValueError(f"x must be [M, {w.K}]")
+    M = x.shape[0]
+    if out is None:
+        out = torch.empty((M, w.N), dtype=out_dtype, device=x.device)
+    _dev(out, "out")
+    need = gemv_workspace_bytes(M, w)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().bq_gemv(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(), _DTYPE[out.dtype],
+                         ws_ptr, ws_bytes, _stream(x.device)))
+    return out
+
+
+def gemm_prefill(x: torch.Tensor, w: BQWeight, out_dtype=torch.float32,
+                 out: torch.Tensor = None) -> torch.Tensor:
+    """Prefill GEMM: Y[M, N] = X[M, K] @ W^T on the tensor cores (fp32 accumulation)."""
+    _dev(x, "x")
+    if x.dim() != 2 or x.shape[1] != w.K:
+        raise ValueError(f"x must be [M, {w.K}]")
+    M = x.shape[0]
+    if out is None:
+        out = torch.empty((M, w.N), dtype=out_dtype, device=x.device)
+    _dev(out, "out")
+    need = int(lib().bq_gemm_prefill_workspace_bytes(M, w.c))
+    ws = torch.empty(need, dtype=torch.uint8, device=x.device) if need else None
+    _check(lib().bq_gemm_prefill(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(),
+                                 _DTYPE[out.dtype], ws.data_ptr() if ws is not None else None,
+                                 need, _stream(x.device)))
+    return out
+
+
+def embed_gather(ids: torch.Tensor, w: BQWeight, out_dtype=torch.bfloat16,
+                 out: torch.Tensor = None) -> torch.Tensor:
+    """Embedding lookup: out[t, :] = dequantised row ids[t] of w."""
+    _dev(ids, "ids")
+    if ids.dtype != torch.int32 or ids.dim() != 1:
+        raise ValueError("ids must be int32 [T]")
+    T = ids.shape[0]
+    if out is None:
+        out = torch.empty((T, w.K), dtype=out_dtype, device=ids.device)
+    _dev(out, "out")
+    _check(lib().bq_embed_gather(ids.data_ptr(), T, w.c, out.data_ptr(), _DTYPE[out.dtype],
+                                 _stream(ids.device)))
+    return out
+
+
+def get_device_error():
+    """Synchronise the current stream and raise BQError if a device-side condition was
+    recorded (an out-of-range embedding id, a bounded wait that gave up)."""
+    _check(lib().bq_get_device_error(_stream()))

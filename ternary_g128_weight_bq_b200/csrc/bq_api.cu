@@ -1,0 +1,329 @@
+// bq_api.cu -- the C ABI of libbq: argument validation, dispatch to the kernels, status
+// codes and the per-device error word.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "bq_internal.cuh"
+
+namespace bq {
+
+// Per-device status array: [kSlotErrBits] sticky device-side error bits,
+// [kSlotInvalidCount] counter for the synchronous pack/unpack validation.
+__device__ unsigned int g_status[4];
+
+static thread_local char t_msg[512] = "no error";
+
+bq_status set_error(bq_status st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_msg, sizeof t_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+bq_status check_launch(const char *what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return BQ_OK;
+}
+
+static constexpr int kMaxDevices = 64;
+static unsigned int *g_status_ptr[kMaxDevices];
+static bool g_checked_arch[kMaxDevices];
+
+unsigned int *device_status(bq_status *st)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        *st = set_error(BQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+        return nullptr;
+    }
+    if (!g_checked_arch[dev]) {
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (major != 10 || minor != 0) {
+            *st = set_error(BQ_ERR_UNSUPPORTED,
+                            "device %d is sm_%d%d; libbq is built for sm_100a only", dev, major, minor);
+            return nullptr;
+        }
+        g_checked_arch[dev] = true;
+    }
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_status);
+        if (e != cudaSuccess) {
+            *st = set_error(BQ_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+            return nullptr;
+        }
+        g_status_ptr[dev] = static_cast<unsigned int *>(p);
+    }
+    *st = BQ_OK;
+    return g_status_ptr[dev];
+}
+
+static bq_status validate_weight(const bq_weight *w)
+{
+    if (!w)
+        return set_error(BQ_ERR_INVALID_ARG, "weight view is NULL");
+    if (w->fmt != BQ_BINARY_G128 && w->fmt != BQ_TERNARY_G128)
+        return set_error(BQ_ERR_INVALID_ARG, "unknown format %d", (int)w->fmt);
+    if (w->N < 1 || w->K < 128 || w->K % 128)
+        return set_error(BQ_ERR_SHAPE, "N=%lld K=%lld: need N >= 1 and K a positive multiple of 128",
+                         (long long)w->N, (long long)w->K);
+    if (w->N > (int64_t(1) << 31) || w->K > (int64_t(1) << 24))
+        return set_error(BQ_ERR_SHAPE, "N=%lld K=%lld beyond the supported range",
+                         (long long)w->N, (long long)w->K);
+    if (!w->words || !w->scales)
+        return set_error(BQ_ERR_INVALID_ARG, "weight words or scales pointer is NULL");
+    if (!aligned16(w->words) || !aligned16(w->scales))
+        return set_error(BQ_ERR_ALIGNMENT, "weight words and scales must be 16-byte aligned");
+    return BQ_OK;
+}
+
+}  // namespace bq
+
+using namespace bq;
+
+extern "C" {
+
+const char *bq_version(void) { return "bq 0.1.0 sm_100a"; }
+
+const char *bq_status_string(bq_status st)
+{
+    switch (st) {
+    case BQ_OK: return "BQ_OK";
+    case BQ_ERR_INVALID_ARG: return "BQ_ERR_INVALID_ARG";
+    case BQ_ERR_SHAPE: return "BQ_ERR_SHAPE";
+    case BQ_ERR_ALIGNMENT: return "BQ_ERR_ALIGNMENT";
+    case BQ_ERR_DTYPE: return "BQ_ERR_DTYPE";
+    case BQ_ERR_INVALID_CODE: return "BQ_ERR_INVALID_CODE";
+    case BQ_ERR_CUDA: return "BQ_ERR_CUDA";
+    case BQ_ERR_TIMEOUT: return "BQ_ERR_TIMEOUT";
+    case BQ_ERR_UNSUPPORTED: return "BQ_ERR_UNSUPPORTED";
+    case BQ_ERR_WORKSPACE: return "BQ_ERR_WORKSPACE";
+    }
+    return "unknown status";
+}
+
+const char *bq_last_error(void) { return t_msg; }
+
+size_t bq_packed_words(bq_format fmt, int64_t N, int64_t K)
+{
+    if (N < 1 || K < 128 || K % 128)
+        return 0;
+    if (fmt == BQ_BINARY_G128)
+        return (size_t)N * (size_t)(K / 32);
+    if (fmt == BQ_TERNARY_G128)
+        return (size_t)N * (size_t)(K / 16);
+    return 0;
+}
+
+static bq_status pack_common(int fmt, const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                             uint32_t *words, uint16_t *s_out, cudaStream_t stream)
+{
+    if (!q || !s_in || !words || !s_out)
+        return set_error(BQ_ERR_INVALID_ARG, "pack: NULL pointer");
+    if (N < 1 || K < 128 || K % 128 || N > (int64_t(1) << 31) || K > (int64_t(1) << 24))
+        return set_error(BQ_ERR_SHAPE, "pack: N=%lld K=%lld invalid", (long long)N, (long long)K);
+    if (!aligned16(q) || !aligned16(words))
+        return set_error(BQ_ERR_ALIGNMENT, "pack: q and words must be 16-byte aligned");
+    bq_status st;
+    unsigned int *status = device_status(&st);
+    if (!status)
+        return st;
+    unsigned int *cnt = status + kSlotInvalidCount;
+    cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(unsigned int), stream);
+    if (e == cudaSuccess)
+        e = fmt == BQ_BINARY_G128 ? launch_pack_binary(q, N, K, words, cnt, stream)
+                                  : launch_pack_ternary(q, N, K, words, cnt, stream);
+    if (e == cudaSuccess && s_out != s_in)
+        e = cudaMemcpyAsync(s_out, s_in, (size_t)N * (size_t)(K / 128) * 2, cudaMemcpyDeviceToDevice,
+                            stream);
+    unsigned int host_cnt = 0;
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(&host_cnt, cnt, sizeof host_cnt, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "pack: %s", cudaGetErrorString(e));
+    if (host_cnt)
+        return set_error(BQ_ERR_INVALID_CODE, "pack: %u weights outside the format's value set",
+                         host_cnt);
+    return BQ_OK;
+}
+
+bq_status bq_pack_binary_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                              uint32_t *words, uint16_t *s_out, cudaStream_t stream)
+{
+    return pack_common(BQ_BINARY_G128, q, s_in, N, K, words, s_out, stream);
+}
+
+bq_status bq_pack_ternary_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                               uint32_t *words, uint16_t *s_out, cudaStream_t stream)
+{
+    return pack_common(BQ_TERNARY_G128, q, s_in, N, K, words, s_out, stream);
+}
+
+bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStream_t stream)
+{
+    bq_status st = validate_weight(w);
+    if (st != BQ_OK)
+        return st;
+    if (!q)
+        return set_error(BQ_ERR_INVALID_ARG, "unpack: q is NULL");
+    if (!aligned16(q))
+        return set_error(BQ_ERR_ALIGNMENT, "unpack: q must be 16-byte aligned");
+    unsigned int *status = device_status(&st);
+    if (!status)
+        return st;
+    unsigned int *cnt = status + kSlotInvalidCount;
+    cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(unsigned int), stream);
+    if (e == cudaSuccess)
+        e = launch_unpack(w->fmt, w->words, w->N, w->K, q, cnt, stream);
+    if (e == cudaSuccess && s_out && s_out != w->scales)
+        e = cudaMemcpyAsync(s_out, w->scales, (size_t)w->N * (size_t)(w->K / 128) * 2,
+                            cudaMemcpyDeviceToDevice, stream);
+    unsigned int host_cnt = 0;
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(&host_cnt, cnt, sizeof host_cnt, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "unpack: %s", cudaGetErrorString(e));
+    if (host_cnt)
+        return set_error(BQ_ERR_INVALID_CODE, "unpack: %u ternary fields hold the invalid code 3",
+                         host_cnt);
+    return BQ_OK;
+}
+
+static bq_status validate_xy(const char *who, const void *x, bq_dtype xt, const void *y, bq_dtype yt)
+{
+    if (!x || !y)
+        return set_error(BQ_ERR_INVALID_ARG, "%s: x or y is NULL", who);
+    if (xt != BQ_F16 && xt != BQ_BF16)
+        return set_error(BQ_ERR_DTYPE, "%s: x must be BQ_F16 or BQ_BF16", who);
+    if (yt != BQ_F32 && yt != BQ_BF16 && yt != BQ_F16)
+        return set_error(BQ_ERR_DTYPE, "%s: y must be BQ_F32, BQ_BF16 or BQ_F16", who);
+    if (!aligned16(x) || !aligned16(y))
+        return set_error(BQ_ERR_ALIGNMENT, "%s: x and y must be 16-byte aligned", who);
+    return BQ_OK;
+}
+
+size_t bq_gemv_workspace_bytes(int64_t M, const bq_weight *w)
+{
+    if (!w || M < 1 || M > 8 || w->N < 1 || w->K < 128 || w->K % 128)
+        return 0;
+    return gemv_workspace_bytes((int)M, w->fmt, w->N, w->K);
+}
+
+bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, void *y, bq_dtype yt,
+                  void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    bq_status st = validate_weight(w);
+    if (st != BQ_OK)
+        return st;
+    if ((st = validate_xy("gemv", x, xt, y, yt)) != BQ_OK)
+        return st;
+    if (M < 1 || M > 8)
+        return set_error(BQ_ERR_SHAPE, "gemv: M=%lld, need 1 <= M <= 8", (long long)M);
+    size_t need = gemv_workspace_bytes((int)M, w->fmt, w->N, w->K);
+    if (need && (!workspace || ws_bytes < need))
+        return set_error(BQ_ERR_WORKSPACE, "gemv: workspace needs %zu bytes, got %zu", need,
+                         workspace ? ws_bytes : (size_t)0);
+    if (workspace && !aligned16(workspace))
+        return set_error(BQ_ERR_ALIGNMENT, "gemv: workspace must be 16-byte aligned");
+    if (!device_status(&st))
+        return st;
+    GemvArgs a{x, (int)xt, (int)M, (int)w->fmt, w->N, w->K, w->words,
+               reinterpret_cast<const __half *>(w->scales), y, (int)yt, workspace, ws_bytes};
+    cudaError_t e = launch_gemv(a, stream);
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "gemv launch: %s", cudaGetErrorString(e));
+    return BQ_OK;
+}
+
+size_t bq_gemm_prefill_workspace_bytes(int64_t M, const bq_weight *w)
+{
+    if (!w || M < 1 || w->N < 1 || w->K < 128 || w->K % 128)
+        return 0;
+    return prefill_workspace_bytes(M, w->fmt, w->N, w->K);
+}
+
+bq_status bq_gemm_prefill(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, void *y,
+                          bq_dtype yt, void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    bq_status st = validate_weight(w);
+    if (st != BQ_OK)
+        return st;
+    if ((st = validate_xy("gemm_prefill", x, xt, y, yt)) != BQ_OK)
+        return st;
+    if (M < 1 || M > (int64_t(1) << 24))
+        return set_error(BQ_ERR_SHAPE, "gemm_prefill: M=%lld out of range", (long long)M);
+    size_t need = prefill_workspace_bytes(M, w->fmt, w->N, w->K);
+    if (need && (!workspace || ws_bytes < need))
+        return set_error(BQ_ERR_WORKSPACE, "gemm_prefill: workspace needs %zu bytes", need);
+    unsigned int *status = device_status(&st);
+    if (!status)
+        return st;
+    PrefillArgs a{x, (int)xt, M, (int)w->fmt, w->N, w->K, w->words,
+                  reinterpret_cast<const __half *>(w->scales), y, (int)yt, status};
+    cudaError_t e = launch_prefill(a, stream);
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "gemm_prefill launch: %s", cudaGetErrorString(e));
+    return BQ_OK;
+}
+
+bq_status bq_embed_gather(const int32_t *ids, int64_t T, const bq_weight *w, void *out, bq_dtype ot,
+                          cudaStream_t stream)
+{
+    bq_status st = validate_weight(w);
+    if (st != BQ_OK)
+        return st;
+    if (T < 0 || T > (int64_t(1) << 31))
+        return set_error(BQ_ERR_SHAPE, "embed_gather: T=%lld out of range", (long long)T);
+    if (T > 0 && (!ids || !out))
+        return set_error(BQ_ERR_INVALID_ARG, "embed_gather: ids or out is NULL");
+    if (ot != BQ_F32 && ot != BQ_BF16 && ot != BQ_F16)
+        return set_error(BQ_ERR_DTYPE, "embed_gather: out must be BQ_F32, BQ_BF16 or BQ_F16");
+    if (!aligned16(out))
+        return set_error(BQ_ERR_ALIGNMENT, "embed_gather: out must be 16-byte aligned");
+    unsigned int *status = device_status(&st);
+    if (!status)
+        return st;
+    if (T == 0)
+        return BQ_OK;
+    cudaError_t e = launch_embed(w->fmt, ids, T, w->words, reinterpret_cast<const __half *>(w->scales),
+                                 w->N, w->K, out, (int)ot, status, stream);
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "embed_gather launch: %s", cudaGetErrorString(e));
+    return BQ_OK;
+}
+
+bq_status bq_get_device_error(cudaStream_t stream)
+{
+    bq_status st;
+    unsigned int *status = device_status(&st);
+    if (!status)
+        return st;
+    unsigned int bits = 0;
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(&bits, status + kSlotErrBits, sizeof bits, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && bits)
+        e = cudaMemset(status + kSlotErrBits, 0, sizeof bits);
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "get_device_error: %s", cudaGetErrorString(e));
+    if (bits & kDevErrTimeout)
+        return set_error(BQ_ERR_TIMEOUT, "a bounded device-side wait gave up");
+    if (bits & kDevErrInvalidId)
+        return set_error(BQ_ERR_INVALID_ARG, "an embedding id was outside [0, N)");
+    return BQ_OK;
+}
+
+}  // extern "C"

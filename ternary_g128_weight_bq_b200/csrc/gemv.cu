@@ -1,0 +1,167 @@
+// gemv.cu -- decode GEMV on packed binary-g128 / ternary-g128 weights, M <= 8 token rows.
+//
+// y[m][n] = sum_g s[n][g] * sum_{k in g} v[n][k] * x[m][k],  v = 2b - 1 (binary) or c - 1
+// (ternary). Model card "prism-ml/Bonsai-27B-mlx-1bit", sections "Weight representation:
+// Binary g128" and "CUDA (NVIDIA GPUs)"; the batch-1 decode (tg128) workload of section
+// "Cross-platform throughput".
+//
+// SIMT kernel: each sign bit is applied to x by select-and-add (never a multiply), each
+// group is reduced in fp32, the group scale is applied once per group, and the lanes that
+// share a row are combined with warp shuffles.
+//   * 8 lanes per row, 4 rows per warp: the 8 lanes of a row read 8 consecutive 16-byte
+//     groups (128 B contiguous), so a warp's load touches 4 full 128-byte lines.
+//   * the activations are staged once per block into shared memory as fp32.
+#include "bq_internal.cuh"
+
+namespace bq {
+namespace {
+
+constexpr int kSimtThreads = 256;        // 8 warps
+constexpr int kRowsPerBlock = 32;        // 4 rows per warp
+constexpr int kSimtMaxSmem = 200 * 1024;
+
+template <typename XT>
+__device__ __forceinline__ float xval(const XT *p) { return load_x(p); }
+
+template <int FMT, int M, typename XT>
+__global__ void __launch_bounds__(kSimtThreads)
+gemv_simt_kernel(const XT *__restrict__ x, int64_t K, const uint32_t *__restrict__ words,
+                 const __half *__restrict__ scales, int64_t N, void *__restrict__ y, int yt)
+{
+    extern __shared__ float xs[];   // [M][K] fp32
+    for (int64_t i = threadIdx.x; i < (int64_t)M * K; i += kSimtThreads)
+        xs[i] = xval(x + i);
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int sub = lane >> 3, j = lane & 7;
+    const int64_t n = (int64_t)blockIdx.x * kRowsPerBlock + warp * 4 + sub;
+    const int64_t G = K / 128;
+    float acc[M];
+#pragma unroll
+    for (int m = 0; m < M; m++)
+        acc[m] = 0.f;
+
+    if (n < N) {
+        constexpr int WPG = FMT == BQ_BINARY_G128 ? 4 : 8;     // words per group
+        const uint32_t *wrow = words + n * G * WPG;
+        for (int64_t g = j; g < G; g += 8) {
+            uint32_t w[WPG];
+#pragma unroll
+            for (int i = 0; i < WPG; i += 4) {
+                uint4 v = __ldg(reinterpret_cast<const uint4 *>(wrow + g * WPG + i));
+                w[i] = v.x; w[i + 1] = v.y; w[i + 2] = v.z; w[i + 3] = v.w;
+            }
+            const float s = __half2float(scales[n * G + g]);
+            float part[M];
+#pragma unroll
+            for (int m = 0; m < M; m++)
+                part[m] = 0.f;
+            const float *xg = xs + g * 128;
+            if (FMT == BQ_BINARY_G128) {
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+#pragma unroll 8
+                    for (int b = 0; b < 32; b++) {
+                        const bool on = (w[i] >> b) & 1u;      // 1 -> +x, 0 -> -x
+#pragma unroll
+                        for (int m = 0; m < M; m++) {
+                            float xv = xg[m * K + i * 32 + b];
+                            part[m] += on ? xv : -xv;
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+#pragma unroll 4
+                    for (int b = 0; b < 16; b++) {
+                        const uint32_t c = (w[i] >> (2 * b)) & 3u;   // 0 -> -x, 1 -> 0, 2 -> +x
+#pragma unroll
+                        for (int m = 0; m < M; m++) {
+                            float xv = xg[m * K + i * 16 + b];
+                            part[m] += c == 2u ? xv : (c == 0u ? -xv : 0.f);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < M; m++)
+                acc[m] = fmaf(s, part[m], acc[m]);     // scale once per group
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < M; m++) {
+        acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 4);
+        acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 2);
+        acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 1);
+    }
+    if (j == 0 && n < N) {
+#pragma unroll
+        for (int m = 0; m < M; m++) {
+            if (yt == BQ_F32)
+                store_out(static_cast<float *>(y) + m * N + n, acc[m]);
+            else if (yt == BQ_BF16)
+                store_out(static_cast<__nv_bfloat16 *>(y) + m * N + n, acc[m]);
+            else
+                store_out(static_cast<__half *>(y) + m * N + n, acc[m]);
+        }
+    }
+}
+
+template <int FMT, int M, typename XT>
+cudaError_t launch_simt_t(const GemvArgs &a, cudaStream_t s)
+{
+    size_t smem = (size_t)M * (size_t)a.K * sizeof(float);
+    auto kern = gemv_simt_kernel<FMT, M, XT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    unsigned blocks = (unsigned)((a.N + kRowsPerBlock - 1) / kRowsPerBlock);
+    kern<<<blocks, kSimtThreads, smem, s>>>(static_cast<const XT *>(a.x), a.K, a.words, a.scales, a.N,
+                                            a.y, a.yt);
+    return cudaGetLastError();
+}
+
+template <int FMT, typename XT>
+cudaError_t launch_simt_m(const GemvArgs &a, cudaStream_t s)
+{
+    switch (a.M) {
+    case 1: return launch_simt_t<FMT, 1, XT>(a, s);
+    case 2: return launch_simt_t<FMT, 2, XT>(a, s);
+    case 3: return launch_simt_t<FMT, 3, XT>(a, s);
+    case 4: return launch_simt_t<FMT, 4, XT>(a, s);
+    case 5: return launch_simt_t<FMT, 5, XT>(a, s);
+    case 6: return launch_simt_t<FMT, 6, XT>(a, s);
+    case 7: return launch_simt_t<FMT, 7, XT>(a, s);
+    default: return launch_simt_t<FMT, 8, XT>(a, s);
+    }
+}
+
+}  // namespace
+
+bool gemv_simt_fits(int M, int64_t K) { return (size_t)M * (size_t)K * sizeof(float) <= kSimtMaxSmem; }
+
+cudaError_t launch_gemv_simt(const GemvArgs &a, cudaStream_t s)
+{
+    if (a.fmt == BQ_BINARY_G128)
+        return a.xt == BQ_F16 ? launch_simt_m<BQ_BINARY_G128, __half>(a, s)
+                              : launch_simt_m<BQ_BINARY_G128, __nv_bfloat16>(a, s);
+    return a.xt == BQ_F16 ? launch_simt_m<BQ_TERNARY_G128, __half>(a, s)
+                          : launch_simt_m<BQ_TERNARY_G128, __nv_bfloat16>(a, s);
+}
+
+size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
+{
+    (void)M; (void)fmt; (void)N; (void)K;
+    return 0;
+}
+
+cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s)
+{
+    if (!gemv_simt_fits(a.M, a.K))
+        return cudaErrorInvalidValue;
+    return launch_gemv_simt(a, s);
+}
+
+}  // namespace bq

@@ -1,0 +1,98 @@
+"""The C-ABI library builds, loads and exports every symbol include/bq.h declares; host-side
+validation rejects bad arguments before any CUDA call (runs without a GPU)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import ternary_g128_weight_bq_b200 as bq
+from ternary_g128_weight_bq_b200 import build as bqbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def libbq():
+    bqbuild.build()
+    return bq.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "bq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("bq_pack_binary_g128", "bq_pack_ternary_g128", "bq_unpack_g128", "bq_gemv",
+                 "bq_gemm_prefill", "bq_embed_gather", "bq_get_device_error"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(libbq):
+    out = subprocess.run(["nm", "-D", "--defined-only", bq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for n in declared_functions():
+        assert getattr(libbq, n) is not None
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    src = tmp_path / "use.c"
+    src.write_text('#include "bq.h"\nint main(void){ return (int)bq_packed_words(BQ_BINARY_G128, 1, 128); }\n')
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-c", "-I", os.path.join(ROOT, "include"),
+                    "-I", "/usr/local/cuda/include", str(src), "-o", str(tmp_path / "use.o")],
+                   check=True)
+
+
+def test_sizes_and_strings(libbq):
+    assert libbq.bq_packed_words(0, 3, 256) == 3 * 8
+    assert libbq.bq_packed_words(1, 3, 256) == 3 * 16
+    assert libbq.bq_packed_words(0, 3, 100) == 0
+    assert libbq.bq_packed_words(7, 3, 128) == 0
+    assert libbq.bq_status_string(5) == b"BQ_ERR_INVALID_CODE"
+    assert b"sm_100a" in libbq.bq_version()
+
+
+def _weight(fmt=0, N=4, K=256, words=16, scales=16):
+    return bq._Weight(fmt, N, K, words, scales)
+
+
+def test_validation_before_any_cuda_call(libbq):
+    """Every one of these fails in host validation, before the library touches CUDA."""
+    W = ctypes.byref
+    # NULL weight view / NULL pointers
+    assert libbq.bq_gemv(16, 1, 1, None, 16, 2, None, 0, None) == 1
+    assert libbq.bq_gemv(16, 1, 1, W(_weight(words=0)), 16, 2, None, 0, None) == 1
+    # K not a multiple of 128, N < 1
+    assert libbq.bq_gemv(16, 1, 1, W(_weight(K=100)), 16, 2, None, 0, None) == 2
+    assert libbq.bq_gemv(16, 1, 1, W(_weight(N=0)), 16, 2, None, 0, None) == 2
+    # unknown format
+    assert libbq.bq_gemv(16, 1, 1, W(_weight(fmt=3)), 16, 2, None, 0, None) == 1
+    # misaligned words / x
+    assert libbq.bq_gemv(16, 1, 1, W(_weight(words=20)), 16, 2, None, 0, None) == 3
+    assert libbq.bq_gemv(18, 1, 1, W(_weight()), 16, 2, None, 0, None) == 3
+    # dtypes
+    assert libbq.bq_gemv(16, 2, 1, W(_weight()), 16, 2, None, 0, None) == 4
+    assert libbq.bq_gemv(16, 1, 1, W(_weight()), 16, 9, None, 0, None) == 4
+    # M range
+    assert libbq.bq_gemv(16, 1, 0, W(_weight()), 16, 2, None, 0, None) == 2
+    assert libbq.bq_gemv(16, 1, 9, W(_weight()), 16, 2, None, 0, None) == 2
+    assert libbq.bq_gemm_prefill(16, 1, 0, W(_weight()), 16, 2, None, 0, None) == 2
+    # pack: NULLs, shapes, alignment
+    assert libbq.bq_pack_binary_g128(None, 16, 1, 128, 16, 16, None) == 1
+    assert libbq.bq_pack_ternary_g128(16, 16, 1, 96, 16, 16, None) == 2
+    assert libbq.bq_pack_binary_g128(17, 16, 1, 128, 16, 16, None) == 3
+    # embed: dtype and NULL ids
+    assert libbq.bq_embed_gather(None, 4, W(_weight()), 16, 1, None) == 1
+    assert libbq.bq_embed_gather(16, 4, W(_weight()), 16, 7, None) == 4
+    assert libbq.bq_embed_gather(16, 4, W(_weight()), 24, 1, None) == 3
+    assert libbq.bq_embed_gather(16, -1, W(_weight()), 16, 1, None) == 2
+    msg = libbq.bq_last_error()
+    assert b"T=-1" in msg

@@ -15,7 +15,7 @@ import numpy as np
 import torch
 
 import oracle
-from ternary_g128_weight_bq_b200 import synth
+import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 B, T = oracle.BINARY, oracle.TERNARY
