@@ -1,0 +1,552 @@
+#!/usr/bin/env python
+"""Benchmark of the packed binary-g128 decode GEMV (and the other hot-path kernels) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {bq,reference}] [--quick]
+
+Headline workload: binary-g128 decode GEMV at K = 5120, N in {5120, 20480}, M in {1, 4, 8},
+x bf16 ~ N(0,1), sign bits Bernoulli(0.5), scales fp16 |N(0, 0.02)| + 1e-3, y fp32. One
+step is the six GEMVs. The metric is algorithmic GB/s: (packed words + scales + x) bytes
+per step / device time per step. The weights of each step are one of several copies that
+together exceed twice the L2 size, so every step streams its weights from HBM.
+
+Prints ONE JSON line (rank 0). With --gpus N > 1 (under torchrun) every rank runs the same
+workload on its own GPU (independent replicas, no data-path collective); the value is the
+bytes of all ranks over the slowest rank's time ("scaling": "weak").
+
+--impl reference times the CPU oracle (fp64, plain C) on the host cores on bounded samples
+of the same workload, in the same metric.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+K_HEAD = 5120
+GEMV_SHAPES = [(5120, 1), (5120, 4), (5120, 8), (20480, 1), (20480, 4), (20480, 8)]   # (N, M)
+METRIC = "packed-weight GEMV HBM GB/s & % of 8 TB/s roofline at K=5120; prefill TFLOP/s"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def gemv_bytes(N, K, M, fmt_bits=1):
+    """Algorithmic bytes of one GEMV: packed weights + fp16 scales + bf16 activations."""
+    return N * K * fmt_bits // 8 + N * (K // 128) * 2 + M * K * 2
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; replicas)
+# --------------------------------------------------------------------------------------
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world <= 1:
+        return 0, 1, None
+    import torch.distributed as dist
+    import datetime
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist.get_rank(), dist.get_world_size(), dist
+
+
+def reduce_max(value: float, dist, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# --------------------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------------------
+# GPU workloads
+# --------------------------------------------------------------------------------------
+
+def l2_bytes(device) -> int:
+    return torch.cuda.get_device_properties(device).L2_cache_size
+
+
+def make_gemv_sets(bq, device, copies: int):
+    """`copies` independent weight sets for the six headline GEMVs (seed = copy index)."""
+    sets = []
+    for c in range(copies):
+        layer = []
+        for (N, M) in GEMV_SHAPES:
+            words = synth.binary_words(c, N, K_HEAD, device=device)
+            s = synth.scales(c, N, K_HEAD // 128).to(device)
+            w = bq.BQWeight(bq.BINARY_G128, N, K_HEAD, words, s)
+            x = synth.activations(c, M, K_HEAD, dtype=torch.bfloat16).to(device)
+            y = torch.empty((M, N), dtype=torch.float32, device=device)
+            layer.append((w, x, y))
+        sets.append(layer)
+    return sets
+
+
+def capture_step_graphs(bq, sets, stream):
+    """One CUDA graph per weight copy; each replays the six GEMVs of a step."""
+    graphs, launches = [], []
+    for layer in sets:
+        for (w, x, y) in layer:                     # eager warm-up outside capture
+            bq.gemv(x, w, out=y)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        before = bq.kernel_launches()
+        with torch.cuda.graph(g, stream=stream):
+            for (w, x, y) in layer:
+                bq.gemv(x, w, out=y)
+        launches.append(bq.kernel_launches() - before)
+        graphs.append(g)
+    return graphs, launches
+
+
+def time_graphs(graphs, steps, warmup, stream, dist, device):
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(steps):
+            graphs[i % len(graphs)].replay()
+        end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    return start.elapsed_time(end)
+
+
+def time_single(fn, reps, warmup, stream):
+    """Average device time (ms) of one call of fn() over reps back-to-back calls."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def per_config_breakdown(bq, sets, stream):
+    """GB/s of each headline GEMV alone, rotating over the weight copies (L2-cold)."""
+    out = []
+    for j, (N, M) in enumerate(GEMV_SHAPES):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for layer in sets:
+                w, x, y = layer[j]
+                bq.gemv(x, w, out=y)
+        ms = time_single(graph.replay, 20, 3, stream) / len(sets)
+        gb = gemv_bytes(N, K_HEAD, M) / 1e9
+        out.append({"N": N, "K": K_HEAD, "M": M, "us": round(ms * 1e3, 3),
+                    "GBps": round(gb / (ms / 1e3), 1)})
+        del graph
+    return out
+
+
+def extra_workloads(bq, device, stream, peaks):
+    """LM head, ternary GEMV, embedding gather, prefill (when available): one line each."""
+    res = {}
+    # LM head: M=1, K=5120, N=248320 (179 MB > L2 on its own)
+    N = 248320
+    w = bq.BQWeight(bq.BINARY_G128, N, K_HEAD, synth.binary_words(0, N, K_HEAD, device=device),
+                    synth.scales(0, N, K_HEAD // 128).to(device))
+    x = synth.activations(0, 1, K_HEAD).to(device)
+    y = torch.empty((1, N), dtype=torch.float32, device=device)
+    ms = time_single(lambda: bq.gemv(x, w, out=y), 50, 5, stream)
+    res["lm_head_gemv"] = {"N": N, "K": K_HEAD, "M": 1, "us": round(ms * 1e3, 2),
+                           "GBps": round(gemv_bytes(N, K_HEAD, 1) / 1e9 / (ms / 1e3), 1)}
+    # embedding gather: 4096 ids over the same matrix, bf16 out
+    ids = synth.random_ids(0, synth.TID_IDS, 4096, N).to(device)
+    out = torch.empty((4096, K_HEAD), dtype=torch.bfloat16, device=device)
+    ms = time_single(lambda: bq.embed_gather(ids, w, out=out), 50, 5, stream)
+    eb = 4096 * (K_HEAD // 8 + K_HEAD // 64 + K_HEAD * 2) + 4096 * 4
+    res["embed_gather"] = {"T": 4096, "K": K_HEAD, "us": round(ms * 1e3, 2),
+                           "GBps": round(eb / 1e9 / (ms / 1e3), 1)}
+    del w, ids, out
+    # ternary GEMV: N=20480, K=5120, M=1 (rotating 12 copies: 334 MB)
+    tsets = []
+    for c in range(12):
+        q = synth.random_ternary(c, synth.TID_TERNARY, (20480, K_HEAD)).to(device)
+        tw = bq.pack_ternary_g128(q, synth.scales(c, 20480, K_HEAD // 128).to(device))
+        tsets.append(tw)
+        del q
+    x = synth.activations(0, 1, K_HEAD).to(device)
+    y = torch.empty((1, 20480), dtype=torch.float32, device=device)
+    it = [0]
+
+    def tstep():
+        bq.gemv(x, tsets[it[0] % len(tsets)], out=y)
+        it[0] += 1
+    ms = time_single(tstep, 48, 4, stream)
+    res["ternary_gemv"] = {"N": 20480, "K": K_HEAD, "M": 1, "us": round(ms * 1e3, 2),
+                           "GBps": round(gemv_bytes(20480, K_HEAD, 1, 2) / 1e9 / (ms / 1e3), 1)}
+    del tsets
+    # prefill GEMM: M=512, K=5120, N=20480 binary and ternary
+    try:
+        for fmt_name in ("binary", "ternary"):
+            if fmt_name == "binary":
+                pw = bq.BQWeight(bq.BINARY_G128, 20480, K_HEAD,
+                                 synth.binary_words(0, 20480, K_HEAD, device=device),
+                                 synth.scales(0, 20480, K_HEAD // 128).to(device))
+            else:
+                q = synth.random_ternary(0, synth.TID_TERNARY, (20480, K_HEAD)).to(device)
+                pw = bq.pack_ternary_g128(q, synth.scales(0, 20480, K_HEAD // 128).to(device))
+            X = synth.activations(0, 512, K_HEAD).to(device)
+            Y = torch.empty((512, 20480), dtype=torch.bfloat16, device=device)
+            ms = time_single(lambda: bq.gemm_prefill(X, pw, out=Y), 20, 3, stream)
+            tf = 2 * 512 * 20480 * K_HEAD / (ms / 1e3) / 1e12
+            res[f"prefill_{fmt_name}"] = {"M": 512, "N": 20480, "K": K_HEAD, "us": round(ms * 1e3, 1),
+                                          "TFLOPs": round(tf, 1),
+                                          "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 3)}
+    except Exception as e:  # reported, not hidden: the line says why there is no number
+        res["prefill"] = {"error": str(e).splitlines()[0][:200]}
+    return res
+
+
+def e2e_gemv(bq, device, steps, warmup, stream):
+    """The headline step through the public API with host buffers: per step, copy the six
+    x from pinned host memory, run the six GEMVs, read the six y back to pinned memory."""
+    sets = make_gemv_sets(bq, device, 6)
+    xh = [[x.cpu().pin_memory() for (_, x, _) in layer] for layer in sets]
+    yh = [[torch.empty(y.shape, dtype=y.dtype).pin_memory() for (_, _, y) in layer] for layer in sets]
+    h2d = sum(x.numel() * x.element_size() for x in xh[0])
+    d2h = sum(y.numel() * y.element_size() for y in yh[0])
+
+    def step(i):
+        layer = sets[i % len(sets)]
+        for j, (w, x, y) in enumerate(layer):
+            x.copy_(xh[i % len(sets)][j], non_blocking=True)
+            bq.gemv(x, w, out=y)
+            yh[i % len(sets)][j].copy_(y, non_blocking=True)
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        step(i)
+    b.record(stream)
+    b.synchronize()
+    ms = a.elapsed_time(b) / steps
+    step_bytes = sum(gemv_bytes(N, K_HEAD, M) for (N, M) in GEMV_SHAPES)
+    del sets
+    return {"value": round(step_bytes / 1e9 / (ms / 1e3), 1), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 5)}
+
+
+def traffic_record(kernel_src: str):
+    """ncu DRAM bytes per launch of the dominant kernel, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "gemv_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    if rec.get("source_sha") != h:
+        return None
+    return rec
+
+
+# --------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and --impl reference)
+# --------------------------------------------------------------------------------------
+
+class OracleSample:
+    """The CPU oracle on bounded samples of the six headline GEMVs: the first R rows of
+    each (all K), run on every host core through a thread pool (ctypes releases the GIL)."""
+
+    def __init__(self, max_rows: int = 512):
+        import oracle
+        self.oracle = oracle
+        self.orc = oracle.default()
+        self.cores = os.cpu_count() or 1
+        self.inputs = []
+        for (N, M) in GEMV_SHAPES:
+            self.inputs.append((synth.activations(0, M, K_HEAD), synth.binary_words(0, max_rows, K_HEAD),
+                                synth.scales(0, max_rows, K_HEAD // 128), M))
+        self.max_rows = max_rows
+        # calibration: seconds per row of all six shapes on one core
+        t0 = time.perf_counter()
+        for (x, w, s, M) in self.inputs:
+            self.orc.gemv(oracle.BINARY, x, oracle.X_BF16, w[:1], s[:1], K_HEAD)
+        self.row_seconds = max(time.perf_counter() - t0, 1e-6)
+
+    def rows_for(self, budget_s: float) -> int:
+        return max(1, min(self.max_rows, int(budget_s * self.cores / self.row_seconds)))
+
+    def run(self, rows: int):
+        """Returns (GB/s, seconds) for one pass over `rows` rows of each shape."""
+        import concurrent.futures as cf
+        o = self.oracle
+        chunks = max(1, min(self.cores, rows))
+        jobs = []
+        for (x, w, s, M) in self.inputs:
+            b = [rows * i // chunks for i in range(chunks + 1)]
+            jobs += [(x, w, s, b[i], b[i + 1]) for i in range(chunks) if b[i + 1] > b[i]]
+
+        def work(a):
+            x, w, s, lo, hi = a
+            return self.orc.gemv(o.BINARY, x, o.X_BF16, w[lo:hi], s[lo:hi], K_HEAD)
+        t0 = time.perf_counter()
+        with cf.ThreadPoolExecutor(max_workers=self.cores) as ex:
+            list(ex.map(work, jobs))
+        dt = time.perf_counter() - t0
+        nbytes = sum(gemv_bytes(rows, K_HEAD, M) for (_, _, _, M) in self.inputs)
+        return nbytes / 1e9 / dt, dt
+
+    def describe(self, rows: int, dt: float) -> str:
+        macs = sum(rows * K_HEAD * M for (_, M) in GEMV_SHAPES)
+        return (f"first {rows} rows of each of the six GEMVs (K=5120, M in 1,4,8; "
+                f"{macs / 1e6:.1f}M fp64 multiply-adds) in {dt:.3f} s")
+
+
+def oracle_gemv_sample(budget_s: float):
+    """One bounded oracle run of about budget_s seconds: (GB/s, cores, description)."""
+    o = OracleSample(max_rows=4096)
+    rows = o.rows_for(budget_s)
+    v, dt = o.run(rows)
+    return v, o.cores, o.describe(rows, dt)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    o = OracleSample(max_rows=512)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    rows = o.rows_for(budget)
+    for _ in range(args.warmup):
+        o.run(rows)
+    vals, dts = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, dt = o.run(rows)
+        vals.append(v)
+        dts.append(dt)
+    wall = time.perf_counter() - t0
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(wall / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "binary g128 decode GEMV, K=5120, N in {5120, 20480}, "
+                               "M in {1, 4, 8}, x bf16; CPU oracle on a row sample per step"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": o.cores,
+                         "kind": "oracle", "sample": o.describe(rows, statistics.median(dts))},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------------
+# main GPU arm
+# --------------------------------------------------------------------------------------
+
+def run_gpu(args):
+    rank, world, dist = dist_init()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import ternary_g128_weight_bq_b200 as bq
+    from ternary_g128_weight_bq_b200 import build as bqbuild
+    bqbuild.build()
+    peaks = read_peaks()
+    stream = torch.cuda.Stream(device)
+
+    step_bytes = sum(gemv_bytes(N, K_HEAD, M) for (N, M) in GEMV_SHAPES)
+    l2 = l2_bytes(device)
+    copies = max(2, math.ceil(2.5 * l2 / step_bytes))
+    with torch.cuda.stream(stream):
+        sets = make_gemv_sets(bq, device, copies)
+        graphs, launches = capture_step_graphs(bq, sets, stream)
+        torch.cuda.synchronize()
+        clocks = ClockSampler(local) if rank == 0 else None
+        ms_total = time_graphs(graphs, args.steps, args.warmup, stream, dist, device)
+        clk = clocks.stop() if clocks else None
+    ms_step = reduce_max(ms_total / args.steps, dist, device)
+    value = world * step_bytes / 1e9 / (ms_step / 1e3)
+    launches_timed = sum(launches[i % len(graphs)] for i in range(args.steps))
+
+    extras = {}
+    breakdown = None
+    e2e = None
+    if rank == 0 and not args.quick:
+        with torch.cuda.stream(stream):
+            breakdown = per_config_breakdown(bq, sets, stream)
+    del graphs, sets
+    torch.cuda.empty_cache()
+    if not args.quick:
+        with torch.cuda.stream(stream):
+            e2e = e2e_gemv(bq, device, min(args.steps, 2000), args.warmup, stream)
+            if rank == 0:
+                extras = extra_workloads(bq, device, stream, peaks)
+        if e2e is not None:
+            e2e_ms = reduce_max(e2e["ms_per_step"], dist, device)
+            e2e["value"] = round(world * step_bytes / 1e9 / (e2e_ms / 1e3), 1)
+
+    if rank == 0:
+        gemv_src = os.path.join(ROOT, "ternary_g128_weight_bq_b200", "csrc", "gemv.cu")
+        tr = traffic_record(gemv_src)
+        achieved = step_bytes / 1e9 / (ms_total / args.steps / 1e3)
+        cpu = None
+        if not args.quick:
+            v, cores, desc = oracle_gemv_sample(args.cpu_seconds)
+            cpu = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                   "sample": desc}
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {
+                "workload": "binary g128 decode GEMV, K=5120, N in {5120, 20480}, M in {1, 4, 8} "
+                            "(six GEMVs per step), x bf16 ~N(0,1), bits Bernoulli(0.5), "
+                            "scales fp16 |N(0,0.02)|+1e-3, y fp32",
+                "l2": f"inputs larger than L2: {copies} weight copies rotated "
+                      f"({copies * step_bytes / 1e6:.0f} MB vs {l2 / 1e6:.0f} MB L2)",
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "bytes_per_step": step_bytes,
+                "timing": "CUDA graph per step (six launches), CUDA events on the launch stream",
+            },
+            "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 1),
+            "roofline": {
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                "peak_source": f"{peaks['source']} (HBM copy, burst)",
+                "kernel": "bq gemv (six launches per step; achieved = algorithmic bytes / "
+                          "device time of the launches)",
+            },
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_timed,
+            "clocks": clk,
+            "breakdown": breakdown,
+            "extras": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["bq", "reference"], default="bq")
+    ap.add_argument("--quick", action="store_true", help="headline number only")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -88,6 +88,10 @@ const char *bq_status_string(bq_status st);
 /* Message describing the last non-OK status returned to the calling thread. */
 const char *bq_last_error(void);
 
+/* Total number of kernel launches this process has enqueued through libbq (all devices,
+ * all threads); instrumentation for benchmarks. */
+unsigned long long bq_kernel_launches(void);
+
 /* Number of uint32 words in a packed matrix: N*K/32 (binary) or N*K/16 (ternary);
  * 0 if the arguments are invalid. Scales always take N*K/128 fp16 values. */
 size_t bq_packed_words(bq_format fmt, int64_t N, int64_t K);

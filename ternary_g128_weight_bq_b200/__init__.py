@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
             "bq_version": ([], ctypes.c_char_p),
             "bq_status_string": ([I], ctypes.c_char_p),
             "bq_last_error": ([], ctypes.c_char_p),
+            "bq_kernel_launches": ([], ctypes.c_ulonglong),
             "bq_packed_words": ([I, I64, I64], ctypes.c_size_t),
             "bq_pack_binary_g128": ([P, P, I64, I64, P, P, P], I),
             "bq_pack_ternary_g128": ([P, P, I64, I64, P, P, P], I),
@@ -130,6 +131,11 @@ class BQWeight:
 
 def version() -> str:
     return lib().bq_version().decode()
+
+
+def kernel_launches() -> int:
+    """Kernel launches enqueued through libbq so far in this process."""
+    return int(lib().bq_kernel_launches())
 
 
 def packed_words(fmt: int, N: int, K: int) -> int:

@@ -13,6 +13,9 @@ namespace bq {
 __device__ unsigned int g_status[4];
 
 static thread_local char t_msg[512] = "no error";
+static unsigned long long g_launches = 0;
+
+void note_launches(unsigned n) { __atomic_fetch_add(&g_launches, (unsigned long long)n, __ATOMIC_RELAXED); }
 
 bq_status set_error(bq_status st, const char *fmt, ...)
 {
@@ -113,6 +116,8 @@ const char *bq_status_string(bq_status st)
 
 const char *bq_last_error(void) { return t_msg; }
 
+unsigned long long bq_kernel_launches(void) { return __atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
+
 size_t bq_packed_words(bq_format fmt, int64_t N, int64_t K)
 {
     if (N < 1 || K < 128 || K % 128)
@@ -142,6 +147,8 @@ static bq_status pack_common(int fmt, const int8_t *q, const uint16_t *s_in, int
     if (e == cudaSuccess)
         e = fmt == BQ_BINARY_G128 ? launch_pack_binary(q, N, K, words, cnt, stream)
                                   : launch_pack_ternary(q, N, K, words, cnt, stream);
+    if (e == cudaSuccess)
+        note_launches(1);
     if (e == cudaSuccess && s_out != s_in)
         e = cudaMemcpyAsync(s_out, s_in, (size_t)N * (size_t)(K / 128) * 2, cudaMemcpyDeviceToDevice,
                             stream);
@@ -186,6 +193,8 @@ bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStr
     cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(unsigned int), stream);
     if (e == cudaSuccess)
         e = launch_unpack(w->fmt, w->words, w->N, w->K, q, cnt, stream);
+    if (e == cudaSuccess)
+        note_launches(1);
     if (e == cudaSuccess && s_out && s_out != w->scales)
         e = cudaMemcpyAsync(s_out, w->scales, (size_t)w->N * (size_t)(w->K / 128) * 2,
                             cudaMemcpyDeviceToDevice, stream);
@@ -242,9 +251,11 @@ bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, voi
         return st;
     GemvArgs a{x, (int)xt, (int)M, (int)w->fmt, w->N, w->K, w->words,
                reinterpret_cast<const __half *>(w->scales), y, (int)yt, workspace, ws_bytes};
-    cudaError_t e = launch_gemv(a, stream);
+    unsigned launches = 0;
+    cudaError_t e = launch_gemv(a, stream, &launches);
     if (e != cudaSuccess)
         return set_error(BQ_ERR_CUDA, "gemv launch: %s", cudaGetErrorString(e));
+    note_launches(launches);
     return BQ_OK;
 }
 
@@ -273,9 +284,11 @@ bq_status bq_gemm_prefill(const void *x, bq_dtype xt, int64_t M, const bq_weight
         return st;
     PrefillArgs a{x, (int)xt, M, (int)w->fmt, w->N, w->K, w->words,
                   reinterpret_cast<const __half *>(w->scales), y, (int)yt, status};
-    cudaError_t e = launch_prefill(a, stream);
+    unsigned launches = 0;
+    cudaError_t e = launch_prefill(a, stream, &launches);
     if (e != cudaSuccess)
         return set_error(BQ_ERR_CUDA, "gemm_prefill launch: %s", cudaGetErrorString(e));
+    note_launches(launches);
     return BQ_OK;
 }
 
@@ -302,6 +315,7 @@ bq_status bq_embed_gather(const int32_t *ids, int64_t T, const bq_weight *w, voi
                                  w->N, w->K, out, (int)ot, status, stream);
     if (e != cudaSuccess)
         return set_error(BQ_ERR_CUDA, "embed_gather launch: %s", cudaGetErrorString(e));
+    note_launches(1);
     return BQ_OK;
 }
 

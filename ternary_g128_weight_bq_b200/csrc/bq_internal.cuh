@@ -23,6 +23,9 @@ constexpr int kSlotInvalidCount = 1;
 unsigned int *device_status(bq_status *st);
 
 bq_status set_error(bq_status st, const char *fmt, ...);
+
+// Count of kernel launches enqueued by the library (instrumentation for benchmarks).
+void note_launches(unsigned n);
 bq_status check_launch(const char *what);
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -50,7 +53,7 @@ struct GemvArgs {
     size_t ws_bytes;
 };
 size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
-cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s);
+cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches);
 
 struct PrefillArgs {
     const void *x;
@@ -65,7 +68,7 @@ struct PrefillArgs {
     unsigned int *dev_status;
 };
 size_t prefill_workspace_bytes(int64_t M, int fmt, int64_t N, int64_t K);
-cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s);
+cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s, unsigned *launches);
 
 cudaError_t launch_embed(int fmt, const int32_t *ids, int64_t T, const uint32_t *words,
                          const __half *scales, int64_t N, int64_t K, void *out, int ot,

@@ -1,7 +1,377 @@
-// gemm_prefill.cu -- prefill GEMM on packed weights (tcgen05 path is added next).
+// gemm_prefill.cu -- prefill GEMM Y[M][N] = X[M][K] * W^T on packed binary-g128 /
+// ternary-g128 weights, on the fifth-generation tensor cores (tcgen05, fp32 accumulation in
+// tensor memory).
+//
+// Model card "prism-ml/Bonsai-27B-mlx-1bit", section "CUDA (NVIDIA GPUs)": the kernel unpacks
+// the sign codes inside the matrix product and applies the group scale; the model is never
+// expanded to a dense FP16 tensor in memory. Section "Cross-platform throughput": pp512 (a
+// 512-token prompt) is the compute-bound phase. Ternary: "Ternary Bonsai 27B vs ..." article
+// (wmrh.cn), PP512 row of its throughput table.
+//
+// One CTA computes a 128 (weight rows) x BN (tokens) tile of Y^T:
+//   * warp 0, one lane: TMA loads of the X tile [BN tokens x 64 k] per k-block into a ring
+//     of shared-memory stages (128-byte swizzle, zero fill past M); warp 0 also owns TMEM.
+//   * warps 2-5 (128 threads, one weight row each): read the row's packed bits and its group
+//     scale straight from global memory, expand each 8-weight chunk to +-s (binary) or
+//     {-s, 0, +s} (ternary) in the operand type through a 256-entry sign-mask table, and
+//     store the 128 x 64 A tile in the same swizzled layout. The scale is folded into the
+//     operand, so a group needs no separate rescaling: +-s is exact in fp16 and rounded to
+//     nearest even in bf16 (x's type decides).
+//   * warp 1, one lane: issues 4 tcgen05.mma (128 x BN x 16) per k-block into a TMEM
+//     accumulator and commits each stage back to the producers.
+//   * warps 2-5 then read the accumulator with tcgen05.ld (lane = weight row, column =
+//     token) and store Y with one coalesced 32-row segment per token.
+// The expanded weights exist only in shared memory. Every mbarrier wait is bounded: after
+// 2 s the kernel records kDevErrTimeout, lets its copies and MMAs drain, frees TMEM and
+// returns.
+#include <cuda.h>
+
 #include "bq_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace bq {
+namespace {
+
+constexpr int kBM = 128;              // weight rows per tile (MMA M)
+constexpr int kBK = 64;               // k per stage: one 128-byte swizzle row of 16-bit values
+constexpr int kThreads = 192;         // 6 warps
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+template <int BN> struct Cfg {
+    static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+    static constexpr int kXBytes = BN * 128;          // X stage: BN rows x 128 B
+    static constexpr int kABytes = kBM * 128;         // A stage: 128 rows x 128 B
+    static constexpr int kLutBytes = 256 * 16;
+    static constexpr int kBarOffset = kStages * (kXBytes + kABytes) + kLutBytes;
+    static constexpr int kSmem = kBarOffset + 256 + 1024;   // barriers + alignment slack
+    static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+};
+
+struct Bars {
+    uint64_t full_x[8];
+    uint64_t full_a[8];
+    uint64_t empty[8];
+    uint64_t acc_full;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast, then every lane
+// observes the (already completed) phase itself so that it acquires the producer's writes.
+// All lanes return the same value, so later warp-collective instructions stay converged.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0)
+        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, kWaitLimitNs);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok)
+        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, kWaitLimitNs);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ uint32_t scale_pair(uint16_t s_f16, bool bf16)
+{
+    uint16_t h = s_f16;
+    if (bf16)
+        h = __bfloat16_as_ushort(__float2bfloat16_rn(__half2float(__ushort_as_half(s_f16))));
+    return (uint32_t)h | ((uint32_t)h << 16);
+}
+
+template <int FMT, int BN, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__restrict__ words,
+               const uint16_t *__restrict__ scales, int64_t M, int64_t N, int64_t K, void *__restrict__ y,
+               int yt, unsigned int *dev_status)
+{
+    using C = Cfg<BN>;
+    constexpr int S = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *xs = smem;                                         // S x kXBytes
+    uint8_t *as = smem + S * C::kXBytes;                        // S x kABytes
+    uint4 *lut = reinterpret_cast<uint4 *>(smem + S * (C::kXBytes + C::kABytes));
+    Bars *bars = reinterpret_cast<Bars *>(smem + C::kBarOffset);
+    volatile int *abort = &bars->abort;
+    unsigned int *err = dev_status + kSlotErrBits;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m0 = (int64_t)blockIdx.x * BN;
+    const int64_t n0 = (int64_t)blockIdx.y * kBM;
+    const int KB = (int)(K / kBK);
+
+    // ---------------------------------------------------------------- set-up
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; s++) {
+            ptx::mbar_init(&bars->full_x[s], 1);
+            ptx::mbar_init(&bars->full_a[s], 4);
+            ptx::mbar_init(&bars->empty[s], 1);
+        }
+        ptx::mbar_init(&bars->acc_full, 1);
+        ptx::mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        ptx::fence_barrier_init();
+        ptx::tma_prefetch_desc(&tmap_x);
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(&bars->tmem_base, C::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (warp >= 2) {
+        // sign-mask table: entry b describes the 8 (binary) or 4 (ternary) weights of byte b
+        for (int b = threadIdx.x - 64; b < 256; b += 128) {
+            uint32_t e[4];
+            if (FMT == BQ_BINARY_G128) {
+                for (int i = 0; i < 4; i++) {
+                    uint32_t lo = ((b >> (2 * i)) & 1) ? 0u : 0x8000u;        // bit 0 -> -s
+                    uint32_t hi = ((b >> (2 * i + 1)) & 1) ? 0u : 0x80000000u;
+                    e[i] = lo | hi;
+                }
+            } else {
+                uint32_t keep[2] = {0, 0}, sign[2] = {0, 0};
+                for (int i = 0; i < 4; i++) {
+                    uint32_t c = (b >> (2 * i)) & 3u;                        // 0:-1 1:0 2:+1 3:invalid
+                    uint32_t sh = 16 * (i & 1);
+                    if (c == 0u || c == 2u)
+                        keep[i >> 1] |= 0xFFFFu << sh;
+                    if (c == 0u)
+                        sign[i >> 1] |= 0x8000u << sh;
+                }
+                e[0] = keep[0]; e[1] = keep[1]; e[2] = sign[0]; e[3] = sign[1];
+            }
+            lut[b] = make_uint4(e[0], e[1], e[2], e[3]);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_d = bars->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < KB; kb++) {
+                const int s = kb % S;
+                const uint32_t ph = (kb / S) & 1;
+                if (!ptx::mbar_wait_bounded(&bars->empty[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
+                    break;
+                ptx::mbar_arrive_expect_tx(&bars->full_x[s], C::kXBytes);
+                ptx::tma_load_2d(xs + s * C::kXBytes, &tmap_x, &bars->full_x[s], kb * kBK, (int32_t)m0);
+                issued++;
+            }
+            // no copy may still be in flight when the CTA exits
+            for (int kb = issued > S ? issued - S : 0; kb < issued; kb++) {
+                volatile int no_abort = 0;
+                ptx::mbar_wait_bounded(&bars->full_x[kb % S], (kb / S) & 1, &no_abort, err, kDevErrTimeout,
+                                       kWaitLimitNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::umma_idesc_f16(BF16 ? 1u : 0u, kBM, BN);
+            int issued = 0;
+            for (int kb = 0; kb < KB; kb++) {
+                const int s = kb % S;
+                const uint32_t ph = (kb / S) & 1;
+                if (!ptx::mbar_wait_bounded(&bars->full_x[s], ph, abort, err, kDevErrTimeout, kWaitLimitNs))
+                    break;
+                if (!ptx::mbar_wait_bounded(&bars->full_a[s], ph, abort, err, kDevErrTimeout, kWaitLimitNs))
+                    break;
+                ptx::tc_fence_after();
+                const uint64_t adesc = ptx::sw128_kmajor_desc(ptx::smem_u32(as + s * C::kABytes));
+                const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(xs + s * C::kXBytes));
+#pragma unroll
+                for (int k = 0; k < kBK / 16; k++)   // advance 16 elements = 32 B inside the swizzle row
+                    ptx::umma_f16(tmem_d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+                ptx::umma_commit(&bars->empty[s]);
+                issued++;
+            }
+            if (issued == KB) {
+                ptx::umma_commit(&bars->acc_full);
+            } else {
+                // aborted: wait for the MMAs already issued before TMEM is released
+                ptx::umma_commit(&bars->drain);
+                volatile int no_abort = 0;
+                ptx::mbar_wait_bounded(&bars->drain, 0, &no_abort, err, kDevErrTimeout, kWaitLimitNs);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ dequant, then epilogue
+        const int r = threadIdx.x - 64;                      // weight row within the tile
+        const int64_t n = n0 + r;
+        const bool row_ok = n < N;
+        const int64_t G = K / 128;
+        constexpr int WPB = FMT == BQ_BINARY_G128 ? 2 : 4;   // words per k-block
+        const uint32_t *wrow = words + (row_ok ? n : 0) * (K / 32 * (FMT == BQ_BINARY_G128 ? 1 : 2));
+        const uint16_t *srow = scales + (row_ok ? n : 0) * G;
+        uint8_t *arow_base = as + r * 128;
+        const int sw = r & 7;
+
+        constexpr int kAhead = 4;                           // k-blocks of bits loaded ahead
+        uint4 wq[kAhead];
+        uint16_t sq[kAhead];
+#pragma unroll
+        for (int i = 0; i < kAhead; i++) {
+            wq[i] = make_uint4(0, 0, 0, 0);
+            sq[i] = 0;
+            if (row_ok && i < KB) {
+                if (WPB == 2) {
+                    uint2 v = __ldg(reinterpret_cast<const uint2 *>(wrow) + i);
+                    wq[i] = make_uint4(v.x, v.y, 0, 0);
+                } else {
+                    wq[i] = __ldg(reinterpret_cast<const uint4 *>(wrow) + i);
+                }
+                sq[i] = __ldg(srow + i / 2);
+            }
+        }
+        for (int kb = 0; kb < KB; kb++) {
+            const uint4 wv = wq[0];
+            const uint16_t sv = sq[0];
+#pragma unroll
+            for (int i = 0; i < kAhead - 1; i++) {
+                wq[i] = wq[i + 1];
+                sq[i] = sq[i + 1];
+            }
+            const int nk = kb + kAhead;
+            wq[kAhead - 1] = make_uint4(0, 0, 0, 0);
+            if (row_ok && nk < KB) {
+                if (WPB == 2) {
+                    uint2 v = __ldg(reinterpret_cast<const uint2 *>(wrow) + nk);
+                    wq[kAhead - 1] = make_uint4(v.x, v.y, 0, 0);
+                } else {
+                    wq[kAhead - 1] = __ldg(reinterpret_cast<const uint4 *>(wrow) + nk);
+                }
+                sq[kAhead - 1] = __ldg(srow + nk / 2);
+            }
+
+            const int s = kb % S;
+            const uint32_t ph = (kb / S) & 1;
+            if (!warp_wait(&bars->empty[s], ph ^ 1, abort, err))
+                break;
+            uint8_t *arow = arow_base + s * C::kABytes;
+            const uint32_t s2 = row_ok ? scale_pair(sv, BF16) : 0u;
+            const uint32_t wds[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int c = 0; c < 8; c++) {                    // 8 chunks of 8 weights (16 B each)
+                uint4 o;
+                if (FMT == BQ_BINARY_G128) {
+                    const uint32_t byte = (wds[c >> 2] >> (8 * (c & 3))) & 0xFFu;
+                    const uint4 e = lut[byte];
+                    o = make_uint4(s2 ^ e.x, s2 ^ e.y, s2 ^ e.z, s2 ^ e.w);
+                } else {
+                    const uint32_t half16 = (wds[c >> 1] >> (16 * (c & 1))) & 0xFFFFu;
+                    const uint4 e0 = lut[half16 & 0xFFu], e1 = lut[half16 >> 8];
+                    o = make_uint4((s2 & e0.x) ^ e0.z, (s2 & e0.y) ^ e0.w, (s2 & e1.x) ^ e1.z, (s2 & e1.y) ^ e1.w);
+                }
+                if (!row_ok)
+                    o = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(arow + ((c ^ sw) << 4)) = o;
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                ptx::mbar_arrive(&bars->full_a[s]);
+        }
+
+        // ------------------------------------------------------------ epilogue
+        if (warp_wait(&bars->acc_full, 0, abort, err)) {
+            ptx::tc_fence_after();
+            const int quad = warp & 3;                       // TMEM lanes 32*quad .. +31
+            const int64_t nrow = n0 + quad * 32 + lane;
+            const bool nok = nrow < N;
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; cc++) {
+                uint32_t v[32];
+                ptx::tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(quad * 32) << 16) + cc * 32, v);
+                ptx::tmem_wait_ld();
+                const int64_t mbase = m0 + cc * 32;
+                if (!nok)
+                    continue;
+#pragma unroll
+                for (int j = 0; j < 32; j++) {
+                    const int64_t m = mbase + j;
+                    if (m < M) {
+                        const float f = __uint_as_float(v[j]);
+                        if (yt == BQ_F32)
+                            store_out(static_cast<float *>(y) + m * N + nrow, f);
+                        else if (yt == BQ_BF16)
+                            store_out(static_cast<__nv_bfloat16 *>(y) + m * N + nrow, f);
+                        else
+                            store_out(static_cast<__half *>(y) + m * N + nrow, f);
+                    }
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_d, C::kTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int FMT, int BN, bool BF16>
+cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return cudaErrorNotSupported;
+    CUtensorMap map;
+    cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
+    cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BN};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&map, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                     const_cast<void *>(a.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    auto kern = prefill_kernel<FMT, BN, BF16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmem);
+    if (e != cudaSuccess)
+        return e;
+    dim3 grid((unsigned)((a.M + BN - 1) / BN), (unsigned)((a.N + kBM - 1) / kBM));
+    kern<<<grid, kThreads, Cfg<BN>::kSmem, s>>>(map, a.words, reinterpret_cast<const uint16_t *>(a.scales), a.M,
+                                                a.N, a.K, a.y, a.yt, a.dev_status);
+    return cudaGetLastError();
+}
+
+template <int FMT, bool BF16>
+cudaError_t launch_bn(const PrefillArgs &a, cudaStream_t s)
+{
+    if (a.M <= 64)
+        return launch_t<FMT, 64, BF16>(a, s);
+    if (a.M <= 128)
+        return launch_t<FMT, 128, BF16>(a, s);
+    return launch_t<FMT, 256, BF16>(a, s);
+}
+
+}  // namespace
 
 size_t prefill_workspace_bytes(int64_t M, int fmt, int64_t N, int64_t K)
 {
@@ -9,10 +379,13 @@ size_t prefill_workspace_bytes(int64_t M, int fmt, int64_t N, int64_t K)
     return 0;
 }
 
-cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s)
+cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s, unsigned *launches)
 {
-    (void)a; (void)s;
-    return cudaErrorNotSupported;
+    *launches = 1;
+    const bool bf16 = a.xt == BQ_BF16;
+    if (a.fmt == BQ_BINARY_G128)
+        return bf16 ? launch_bn<BQ_BINARY_G128, true>(a, s) : launch_bn<BQ_BINARY_G128, false>(a, s);
+    return bf16 ? launch_bn<BQ_TERNARY_G128, true>(a, s) : launch_bn<BQ_TERNARY_G128, false>(a, s);
 }
 
 }  // namespace bq

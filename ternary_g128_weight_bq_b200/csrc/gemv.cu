@@ -157,10 +157,11 @@ size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
     return 0;
 }
 
-cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s)
+cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches)
 {
     if (!gemv_simt_fits(a.M, a.K))
         return cudaErrorInvalidValue;
+    *launches = 1;
     return launch_gemv_simt(a, s);
 }
 

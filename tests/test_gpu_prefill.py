@@ -1,0 +1,77 @@
+"""GPU prefill GEMM (tcgen05) against the CPU oracle, within 2e-3 * sum_k |x s| per output.
+Small ragged shapes are checked on every output; the M=512, K=5120, N=20480 binary and
+ternary workloads on sampled weight rows (all 512 tokens), launched as the benchmark
+launches them."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.gpu_common import (assert_within_bound, bq, requires_gpu, sample_rows, ternary_q,
+                              x_dtype_code)
+
+pytestmark = requires_gpu
+
+
+def weight(m, fmt, seed, N, K):
+    s = synth.scales(seed, N, K // 128)
+    if fmt == oracle.BINARY:
+        words = synth.binary_words(seed, N, K)
+        return m.BQWeight(m.BINARY_G128, N, K, words.cuda(), s.cuda()), words.numpy(), s
+    q = ternary_q(seed, N, K)
+    w = m.pack_ternary_g128(q.cuda(), s.cuda())
+    return w, w.words.cpu().numpy(), s
+
+
+def check(orc, fmt, seed, M, N, K, xdt=torch.bfloat16, ydt=torch.float32, rows=None):
+    m = bq()
+    w, words_np, s = weight(m, fmt, seed, N, K)
+    if fmt == oracle.TERNARY:
+        # the oracle packs the same q itself; the device words must agree bit for bit
+        q = ternary_q(seed, N, K)
+        st, words_ref, _ = orc.pack(oracle.TERNARY, q.numpy(), s.numpy())
+        assert np.array_equal(words_np.view(np.uint32), words_ref)
+        words_np = words_ref
+    x = synth.activations(seed + 1, M, K, dtype=xdt)
+    y = m.gemm_prefill(x.cuda(), w, out_dtype=ydt)
+    torch.cuda.synchronize()
+    m.get_device_error()
+    y_ref, bound = orc.gemv(fmt, x, x_dtype_code(xdt), words_np, s, K, rows=rows)
+    yg = y if rows is None else y[:, torch.from_numpy(rows).cuda()]
+    return assert_within_bound(yg, y_ref, bound, f"prefill fmt={fmt} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("fmt", [oracle.BINARY, oracle.TERNARY])
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (17, 300, 640), (77, 1000, 256), (64, 129, 384),
+                                   (130, 256, 1152), (300, 200, 512), (512, 384, 640)])
+def test_prefill_ragged_all_outputs(orc, fmt, M, N, K):
+    check(orc, fmt, 300 + M, M, N, K)
+
+
+@pytest.mark.parametrize("ydt", [torch.float32, torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("xdt", [torch.float16, torch.bfloat16])
+def test_prefill_dtypes(orc, xdt, ydt):
+    check(orc, oracle.BINARY, 9, 200, 256, 1024, xdt=xdt, ydt=ydt)
+
+
+@pytest.mark.parametrize("fmt", [oracle.BINARY, oracle.TERNARY])
+def test_prefill_m512_k5120_n20480_sampled(orc, fmt):
+    check(orc, fmt, 0, 512, 20480, 5120, rows=sample_rows(20480, 96, 5))
+
+
+def test_prefill_fp16_is_exact_scale(orc):
+    """With fp16 x the +-s operand is exact: the error is fp32 accumulation only."""
+    r = check(orc, oracle.BINARY, 11, 256, 512, 2048, xdt=torch.float16)
+    assert r < 0.05
+
+
+def test_prefill_matches_gemv(orc):
+    """For M <= 8 the prefill kernel and the decode GEMV compute the same product."""
+    m = bq()
+    w, _, _ = weight(m, oracle.BINARY, 12, 1000, 1024)
+    x = synth.activations(13, 8, 1024, dtype=torch.float16).cuda()
+    a = m.gemm_prefill(x, w)
+    b = m.gemv(x, w)
+    assert torch.allclose(a, b, rtol=1e-4, atol=1e-4)
