@@ -247,10 +247,11 @@ bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, voi
                          workspace ? ws_bytes : (size_t)0);
     if (workspace && !aligned16(workspace))
         return set_error(BQ_ERR_ALIGNMENT, "gemv: workspace must be 16-byte aligned");
-    if (!device_status(&st))
+    unsigned int *status = device_status(&st);
+    if (!status)
         return st;
     GemvArgs a{x, (int)xt, (int)M, (int)w->fmt, w->N, w->K, w->words,
-               reinterpret_cast<const __half *>(w->scales), y, (int)yt, workspace, ws_bytes};
+               reinterpret_cast<const __half *>(w->scales), y, (int)yt, workspace, ws_bytes, status};
     unsigned launches = 0;
     cudaError_t e = launch_gemv(a, stream, &launches);
     if (e != cudaSuccess)

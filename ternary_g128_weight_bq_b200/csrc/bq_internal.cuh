@@ -51,8 +51,13 @@ struct GemvArgs {
     int yt;           // bq_dtype
     void *workspace;
     size_t ws_bytes;
+    unsigned int *dev_status;
 };
 size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
+// integer tensor-core path (gemv_tc.cu): K a multiple of 1024
+bool gemv_tc_supported(int M, int fmt, int64_t K);
+size_t gemv_tc_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
+cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s);
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches);
 
 struct PrefillArgs {

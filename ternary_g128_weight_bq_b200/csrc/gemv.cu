@@ -10,7 +10,10 @@
 // share a row are combined with warp shuffles.
 //   * 8 lanes per row, 4 rows per warp: the 8 lanes of a row read 8 consecutive 16-byte
 //     groups (128 B contiguous), so a warp's load touches 4 full 128-byte lines.
-//   * the activations are staged once per block into shared memory as fp32.
+//   * the activations are staged once per block into shared memory as fp32 when they fit
+//     (M*K*4 <= 200 KB), else read from global memory (L1/L2-resident).
+// This kernel serves the shapes the tensor-core kernel (gemv_tc.cu) does not take: K not a
+// multiple of 1024, or digit fragments too large for shared memory.
 #include "bq_internal.cuh"
 
 namespace bq {
@@ -23,15 +26,26 @@ constexpr int kSimtMaxSmem = 200 * 1024;
 template <typename XT>
 __device__ __forceinline__ float xval(const XT *p) { return load_x(p); }
 
-template <int FMT, int M, typename XT>
+// x is read from shared memory (fp32, when M*K*4 fits) or straight from global memory.
+template <bool SMEM_X, typename XT>
+struct XSrc {
+    const float *s;
+    const XT *g;
+    __device__ __forceinline__ float operator[](int64_t i) const { return SMEM_X ? s[i] : xval(g + i); }
+};
+
+template <int FMT, int M, typename XT, bool SMEM_X>
 __global__ void __launch_bounds__(kSimtThreads)
 gemv_simt_kernel(const XT *__restrict__ x, int64_t K, const uint32_t *__restrict__ words,
                  const __half *__restrict__ scales, int64_t N, void *__restrict__ y, int yt)
 {
-    extern __shared__ float xs[];   // [M][K] fp32
-    for (int64_t i = threadIdx.x; i < (int64_t)M * K; i += kSimtThreads)
-        xs[i] = xval(x + i);
-    __syncthreads();
+    extern __shared__ float xs_raw[];   // [M][K] fp32 when SMEM_X
+    if (SMEM_X) {
+        for (int64_t i = threadIdx.x; i < (int64_t)M * K; i += kSimtThreads)
+            xs_raw[i] = xval(x + i);
+        __syncthreads();
+    }
+    const XSrc<SMEM_X, XT> xs{xs_raw, x};
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = lane >> 3, j = lane & 7;
@@ -57,7 +71,7 @@ gemv_simt_kernel(const XT *__restrict__ x, int64_t K, const uint32_t *__restrict
 #pragma unroll
             for (int m = 0; m < M; m++)
                 part[m] = 0.f;
-            const float *xg = xs + g * 128;
+            const int64_t xg = g * 128;
             if (FMT == BQ_BINARY_G128) {
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
@@ -66,7 +80,7 @@ gemv_simt_kernel(const XT *__restrict__ x, int64_t K, const uint32_t *__restrict
                         const bool on = (w[i] >> b) & 1u;      // 1 -> +x, 0 -> -x
 #pragma unroll
                         for (int m = 0; m < M; m++) {
-                            float xv = xg[m * K + i * 32 + b];
+                            float xv = xs[xg + m * K + i * 32 + b];
                             part[m] += on ? xv : -xv;
                         }
                     }
@@ -79,7 +93,7 @@ gemv_simt_kernel(const XT *__restrict__ x, int64_t K, const uint32_t *__restrict
                         const uint32_t c = (w[i] >> (2 * b)) & 3u;   // 0 -> -x, 1 -> 0, 2 -> +x
 #pragma unroll
                         for (int m = 0; m < M; m++) {
-                            float xv = xg[m * K + i * 16 + b];
+                            float xv = xs[xg + m * K + i * 16 + b];
                             part[m] += c == 2u ? xv : (c == 0u ? -xv : 0.f);
                         }
                     }
@@ -112,14 +126,19 @@ gemv_simt_kernel(const XT *__restrict__ x, int64_t K, const uint32_t *__restrict
 template <int FMT, int M, typename XT>
 cudaError_t launch_simt_t(const GemvArgs &a, cudaStream_t s)
 {
-    size_t smem = (size_t)M * (size_t)a.K * sizeof(float);
-    auto kern = gemv_simt_kernel<FMT, M, XT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess)
-        return e;
-    unsigned blocks = (unsigned)((a.N + kRowsPerBlock - 1) / kRowsPerBlock);
-    kern<<<blocks, kSimtThreads, smem, s>>>(static_cast<const XT *>(a.x), a.K, a.words, a.scales, a.N,
-                                            a.y, a.yt);
+    const size_t smem = (size_t)M * (size_t)a.K * sizeof(float);
+    const unsigned blocks = (unsigned)((a.N + kRowsPerBlock - 1) / kRowsPerBlock);
+    if (smem <= kSimtMaxSmem) {
+        auto kern = gemv_simt_kernel<FMT, M, XT, true>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        kern<<<blocks, kSimtThreads, smem, s>>>(static_cast<const XT *>(a.x), a.K, a.words, a.scales, a.N,
+                                                a.y, a.yt);
+    } else {
+        gemv_simt_kernel<FMT, M, XT, false><<<blocks, kSimtThreads, 0, s>>>(
+            static_cast<const XT *>(a.x), a.K, a.words, a.scales, a.N, a.y, a.yt);
+    }
     return cudaGetLastError();
 }
 
@@ -140,8 +159,6 @@ cudaError_t launch_simt_m(const GemvArgs &a, cudaStream_t s)
 
 }  // namespace
 
-bool gemv_simt_fits(int M, int64_t K) { return (size_t)M * (size_t)K * sizeof(float) <= kSimtMaxSmem; }
-
 cudaError_t launch_gemv_simt(const GemvArgs &a, cudaStream_t s)
 {
     if (a.fmt == BQ_BINARY_G128)
@@ -151,17 +168,22 @@ cudaError_t launch_gemv_simt(const GemvArgs &a, cudaStream_t s)
                           : launch_simt_m<BQ_TERNARY_G128, __nv_bfloat16>(a, s);
 }
 
+// Workspace of the tensor-core path (partial sums of row blocks split between CTAs and
+// their counters); the SIMT kernel needs none.
 size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
 {
-    (void)M; (void)fmt; (void)N; (void)K;
-    return 0;
+    if (!gemv_tc_supported(M, fmt, K))
+        return 0;
+    return gemv_tc_workspace_bytes(M, fmt, N, K);
 }
 
+// K a multiple of 1024 (and its digit fragments fit in shared memory): the integer
+// tensor-core kernel; otherwise the SIMT kernel. One launch either way.
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches)
 {
-    if (!gemv_simt_fits(a.M, a.K))
-        return cudaErrorInvalidValue;
     *launches = 1;
+    if (gemv_tc_supported(a.M, a.fmt, a.K))
+        return launch_gemv_tc(a, s);
     return launch_gemv_simt(a, s);
 }
 

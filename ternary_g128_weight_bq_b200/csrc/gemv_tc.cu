@@ -1,0 +1,626 @@
+// gemv_tc.cu -- decode GEMV (M <= 8) on packed binary-g128 / ternary-g128 weights that streams
+// the packed words at HBM speed and sums on the integer tensor cores.
+//
+// Model card "prism-ml/Bonsai-27B-mlx-1bit", sections "Weight representation: Binary g128" and
+// "CUDA (NVIDIA GPUs)": y[m][n] = sum_g s[n][g] * sum_{k in g} v[n][k] x[m][k], v = +-1
+// (binary) or {-1, 0, +1} (ternary: "Ternary Bonsai 27B vs ..." article, wmrh.cn); the packed
+// weights are unpacked inside the product and each group scale is applied once per group.
+// Batch-1 decode (tg128) is the memory-bound phase of section "Cross-platform throughput".
+//
+// Why this shape. At B200's HBM rate one SM receives ~174 binary weights per clock. A
+// select-and-add per weight on the CUDA cores costs more issue slots than that, so each
+// sign bit is turned into the 8-bit integer +-64 (one IMAD shift on the FMA pipe and one LOP3
+// on the ALU pipe per four weights) and mma.sync m16n8k32 s8 (measured ~177 weights per SM
+// clock with fresh operands) does the additions, exactly, in int32: the "add" of select-and-add
+// runs on the tensor pipe. Ternary codes become {-64, 0, +64} with one PRMT per four codes.
+//
+// x as integers. Per (token, group of 128), x is written as X = round(x * 2^(21-e)) with
+// e = floor(log2 max|x|) over the group, |X| < 2^22, split into three balanced base-256 digits
+// d0 + 256 d1 + 65536 d2 (each in [-128, 127]); every digit is one MMA column. The rounding
+// error is at most 2^-22 max|x| per element, 2^-15 max|x| s per group: below 1/60 of that
+// group's share of the 2e-3 sum|x s| tolerance. The int32 column sums are exact; the group
+// scale times 2^(e-27+8d) is applied once per group in fp32.
+//
+// One kernel per call (programmatic dependent launch):
+//   * prologue: the CTA's consumer warps turn x into MMA B fragments (digits) for the k-chunks
+//     the CTA will touch, straight into shared memory, while the producer already streams the
+//     first weight tiles;
+//   * units = (block of 128 rows, 512-k chunk); CTA i owns units [i U / P, (i+1) U / P)
+//     (stream-K), so every shape is balanced to one unit;
+//   * the producer lane TMA-loads, per unit, the 128 x 64 B (binary, 64B swizzle) or
+//     128 x 128 B (ternary, 128B swizzle) tile of packed words and the 128 x 8 scales into a
+//     ring of stages; consumer warp w owns rows 16 w .. 16 w + 15;
+//   * a block owned by one CTA is written directly; a block split between CTAs leaves partial
+//     sums in the workspace, and the last warp to finish its 16 rows (a counter tagged with
+//     the call id, so it needs no zero-filled workspace) adds them in a fixed order.
+#include <cuda.h>
+
+#include "bq_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace bq {
+namespace {
+
+constexpr int kRows = 128;           // weight rows per block (8 warps x 16)
+constexpr int kChunkK = 512;         // k per unit (4 groups)
+constexpr int kConsumers = 8;
+constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kDigits = 3;           // base-256 digits of x per token
+constexpr int kMaxStages = 8;
+constexpr int kSmemLimit = 227 * 1024;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Position of weight k of a group in the MMA operands: quad-thread t (lane % 4) holds register
+// rho (0..7) of the A fragment of its two rows; byte b of it is weight k_local(t, rho, b).
+// MMA j of the group takes registers 2j (k slots 0..15) and 2j+1 (slots 16..31); the B
+// fragment uses the same (t, rho, b) -> k map.
+template <int FMT>
+__device__ __forceinline__ int k_local(int t, int rho, int b)
+{
+    if (FMT == BQ_BINARY_G128)
+        return 32 * t + 8 * b + rho;                 // bit 8b + rho of word t of the group
+    const int h = rho >> 2, r = rho & 3;             // word 2t + h of the group (16 codes)
+    const int i = (r == 0) ? 2 * b : (r == 1) ? 8 + 2 * b : (r == 2) ? 2 * b + 1 : 9 + 2 * b;
+    return 16 * (2 * t + h) + i;
+}
+
+template <int FMT> struct StageCfg {
+    static constexpr int kWordBytes = kRows * (FMT == BQ_BINARY_G128 ? 64 : 128);
+    static constexpr int kScaleBytes = kRows * 16;   // 8 fp16 scales per row
+    static constexpr int kBytes = kWordBytes + kScaleBytes;
+};
+
+struct Layout {
+    int frag_off, colf_off, stage_off, red_off, bar_off, total, stages;
+};
+
+// Shared-memory layout for a call (host and device compute the same thing).
+template <int FMT, int CS>
+__host__ __device__ inline Layout make_layout(int G, int stages)
+{
+    Layout L;
+    L.frag_off = 0;
+    L.colf_off = CS * G * 1024;
+    L.stage_off = (L.colf_off + CS * G * 32 + 1023) / 1024 * 1024;
+    L.red_off = L.stage_off + stages * StageCfg<FMT>::kBytes;
+    L.bar_off = L.red_off + kConsumers * 16 * CS * 8 * 4;
+    L.total = L.bar_off + 256 + 1024;                // barriers + alignment slack
+    L.stages = stages;
+    return L;
+}
+
+struct Bars {
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    int abort;
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0)
+        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, kWaitLimitNs);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok)
+        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, kWaitLimitNs);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// 8 A registers (s8 +-64) of one binary word: register i holds, in byte b, bit 8b + i
+// (1 -> +64 = 0x40, 0 -> -64 = 0xC0). The shift is a multiply by mul[i] = 2^(7-i) held in a
+// register, so it issues on the FMA pipe; the LOP3 issues on the ALU pipe.
+__device__ __forceinline__ void expand_binary(uint32_t w, const uint32_t (&mul)[8], uint32_t *a)
+{
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        uint32_t sh;
+        asm("mad.lo.u32 %0, %1, %2, 0;" : "=r"(sh) : "r"(w), "r"(mul[i]));   // bit 8b+i -> 8b+7
+        uint32_t r;
+        asm("lop3.b32 %0, %1, %2, %3, 0xAE;" : "=r"(r) : "r"(sh), "r"(0x80808080u), "r"(0x40404040u));
+        a[i] = r;                                    // (~sh & 0x80808080) | 0x40404040
+    }
+}
+
+// 4 A registers of one ternary word (16 codes), through a PRMT byte table:
+// code 0 -> -64 (0xC0), 1 -> 0, 2 -> +64 (0x40), 3 (invalid) -> 0.
+__device__ __forceinline__ void expand_ternary(uint32_t w, uint32_t *a)
+{
+    const uint32_t table = 0x004000C0u;
+    const uint32_t e = w & 0x33333333u;              // codes 0, 2, .., 14 in nibbles 0..7
+    const uint32_t o = (w >> 2) & 0x33333333u;       // codes 1, 3, .., 15
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a[0]) : "r"(table), "r"(e));
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a[1]) : "r"(table), "r"(e >> 16));
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a[2]) : "r"(table), "r"(o));
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a[3]) : "r"(table), "r"(o >> 16));
+}
+
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <typename T>
+__device__ __forceinline__ void store_y(void *y, int yt, int64_t idx, float v)
+{
+    (void)sizeof(T);
+    if (yt == BQ_F32)
+        store_out(static_cast<float *>(y) + idx, v);
+    else if (yt == BQ_BF16)
+        store_out(static_cast<__nv_bfloat16 *>(y) + idx, v);
+    else
+        store_out(static_cast<__half *>(y) + idx, v);
+}
+
+// Turn x[m][128 q .. 128 q + 127] into the digit fragments of group q (all column sets) and
+// the column factors. One warp; lane (t, rho) builds register rho of quad-thread t.
+template <int FMT, int CS, typename XT>
+__device__ __forceinline__ void build_fragments(const XT *__restrict__ x, int M, int64_t K, int G, int q, int lane,
+                                                uint32_t *frag_s, float *colf_s)
+{
+    const int t = lane >> 3, rho = lane & 7;
+    uint32_t outw[CS * 8];
+    float fac[CS * 8];
+#pragma unroll
+    for (int c = 0; c < CS * 8; c++) {
+        outw[c] = 0u;
+        fac[c] = 0.f;
+    }
+    float v[8][4];
+#pragma unroll
+    for (int m = 0; m < 8; m++)
+        if (m < M)
+#pragma unroll
+            for (int b = 0; b < 4; b++)
+                v[m][b] = load_x(x + (int64_t)m * K + 128 * q + k_local<FMT>(t, rho, b));
+#pragma unroll
+    for (int m = 0; m < 8; m++) {
+        if (m >= M)
+            break;
+        float amax = fmaxf(fmaxf(fabsf(v[m][0]), fabsf(v[m][1])), fmaxf(fabsf(v[m][2]), fabsf(v[m][3])));
+#pragma unroll
+        for (int o = 16; o; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        int e = 0;
+        if (amax > 0.f) {
+            frexpf(amax, &e);                        // amax = f 2^e, f in [0.5, 1)
+            e -= 1;                                  // amax in [2^e, 2^(e+1))
+        }
+        uint32_t dw[kDigits] = {0u, 0u, 0u};
+#pragma unroll
+        for (int b = 0; b < 4; b++) {
+            int X = amax > 0.f ? __float2int_rn(ldexpf(v[m][b], 21 - e)) : 0;   // |X| < 2^22
+#pragma unroll
+            for (int d = 0; d < kDigits; d++) {
+                const int dig = ((X + 128) & 255) - 128;                     // balanced digit
+                dw[d] |= ((uint32_t)dig & 0xFFu) << (8 * b);
+                X = (X - dig) >> 8;                                          // exact
+            }
+        }
+#pragma unroll
+        for (int d = 0; d < kDigits; d++) {
+            const int c = m * kDigits + d;
+            if (c < CS * 8) {
+                outw[c] = dw[d];
+                fac[c] = amax > 0.f ? ldexpf(1.f, e - 27 + 8 * d) : 0.f;    // 2^(e-21+8d) / 64
+            }
+        }
+    }
+    // fragment layout in shared memory: [cs][q][half][lane][4] u32, register rho = 4 half + r
+#pragma unroll
+    for (int c = 0; c < CS * 8; c++) {
+        const int cs = c >> 3, ln = 4 * (c & 7) + t;
+        frag_s[(((cs * G + q) * 2 + (rho >> 2)) * 32 + ln) * 4 + (rho & 3)] = outw[c];
+    }
+    if (lane < CS * 8)
+        colf_s[((lane >> 3) * G + q) * 8 + (lane & 7)] = fac[lane];
+}
+
+template <int FMT, int CS, typename XT>
+__global__ void __launch_bounds__(kThreads, 1)
+gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
+               const XT *__restrict__ x, int M, int64_t N, int64_t K, void *__restrict__ y, int yt,
+               float *__restrict__ part, unsigned long long *__restrict__ counters, int64_t U, int C, int maxseg,
+               int stages, uint32_t call_id, uint32_t one, unsigned int *dev_status)
+{
+    using SC = StageCfg<FMT>;
+    const int G = (int)(K / 128);
+    const Layout L = make_layout<FMT, CS>(G, stages);
+    const int S = stages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t *frag_s = reinterpret_cast<uint32_t *>(smem + L.frag_off);
+    float *colf_s = reinterpret_cast<float *>(smem + L.colf_off);
+    float *red = reinterpret_cast<float *>(smem + L.red_off);
+    Bars *bars = reinterpret_cast<Bars *>(smem + L.bar_off);
+    volatile int *abort = &bars->abort;
+    unsigned int *err = dev_status + kSlotErrBits;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t Pn = gridDim.x;
+    const int64_t u0 = (int64_t)blockIdx.x * U / Pn, u1 = ((int64_t)blockIdx.x + 1) * U / Pn;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; s++) {
+            ptx::mbar_init(&bars->full[s], 1);
+            ptx::mbar_init(&bars->empty[s], kConsumers);
+        }
+        bars->abort = 0;
+        ptx::fence_barrier_init();
+    }
+    __syncthreads();
+    // the next kernel in the stream may start its own prologue now; it still waits for this
+    // grid to finish before it reads anything this grid writes
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    if (warp == kConsumers) {
+        // ------------------------------------------------------------------- producer
+        if (lane == 0) {
+            ptx::tma_prefetch_desc(&tmap_w);
+            ptx::tma_prefetch_desc(&tmap_s);
+            int64_t it = 0;
+            for (int64_t u = u0; u < u1; u++, it++) {
+                const int s = (int)(it % S);
+                const uint32_t ph = (uint32_t)((it / S) & 1);
+                if (!ptx::mbar_wait_bounded(&bars->empty[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
+                    break;
+                const int64_t rb = u / C;
+                const int c = (int)(u % C);
+                uint8_t *st = smem + L.stage_off + s * SC::kBytes;
+                ptx::mbar_arrive_expect_tx(&bars->full[s], SC::kBytes);
+                ptx::tma_load_2d(st, &tmap_w, &bars->full[s], c * (FMT == BQ_BINARY_G128 ? 16 : 32),
+                                 (int32_t)(rb * kRows));
+                ptx::tma_load_2d(st + SC::kWordBytes, &tmap_s, &bars->full[s], (4 * c) & ~7, (int32_t)(rb * kRows));
+            }
+            // no copy may still be in flight when the CTA exits
+            for (int64_t k = it > S ? it - S : 0; k < it; k++) {
+                volatile int no_abort = 0;
+                ptx::mbar_wait_bounded(&bars->full[k % S], (uint32_t)((k / S) & 1), &no_abort, err,
+                                       kDevErrTimeout, kWaitLimitNs);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------- consumers
+        // x may be the output of the previous kernel in the stream
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        {
+            // digit fragments of the chunks this CTA touches (all of them if it owns >= C units)
+            const int64_t span = u1 - u0 < C ? u1 - u0 : C;
+            const int nitems = (int)span * 4;
+            for (int i = warp; i < nitems; i += kConsumers) {
+                const int c = (int)((u0 + i / 4) % C);
+                build_fragments<FMT, CS, XT>(x, M, K, G, 4 * c + (i & 3), lane, frag_s, colf_s);
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");   // fragments ready
+
+        const int g8 = lane >> 2, t = lane & 3;
+        const int r0 = warp * 16 + g8, r1 = r0 + 8;          // rows of this thread in the block
+        uint32_t mul[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+            mul[i] = one << (7 - i);
+        float *wred = red + warp * (16 * CS * 8);            // [16 rows][CS*8 columns]
+        int64_t it = 0;
+        bool ok = true;
+        for (int64_t rb = u0 / C; ok && rb * C < u1; rb++) {
+            const int c_lo = (int)(rb == u0 / C ? u0 % C : 0);
+            const int c_hi = (int)((rb + 1) * C <= u1 ? C : u1 - rb * C);
+            float acc[CS][4];
+#pragma unroll
+            for (int cs = 0; cs < CS; cs++)
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    acc[cs][i] = 0.f;
+            for (int c = c_lo; c < c_hi; c++, it++) {
+                const int s = (int)(it % S);
+                const uint32_t ph = (uint32_t)((it / S) & 1);
+                if (!warp_wait(&bars->full[s], ph, abort, err)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *st = smem + L.stage_off + s * SC::kBytes;
+                const uint16_t *sc = reinterpret_cast<const uint16_t *>(st + SC::kWordBytes);
+                const int soff = (4 * c) & 7;
+#pragma unroll
+                for (int qp = 0; qp < 4; qp += 2) {         // two groups at a time: independent chains
+                    uint32_t A[2][2][8];                    // [group][row r0/r1][register]
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const int q = qp + h;
+                        if (FMT == BQ_BINARY_G128) {
+                            const int ch0 = q ^ ((r0 >> 1) & 3), ch1 = q ^ ((r1 >> 1) & 3);
+                            const uint32_t w0 = *reinterpret_cast<const uint32_t *>(st + r0 * 64 + ch0 * 16 + 4 * t);
+                            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(st + r1 * 64 + ch1 * 16 + 4 * t);
+                            expand_binary(w0, mul, A[h][0]);
+                            expand_binary(w1, mul, A[h][1]);
+                        } else {
+                            const int c16 = 2 * q + (t >> 1);
+                            const uint2 w0 = *reinterpret_cast<const uint2 *>(st + r0 * 128 + ((c16 ^ (r0 & 7)) << 4) + 8 * (t & 1));
+                            const uint2 w1 = *reinterpret_cast<const uint2 *>(st + r1 * 128 + ((c16 ^ (r1 & 7)) << 4) + 8 * (t & 1));
+                            expand_ternary(w0.x, A[h][0]);
+                            expand_ternary(w0.y, A[h][0] + 4);
+                            expand_ternary(w1.x, A[h][1]);
+                            expand_ternary(w1.y, A[h][1] + 4);
+                        }
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const int q = qp + h;
+                        const int gq = 4 * c + q;          // group index within K
+                        const float s0 = __half2float(__ushort_as_half(sc[r0 * 8 + soff + q]));
+                        const float s1 = __half2float(__ushort_as_half(sc[r1 * 8 + soff + q]));
+#pragma unroll
+                        for (int cs = 0; cs < CS; cs++) {
+                            const uint4 bA = *reinterpret_cast<const uint4 *>(frag_s + (((cs * G + gq) * 2 + 0) * 32 + lane) * 4);
+                            const uint4 bB = *reinterpret_cast<const uint4 *>(frag_s + (((cs * G + gq) * 2 + 1) * 32 + lane) * 4);
+                            const uint32_t b[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
+                            int de[4] = {0, 0, 0, 0}, dd[4] = {0, 0, 0, 0};   // two independent chains
+                            mma_s8(de, A[h][0][0], A[h][1][0], A[h][0][1], A[h][1][1], b[0], b[1]);
+                            mma_s8(dd, A[h][0][2], A[h][1][2], A[h][0][3], A[h][1][3], b[2], b[3]);
+                            mma_s8(de, A[h][0][4], A[h][1][4], A[h][0][5], A[h][1][5], b[4], b[5]);
+                            mma_s8(dd, A[h][0][6], A[h][1][6], A[h][0][7], A[h][1][7], b[6], b[7]);
+                            const float2 f = *reinterpret_cast<const float2 *>(colf_s + (cs * G + gq) * 8 + 2 * t);
+                            // (r0, col 2t) (r0, 2t+1) (r1, 2t) (r1, 2t+1)
+                            acc[cs][0] = fmaf((float)(de[0] + dd[0]), s0 * f.x, acc[cs][0]);
+                            acc[cs][1] = fmaf((float)(de[1] + dd[1]), s0 * f.y, acc[cs][1]);
+                            acc[cs][2] = fmaf((float)(de[2] + dd[2]), s1 * f.x, acc[cs][2]);
+                            acc[cs][3] = fmaf((float)(de[3] + dd[3]), s1 * f.y, acc[cs][3]);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0)
+                    ptx::mbar_arrive(&bars->empty[s]);
+            }
+            if (!ok)
+                break;
+
+            // ---- digits of a token: y[row][m] = sum_d acc[row][3m + d]
+#pragma unroll
+            for (int cs = 0; cs < CS; cs++) {
+                wred[g8 * (CS * 8) + cs * 8 + 2 * t] = acc[cs][0];
+                wred[g8 * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][1];
+                wred[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t] = acc[cs][2];
+                wred[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][3];
+            }
+            __syncwarp();
+            const int64_t row0 = rb * kRows + warp * 16;
+            const bool whole = c_lo == 0 && c_hi == C;
+            const int64_t x0 = rb * C, x1 = rb * C + C;     // owners of the block's first/last unit
+            const int64_t i_first = (x0 + 1) * Pn / U + (((x0 + 1) * Pn) % U != 0) - 1;
+            const int64_t i_last = x1 * Pn / U + ((x1 * Pn) % U != 0) - 1;
+            const int nseg = (int)(i_last - i_first + 1);
+            const int seg = (int)(blockIdx.x - i_first);
+            for (int e = lane; e < 16 * M; e += 32) {
+                const int rr = e / M, m = e % M;
+                float v = 0.f;
+#pragma unroll
+                for (int d = 0; d < kDigits; d++)
+                    v += wred[rr * (CS * 8) + m * kDigits + d];
+                const int64_t n = row0 + rr;
+                if (whole) {
+                    if (n < N)
+                        store_y<float>(y, yt, (int64_t)m * N + n, v);
+                } else {
+                    part[((rb * maxseg + seg) * kRows + warp * 16 + rr) * M + m] = v;
+                }
+            }
+            __syncwarp();
+            if (!whole) {
+                // the last of the nseg warps that own these 16 rows sums the partials in
+                // segment order; the counter holds (call id << 32) | arrivals and is reset to 0
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) {
+                    unsigned long long *ctr = counters + rb * kConsumers + warp;
+                    const unsigned long long tag = (unsigned long long)call_id << 32;
+                    unsigned long long cur = atomicAdd(ctr, 0ull);
+                    for (int tries = 0; tries < (1 << 20); tries++) {
+                        const unsigned long long next = (cur >> 32) == call_id ? cur + 1 : (tag | 1ull);
+                        const unsigned long long prev = atomicCAS(ctr, cur, next);
+                        if (prev == cur) {
+                            last = (int)(next & 0xFFFFFFFFull) == nseg;
+                            if (last)
+                                atomicExch(ctr, 0ull);
+                            break;
+                        }
+                        cur = prev;
+                    }
+                }
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {
+                    __threadfence();
+                    for (int e = lane; e < 16 * M; e += 32) {
+                        const int rr = e / M, m = e % M;
+                        float v = 0.f;
+                        for (int sg = 0; sg < nseg; sg++)           // fixed order: deterministic
+                            v += __ldcg(part + ((rb * maxseg + sg) * kRows + warp * 16 + rr) * M + m);
+                        const int64_t n = row0 + rr;
+                        if (n < N)
+                            store_y<float>(y, yt, (int64_t)m * N + n, v);
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+int sm_count()
+{
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+struct Plan {
+    int CS, stages, grid, maxseg;
+    int64_t NB, C, U;
+    int smem;
+    size_t part_bytes, counter_bytes;
+};
+
+template <int FMT, int CS>
+int plan_stages(int G)
+{
+    for (int s = kMaxStages; s >= 2; s--)
+        if (make_layout<FMT, CS>(G, s).total <= kSmemLimit)
+            return s;
+    return 0;
+}
+
+int stages_for(int fmt, int CS, int G)
+{
+    if (fmt == BQ_BINARY_G128)
+        return CS == 1 ? plan_stages<BQ_BINARY_G128, 1>(G) : CS == 2 ? plan_stages<BQ_BINARY_G128, 2>(G)
+                                                                     : plan_stages<BQ_BINARY_G128, 3>(G);
+    return CS == 1 ? plan_stages<BQ_TERNARY_G128, 1>(G) : CS == 2 ? plan_stages<BQ_TERNARY_G128, 2>(G)
+                                                                  : plan_stages<BQ_TERNARY_G128, 3>(G);
+}
+
+Plan make_plan(int M, int fmt, int64_t N, int64_t K)
+{
+    Plan p;
+    p.CS = (M * kDigits + 7) / 8;
+    const int G = (int)(K / 128);
+    p.stages = stages_for(fmt, p.CS, G);
+    p.NB = (N + kRows - 1) / kRows;
+    p.C = K / kChunkK;
+    p.U = p.NB * p.C;
+    const int64_t sms = sm_count();
+    p.grid = (int)(p.U < sms ? p.U : sms);
+    const int64_t per = p.U / p.grid;                 // every CTA owns at least `per` units
+    p.maxseg = (int)((p.C + per - 1) / per + 1);
+    if (p.maxseg > p.grid)
+        p.maxseg = p.grid;
+    auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
+    p.part_bytes = al((size_t)p.NB * p.maxseg * kRows * M * 4);
+    p.counter_bytes = al((size_t)p.NB * kConsumers * 8);
+    if (p.stages)
+        p.smem = fmt == BQ_BINARY_G128 ? 0 : 0;      // filled by the launcher
+    return p;
+}
+
+uint32_t next_call_id()
+{
+    static uint32_t ctr = 0;
+    uint32_t v = __atomic_add_fetch(&ctr, 1u, __ATOMIC_RELAXED);
+    return v ? v : __atomic_add_fetch(&ctr, 1u, __ATOMIC_RELAXED);
+}
+
+template <int FMT, int CS, typename XT>
+cudaError_t launch_tc_t(const GemvArgs &a, const Plan &pl, cudaStream_t s)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return cudaErrorNotSupported;
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    float *part = reinterpret_cast<float *>(ws);
+    unsigned long long *counters = reinterpret_cast<unsigned long long *>(ws + pl.part_bytes);
+
+    CUtensorMap mw, ms;
+    const cuuint64_t wpr = (cuuint64_t)(FMT == BQ_BINARY_G128 ? a.K / 32 : a.K / 16);
+    cuuint64_t wdims[2] = {wpr, (cuuint64_t)a.N};
+    cuuint64_t wstr[1] = {wpr * 4};
+    cuuint32_t wbox[2] = {(cuuint32_t)(FMT == BQ_BINARY_G128 ? 16 : 32), (cuuint32_t)kRows};
+    cuuint32_t est[2] = {1, 1};
+    CUresult r = enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(a.words), wdims, wstr, wbox, est,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     FMT == BQ_BINARY_G128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const cuuint64_t G = (cuuint64_t)(a.K / 128);
+    cuuint64_t sdims[2] = {G, (cuuint64_t)a.N};
+    cuuint64_t sstr[1] = {G * 2};
+    cuuint32_t sbox[2] = {8, (cuuint32_t)kRows};
+    r = enc(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<__half *>(a.scales), sdims, sstr, sbox, est,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+
+    const int smem = make_layout<FMT, CS>((int)G, pl.stages).total;
+    auto kern = gemv_tc_kernel<FMT, CS, XT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mw, ms, static_cast<const XT *>(a.x), a.M, a.N, a.K, a.y, a.yt, part,
+                              counters, pl.U, (int)pl.C, pl.maxseg, pl.stages, next_call_id(), 1u, a.dev_status);
+}
+
+template <int FMT, typename XT>
+cudaError_t launch_tc_cs(const GemvArgs &a, const Plan &pl, cudaStream_t s)
+{
+    switch (pl.CS) {
+    case 1: return launch_tc_t<FMT, 1, XT>(a, pl, s);
+    case 2: return launch_tc_t<FMT, 2, XT>(a, pl, s);
+    default: return launch_tc_t<FMT, 3, XT>(a, pl, s);
+    }
+}
+
+}  // namespace
+
+// K a multiple of 1024 (whole 8-scale TMA boxes) and the digit fragments of all of K in
+// shared memory next to at least two stages.
+bool gemv_tc_supported(int M, int fmt, int64_t K)
+{
+    if (M < 1 || M > 8 || K % 1024 != 0)
+        return false;
+    return stages_for(fmt, (M * kDigits + 7) / 8, (int)(K / 128)) >= 2;
+}
+
+size_t gemv_tc_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
+{
+    Plan p = make_plan(M, fmt, N, K);
+    return p.part_bytes + p.counter_bytes;
+}
+
+cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s)
+{
+    Plan pl = make_plan(a.M, a.fmt, a.N, a.K);
+    if (a.fmt == BQ_BINARY_G128)
+        return a.xt == BQ_F16 ? launch_tc_cs<BQ_BINARY_G128, __half>(a, pl, s)
+                              : launch_tc_cs<BQ_BINARY_G128, __nv_bfloat16>(a, pl, s);
+    return a.xt == BQ_F16 ? launch_tc_cs<BQ_TERNARY_G128, __half>(a, pl, s)
+                          : launch_tc_cs<BQ_TERNARY_G128, __nv_bfloat16>(a, pl, s);
+}
+
+}  // namespace bq

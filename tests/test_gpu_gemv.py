@@ -123,3 +123,73 @@ def test_api_errors_on_device():
     assert e.value.status_name == "BQ_ERR_ALIGNMENT"
     m.gemv(xd, w)                                              # still works afterwards
     torch.cuda.synchronize()
+
+
+# ---- tensor-core path (K a multiple of 1024): fp8 pieces of x, stream-K split ----------
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("xdt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("N,K", [(1, 1024), (127, 2048), (129, 1024), (1000, 3072)])
+def test_tensor_path_ragged_all_outputs(orc, M, xdt, N, K):
+    run_binary(orc, 400 + M, N, K, M, xdt=xdt)
+
+
+@pytest.mark.parametrize("M", [1, 4, 8])
+@pytest.mark.parametrize("N,K", [(5, 1024), (333, 2048), (2000, 5120)])
+def test_tensor_path_ternary(orc, M, N, K):
+    run_ternary(orc, 500 + M, N, K, M)
+
+
+def test_tensor_path_wide_dynamic_range(orc):
+    """x spanning 40 binades inside each group: the e4m3 pieces stay within the bound."""
+    m = bq()
+    N, K, M = 300, 2048, 3
+    x = synth.activations(7, M, K, dtype=torch.float32)
+    mag = torch.tensor([2.0 ** (-30 + (k % 41)) for k in range(K)])
+    x = (x * mag).to(torch.bfloat16)
+    words = synth.binary_words(7, N, K)
+    s = synth.scales(7, N, K // 128)
+    w = m.BQWeight(m.BINARY_G128, N, K, words.cuda(), s.cuda())
+    y = m.gemv(x.cuda(), w)
+    y_ref, bound = orc.gemv(oracle.BINARY, x, oracle.X_BF16, words, s, K)
+    assert_within_bound(y, y_ref, bound, "wide range")
+
+
+def test_tensor_path_zero_and_tiny_groups(orc):
+    m = bq()
+    N, K, M = 200, 1024, 2
+    x = synth.activations(8, M, K).float()
+    x[0, :128] = 0.0                                   # an all-zero group
+    x[1, 128:256] = 1e-30                              # a group of tiny values
+    x = x.to(torch.bfloat16)
+    words = synth.binary_words(8, N, K)
+    s = synth.scales(8, N, K // 128)
+    w = m.BQWeight(m.BINARY_G128, N, K, words.cuda(), s.cuda())
+    y = m.gemv(x.cuda(), w)
+    y_ref, bound = orc.gemv(oracle.BINARY, x, oracle.X_BF16, words, s, K)
+    assert_within_bound(y, y_ref, bound, "zero/tiny groups")
+
+
+def test_tensor_path_deterministic():
+    """Split blocks are summed in a fixed order: repeated calls give identical bits."""
+    m = bq()
+    x, words, s = binary_inputs(9, 5120, 5120, 8)
+    w = m.BQWeight(m.BINARY_G128, 5120, 5120, words.cuda(), s.cuda())
+    xd = x.cuda()
+    y1 = m.gemv(xd, w).clone()
+    for _ in range(5):
+        assert torch.equal(m.gemv(xd, w), y1)
+
+
+def test_workspace_too_small_is_rejected():
+    m = bq()
+    x, words, s = binary_inputs(10, 256, 1024, 2)
+    w = m.BQWeight(m.BINARY_G128, 256, 1024, words.cuda(), s.cuda())
+    need = m.gemv_workspace_bytes(2, w)
+    assert need > 0
+    y = torch.empty((2, 256), dtype=torch.float32, device="cuda")
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(m.BQError) as e:
+        m._check(m.lib().bq_gemv(x.cuda().data_ptr(), 1, 2, w.c, y.data_ptr(), 2, ws.data_ptr(),
+                                 need - 256, m._stream()))
+    assert e.value.status_name == "BQ_ERR_WORKSPACE"
