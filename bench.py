@@ -276,6 +276,7 @@ def extra_workloads(bq, device, stream, peaks):
     res["ternary_gemv"] = {"N": 20480, "K": K_HEAD, "M": 1, "us": round(ms * 1e3, 2),
                            "GBps": round(gemv_bytes(20480, K_HEAD, 1, 2) / 1e9 / (ms / 1e3), 1)}
     del tsets
+    res["full_depth_decode_step"] = full_depth_step(bq, device, stream, peaks)
     # prefill GEMM: M=512, K=5120, N=20480 binary and ternary
     try:
         for fmt_name in ("binary", "ternary"):
@@ -296,6 +297,42 @@ def extra_workloads(bq, device, stream, peaks):
     except Exception as e:  # reported, not hidden: the line says why there is no number
         res["prefill"] = {"error": str(e).splitlines()[0][:200]}
     return res
+
+
+# the 64 blocks of the full-depth decode step: (N, K) of each block's four binary GEMVs
+FULL_DEPTH_BLOCK = [(9120, 5120), (5120, 5120), (40960, 5120), (5120, 20480)]
+FULL_DEPTH_BLOCKS = 64
+
+
+def full_depth_step(bq, device, stream, peaks):
+    """One decode token through all 64 blocks: 256 binary GEMVs at M = 1 (24.8e9 weights,
+    3.49 GB, every block's weights distinct), replayed as one CUDA graph."""
+    mats = []
+    for b in range(FULL_DEPTH_BLOCKS):
+        for j, (N, K) in enumerate(FULL_DEPTH_BLOCK):
+            seed = 1000 + 4 * b + j
+            mats.append(bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(seed, N, K, device=device),
+                                    synth.scales(seed, N, K // 128, device=device)))
+    xs = {K: synth.activations(0, 1, K).to(device) for K in (5120, 20480)}
+    ys = {N: torch.empty((1, N), dtype=torch.float32, device=device) for (N, _) in FULL_DEPTH_BLOCK}
+    ws_bytes = max(bq.gemv_workspace_bytes(1, w) for w in mats[:4])
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+    total = sum(gemv_bytes(w.N, w.K, 1) for w in mats)
+    with torch.cuda.stream(stream):
+        for w in mats[:4]:
+            bq.gemv(xs[w.K], w, out=ys[w.N], workspace=ws)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for w in mats:
+                bq.gemv(xs[w.K], w, out=ys[w.N], workspace=ws)
+        ms = time_single(g.replay, 20, 3, stream)
+    del g, mats
+    torch.cuda.empty_cache()
+    gbs = total / 1e9 / (ms / 1e3)
+    return {"blocks": FULL_DEPTH_BLOCKS, "gemvs": 4 * FULL_DEPTH_BLOCKS, "bytes": total,
+            "us": round(ms * 1e3, 1), "tokens_per_s": round(1e3 / ms, 1), "GBps": round(gbs, 1),
+            "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4)}
 
 
 def e2e_gemv(bq, device, steps, warmup, stream):
@@ -529,6 +566,50 @@ def run_gpu(args):
     return 0
 
 
+def run_case(args):
+    """One workload alone, --steps calls after --warmup, for profiling (ncu -k / -c) and
+    spot timing; prints one JSON line with the average device time per call."""
+    import ternary_g128_weight_bq_b200 as bq
+    from ternary_g128_weight_bq_b200 import build as bqbuild
+    bqbuild.build()
+    device = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device)
+    N, M, K = args.N, args.M, args.K
+    with torch.cuda.stream(stream):
+        if args.case in ("gemv", "prefill"):
+            if args.fmt == "binary":
+                w = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(0, N, K, device=device),
+                                synth.scales(0, N, K // 128, device=device))
+            else:
+                q = synth.random_ternary(0, synth.TID_TERNARY, (N, K), device=device)
+                w = bq.pack_ternary_g128(q, synth.scales(0, N, K // 128, device=device))
+                del q
+            x = synth.activations(0, M, K).to(device)
+            if args.case == "gemv":
+                y = torch.empty((M, N), dtype=torch.float32, device=device)
+                ws = torch.empty(max(bq.gemv_workspace_bytes(M, w), 16), dtype=torch.uint8, device=device)
+                fn = lambda: bq.gemv(x, w, out=y, workspace=ws)
+                work = {"GBps": gemv_bytes(N, K, M, 1 if args.fmt == "binary" else 2) / 1e9}
+            else:
+                y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+                fn = lambda: bq.gemm_prefill(x, w, out=y)
+                work = {"TFLOPs": 2 * M * N * K / 1e12}
+        elif args.case == "embed":
+            w = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(0, N, K, device=device),
+                            synth.scales(0, N, K // 128, device=device))
+            ids = synth.random_ids(0, synth.TID_IDS, M, N).to(device)
+            out = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+            fn = lambda: bq.embed_gather(ids, w, out=out)
+            work = {"GBps": M * (K // 8 + K // 64 + K * 2 + 4) / 1e9}
+        ms = time_single(fn, args.steps, args.warmup, stream)
+    line = {"case": args.case, "fmt": args.fmt, "N": N, "M": M, "K": K, "steps": args.steps,
+            "us_per_call": round(ms * 1e3, 3)}
+    for k, v in work.items():
+        line[k] = round(v / (ms / 1e3), 1)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -537,6 +618,12 @@ def main():
     ap.add_argument("--impl", choices=["bq", "reference"], default="bq")
     ap.add_argument("--quick", action="store_true", help="headline number only")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--case", choices=["gemv", "prefill", "embed"],
+                    help="time one workload alone (for profiling) instead of the benchmark")
+    ap.add_argument("--fmt", choices=["binary", "ternary"], default="binary")
+    ap.add_argument("--N", type=int, default=248320)
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--K", type=int, default=K_HEAD)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -545,6 +632,8 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
         return 1
+    if args.case:
+        return run_case(args)
     return run_gpu(args)
 
 

@@ -108,9 +108,10 @@ def random_ids(seed: int, tid: int, count: int, vocab: int) -> torch.Tensor:
     return ((u * vocab) >> 32).to(torch.int32)
 
 
-def normal(seed: int, tid: int, count: int, start: int = 0) -> torch.Tensor:
-    """``count`` N(0,1) samples in fp64 on the host (Box-Muller, cosine branch)."""
-    u = u32_stream(seed, tid, 2 * start, 2 * count).to(torch.float64)
+def normal(seed: int, tid: int, count: int, start: int = 0, device="cpu") -> torch.Tensor:
+    """``count`` N(0,1) samples in fp64 (Box-Muller, cosine branch), on the host unless a
+    device is given (device values may differ from host ones in the last bits of log/cos)."""
+    u = u32_stream(seed, tid, 2 * start, 2 * count, device).to(torch.float64)
     u1 = (u[0::2] + 0.5) / 2.0**32
     u2 = u[1::2] / 2.0**32
     return torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(2.0 * math.pi * u2)
@@ -122,12 +123,12 @@ def activations(seed: int, M: int, K: int, dtype=torch.bfloat16, tid: int = TID_
 
 
 def scales(seed: int, N: int, G: int, tid: int = TID_SCALES, row0: int = 0,
-           chunk: int = 1 << 24) -> torch.Tensor:
+           chunk: int = 1 << 24, device="cpu") -> torch.Tensor:
     """Group scales fp16[N, G] = fp16(|N(0, 0.02)| + 1e-3), rows [row0, row0 + N) of the stream."""
-    out = torch.empty(N * G, dtype=torch.float16)
+    out = torch.empty(N * G, dtype=torch.float16, device=device)
     for a in range(0, N * G, chunk):
         b = min(N * G, a + chunk)
-        z = normal(seed, tid, b - a, start=row0 * G + a)
+        z = normal(seed, tid, b - a, start=row0 * G + a, device=device)
         out[a:b] = (z.abs() * 0.02 + 1e-3).to(torch.float16)
     return out.reshape(N, G)
 

@@ -16,23 +16,28 @@
 //
 // x as integers. Per (token, group of 128), x is written as X = round(x * 2^(21-e)) with
 // e = floor(log2 max|x|) over the group, |X| < 2^22, split into three balanced base-256 digits
-// d0 + 256 d1 + 65536 d2 (each in [-128, 127]); every digit is one MMA column. The rounding
-// error is at most 2^-22 max|x| per element, 2^-15 max|x| s per group: below 1/60 of that
-// group's share of the 2e-3 sum|x s| tolerance. The int32 column sums are exact; the group
-// scale times 2^(e-27+8d) is applied once per group in fp32.
+// d0 + 256 d1 + 65536 d2 (each in [-128, 127]); every digit is one MMA column (a token owns
+// four columns: three digits and a zero one). The rounding error is at most 2^-22 max|x| per
+// element, 2^-15 max|x| s per group: below 1/60 of that group's share of the 2e-3 sum|x s|
+// tolerance. The int32 column sums are exact (each starts at the bits of 1.5 * 2^23, so one
+// fp32 subtraction turns it into a float without rounding); the group scale times 2^(e-27) is
+// applied once per group in fp32, and the digit weight 256^d once per block.
 //
 // One kernel per call (programmatic dependent launch):
 //   * prologue: the CTA's consumer warps turn x into MMA B fragments (digits) for the k-chunks
 //     the CTA will touch, straight into shared memory, while the producer already streams the
 //     first weight tiles;
-//   * units = (block of 128 rows, 512-k chunk); CTA i owns units [i U / P, (i+1) U / P)
+//   * units = (block of 128 rows, one stage of k); CTA i owns units [i U / P, (i+1) U / P)
 //     (stream-K), so every shape is balanced to one unit;
-//   * the producer lane TMA-loads, per unit, the 128 x 64 B (binary, 64B swizzle) or
-//     128 x 128 B (ternary, 128B swizzle) tile of packed words and the 128 x 8 scales into a
-//     ring of stages; consumer warp w owns rows 16 w .. 16 w + 15;
+//   * the producer lane TMA-loads, per unit, a 128 rows x 128 bytes tile of packed words (1024
+//     binary / 512 ternary weights per row; 128B swizzle; 128-byte rows stream measurably
+//     faster than 64-byte ones) into a ring of stages; 8 consumer warps, one per 16-row
+//     tile, expand the stage's groups four at a time (four independent MMA chains); the
+//     group scales come straight from global memory, each stage's loaded one stage early;
 //   * a block owned by one CTA is written directly; a block split between CTAs leaves partial
-//     sums in the workspace, and the last warp to finish its 16 rows (a counter tagged with
-//     the call id, so it needs no zero-filled workspace) adds them in a fixed order.
+//     sums in the workspace (two 128-row slots per CTA: its first and its last block), and the
+//     last warp to finish its 16 rows (a counter tagged with the call id, so it needs no
+//     zero-filled workspace) adds them in a fixed order.
 #include <cuda.h>
 
 #include "bq_internal.cuh"
@@ -41,11 +46,15 @@
 namespace bq {
 namespace {
 
-constexpr int kRows = 128;           // weight rows per block (8 warps x 16)
-constexpr int kChunkK = 512;         // k per unit (4 groups)
-constexpr int kConsumers = 8;
+constexpr int kRows = 128;           // weight rows per block (8 tiles of 16 rows)
+constexpr int kTiles = 8;
+constexpr int kHalves = 1;           // consumer warps per 16-row tile (each takes 1/kHalves of a stage's groups)
+constexpr int kConsumers = kTiles * kHalves;
+constexpr int kGP = 4;               // groups a warp expands and multiplies at once (independent chains)
 constexpr int kThreads = (kConsumers + 1) * 32;
 constexpr int kDigits = 3;           // base-256 digits of x per token
+constexpr int kColsPerTok = 4;       // MMA columns per token: the 3 digits and one zero column
+constexpr int kMagic = 0x4B400000;   // bits of 1.5 * 2^23: int n in |n| < 2^22 -> float(bits + n) = 1.5*2^23 + n
 constexpr int kMaxStages = 8;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -64,10 +73,11 @@ __device__ __forceinline__ int k_local(int t, int rho, int b)
     return 16 * (2 * t + h) + i;
 }
 
+// One stage = 128 rows x 128 bytes of packed words (one 128-byte-swizzled TMA box):
+// 1024 k (8 groups) of binary weights or 512 k (4 groups) of ternary codes.
 template <int FMT> struct StageCfg {
-    static constexpr int kWordBytes = kRows * (FMT == BQ_BINARY_G128 ? 64 : 128);
-    static constexpr int kScaleBytes = kRows * 16;   // 8 fp16 scales per row
-    static constexpr int kBytes = kWordBytes + kScaleBytes;
+    static constexpr int kGroups = FMT == BQ_BINARY_G128 ? 8 : 4;
+    static constexpr int kBytes = kRows * 128;
 };
 
 struct Layout {
@@ -81,9 +91,9 @@ __host__ __device__ inline Layout make_layout(int G, int stages)
     Layout L;
     L.frag_off = 0;
     L.colf_off = CS * G * 1024;
-    L.stage_off = (L.colf_off + CS * G * 32 + 1023) / 1024 * 1024;
+    L.stage_off = (L.colf_off + 2 * CS * G * 4 + 1023) / 1024 * 1024;   // one factor per token slot
     L.red_off = L.stage_off + stages * StageCfg<FMT>::kBytes;
-    L.bar_off = L.red_off + kConsumers * 16 * CS * 8 * 4;
+    L.bar_off = L.red_off + kTiles * 16 * CS * 8 * 4;
     L.total = L.bar_off + 256 + 1024;                // barriers + alignment slack
     L.stages = stages;
     return L;
@@ -95,28 +105,18 @@ struct Bars {
     int abort;
 };
 
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err)
-{
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0)
-        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, kWaitLimitNs);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (ok)
-        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, kWaitLimitNs);
-    return __all_sync(0xffffffffu, ok);
-}
-
 // 8 A registers (s8 +-64) of one binary word: register i holds, in byte b, bit 8b + i
 // (1 -> +64 = 0x40, 0 -> -64 = 0xC0). The shift is a multiply by mul[i] = 2^(7-i) held in a
 // register, so it issues on the FMA pipe; the LOP3 issues on the ALU pipe.
-__device__ __forceinline__ void expand_binary(uint32_t w, const uint32_t (&mul)[8], uint32_t *a)
+// mul[8] = {2^7, .., 2^1, 0x80808080, 0x40404040}: the masks live in registers (they come
+// from a kernel argument), so each byte select is a single three-register LOP3.
+__device__ __forceinline__ void expand_binary(uint32_t w, const uint32_t (&mul)[9], uint32_t *a)
 {
 #pragma unroll
     for (int i = 0; i < 8; i++) {
-        uint32_t sh;
-        asm("mad.lo.u32 %0, %1, %2, 0;" : "=r"(sh) : "r"(w), "r"(mul[i]));   // bit 8b+i -> 8b+7
+        const uint32_t sh = i < 7 ? w * mul[i] : w;  // bit 8b+i -> 8b+7 (mul[i] = 2^(7-i), a register)
         uint32_t r;
-        asm("lop3.b32 %0, %1, %2, %3, 0xAE;" : "=r"(r) : "r"(sh), "r"(0x80808080u), "r"(0x40404040u));
+        asm("lop3.b32 %0, %1, %2, %3, 0xAE;" : "=r"(r) : "r"(sh), "r"(mul[7]), "r"(mul[8]));
         a[i] = r;                                    // (~sh & 0x80808080) | 0x40404040
     }
 }
@@ -134,6 +134,34 @@ __device__ __forceinline__ void expand_ternary(uint32_t w, uint32_t *a)
     asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a[3]) : "r"(table), "r"(o >> 16));
 }
 
+// Expand one group of this thread's two rows straight into the four MMA A operands:
+// quad[j] = {row r0 reg 2j, row r1 reg 2j, row r0 reg 2j+1, row r1 reg 2j+1}, the register
+// order mma.sync wants, so no copies are needed to form the operand tuples.
+template <int FMT>
+__device__ __forceinline__ void expand_group(const uint8_t *p0, const uint8_t *p1, const uint32_t (&mul)[9],
+                                             uint32_t (&quad)[4][4])
+{
+    uint32_t a0[8], a1[8];
+    if (FMT == BQ_BINARY_G128) {
+        expand_binary(*reinterpret_cast<const uint32_t *>(p0), mul, a0);
+        expand_binary(*reinterpret_cast<const uint32_t *>(p1), mul, a1);
+    } else {
+        const uint2 w0 = *reinterpret_cast<const uint2 *>(p0);
+        const uint2 w1 = *reinterpret_cast<const uint2 *>(p1);
+        expand_ternary(w0.x, a0);
+        expand_ternary(w0.y, a0 + 4);
+        expand_ternary(w1.x, a1);
+        expand_ternary(w1.y, a1 + 4);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        quad[j][0] = a0[2 * j];
+        quad[j][1] = a1[2 * j];
+        quad[j][2] = a0[2 * j + 1];
+        quad[j][3] = a1[2 * j + 1];
+    }
+}
+
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1)
 {
@@ -141,6 +169,16 @@ __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, ui
         "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// First MMA of a chain: the accumulator input is a constant quad c (kept in registers).
+__device__ __forceinline__ void mma_s8_first(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1, const int (&c)[4])
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]), "r"(c[2]), "r"(c[3]));
 }
 
 template <typename T>
@@ -156,19 +194,19 @@ __device__ __forceinline__ void store_y(void *y, int yt, int64_t idx, float v)
 }
 
 // Turn x[m][128 q .. 128 q + 127] into the digit fragments of group q (all column sets) and
-// the column factors. One warp; lane (t, rho) builds register rho of quad-thread t.
+// the per-(token, group) factors 2^(e-27) (the 2^(8d) of digit d is applied per block).
+// One warp; lane (t, rho) builds register rho of quad-thread t. Token m owns the MMA columns
+// 4m .. 4m+3 (digits 0, 1, 2 and a zero column), so a quad-thread's two accumulator
+// columns always belong to one token.
 template <int FMT, int CS, typename XT>
 __device__ __forceinline__ void build_fragments(const XT *__restrict__ x, int M, int64_t K, int G, int q, int lane,
                                                 uint32_t *frag_s, float *colf_s)
 {
     const int t = lane >> 3, rho = lane & 7;
     uint32_t outw[CS * 8];
-    float fac[CS * 8];
 #pragma unroll
-    for (int c = 0; c < CS * 8; c++) {
+    for (int c = 0; c < CS * 8; c++)
         outw[c] = 0u;
-        fac[c] = 0.f;
-    }
     float v[8][4];
 #pragma unroll
     for (int m = 0; m < 8; m++)
@@ -176,6 +214,7 @@ __device__ __forceinline__ void build_fragments(const XT *__restrict__ x, int M,
 #pragma unroll
             for (int b = 0; b < 4; b++)
                 v[m][b] = load_x(x + (int64_t)m * K + 128 * q + k_local<FMT>(t, rho, b));
+    float fac = 0.f;                                 // lane m < 2 CS keeps token m's factor
 #pragma unroll
     for (int m = 0; m < 8; m++) {
         if (m >= M)
@@ -202,12 +241,12 @@ __device__ __forceinline__ void build_fragments(const XT *__restrict__ x, int M,
         }
 #pragma unroll
         for (int d = 0; d < kDigits; d++) {
-            const int c = m * kDigits + d;
-            if (c < CS * 8) {
+            const int c = m * kColsPerTok + d;
+            if (c < CS * 8)
                 outw[c] = dw[d];
-                fac[c] = amax > 0.f ? ldexpf(1.f, e - 27 + 8 * d) : 0.f;    // 2^(e-21+8d) / 64
-            }
         }
+        if (lane == m)
+            fac = amax > 0.f ? ldexpf(1.f, e - 27) : 0.f;                   // 2^(e-21) / 64
     }
     // fragment layout in shared memory: [cs][q][half][lane][4] u32, register rho = 4 half + r
 #pragma unroll
@@ -215,15 +254,15 @@ __device__ __forceinline__ void build_fragments(const XT *__restrict__ x, int M,
         const int cs = c >> 3, ln = 4 * (c & 7) + t;
         frag_s[(((cs * G + q) * 2 + (rho >> 2)) * 32 + ln) * 4 + (rho & 3)] = outw[c];
     }
-    if (lane < CS * 8)
-        colf_s[((lane >> 3) * G + q) * 8 + (lane & 7)] = fac[lane];
+    if (lane < 2 * CS)
+        colf_s[lane * G + q] = fac;                  // tokens past M get 0
 }
 
 template <int FMT, int CS, typename XT>
 __global__ void __launch_bounds__(kThreads, 1)
-gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
+gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restrict__ scales,
                const XT *__restrict__ x, int M, int64_t N, int64_t K, void *__restrict__ y, int yt,
-               float *__restrict__ part, unsigned long long *__restrict__ counters, int64_t U, int C, int maxseg,
+               float *__restrict__ part, unsigned long long *__restrict__ counters, int64_t U, int C,
                int stages, uint32_t call_id, uint32_t one, unsigned int *dev_status)
 {
     using SC = StageCfg<FMT>;
@@ -231,7 +270,8 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const Layout L = make_layout<FMT, CS>(G, stages);
     const int S = stages;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // align by an offset on the shared array itself, so every access stays a shared-memory one
+    uint8_t *smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint32_t *frag_s = reinterpret_cast<uint32_t *>(smem + L.frag_off);
     float *colf_s = reinterpret_cast<float *>(smem + L.colf_off);
     float *red = reinterpret_cast<float *>(smem + L.red_off);
@@ -259,20 +299,25 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         // ------------------------------------------------------------------- producer
         if (lane == 0) {
             ptx::tma_prefetch_desc(&tmap_w);
-            ptx::tma_prefetch_desc(&tmap_s);
             int64_t it = 0;
+            int s = 0;
+            uint32_t ph = 0;
+            int64_t rb = u0 / C;
+            int c = (int)(u0 % C);
             for (int64_t u = u0; u < u1; u++, it++) {
-                const int s = (int)(it % S);
-                const uint32_t ph = (uint32_t)((it / S) & 1);
                 if (!ptx::mbar_wait_bounded(&bars->empty[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
                     break;
-                const int64_t rb = u / C;
-                const int c = (int)(u % C);
                 uint8_t *st = smem + L.stage_off + s * SC::kBytes;
                 ptx::mbar_arrive_expect_tx(&bars->full[s], SC::kBytes);
-                ptx::tma_load_2d(st, &tmap_w, &bars->full[s], c * (FMT == BQ_BINARY_G128 ? 16 : 32),
-                                 (int32_t)(rb * kRows));
-                ptx::tma_load_2d(st + SC::kWordBytes, &tmap_s, &bars->full[s], (4 * c) & ~7, (int32_t)(rb * kRows));
+                ptx::tma_load_2d(st, &tmap_w, &bars->full[s], c * 32, (int32_t)(rb * kRows));
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1;
+                }
+                if (++c == C) {
+                    c = 0;
+                    rb++;
+                }
             }
             // no copy may still be in flight when the CTA exits
             for (int64_t k = it > S ? it - S : 0; k < it; k++) {
@@ -288,24 +333,65 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         {
             // digit fragments of the chunks this CTA touches (all of them if it owns >= C units)
             const int64_t span = u1 - u0 < C ? u1 - u0 : C;
-            const int nitems = (int)span * 4;
+            const int nitems = (int)span * SC::kGroups;
             for (int i = warp; i < nitems; i += kConsumers) {
-                const int c = (int)((u0 + i / 4) % C);
-                build_fragments<FMT, CS, XT>(x, M, K, G, 4 * c + (i & 3), lane, frag_s, colf_s);
+                const int c = (int)((u0 + i / SC::kGroups) % C);
+                build_fragments<FMT, CS, XT>(x, M, K, G, SC::kGroups * c + i % SC::kGroups, lane, frag_s, colf_s);
             }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");   // fragments ready
 
+        const int tile = warp & (kTiles - 1), half = warp / kTiles;   // this warp's share of the groups
         const int g8 = lane >> 2, t = lane & 3;
-        const int r0 = warp * 16 + g8, r1 = r0 + 8;          // rows of this thread in the block
-        uint32_t mul[8];
+        const int r0 = tile * 16 + g8, r1 = r0 + 8;          // rows of this thread in the block
+        uint32_t mul[9];                                  // runtime values: kept in registers
 #pragma unroll
-        for (int i = 0; i < 8; i++)
+        for (int i = 0; i < 7; i++)
             mul[i] = one << (7 - i);
-        float *wred = red + warp * (16 * CS * 8);            // [16 rows][CS*8 columns]
-        int64_t it = 0;
+        mul[7] = one * 0x80808080u;
+        mul[8] = one * 0x40404040u;
+        const int m0 = (int)(one - 1u) + kMagic;      // the accumulators start at 1.5 * 2^23 (as float bits)
+        const int magic[4] = {m0, m0, m0, m0};
+        // this warp takes groups [half GH, (half + 1) GH) of every stage, two at a time
+        constexpr int GH = SC::kGroups / kHalves;
+        // byte offsets of this thread's packed word(s) of each of those groups in rows r0 / r1
+        // (128-byte rows, 128B swizzle: 16-byte chunk j of row r sits at j ^ (r & 7))
+        int woff[GH][2];
+#pragma unroll
+        for (int h = 0; h < GH; h++) {
+            const int q = half * GH + h;
+            const int j = FMT == BQ_BINARY_G128 ? q : 2 * q + (t >> 1);          // 16-byte chunk
+            const int within = FMT == BQ_BINARY_G128 ? 4 * t : 8 * (t & 1);
+            woff[h][0] = r0 * 128 + ((j ^ (r0 & 7)) << 4) + within;
+            woff[h][1] = r1 * 128 + ((j ^ (r1 & 7)) << 4) + within;
+        }
+        // this thread's GH scales of rows r0 / r1 for unit (rb, c) (0 past row N); the loads
+        // are issued one stage before the scales are needed
+        auto load_scales = [&](int64_t rb_, int c_, uint32_t (&o0)[GH / 2], uint32_t (&o1)[GH / 2]) {
+            const int64_t n0 = rb_ * kRows + r0, n1 = n0 + 8;
+            const uint16_t *p0 = scales + (n0 < N ? n0 : 0) * G + c_ * SC::kGroups + half * GH;
+            const uint16_t *p1 = scales + (n1 < N ? n1 : 0) * G + c_ * SC::kGroups + half * GH;
+            if (GH == 8) {
+                const uint4 a = n0 < N ? __ldg(reinterpret_cast<const uint4 *>(p0)) : make_uint4(0, 0, 0, 0);
+                const uint4 b = n1 < N ? __ldg(reinterpret_cast<const uint4 *>(p1)) : make_uint4(0, 0, 0, 0);
+                o0[0] = a.x; o0[1 % (GH / 2)] = a.y; o0[2 % (GH / 2)] = a.z; o0[3 % (GH / 2)] = a.w;
+                o1[0] = b.x; o1[1 % (GH / 2)] = b.y; o1[2 % (GH / 2)] = b.z; o1[3 % (GH / 2)] = b.w;
+            } else if (GH == 4) {
+                const uint2 a = n0 < N ? __ldg(reinterpret_cast<const uint2 *>(p0)) : make_uint2(0, 0);
+                const uint2 b = n1 < N ? __ldg(reinterpret_cast<const uint2 *>(p1)) : make_uint2(0, 0);
+                o0[0] = a.x; o0[GH / 2 - 1] = a.y;
+                o1[0] = b.x; o1[GH / 2 - 1] = b.y;
+            } else {
+                o0[0] = n0 < N ? __ldg(reinterpret_cast<const uint32_t *>(p0)) : 0u;
+                o1[0] = n1 < N ? __ldg(reinterpret_cast<const uint32_t *>(p1)) : 0u;
+            }
+        };
+        uint32_t nx0[GH / 2], nx1[GH / 2];
+        load_scales(u0 / C, (int)(u0 % C), nx0, nx1);
+        int s = 0;
+        uint32_t ph = 0;
         bool ok = true;
-        for (int64_t rb = u0 / C; ok && rb * C < u1; rb++) {
+        for (int64_t rb = u0 / C; rb * C < u1; rb++) {
             const int c_lo = (int)(rb == u0 / C ? u0 % C : 0);
             const int c_hi = (int)((rb + 1) * C <= u1 ? C : u1 - rb * C);
             float acc[CS][4];
@@ -314,98 +400,147 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < 4; i++)
                     acc[cs][i] = 0.f;
-            for (int c = c_lo; c < c_hi; c++, it++) {
-                const int s = (int)(it % S);
-                const uint32_t ph = (uint32_t)((it / S) & 1);
-                if (!warp_wait(&bars->full[s], ph, abort, err)) {
-                    ok = false;
-                    break;
+            for (int c = c_lo; ok && c < c_hi; c++) {
+                // this stage's scales were loaded one stage ago; start the next stage's now
+                uint32_t sw0[GH / 2], sw1[GH / 2];
+#pragma unroll
+                for (int i = 0; i < GH / 2; i++) {
+                    sw0[i] = nx0[i];
+                    sw1[i] = nx1[i];
                 }
+                if (c + 1 < c_hi)
+                    load_scales(rb, c + 1, nx0, nx1);
+                else if ((rb + 1) * C < u1)
+                    load_scales(rb + 1, 0, nx0, nx1);
+                // every lane observes the stage's phase itself; the verdict is made warp-uniform
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&bars->full[s], ph, abort, err,
+                                                                    kDevErrTimeout, kWaitLimitNs));
+                if (!ok)
+                    break;                          // still meet the partner warp below
                 const uint8_t *st = smem + L.stage_off + s * SC::kBytes;
-                const uint16_t *sc = reinterpret_cast<const uint16_t *>(st + SC::kWordBytes);
-                const int soff = (4 * c) & 7;
+                constexpr int GP = GH < kGP ? GH : kGP;
 #pragma unroll
-                for (int qp = 0; qp < 4; qp += 2) {         // two groups at a time: independent chains
-                    uint32_t A[2][2][8];                    // [group][row r0/r1][register]
+                for (int h0 = 0; h0 < GH; h0 += GP) {          // GP groups at a time
+                    uint32_t A[GP][4][4];                       // [group][mma][a0..a3]
 #pragma unroll
-                    for (int h = 0; h < 2; h++) {
-                        const int q = qp + h;
-                        if (FMT == BQ_BINARY_G128) {
-                            const int ch0 = q ^ ((r0 >> 1) & 3), ch1 = q ^ ((r1 >> 1) & 3);
-                            const uint32_t w0 = *reinterpret_cast<const uint32_t *>(st + r0 * 64 + ch0 * 16 + 4 * t);
-                            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(st + r1 * 64 + ch1 * 16 + 4 * t);
-                            expand_binary(w0, mul, A[h][0]);
-                            expand_binary(w1, mul, A[h][1]);
-                        } else {
-                            const int c16 = 2 * q + (t >> 1);
-                            const uint2 w0 = *reinterpret_cast<const uint2 *>(st + r0 * 128 + ((c16 ^ (r0 & 7)) << 4) + 8 * (t & 1));
-                            const uint2 w1 = *reinterpret_cast<const uint2 *>(st + r1 * 128 + ((c16 ^ (r1 & 7)) << 4) + 8 * (t & 1));
-                            expand_ternary(w0.x, A[h][0]);
-                            expand_ternary(w0.y, A[h][0] + 4);
-                            expand_ternary(w1.x, A[h][1]);
-                            expand_ternary(w1.y, A[h][1] + 4);
-                        }
+                    for (int h = 0; h < GP; h++)
+                        expand_group<FMT>(st + woff[h0 + h][0], st + woff[h0 + h][1], mul, A[h]);
+                    if (h0 + GP == GH) {
+                        __syncwarp();
+                        if (lane == 0)
+                            ptx::mbar_arrive(&bars->empty[s]);  // the stage's words are in registers
                     }
 #pragma unroll
-                    for (int h = 0; h < 2; h++) {
-                        const int q = qp + h;
-                        const int gq = 4 * c + q;          // group index within K
-                        const float s0 = __half2float(__ushort_as_half(sc[r0 * 8 + soff + q]));
-                        const float s1 = __half2float(__ushort_as_half(sc[r1 * 8 + soff + q]));
+                    for (int cs = 0; cs < CS; cs++) {
+                        int d[GP][4];
 #pragma unroll
-                        for (int cs = 0; cs < CS; cs++) {
+                        for (int h = 0; h < GP; h++) {          // GP independent chains
+                            const int gq = SC::kGroups * c + half * GH + h0 + h;
                             const uint4 bA = *reinterpret_cast<const uint4 *>(frag_s + (((cs * G + gq) * 2 + 0) * 32 + lane) * 4);
                             const uint4 bB = *reinterpret_cast<const uint4 *>(frag_s + (((cs * G + gq) * 2 + 1) * 32 + lane) * 4);
-                            const uint32_t b[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
-                            int de[4] = {0, 0, 0, 0}, dd[4] = {0, 0, 0, 0};   // two independent chains
-                            mma_s8(de, A[h][0][0], A[h][1][0], A[h][0][1], A[h][1][1], b[0], b[1]);
-                            mma_s8(dd, A[h][0][2], A[h][1][2], A[h][0][3], A[h][1][3], b[2], b[3]);
-                            mma_s8(de, A[h][0][4], A[h][1][4], A[h][0][5], A[h][1][5], b[4], b[5]);
-                            mma_s8(dd, A[h][0][6], A[h][1][6], A[h][0][7], A[h][1][7], b[6], b[7]);
-                            const float2 f = *reinterpret_cast<const float2 *>(colf_s + (cs * G + gq) * 8 + 2 * t);
-                            // (r0, col 2t) (r0, 2t+1) (r1, 2t) (r1, 2t+1)
-                            acc[cs][0] = fmaf((float)(de[0] + dd[0]), s0 * f.x, acc[cs][0]);
-                            acc[cs][1] = fmaf((float)(de[1] + dd[1]), s0 * f.y, acc[cs][1]);
-                            acc[cs][2] = fmaf((float)(de[2] + dd[2]), s1 * f.x, acc[cs][2]);
-                            acc[cs][3] = fmaf((float)(de[3] + dd[3]), s1 * f.y, acc[cs][3]);
+                            mma_s8_first(d[h], A[h][0][0], A[h][0][1], A[h][0][2], A[h][0][3], bA.x, bA.y, magic);
+                            mma_s8(d[h], A[h][1][0], A[h][1][1], A[h][1][2], A[h][1][3], bA.z, bA.w);
+                            mma_s8(d[h], A[h][2][0], A[h][2][1], A[h][2][2], A[h][2][3], bB.x, bB.y);
+                            mma_s8(d[h], A[h][3][0], A[h][3][1], A[h][3][2], A[h][3][3], bB.z, bB.w);
+                        }
+#pragma unroll
+                        for (int h = 0; h < GP; h++) {
+                            const int gq = SC::kGroups * c + half * GH + h0 + h;
+                            const __half2 p0 = *reinterpret_cast<const __half2 *>(&sw0[(h0 + h) >> 1]);
+                            const __half2 p1 = *reinterpret_cast<const __half2 *>(&sw1[(h0 + h) >> 1]);
+                            // 2^(e-27) of this quad-thread's token (2 cs + t/2) in group gq, times the scales
+                            const float f = colf_s[(2 * cs + (t >> 1)) * G + gq];
+                            const float sf0 = ((h & 1) ? __high2float(p0) : __low2float(p0)) * f;
+                            const float sf1 = ((h & 1) ? __high2float(p1) : __low2float(p1)) * f;
+                            // exact int -> float: the accumulator started at the bits of 1.5 * 2^23
+                            const float t0 = __int_as_float(d[h][0]) - 12582912.f;
+                            const float t1 = __int_as_float(d[h][1]) - 12582912.f;
+                            const float t2 = __int_as_float(d[h][2]) - 12582912.f;
+                            const float t3 = __int_as_float(d[h][3]) - 12582912.f;
+                            // (r0, col 2t) (r0, 2t+1) (r1, 2t) (r1, 2t+1): columns 2t, 2t+1 are digits of one token
+                            acc[cs][0] = fmaf(t0, sf0, acc[cs][0]);
+                            acc[cs][1] = fmaf(t1, sf0, acc[cs][1]);
+                            acc[cs][2] = fmaf(t2, sf1, acc[cs][2]);
+                            acc[cs][3] = fmaf(t3, sf1, acc[cs][3]);
                         }
                     }
                 }
-                __syncwarp();
-                if (lane == 0)
-                    ptx::mbar_arrive(&bars->empty[s]);
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1;
+                }
             }
-            if (!ok)
-                break;
 
-            // ---- digits of a token: y[row][m] = sum_d acc[row][3m + d]
+            // ---- the two warps of a tile meet: half 1 hands its sums to half 0 through a slot
+            // (barrier 1: written; barrier 2: read), then half 0 adds the digits and writes.
+            float *slot = red + (tile * 16) * (CS * 8);   // [16 rows][CS*8]
+            if (kHalves == 1) {
 #pragma unroll
-            for (int cs = 0; cs < CS; cs++) {
-                wred[g8 * (CS * 8) + cs * 8 + 2 * t] = acc[cs][0];
-                wred[g8 * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][1];
-                wred[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t] = acc[cs][2];
-                wred[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][3];
+                for (int cs = 0; cs < CS; cs++) {
+                    slot[g8 * (CS * 8) + cs * 8 + 2 * t] = acc[cs][0];
+                    slot[g8 * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][1];
+                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t] = acc[cs][2];
+                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][3];
+                }
+                __syncwarp();
+                if (!ok || *abort)
+                    break;
+            } else if (half == 1) {
+#pragma unroll
+                for (int cs = 0; cs < CS; cs++) {
+                    slot[g8 * (CS * 8) + cs * 8 + 2 * t] = acc[cs][0];
+                    slot[g8 * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][1];
+                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t] = acc[cs][2];
+                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][3];
+                }
             }
-            __syncwarp();
-            const int64_t row0 = rb * kRows + warp * 16;
+            if (kHalves == 2)
+                asm volatile("bar.sync %0, 64;" ::"r"(2 + tile) : "memory");   // id 1 is the prologue barrier
+            if (!ok || *abort)
+                break;                                      // both warps of the tile stop here
+            if (kHalves == 2 && half == 0) {
+#pragma unroll
+                for (int cs = 0; cs < CS; cs++) {
+                    slot[g8 * (CS * 8) + cs * 8 + 2 * t] += acc[cs][0];
+                    slot[g8 * (CS * 8) + cs * 8 + 2 * t + 1] += acc[cs][1];
+                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t] += acc[cs][2];
+                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t + 1] += acc[cs][3];
+                }
+                __syncwarp();
+            }
+            float fin[16];                                  // half 0: the tile's (row, token) sums
+            for (int e = lane, i = 0; e < 16 * M; e += 32, i++) {
+                const int rr = e / M, m = e % M;
+                float v = 0.f;
+#pragma unroll
+                for (int dg = kDigits - 1; dg >= 0; dg--)                    // digit d weighs 256^d
+                    v = fmaf(v, 256.f, slot[rr * (CS * 8) + m * kColsPerTok + dg]);
+                fin[i] = v;
+            }
+            if (kHalves == 2) {
+                asm volatile("bar.sync %0, 64;" ::"r"(2 + tile) : "memory");   // the slot is free again
+                if (half == 1)
+                    continue;
+            }
+            const int64_t row0 = rb * kRows + tile * 16;
             const bool whole = c_lo == 0 && c_hi == C;
             const int64_t x0 = rb * C, x1 = rb * C + C;     // owners of the block's first/last unit
             const int64_t i_first = (x0 + 1) * Pn / U + (((x0 + 1) * Pn) % U != 0) - 1;
             const int64_t i_last = x1 * Pn / U + ((x1 * Pn) % U != 0) - 1;
             const int nseg = (int)(i_last - i_first + 1);
-            const int seg = (int)(blockIdx.x - i_first);
-            for (int e = lane; e < 16 * M; e += 32) {
+            // a split block is the first (slot 0) or the last (slot 1) block of each CTA that
+            // shares it; only its first owner can hold it in slot 1, and a CTA is the first
+            // owner of at most one split block, so the counter is indexed by that owner
+            const int end = rb == u0 / C ? 0 : 1;
+            for (int e = lane, i = 0; e < 16 * M; e += 32, i++) {
                 const int rr = e / M, m = e % M;
-                float v = 0.f;
-#pragma unroll
-                for (int d = 0; d < kDigits; d++)
-                    v += wred[rr * (CS * 8) + m * kDigits + d];
+                const float v = fin[i];
                 const int64_t n = row0 + rr;
                 if (whole) {
                     if (n < N)
                         store_y<float>(y, yt, (int64_t)m * N + n, v);
                 } else {
-                    part[((rb * maxseg + seg) * kRows + warp * 16 + rr) * M + m] = v;
+                    part[(((int64_t)blockIdx.x * 2 + end) * kRows + tile * 16 + rr) * M + m] = v;
                 }
             }
             __syncwarp();
@@ -416,7 +551,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                 __syncwarp();
                 int last = 0;
                 if (lane == 0) {
-                    unsigned long long *ctr = counters + rb * kConsumers + warp;
+                    unsigned long long *ctr = counters + i_first * kTiles + tile;
                     const unsigned long long tag = (unsigned long long)call_id << 32;
                     unsigned long long cur = atomicAdd(ctr, 0ull);
                     for (int tries = 0; tries < (1 << 20); tries++) {
@@ -437,8 +572,11 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                     for (int e = lane; e < 16 * M; e += 32) {
                         const int rr = e / M, m = e % M;
                         float v = 0.f;
-                        for (int sg = 0; sg < nseg; sg++)           // fixed order: deterministic
-                            v += __ldcg(part + ((rb * maxseg + sg) * kRows + warp * 16 + rr) * M + m);
+                        for (int sg = 0; sg < nseg; sg++) {         // fixed order: deterministic
+                            const int64_t i = i_first + sg;
+                            const int slot_i = sg == 0 && i * U / Pn != x0 ? 1 : 0;
+                            v += __ldcg(part + ((i * 2 + slot_i) * kRows + tile * 16 + rr) * M + m);
+                        }
                         const int64_t n = row0 + rr;
                         if (n < N)
                             store_y<float>(y, yt, (int64_t)m * N + n, v);
@@ -481,9 +619,8 @@ int sm_count()
 }
 
 struct Plan {
-    int CS, stages, grid, maxseg;
+    int CS, stages, grid;
     int64_t NB, C, U;
-    int smem;
     size_t part_bytes, counter_bytes;
 };
 
@@ -500,31 +637,27 @@ int stages_for(int fmt, int CS, int G)
 {
     if (fmt == BQ_BINARY_G128)
         return CS == 1 ? plan_stages<BQ_BINARY_G128, 1>(G) : CS == 2 ? plan_stages<BQ_BINARY_G128, 2>(G)
-                                                                     : plan_stages<BQ_BINARY_G128, 3>(G);
+             : CS == 3 ? plan_stages<BQ_BINARY_G128, 3>(G) : plan_stages<BQ_BINARY_G128, 4>(G);
     return CS == 1 ? plan_stages<BQ_TERNARY_G128, 1>(G) : CS == 2 ? plan_stages<BQ_TERNARY_G128, 2>(G)
-                                                                  : plan_stages<BQ_TERNARY_G128, 3>(G);
+         : CS == 3 ? plan_stages<BQ_TERNARY_G128, 3>(G) : plan_stages<BQ_TERNARY_G128, 4>(G);
 }
 
 Plan make_plan(int M, int fmt, int64_t N, int64_t K)
 {
     Plan p;
-    p.CS = (M * kDigits + 7) / 8;
+    p.CS = (M * kColsPerTok + 7) / 8;
     const int G = (int)(K / 128);
     p.stages = stages_for(fmt, p.CS, G);
     p.NB = (N + kRows - 1) / kRows;
-    p.C = K / kChunkK;
+    p.C = K / (fmt == BQ_BINARY_G128 ? 1024 : 512);
     p.U = p.NB * p.C;
     const int64_t sms = sm_count();
     p.grid = (int)(p.U < sms ? p.U : sms);
-    const int64_t per = p.U / p.grid;                 // every CTA owns at least `per` units
-    p.maxseg = (int)((p.C + per - 1) / per + 1);
-    if (p.maxseg > p.grid)
-        p.maxseg = p.grid;
+    // partial sums: two 128-row slots per CTA (its first and last block, the only ones it
+    // may share); one counter per tile of the split block each CTA opens
     auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
-    p.part_bytes = al((size_t)p.NB * p.maxseg * kRows * M * 4);
-    p.counter_bytes = al((size_t)p.NB * kConsumers * 8);
-    if (p.stages)
-        p.smem = fmt == BQ_BINARY_G128 ? 0 : 0;      // filled by the launcher
+    p.part_bytes = al((size_t)p.grid * 2 * kRows * M * 4);
+    p.counter_bytes = al((size_t)p.grid * kTiles * 8);
     return p;
 }
 
@@ -545,28 +678,18 @@ cudaError_t launch_tc_t(const GemvArgs &a, const Plan &pl, cudaStream_t s)
     float *part = reinterpret_cast<float *>(ws);
     unsigned long long *counters = reinterpret_cast<unsigned long long *>(ws + pl.part_bytes);
 
-    CUtensorMap mw, ms;
+    CUtensorMap mw;
     const cuuint64_t wpr = (cuuint64_t)(FMT == BQ_BINARY_G128 ? a.K / 32 : a.K / 16);
     cuuint64_t wdims[2] = {wpr, (cuuint64_t)a.N};
     cuuint64_t wstr[1] = {wpr * 4};
-    cuuint32_t wbox[2] = {(cuuint32_t)(FMT == BQ_BINARY_G128 ? 16 : 32), (cuuint32_t)kRows};
+    cuuint32_t wbox[2] = {32, (cuuint32_t)kRows};        // 128 bytes x 128 rows
     cuuint32_t est[2] = {1, 1};
     CUresult r = enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(a.words), wdims, wstr, wbox, est,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     FMT == BQ_BINARY_G128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     const cuuint64_t G = (cuuint64_t)(a.K / 128);
-    cuuint64_t sdims[2] = {G, (cuuint64_t)a.N};
-    cuuint64_t sstr[1] = {G * 2};
-    cuuint32_t sbox[2] = {8, (cuuint32_t)kRows};
-    r = enc(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<__half *>(a.scales), sdims, sstr, sbox, est,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
-
     const int smem = make_layout<FMT, CS>((int)G, pl.stages).total;
     auto kern = gemv_tc_kernel<FMT, CS, XT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -582,8 +705,8 @@ cudaError_t launch_tc_t(const GemvArgs &a, const Plan &pl, cudaStream_t s)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mw, ms, static_cast<const XT *>(a.x), a.M, a.N, a.K, a.y, a.yt, part,
-                              counters, pl.U, (int)pl.C, pl.maxseg, pl.stages, next_call_id(), 1u, a.dev_status);
+    return cudaLaunchKernelEx(&cfg, kern, mw, reinterpret_cast<const uint16_t *>(a.scales), static_cast<const XT *>(a.x), a.M, a.N, a.K, a.y, a.yt, part,
+                              counters, pl.U, (int)pl.C, pl.stages, next_call_id(), 1u, a.dev_status);
 }
 
 template <int FMT, typename XT>
@@ -592,7 +715,8 @@ cudaError_t launch_tc_cs(const GemvArgs &a, const Plan &pl, cudaStream_t s)
     switch (pl.CS) {
     case 1: return launch_tc_t<FMT, 1, XT>(a, pl, s);
     case 2: return launch_tc_t<FMT, 2, XT>(a, pl, s);
-    default: return launch_tc_t<FMT, 3, XT>(a, pl, s);
+    case 3: return launch_tc_t<FMT, 3, XT>(a, pl, s);
+    default: return launch_tc_t<FMT, 4, XT>(a, pl, s);
     }
 }
 
@@ -604,7 +728,7 @@ bool gemv_tc_supported(int M, int fmt, int64_t K)
 {
     if (M < 1 || M > 8 || K % 1024 != 0)
         return false;
-    return stages_for(fmt, (M * kDigits + 7) / 8, (int)(K / 128)) >= 2;
+    return stages_for(fmt, (M * kColsPerTok + 7) / 8, (int)(K / 128)) >= 2;
 }
 
 size_t gemv_tc_workspace_bytes(int M, int fmt, int64_t N, int64_t K)

@@ -54,6 +54,13 @@ def test_binary_k5120_n20480_sampled(orc, M):
     run_binary(orc, 0, 20480, 5120, M, rows=sample_rows(20480, 1500, M))
 
 
+@pytest.mark.parametrize("N,K", [(9120, 5120), (40960, 5120), (5120, 20480)])
+def test_full_depth_block_shapes_sampled(orc, N, K):
+    """The shapes of one block of the full-depth decode step (attention in, MLP gate/up,
+    MLP down; attention out is the 5120 x 5120 case above), M=1, as the step launches them."""
+    run_binary(orc, 64, N, K, 1, rows=sample_rows(N, 800, 1))
+
+
 def test_binary_lm_head_sampled(orc):
     """LM head: M=1, K=5120, N=248320 (~159 MB packed + ~20 MB scales)."""
     run_binary(orc, 0, 248320, 5120, 1, rows=sample_rows(248320, 1500))
