@@ -144,6 +144,30 @@ bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w,
 size_t bq_gemv_workspace_bytes(int64_t M, const bq_weight *w);
 
 /*
+ * bq_gemv without a workspace argument: the same product, same kernels, same arguments and
+ * results, with the scratch taken from a fixed array inside the library. It allocates no
+ * device memory. The model card and the Ternary Bonsai article have no counterpart: this
+ * call exists for callers that cannot allocate device memory per call, or do not want to:
+ *   - code that already handed all free device memory to its own pools (weights, KV cache)
+ *     and has no allocator to draw a workspace from;
+ *   - a decode loop that must not call cudaMalloc or cudaFree between steps, since those
+ *     calls can synchronise the device and stall the queued work;
+ *   - plain C hosts that do not want to size, own and free a buffer per weight shape.
+ * Limit: the array is 1.26 MiB per device, enough for every M <= 8 on a device with up to
+ * 160 SMs; a shape that needs more returns BQ_ERR_WORKSPACE with the two sizes in
+ * bq_last_error(), and bq_gemv with a workspace then serves it.
+ * Set-up: the first call on each device (with that device current) resolves the array's
+ * address; make that first call before any stream capture. Later calls do no set-up.
+ * Sharing: all calls on a device share the one array. Its counters start at zero and every
+ * call leaves them at zero; the partial sums need no initial value. Calls that may overlap
+ * on the device (different streams, several host threads) race on the array and give wrong
+ * results: order them on one stream, or use bq_gemv with a workspace per stream.
+ * Errors: as bq_gemv, plus BQ_ERR_WORKSPACE for the limit above.
+ */
+bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight *w,
+                          void *y, bq_dtype yt, cudaStream_t stream);
+
+/*
  * Prefill GEMM: the same product for M up to 512 token rows (larger M is accepted),
  * Y[M][N] = X[M][K] * W^T with W the dequantised +-s (binary) or {-s, 0, +s} (ternary)
  * matrix. The packed tiles are unpacked into shared memory next to the tensor cores

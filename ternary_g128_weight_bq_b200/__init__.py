@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "bq_unpack_g128": ([W, P, P, P], I),
             "bq_gemv": ([P, I, I64, W, P, I, P, ctypes.c_size_t, P], I),
             "bq_gemv_workspace_bytes": ([I64, W], ctypes.c_size_t),
+            "bq_gemv_noalloc": ([P, I, I64, W, P, I, P], I),
             "bq_gemm_prefill": ([P, I, I64, W, P, I, P, ctypes.c_size_t, P], I),
             "bq_gemm_prefill_workspace_bytes": ([I64, W], ctypes.c_size_t),
             "bq_embed_gather": ([P, I64, W, P, I, P], I),
@@ -197,6 +198,22 @@ def gemv(x: torch.Tensor, w: BQWeight, out_dtype=torch.float32, out: torch.Tenso
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().bq_gemv(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(), _DTYPE[out.dtype],
                          ws_ptr, ws_bytes, _stream(x.device)))
+    return out
+
+
+def gemv_noalloc(x: torch.Tensor, w: BQWeight, out_dtype=torch.float32,
+                 out: torch.Tensor = None) -> torch.Tensor:
+    """gemv with the library's fixed scratch array instead of a workspace (no device
+    allocation inside the call; calls on one device must not overlap)."""
+    _dev(x, "x")
+    if x.dim() != 2 or x.shape[1] != w.K:
+        raise ValueError(f"x must be [M, {w.K}]")
+    M = x.shape[0]
+    if out is None:
+        out = torch.empty((M, w.N), dtype=out_dtype, device=x.device)
+    _dev(out, "out")
+    _check(lib().bq_gemv_noalloc(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(),
+                                 _DTYPE[out.dtype], _stream(x.device)))
     return out
 
 

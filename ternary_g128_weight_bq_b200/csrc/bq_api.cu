@@ -260,6 +260,43 @@ bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, voi
     return BQ_OK;
 }
 
+bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, void *y,
+                          bq_dtype yt, cudaStream_t stream)
+{
+    bq_status st = validate_weight(w);
+    if (st != BQ_OK)
+        return st;
+    if ((st = validate_xy("gemv_noalloc", x, xt, y, yt)) != BQ_OK)
+        return st;
+    if (M < 1 || M > 8)
+        return set_error(BQ_ERR_SHAPE, "gemv_noalloc: M=%lld, need 1 <= M <= 8", (long long)M);
+    unsigned int *status = device_status(&st);
+    if (!status)
+        return st;
+    const size_t need = gemv_workspace_bytes((int)M, w->fmt, w->N, w->K);
+    void *scratch = nullptr;
+    size_t cap = 0;
+    if (need) {
+        cudaError_t e = gemv_static_scratch(&scratch, &cap);
+        if (e != cudaSuccess)
+            return set_error(BQ_ERR_CUDA, "gemv_noalloc: cudaGetSymbolAddress of the scratch array: %s",
+                             cudaGetErrorString(e));
+        if (need > cap)
+            return set_error(BQ_ERR_WORKSPACE,
+                             "gemv_noalloc: this shape on this device needs %zu bytes of scratch, more than "
+                             "the %zu bytes of the library's fixed array; call bq_gemv with a workspace",
+                             need, cap);
+    }
+    GemvArgs a{x, (int)xt, (int)M, (int)w->fmt, w->N, w->K, w->words,
+               reinterpret_cast<const __half *>(w->scales), y, (int)yt, scratch, cap, status};
+    unsigned launches = 0;
+    cudaError_t e = launch_gemv(a, stream, &launches);
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "gemv_noalloc launch: %s", cudaGetErrorString(e));
+    note_launches(launches);
+    return BQ_OK;
+}
+
 size_t bq_gemm_prefill_workspace_bytes(int64_t M, const bq_weight *w)
 {
     if (!w || M < 1 || w->N < 1 || w->K < 128 || w->K % 128)

@@ -59,6 +59,9 @@ bool gemv_tc_supported(int M, int fmt, int64_t K);
 size_t gemv_tc_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
 cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s);
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches);
+// Device address and size of the fixed scratch array of bq_gemv_noalloc on the current
+// device (gemv_tc.cu); resolved once per device.
+cudaError_t gemv_static_scratch(void **ptr, size_t *bytes);
 
 struct PrefillArgs {
     const void *x;

@@ -40,6 +40,8 @@
 //     zero-filled workspace) adds them in a fixed order.
 #include <cuda.h>
 
+#include <mutex>
+
 #include "bq_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -745,6 +747,45 @@ cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s)
                               : launch_tc_cs<BQ_BINARY_G128, __nv_bfloat16>(a, pl, s);
     return a.xt == BQ_F16 ? launch_tc_cs<BQ_TERNARY_G128, __half>(a, pl, s)
                           : launch_tc_cs<BQ_TERNARY_G128, __nv_bfloat16>(a, pl, s);
+}
+
+// ---------------------------------------------------------------------------------------
+// fixed scratch of bq_gemv_noalloc
+// ---------------------------------------------------------------------------------------
+// The workspace this kernel needs is at most two 128-row slots of M <= 8 fp32 partial sums
+// per CTA plus one counter per 16-row tile per CTA, and the grid is at most one CTA per SM.
+// This array holds that for grids of up to kStaticMaxCtas CTAs (1.26 MiB). Static device
+// storage starts zeroed; the counters are the only part that must, and every call returns
+// each counter it used to zero (a call cut short by a timeout may leave one tagged with its
+// own call id, which later calls treat as zero).
+constexpr int kStaticMaxCtas = 160;
+constexpr size_t kStaticPartBytes = (size_t)kStaticMaxCtas * 2 * kRows * 8 * sizeof(float);
+constexpr size_t kStaticCounterBytes = ((size_t)kStaticMaxCtas * kTiles * 8 + 255) & ~size_t(255);
+static __device__ __align__(256) unsigned char g_gemv_scratch[kStaticPartBytes + kStaticCounterBytes];
+
+cudaError_t gemv_static_scratch(void **ptr, size_t *bytes)
+{
+    constexpr int kMaxDev = 64;
+    static std::mutex mu;
+    static void *addr[kMaxDev] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        // first use on this device (the device is current): resolve the array's address
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_gemv_scratch);
+        if (e != cudaSuccess)
+            return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    *bytes = sizeof(g_gemv_scratch);
+    return cudaSuccess;
 }
 
 }  // namespace bq
