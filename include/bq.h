@@ -153,13 +153,13 @@ size_t bq_gemv_workspace_bytes(int64_t M, const bq_weight *w);
  *   - a decode loop that must not call cudaMalloc or cudaFree between steps, since those
  *     calls can synchronise the device and stall the queued work;
  *   - plain C hosts that do not want to size, own and free a buffer per weight shape.
- * Limit: the array is 1.26 MiB per device, enough for every M <= 8 on a device with up to
- * 160 SMs; a shape that needs more returns BQ_ERR_WORKSPACE with the two sizes in
+ * Limit: the array is 1.55 MiB per device, enough for every M <= 8 and every K on a device
+ * with up to 160 SMs; a shape that needs more returns BQ_ERR_WORKSPACE with the two sizes in
  * bq_last_error(), and bq_gemv with a workspace then serves it.
  * Set-up: the first call on each device (with that device current) resolves the array's
  * address; make that first call before any stream capture. Later calls do no set-up.
- * Sharing: all calls on a device share the one array. Its counters start at zero and every
- * call leaves them at zero; the partial sums need no initial value. Calls that may overlap
+ * Sharing: all calls on a device share the one array. Nothing in it needs an initial value
+ * (each call zeroes the counters it uses before using them). Calls that may overlap
  * on the device (different streams, several host threads) race on the array and give wrong
  * results: order them on one stream, or use bq_gemv with a workspace per stream.
  * Errors: as bq_gemv, plus BQ_ERR_WORKSPACE for the limit above.

@@ -181,9 +181,11 @@ size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
 // tensor-core kernel; otherwise the SIMT kernel. One launch either way.
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches)
 {
-    *launches = 1;
-    if (gemv_tc_supported(a.M, a.fmt, a.K))
+    if (gemv_tc_supported(a.M, a.fmt, a.K)) {
+        *launches = 2;                               // fragment prep + the GEMV
         return launch_gemv_tc(a, s);
+    }
+    *launches = 1;
     return launch_gemv_simt(a, s);
 }
 

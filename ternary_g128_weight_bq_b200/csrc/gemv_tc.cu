@@ -23,10 +23,12 @@
 // fp32 subtraction turns it into a float without rounding); the group scale times 2^(e-27) is
 // applied once per group in fp32, and the digit weight 256^d once per block.
 //
-// One kernel per call (programmatic dependent launch):
-//   * prologue: the CTA's consumer warps turn x into MMA B fragments (digits) for the k-chunks
-//     the CTA will touch, straight into shared memory, while the producer already streams the
-//     first weight tiles;
+// Two kernels per call, both with programmatic dependent launch:
+//   * a prep kernel turns x into the MMA B fragments (digits) and per-(token, group) factors
+//     once, one warp per (group, token slot), and zeroes the split-block counters; every CTA
+//     of the GEMV then bulk-copies the fragments of the k-chunks it touches into shared memory
+//     (building them in each CTA cost up to 25 us at M = 8, all of it after the previous
+//     kernel had finished), while its producer already streams the first weight tiles;
 //   * units = (block of 128 rows, one stage of k); CTA i owns units [i U / P, (i+1) U / P)
 //     (stream-K), so every shape is balanced to one unit;
 //   * the producer lane TMA-loads, per unit, a 128 rows x 128 bytes tile of packed words (1024
@@ -36,8 +38,8 @@
 //     group scales come straight from global memory, each stage's loaded one stage early;
 //   * a block owned by one CTA is written directly; a block split between CTAs leaves partial
 //     sums in the workspace (two 128-row slots per CTA: its first and its last block), and the
-//     last warp to finish its 16 rows (a counter tagged with the call id, so it needs no
-//     zero-filled workspace) adds them in a fixed order.
+//     last warp to finish its 16 rows (one atomic on a counter the prep kernel zeroed) adds
+//     them in a fixed order.
 #include <cuda.h>
 
 #include <mutex>
@@ -104,6 +106,7 @@ __host__ __device__ inline Layout make_layout(int G, int stages)
 struct Bars {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
+    uint64_t frag;                    // the digit fragments and factors have landed
     int abort;
 };
 
@@ -195,33 +198,24 @@ __device__ __forceinline__ void store_y(void *y, int yt, int64_t idx, float v)
         store_out(static_cast<__half *>(y) + idx, v);
 }
 
-// Turn x[m][128 q .. 128 q + 127] into the digit fragments of group q (all column sets) and
-// the per-(token, group) factors 2^(e-27) (the 2^(8d) of digit d is applied per block).
-// One warp; lane (t, rho) builds register rho of quad-thread t. Token m owns the MMA columns
-// 4m .. 4m+3 (digits 0, 1, 2 and a zero column), so a quad-thread's two accumulator
-// columns always belong to one token.
-template <int FMT, int CS, typename XT>
-__device__ __forceinline__ void build_fragments(const XT *__restrict__ x, int M, int64_t K, int G, int q, int lane,
-                                                uint32_t *frag_s, float *colf_s)
+// Digit fragments of token slot m (MMA columns 4m .. 4m+3: digits 0, 1, 2 and a zero column)
+// in group q, and the token's factor 2^(e-27) (the 2^(8d) of digit d is applied per block),
+// written with the shared-memory layout [cs][q][half][lane][4] u32 / [slot][G] f32. One warp;
+// lane (t, rho) builds register rho of quad-thread t. Slots m >= M (the padding of the last
+// column set) get zeros, so a quad-thread's two accumulator columns always belong to one token.
+template <int FMT, typename XT>
+__device__ __forceinline__ void build_token(const XT *__restrict__ x, int M, int64_t K, int G, int q, int m,
+                                            int lane, uint32_t *__restrict__ frag, float *__restrict__ colf)
 {
     const int t = lane >> 3, rho = lane & 7;
-    uint32_t outw[CS * 8];
+    uint32_t dw[kDigits] = {0u, 0u, 0u};
+    float fac = 0.f;
+    if (m < M) {
+        float v[4];
 #pragma unroll
-    for (int c = 0; c < CS * 8; c++)
-        outw[c] = 0u;
-    float v[8][4];
-#pragma unroll
-    for (int m = 0; m < 8; m++)
-        if (m < M)
-#pragma unroll
-            for (int b = 0; b < 4; b++)
-                v[m][b] = load_x(x + (int64_t)m * K + 128 * q + k_local<FMT>(t, rho, b));
-    float fac = 0.f;                                 // lane m < 2 CS keeps token m's factor
-#pragma unroll
-    for (int m = 0; m < 8; m++) {
-        if (m >= M)
-            break;
-        float amax = fmaxf(fmaxf(fabsf(v[m][0]), fabsf(v[m][1])), fmaxf(fabsf(v[m][2]), fabsf(v[m][3])));
+        for (int b = 0; b < 4; b++)
+            v[b] = load_x(x + (int64_t)m * K + 128 * q + k_local<FMT>(t, rho, b));
+        float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
         for (int o = 16; o; o >>= 1)
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -230,10 +224,9 @@ __device__ __forceinline__ void build_fragments(const XT *__restrict__ x, int M,
             frexpf(amax, &e);                        // amax = f 2^e, f in [0.5, 1)
             e -= 1;                                  // amax in [2^e, 2^(e+1))
         }
-        uint32_t dw[kDigits] = {0u, 0u, 0u};
 #pragma unroll
         for (int b = 0; b < 4; b++) {
-            int X = amax > 0.f ? __float2int_rn(ldexpf(v[m][b], 21 - e)) : 0;   // |X| < 2^22
+            int X = amax > 0.f ? __float2int_rn(ldexpf(v[b], 21 - e)) : 0;   // |X| < 2^22
 #pragma unroll
             for (int d = 0; d < kDigits; d++) {
                 const int dig = ((X + 128) & 255) - 128;                     // balanced digit
@@ -241,31 +234,48 @@ __device__ __forceinline__ void build_fragments(const XT *__restrict__ x, int M,
                 X = (X - dig) >> 8;                                          // exact
             }
         }
-#pragma unroll
-        for (int d = 0; d < kDigits; d++) {
-            const int c = m * kColsPerTok + d;
-            if (c < CS * 8)
-                outw[c] = dw[d];
-        }
-        if (lane == m)
-            fac = amax > 0.f ? ldexpf(1.f, e - 27) : 0.f;                   // 2^(e-21) / 64
+        fac = amax > 0.f ? ldexpf(1.f, e - 27) : 0.f;                       // 2^(e-21) / 64
     }
-    // fragment layout in shared memory: [cs][q][half][lane][4] u32, register rho = 4 half + r
 #pragma unroll
-    for (int c = 0; c < CS * 8; c++) {
+    for (int d = 0; d < kColsPerTok; d++) {
+        const int c = m * kColsPerTok + d;
         const int cs = c >> 3, ln = 4 * (c & 7) + t;
-        frag_s[(((cs * G + q) * 2 + (rho >> 2)) * 32 + ln) * 4 + (rho & 3)] = outw[c];
+        frag[(((cs * G + q) * 2 + (rho >> 2)) * 32 + ln) * 4 + (rho & 3)] = d < kDigits ? dw[d] : 0u;
     }
-    if (lane < 2 * CS)
-        colf_s[lane * G + q] = fac;                  // tokens past M get 0
+    if (lane == 0)
+        colf[m * G + q] = fac;
 }
 
+// x -> digit fragments and factors of every (group, token slot), once per call, into the
+// workspace; block 0 also zeroes the split-block counters. One warp per (group, slot).
+constexpr int kPrepThreads = 256;
+
 template <int FMT, int CS, typename XT>
+__global__ void __launch_bounds__(kPrepThreads)
+gemv_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint32_t *__restrict__ frag,
+                 float *__restrict__ colf, unsigned int *__restrict__ counters, int n_counters)
+{
+    // the GEMV that reads these fragments may start its weight stream now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // x may be the output of the previous kernel, and the previous GEMV may still be reading
+    // the workspace: wait for it to finish before writing anything
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int G = (int)(K / 128);
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < n_counters; i += kPrepThreads)
+            counters[i] = 0u;
+    const int item = (int)((blockIdx.x * kPrepThreads + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (item < G * 2 * CS)
+        build_token<FMT, XT>(x, M, K, G, item / (2 * CS), item % (2 * CS), lane, frag, colf);
+}
+
+template <int FMT, int CS>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restrict__ scales,
-               const XT *__restrict__ x, int M, int64_t N, int64_t K, void *__restrict__ y, int yt,
-               float *__restrict__ part, unsigned long long *__restrict__ counters, int64_t U, int C,
-               int stages, uint32_t call_id, uint32_t one, unsigned int *dev_status)
+               int M, int64_t N, int64_t K, void *__restrict__ y, int yt,
+               float *__restrict__ part, unsigned int *__restrict__ counters,
+               const uint32_t *__restrict__ frag_g, const float *__restrict__ colf_g, int64_t U, int C,
+               int stages, uint32_t one, unsigned int *dev_status)
 {
     using SC = StageCfg<FMT>;
     const int G = (int)(K / 128);
@@ -289,6 +299,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
             ptx::mbar_init(&bars->full[s], 1);
             ptx::mbar_init(&bars->empty[s], kConsumers);
         }
+        ptx::mbar_init(&bars->frag, 1);
         bars->abort = 0;
         ptx::fence_barrier_init();
     }
@@ -330,18 +341,37 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
         }
     } else {
         // ------------------------------------------------------------------- consumers
-        // x may be the output of the previous kernel in the stream
+        // the fragments are written by the prep kernel launched just before this one
         asm volatile("griddepcontrol.wait;" ::: "memory");
-        {
-            // digit fragments of the chunks this CTA touches (all of them if it owns >= C units)
-            const int64_t span = u1 - u0 < C ? u1 - u0 : C;
-            const int nitems = (int)span * SC::kGroups;
-            for (int i = warp; i < nitems; i += kConsumers) {
-                const int c = (int)((u0 + i / SC::kGroups) % C);
-                build_fragments<FMT, CS, XT>(x, M, K, G, SC::kGroups * c + i % SC::kGroups, lane, frag_s, colf_s);
+        if (threadIdx.x == 0) {
+            // bulk-copy the digit fragments of the k-chunks this CTA touches (one range, two
+            // when its units wrap into the next row block, all of them if it owns >= C units)
+            // and all the factors
+            int ra0 = 0, ra1 = C, rb0 = 0, rb1 = 0;
+            if (u1 - u0 < C) {
+                const int cA = (int)(u0 % C), cB = (int)((u1 - 1) % C);
+                ra0 = cA;
+                if (cA <= cB) {
+                    ra1 = cB + 1;
+                } else {
+                    ra1 = C;
+                    rb1 = cB + 1;
+                }
             }
+            constexpr uint32_t kChunkBytes = SC::kGroups * 1024;
+            const uint32_t colf_bytes = (uint32_t)(2 * CS * G * 4);
+            ptx::mbar_arrive_expect_tx(&bars->frag,
+                                       (uint32_t)CS * (uint32_t)(ra1 - ra0 + rb1 - rb0) * kChunkBytes + colf_bytes);
+#pragma unroll
+            for (int cs = 0; cs < CS; cs++) {
+                const size_t o = (size_t)cs * G * 256;
+                ptx::bulk_load(frag_s + o + ra0 * SC::kGroups * 256, frag_g + o + ra0 * SC::kGroups * 256,
+                               (uint32_t)(ra1 - ra0) * kChunkBytes, &bars->frag);
+                if (rb1 > rb0)
+                    ptx::bulk_load(frag_s + o, frag_g + o, (uint32_t)(rb1 - rb0) * kChunkBytes, &bars->frag);
+            }
+            ptx::bulk_load(colf_s, colf_g, colf_bytes, &bars->frag);
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");   // fragments ready
 
         const int tile = warp & (kTiles - 1), half = warp / kTiles;   // this warp's share of the groups
         const int g8 = lane >> 2, t = lane & 3;
@@ -367,32 +397,51 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
             woff[h][0] = r0 * 128 + ((j ^ (r0 & 7)) << 4) + within;
             woff[h][1] = r1 * 128 + ((j ^ (r1 & 7)) << 4) + within;
         }
-        // this thread's GH scales of rows r0 / r1 for unit (rb, c) (0 past row N); the loads
-        // are issued one stage before the scales are needed
-        auto load_scales = [&](int64_t rb_, int c_, uint32_t (&o0)[GH / 2], uint32_t (&o1)[GH / 2]) {
+        // this thread's GH scales of rows r0 / r1, loaded one stage before they are needed:
+        // row pointers are set once per block (rows past N read row 0 and are zeroed)
+        struct ScaleRows {
+            const uint16_t *p0, *p1;
+            bool v0, v1;
+        };
+        auto scale_rows = [&](int64_t rb_) {
             const int64_t n0 = rb_ * kRows + r0, n1 = n0 + 8;
-            const uint16_t *p0 = scales + (n0 < N ? n0 : 0) * G + c_ * SC::kGroups + half * GH;
-            const uint16_t *p1 = scales + (n1 < N ? n1 : 0) * G + c_ * SC::kGroups + half * GH;
+            ScaleRows sr;
+            sr.v0 = n0 < N;
+            sr.v1 = n1 < N;
+            sr.p0 = scales + (sr.v0 ? n0 : 0) * G + half * GH;
+            sr.p1 = scales + (sr.v1 ? n1 : 0) * G + half * GH;
+            return sr;
+        };
+        auto load_scales = [&](const ScaleRows &sr, int c_, uint32_t (&o0)[GH / 2], uint32_t (&o1)[GH / 2]) {
+            const uint16_t *p0 = sr.p0 + c_ * SC::kGroups, *p1 = sr.p1 + c_ * SC::kGroups;
             if (GH == 8) {
-                const uint4 a = n0 < N ? __ldg(reinterpret_cast<const uint4 *>(p0)) : make_uint4(0, 0, 0, 0);
-                const uint4 b = n1 < N ? __ldg(reinterpret_cast<const uint4 *>(p1)) : make_uint4(0, 0, 0, 0);
+                const uint4 a = sr.v0 ? __ldg(reinterpret_cast<const uint4 *>(p0)) : make_uint4(0, 0, 0, 0);
+                const uint4 b = sr.v1 ? __ldg(reinterpret_cast<const uint4 *>(p1)) : make_uint4(0, 0, 0, 0);
                 o0[0] = a.x; o0[1 % (GH / 2)] = a.y; o0[2 % (GH / 2)] = a.z; o0[3 % (GH / 2)] = a.w;
                 o1[0] = b.x; o1[1 % (GH / 2)] = b.y; o1[2 % (GH / 2)] = b.z; o1[3 % (GH / 2)] = b.w;
             } else if (GH == 4) {
-                const uint2 a = n0 < N ? __ldg(reinterpret_cast<const uint2 *>(p0)) : make_uint2(0, 0);
-                const uint2 b = n1 < N ? __ldg(reinterpret_cast<const uint2 *>(p1)) : make_uint2(0, 0);
+                const uint2 a = sr.v0 ? __ldg(reinterpret_cast<const uint2 *>(p0)) : make_uint2(0, 0);
+                const uint2 b = sr.v1 ? __ldg(reinterpret_cast<const uint2 *>(p1)) : make_uint2(0, 0);
                 o0[0] = a.x; o0[GH / 2 - 1] = a.y;
                 o1[0] = b.x; o1[GH / 2 - 1] = b.y;
             } else {
-                o0[0] = n0 < N ? __ldg(reinterpret_cast<const uint32_t *>(p0)) : 0u;
-                o1[0] = n1 < N ? __ldg(reinterpret_cast<const uint32_t *>(p1)) : 0u;
+                o0[0] = sr.v0 ? __ldg(reinterpret_cast<const uint32_t *>(p0)) : 0u;
+                o1[0] = sr.v1 ? __ldg(reinterpret_cast<const uint32_t *>(p1)) : 0u;
             }
         };
+        // per-stage bases: digit fragments [cs][q][half][lane][4] (q stride 256 words, cs
+        // stride 256 G), factors [slot][G] (slot 2 cs + t/2)
+        const int fstride = G * 256, cstride = 2 * G;
+        const uint32_t *frag_lane = frag_s + lane * 4 + half * GH * 256;
+        const float *colf_tok = colf_s + (t >> 1) * G + half * GH;
         uint32_t nx0[GH / 2], nx1[GH / 2];
-        load_scales(u0 / C, (int)(u0 % C), nx0, nx1);
+        ScaleRows rows = scale_rows(u0 / C);
+        load_scales(rows, (int)(u0 % C), nx0, nx1);
         int s = 0;
         uint32_t ph = 0;
-        bool ok = true;
+        const uint8_t *stage = smem + L.stage_off;
+        bool ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&bars->frag, 0, abort, err, kDevErrTimeout,
+                                                                kWaitLimitNs));
         for (int64_t rb = u0 / C; rb * C < u1; rb++) {
             const int c_lo = (int)(rb == u0 / C ? u0 % C : 0);
             const int c_hi = (int)((rb + 1) * C <= u1 ? C : u1 - rb * C);
@@ -410,23 +459,29 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                     sw0[i] = nx0[i];
                     sw1[i] = nx1[i];
                 }
-                if (c + 1 < c_hi)
-                    load_scales(rb, c + 1, nx0, nx1);
-                else if ((rb + 1) * C < u1)
-                    load_scales(rb + 1, 0, nx0, nx1);
+                if (c + 1 < c_hi) {
+                    load_scales(rows, c + 1, nx0, nx1);
+                } else if ((rb + 1) * C < u1) {
+                    rows = scale_rows(rb + 1);              // the next block's rows, once per block
+                    load_scales(rows, 0, nx0, nx1);
+                }
                 // every lane observes the stage's phase itself; the verdict is made warp-uniform
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&bars->full[s], ph, abort, err,
                                                                     kDevErrTimeout, kWaitLimitNs));
                 if (!ok)
                     break;                          // still meet the partner warp below
-                const uint8_t *st = smem + L.stage_off + s * SC::kBytes;
-                constexpr int GP = GH < kGP ? GH : kGP;
+                const uint32_t *fb = frag_lane + c * (SC::kGroups * 256);
+                const float *cb = colf_tok + c * SC::kGroups;
+                // groups expanded at once: four independent MMA chains at one column set, two
+                // per column set beyond (fewer live A registers where there are more chains)
+                constexpr int GPW = CS >= 2 ? 2 : kGP;
+                constexpr int GP = GH < GPW ? GH : GPW;
 #pragma unroll
                 for (int h0 = 0; h0 < GH; h0 += GP) {          // GP groups at a time
                     uint32_t A[GP][4][4];                       // [group][mma][a0..a3]
 #pragma unroll
                     for (int h = 0; h < GP; h++)
-                        expand_group<FMT>(st + woff[h0 + h][0], st + woff[h0 + h][1], mul, A[h]);
+                        expand_group<FMT>(stage + woff[h0 + h][0], stage + woff[h0 + h][1], mul, A[h]);
                     if (h0 + GP == GH) {
                         __syncwarp();
                         if (lane == 0)
@@ -437,9 +492,9 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                         int d[GP][4];
 #pragma unroll
                         for (int h = 0; h < GP; h++) {          // GP independent chains
-                            const int gq = SC::kGroups * c + half * GH + h0 + h;
-                            const uint4 bA = *reinterpret_cast<const uint4 *>(frag_s + (((cs * G + gq) * 2 + 0) * 32 + lane) * 4);
-                            const uint4 bB = *reinterpret_cast<const uint4 *>(frag_s + (((cs * G + gq) * 2 + 1) * 32 + lane) * 4);
+                            const uint32_t *fq = fb + cs * fstride + (h0 + h) * 256;
+                            const uint4 bA = *reinterpret_cast<const uint4 *>(fq);
+                            const uint4 bB = *reinterpret_cast<const uint4 *>(fq + 128);
                             mma_s8_first(d[h], A[h][0][0], A[h][0][1], A[h][0][2], A[h][0][3], bA.x, bA.y, magic);
                             mma_s8(d[h], A[h][1][0], A[h][1][1], A[h][1][2], A[h][1][3], bA.z, bA.w);
                             mma_s8(d[h], A[h][2][0], A[h][2][1], A[h][2][2], A[h][2][3], bB.x, bB.y);
@@ -447,11 +502,10 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                         }
 #pragma unroll
                         for (int h = 0; h < GP; h++) {
-                            const int gq = SC::kGroups * c + half * GH + h0 + h;
                             const __half2 p0 = *reinterpret_cast<const __half2 *>(&sw0[(h0 + h) >> 1]);
                             const __half2 p1 = *reinterpret_cast<const __half2 *>(&sw1[(h0 + h) >> 1]);
-                            // 2^(e-27) of this quad-thread's token (2 cs + t/2) in group gq, times the scales
-                            const float f = colf_s[(2 * cs + (t >> 1)) * G + gq];
+                            // 2^(e-27) of this quad-thread's token (2 cs + t/2) in this group, times the scales
+                            const float f = cb[cs * cstride + h0 + h];
                             const float sf0 = ((h & 1) ? __high2float(p0) : __low2float(p0)) * f;
                             const float sf1 = ((h & 1) ? __high2float(p1) : __low2float(p1)) * f;
                             // exact int -> float: the accumulator started at the bits of 1.5 * 2^23
@@ -467,9 +521,11 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                         }
                     }
                 }
+                stage += SC::kBytes;
                 if (++s == S) {
                     s = 0;
                     ph ^= 1;
+                    stage = smem + L.stage_off;
                 }
             }
 
@@ -510,13 +566,17 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                 }
                 __syncwarp();
             }
-            float fin[16];                                  // half 0: the tile's (row, token) sums
-            for (int e = lane, i = 0; e < 16 * M; e += 32, i++) {
-                const int rr = e / M, m = e % M;
-                float v = 0.f;
+            // the tile's 16 M (row, token) sums, element e = lane + 32 i (16 M <= 128)
+            float fin[4];
 #pragma unroll
-                for (int dg = kDigits - 1; dg >= 0; dg--)                    // digit d weighs 256^d
-                    v = fmaf(v, 256.f, slot[rr * (CS * 8) + m * kColsPerTok + dg]);
+            for (int i = 0; i < 4; i++) {
+                const int e = lane + 32 * i, rr = e / M, m = e % M;
+                float v = 0.f;
+                if (e < 16 * M) {
+#pragma unroll
+                    for (int dg = kDigits - 1; dg >= 0; dg--)                // digit d weighs 256^d
+                        v = fmaf(v, 256.f, slot[rr * (CS * 8) + m * kColsPerTok + dg]);
+                }
                 fin[i] = v;
             }
             if (kHalves == 2) {
@@ -534,40 +594,27 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
             // shares it; only its first owner can hold it in slot 1, and a CTA is the first
             // owner of at most one split block, so the counter is indexed by that owner
             const int end = rb == u0 / C ? 0 : 1;
-            for (int e = lane, i = 0; e < 16 * M; e += 32, i++) {
-                const int rr = e / M, m = e % M;
-                const float v = fin[i];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const int e = lane + 32 * i, rr = e / M, m = e % M;
                 const int64_t n = row0 + rr;
-                if (whole) {
-                    if (n < N)
-                        store_y<float>(y, yt, (int64_t)m * N + n, v);
-                } else {
-                    part[(((int64_t)blockIdx.x * 2 + end) * kRows + tile * 16 + rr) * M + m] = v;
+                if (e < 16 * M) {
+                    if (whole) {
+                        if (n < N)
+                            store_y<float>(y, yt, (int64_t)m * N + n, fin[i]);
+                    } else {
+                        part[(((int64_t)blockIdx.x * 2 + end) * kRows + tile * 16 + rr) * M + m] = fin[i];
+                    }
                 }
             }
-            __syncwarp();
             if (!whole) {
                 // the last of the nseg warps that own these 16 rows sums the partials in
-                // segment order; the counter holds (call id << 32) | arrivals and is reset to 0
+                // segment order; the counters were zeroed by this call's prep kernel
                 __threadfence();
                 __syncwarp();
                 int last = 0;
-                if (lane == 0) {
-                    unsigned long long *ctr = counters + i_first * kTiles + tile;
-                    const unsigned long long tag = (unsigned long long)call_id << 32;
-                    unsigned long long cur = atomicAdd(ctr, 0ull);
-                    for (int tries = 0; tries < (1 << 20); tries++) {
-                        const unsigned long long next = (cur >> 32) == call_id ? cur + 1 : (tag | 1ull);
-                        const unsigned long long prev = atomicCAS(ctr, cur, next);
-                        if (prev == cur) {
-                            last = (int)(next & 0xFFFFFFFFull) == nseg;
-                            if (last)
-                                atomicExch(ctr, 0ull);
-                            break;
-                        }
-                        cur = prev;
-                    }
-                }
+                if (lane == 0)
+                    last = atomicAdd(counters + i_first * kTiles + tile, 1u) == (unsigned)(nseg - 1);
                 last = __shfl_sync(0xffffffffu, last, 0);
                 if (last) {
                     __threadfence();
@@ -586,6 +633,11 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                 }
             }
         }
+    }
+    if (threadIdx.x == 0) {
+        // the fragment copy this thread issued must have landed before the CTA exits
+        volatile int no_abort = 0;
+        ptx::mbar_wait_bounded(&bars->frag, 0, &no_abort, err, kDevErrTimeout, kWaitLimitNs);
     }
     __syncthreads();
 }
@@ -623,7 +675,8 @@ int sm_count()
 struct Plan {
     int CS, stages, grid;
     int64_t NB, C, U;
-    size_t part_bytes, counter_bytes;
+    size_t part_bytes, counter_bytes, frag_bytes, colf_bytes;
+    int n_counters;
 };
 
 template <int FMT, int CS>
@@ -659,15 +712,12 @@ Plan make_plan(int M, int fmt, int64_t N, int64_t K)
     // may share); one counter per tile of the split block each CTA opens
     auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
     p.part_bytes = al((size_t)p.grid * 2 * kRows * M * 4);
-    p.counter_bytes = al((size_t)p.grid * kTiles * 8);
+    p.n_counters = p.grid * kTiles;
+    p.counter_bytes = al((size_t)p.n_counters * 4);
+    // the digit fragments and factors the prep kernel writes (the shared-memory images)
+    p.frag_bytes = al((size_t)p.CS * G * 1024);
+    p.colf_bytes = al((size_t)2 * p.CS * G * 4);
     return p;
-}
-
-uint32_t next_call_id()
-{
-    static uint32_t ctr = 0;
-    uint32_t v = __atomic_add_fetch(&ctr, 1u, __ATOMIC_RELAXED);
-    return v ? v : __atomic_add_fetch(&ctr, 1u, __ATOMIC_RELAXED);
 }
 
 template <int FMT, int CS, typename XT>
@@ -678,7 +728,9 @@ cudaError_t launch_tc_t(const GemvArgs &a, const Plan &pl, cudaStream_t s)
         return cudaErrorNotSupported;
     uint8_t *ws = static_cast<uint8_t *>(a.workspace);
     float *part = reinterpret_cast<float *>(ws);
-    unsigned long long *counters = reinterpret_cast<unsigned long long *>(ws + pl.part_bytes);
+    unsigned int *counters = reinterpret_cast<unsigned int *>(ws + pl.part_bytes);
+    uint32_t *frag = reinterpret_cast<uint32_t *>(ws + pl.part_bytes + pl.counter_bytes);
+    float *colf = reinterpret_cast<float *>(ws + pl.part_bytes + pl.counter_bytes + pl.frag_bytes);
 
     CUtensorMap mw;
     const cuuint64_t wpr = (cuuint64_t)(FMT == BQ_BINARY_G128 ? a.K / 32 : a.K / 16);
@@ -693,8 +745,24 @@ cudaError_t launch_tc_t(const GemvArgs &a, const Plan &pl, cudaStream_t s)
         return cudaErrorInvalidValue;
     const cuuint64_t G = (cuuint64_t)(a.K / 128);
     const int smem = make_layout<FMT, CS>((int)G, pl.stages).total;
-    auto kern = gemv_tc_kernel<FMT, CS, XT>;
+    auto kern = gemv_tc_kernel<FMT, CS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    // both kernels may start before their predecessor in the stream finishes (programmatic
+    // dependent launch); each waits for it (griddepcontrol.wait) before touching its outputs
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t pcfg = {};
+    const int items = (int)G * 2 * CS;
+    pcfg.gridDim = dim3((unsigned)((items * 32 + kPrepThreads - 1) / kPrepThreads));
+    pcfg.blockDim = dim3(kPrepThreads);
+    pcfg.stream = s;
+    pcfg.attrs = attr;
+    pcfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&pcfg, gemv_prep_kernel<FMT, CS, XT>, static_cast<const XT *>(a.x), a.M, a.K, frag, colf,
+                           counters, pl.n_counters);
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
@@ -702,13 +770,10 @@ cudaError_t launch_tc_t(const GemvArgs &a, const Plan &pl, cudaStream_t s)
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mw, reinterpret_cast<const uint16_t *>(a.scales), static_cast<const XT *>(a.x), a.M, a.N, a.K, a.y, a.yt, part,
-                              counters, pl.U, (int)pl.C, pl.stages, next_call_id(), 1u, a.dev_status);
+    return cudaLaunchKernelEx(&cfg, kern, mw, reinterpret_cast<const uint16_t *>(a.scales), a.M, a.N, a.K, a.y, a.yt, part, counters, frag, colf, pl.U, (int)pl.C, pl.stages, 1u,
+                              a.dev_status);
 }
 
 template <int FMT, typename XT>
@@ -736,7 +801,7 @@ bool gemv_tc_supported(int M, int fmt, int64_t K)
 size_t gemv_tc_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
 {
     Plan p = make_plan(M, fmt, N, K);
-    return p.part_bytes + p.counter_bytes;
+    return p.part_bytes + p.counter_bytes + p.frag_bytes + p.colf_bytes;
 }
 
 cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s)
@@ -753,15 +818,17 @@ cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s)
 // fixed scratch of bq_gemv_noalloc
 // ---------------------------------------------------------------------------------------
 // The workspace this kernel needs is at most two 128-row slots of M <= 8 fp32 partial sums
-// per CTA plus one counter per 16-row tile per CTA, and the grid is at most one CTA per SM.
-// This array holds that for grids of up to kStaticMaxCtas CTAs (1.26 MiB). Static device
-// storage starts zeroed; the counters are the only part that must, and every call returns
-// each counter it used to zero (a call cut short by a timeout may leave one tagged with its
-// own call id, which later calls treat as zero).
+// per CTA, one counter per 16-row tile per CTA (the grid is at most one CTA per SM), and the
+// digit fragments and factors, which fit in shared memory. This array holds that for grids of
+// up to kStaticMaxCtas CTAs (1.55 MiB). Nothing in it needs an initial value: each call's
+// prep kernel zeroes the counters before the GEMV uses them.
 constexpr int kStaticMaxCtas = 160;
 constexpr size_t kStaticPartBytes = (size_t)kStaticMaxCtas * 2 * kRows * 8 * sizeof(float);
-constexpr size_t kStaticCounterBytes = ((size_t)kStaticMaxCtas * kTiles * 8 + 255) & ~size_t(255);
-static __device__ __align__(256) unsigned char g_gemv_scratch[kStaticPartBytes + kStaticCounterBytes];
+constexpr size_t kStaticCounterBytes = ((size_t)kStaticMaxCtas * kTiles * 4 + 255) & ~size_t(255);
+constexpr size_t kStaticFragBytes = (size_t)kSmemLimit;        // the fragments fit in shared memory
+constexpr size_t kStaticColfBytes = ((size_t)kSmemLimit / 128 + 255) & ~size_t(255);
+static __device__ __align__(256) unsigned char
+    g_gemv_scratch[kStaticPartBytes + kStaticCounterBytes + kStaticFragBytes + kStaticColfBytes];
 
 cudaError_t gemv_static_scratch(void **ptr, size_t *bytes)
 {
