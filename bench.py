@@ -368,7 +368,8 @@ def e2e_gemv(bq, device, steps, warmup, stream):
 
 
 def traffic_record(kernel_src: str):
-    """ncu DRAM bytes per launch of the dominant kernel, if taken on the current source."""
+    """ncu DRAM bytes (read + write) of one bench step's launches, if taken on the current
+    kernel source (profiles/gemv_traffic.json records the source hash and the command)."""
     p = os.path.join(ROOT, "profiles", "gemv_traffic.json")
     if not os.path.exists(p):
         return None
@@ -521,7 +522,7 @@ def run_gpu(args):
             e2e["value"] = round(world * step_bytes / 1e9 / (e2e_ms / 1e3), 1)
 
     if rank == 0:
-        gemv_src = os.path.join(ROOT, "ternary_g128_weight_bq_b200", "csrc", "gemv.cu")
+        gemv_src = os.path.join(ROOT, "ternary_g128_weight_bq_b200", "csrc", "gemv_tc.cu")
         tr = traffic_record(gemv_src)
         achieved = step_bytes / 1e9 / (ms_total / args.steps / 1e3)
         cpu = None
@@ -548,10 +549,12 @@ def run_gpu(args):
             "roofline": {
                 "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                "traffic": tr["dram_bytes_per_step"] if tr else None,
+                "traffic_unit": "DRAM bytes per step (the twelve launches of six GEMVs), one ncu capture",
+                "bytes_per_step": step_bytes,
                 "peak_source": f"{peaks['source']} (HBM copy, burst)",
-                "kernel": "bq gemv (six launches per step; achieved = algorithmic bytes / "
-                          "device time of the launches)",
+                "kernel": "bq gemv: gemv_prep_kernel + gemv_tc_kernel per GEMV, six GEMVs per step; "
+                          "achieved = algorithmic bytes per step / device time per step",
             },
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -318,7 +318,8 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
             int64_t rb = u0 / C;
             int c = (int)(u0 % C);
             for (int64_t u = u0; u < u1; u++, it++) {
-                if (!ptx::mbar_wait_bounded(&bars->empty[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
+                // a free slot: the producer sleeps in the wait, leaving the issue slots to the consumers
+                if (!ptx::mbar_wait_bounded_sleep(&bars->empty[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
                     break;
                 uint8_t *st = smem + L.stage_off + s * SC::kBytes;
                 ptx::mbar_arrive_expect_tx(&bars->full[s], SC::kBytes);

@@ -56,6 +56,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to `hint_ns` for the phase to complete instead
+// of returning at once: for waiters that are not on the critical path (a producer waiting for a
+// free slot), so that they do not take issue slots from the warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed. Gives up after `limit_ns` of
 // device time, or as soon as *abort is set by another thread; returns false then, after
 // recording kTimeout in *err (only for a real timeout).
@@ -77,6 +93,27 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
                 *abort = 1;
                 return false;
             }
+        }
+    }
+}
+
+// mbar_wait_bounded for a waiter off the critical path: each attempt may sleep up to 2 us.
+__device__ __forceinline__ bool mbar_wait_bounded_sleep(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                        unsigned int *err, unsigned int timeout_bit,
+                                                        uint64_t limit_ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 2000u))
+            return true;
+        if (*abort)
+            return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            atomicOr(err, timeout_bit);
+            *abort = 1;
+            return false;
         }
     }
 }
