@@ -153,7 +153,7 @@ size_t bq_gemv_workspace_bytes(int64_t M, const bq_weight *w);
  *   - a decode loop that must not call cudaMalloc or cudaFree between steps, since those
  *     calls can synchronise the device and stall the queued work;
  *   - plain C hosts that do not want to size, own and free a buffer per weight shape.
- * Limit: the array is 1.55 MiB per device, enough for every M <= 8 and every K on a device
+ * Limit: the array is 1.56 MB per device, enough for every M <= 8 and every K on a device
  * with up to 160 SMs; a shape that needs more returns BQ_ERR_WORKSPACE with the two sizes in
  * bq_last_error(), and bq_gemv with a workspace then serves it.
  * Set-up: the first call on each device (with that device current) resolves the array's

@@ -8,36 +8,40 @@
 // Batch-1 decode (tg128) is the memory-bound phase of section "Cross-platform throughput".
 //
 // Why this shape. At B200's HBM rate one SM receives ~174 binary weights per clock. A
-// select-and-add per weight on the CUDA cores costs more issue slots than that, so each
-// sign bit is turned into the 8-bit integer +-64 (one IMAD shift on the FMA pipe and one LOP3
-// on the ALU pipe per four weights) and mma.sync m16n8k32 s8 (measured ~177 weights per SM
-// clock with fresh operands) does the additions, exactly, in int32: the "add" of select-and-add
-// runs on the tensor pipe. Ternary codes become {-64, 0, +64} with one PRMT per four codes.
+// select-and-add per weight on the CUDA cores costs more issue slots than that, so the sign
+// bits go to mma.sync m16n8k32 s8 (measured ~177 weights per SM clock with fresh operands),
+// which does the additions exactly in int32: the "add" of select-and-add runs on the tensor
+// pipe. A binary register of four weights is one AND of the word (or of the word shifted by 3
+// or 6 bits) with a byte mask: bit b of a byte becomes b * 2^p, p in {5, 6, 7}; two shifts and
+// eight ANDs per 32 weights. Ternary codes become {-64, 0, +64} with one PRMT per four codes.
 //
 // x as integers. Per (token, group of 128), x is written as X = round(x * 2^(21-e)) with
-// e = floor(log2 max|x|) over the group, |X| < 2^22, split into three balanced base-256 digits
-// d0 + 256 d1 + 65536 d2 (each in [-128, 127]); every digit is one MMA column (a token owns
-// four columns: three digits and a zero one). The rounding error is at most 2^-22 max|x| per
-// element, 2^-15 max|x| s per group: below 1/60 of that group's share of the 2e-3 sum|x s|
-// tolerance. The int32 column sums are exact (each starts at the bits of 1.5 * 2^23, so one
-// fp32 subtraction turns it into a float without rounding); the group scale times 2^(e-27) is
-// applied once per group in fp32, and the digit weight 256^d once per block.
+// e = floor(log2 max|x|) over the group, |X| < 2^22, split into balanced digits: four of base
+// 64 for binary (|d| <= 32; the B byte is d * 2^(7-p), so each product is 128 b d, and the
+// accumulator starts at -64 sum(d) over the group, which turns sum(b d) into the sum of
+// (2b - 1) d / 2), three of base 256 and a zero column for ternary. Every digit is one MMA
+// column; a token owns four. The rounding error is at most 2^-22 max|x| per element,
+// 2^-15 max|x| s per group: below 1/60 of that group's share of the 2e-3 sum|x s| tolerance.
+// The int32 column sums are exact (each also starts at the bits of 1.5 * 2^23, so one fp32
+// subtraction turns it into a float without rounding); the group scale times 2^(e-27) is
+// applied once per group in fp32, and the digit weight once per block.
 //
 // Two kernels per call, both with programmatic dependent launch:
-//   * a prep kernel turns x into the MMA B fragments (digits) and per-(token, group) factors
-//     once, one warp per (group, token slot), and zeroes the split-block counters; every CTA
-//     of the GEMV then bulk-copies the fragments of the k-chunks it touches into shared memory
-//     (building them in each CTA cost up to 25 us at M = 8, all of it after the previous
-//     kernel had finished), while its producer already streams the first weight tiles;
-//   * units = (block of 128 rows, one stage of k); CTA i owns units [i U / P, (i+1) U / P)
+//   * a prep kernel turns x into the MMA B fragments (digits), the per-(token, group) factors
+//     and accumulator inputs once, one warp per (group, token slot), and zeroes the split-block
+//     counters; every CTA of the GEMV then bulk-copies the fragments of the k-chunks it touches
+//     into shared memory (building them in each CTA cost up to 25 us at M = 8, all of it after
+//     the previous kernel had finished), while its producer already streams the first weight
+//     tiles;
+//   * units = (block of ROWS rows, one stage of k); CTA i owns units [i U / P, (i+1) U / P)
 //     (stream-K), so every shape is balanced to one unit;
-//   * the producer lane TMA-loads, per unit, a 128 rows x 128 bytes tile of packed words (1024
+//   * the producer lane TMA-loads, per unit, a ROWS x 128 bytes tile of packed words (1024
 //     binary / 512 ternary weights per row; 128B swizzle; 128-byte rows stream measurably
-//     faster than 64-byte ones) into a ring of stages; 8 consumer warps, one per 16-row
-//     tile, expand the stage's groups four at a time (four independent MMA chains); the
-//     group scales come straight from global memory, each stage's loaded one stage early;
+//     faster than 64-byte ones) into a ring of stages; one consumer warp per 16-row tile
+//     expands the stage's groups two or four at a time (independent MMA chains); the group
+//     scales come straight from global memory, each stage's loaded one stage early;
 //   * a block owned by one CTA is written directly; a block split between CTAs leaves partial
-//     sums in the workspace (two 128-row slots per CTA: its first and its last block), and the
+//     sums in the workspace (two block slots per CTA: its first and its last block), and the
 //     last warp to finish its 16 rows (one atomic on a counter the prep kernel zeroed) adds
 //     them in a fixed order.
 #include <cuda.h>
@@ -50,14 +54,19 @@
 namespace bq {
 namespace {
 
-constexpr int kRows = 128;           // weight rows per block (8 tiles of 16 rows)
-constexpr int kTiles = 8;
-constexpr int kHalves = 1;           // consumer warps per 16-row tile (each takes 1/kHalves of a stage's groups)
-constexpr int kConsumers = kTiles * kHalves;
-constexpr int kGP = 4;               // groups a warp expands and multiplies at once (independent chains)
-constexpr int kThreads = (kConsumers + 1) * 32;
-constexpr int kDigits = 3;           // base-256 digits of x per token
-constexpr int kColsPerTok = 4;       // MMA columns per token: the 3 digits and one zero column
+// A block is ROWS weight rows: one consumer warp per 16-row tile plus one producer warp.
+// 192 rows (12 consumer warps, registers capped at 128 by the 13-warp block) at one column set,
+// where more warps hide more latency; 128 rows (8 consumer warps, up to 168 registers) where
+// the wider accumulators of two to four column sets need the registers.
+template <int ROWS> struct Geo {
+    static constexpr int kRows = ROWS;
+    static constexpr int kTiles = ROWS / 16;
+    static constexpr int kConsumers = kTiles;
+    static constexpr int kThreads = (kConsumers + 1) * 32;
+};
+constexpr int rows_for(int fmt, int CS) { return fmt == BQ_BINARY_G128 && CS == 1 ? 192 : 128; }
+constexpr int kMaxTiles = 12;
+constexpr int kColsPerTok = 4;       // MMA columns per token (one per digit of x; see Digits)
 constexpr int kMagic = 0x4B400000;   // bits of 1.5 * 2^23: int n in |n| < 2^22 -> float(bits + n) = 1.5*2^23 + n
 constexpr int kMaxStages = 8;
 constexpr int kSmemLimit = 227 * 1024;
@@ -79,25 +88,50 @@ __device__ __forceinline__ int k_local(int t, int rho, int b)
 
 // One stage = 128 rows x 128 bytes of packed words (one 128-byte-swizzled TMA box):
 // 1024 k (8 groups) of binary weights or 512 k (4 groups) of ternary codes.
-template <int FMT> struct StageCfg {
+template <int FMT, int ROWS> struct StageCfg {
     static constexpr int kGroups = FMT == BQ_BINARY_G128 ? 8 : 4;
-    static constexpr int kBytes = kRows * 128;
+    static constexpr int kBytes = ROWS * 128;
 };
 
+// How x and the weights enter the MMA.
+//   kMask (binary, one column set, where the expansion is most of the work): four balanced
+//     base-64 digits per token (|d| <= 32); the sign bits enter as b * 2^p with b in {0, 1}
+//     (one AND per four weights, p = 5, 6 or 7 by register) and the B byte is d * 2^(7-p)
+//     (negated for p = 7, where b * 2^7 is the s8 value -128), so every product is 128 b d; the
+//     -64 sum(d) that turns b into 2b - 1 is the MMA's accumulator input, a per-(group, column)
+//     value.
+//   otherwise (binary at two to four column sets, where the tensor pipe is the limit and a
+//     per-group accumulator input would cost a load per column set; ternary): three balanced
+//     base-256 digits and a zero column; sign bits enter as +-64 (one shift and one LOP3 per
+//     four weights), ternary codes as {-64, 0, +64} (one PRMT per four codes); the accumulator
+//     input is a constant.
+template <int FMT, int CS> struct Scheme {
+    static constexpr bool kMask = FMT == BQ_BINARY_G128 && CS == 1;
+    static constexpr int kCount = kMask ? 4 : 3;
+    static constexpr int kBits = kMask ? 6 : 8;
+    static constexpr int kRows = rows_for(FMT, CS);
+};
+
+// Binary: bit position p that bit (8b + rho) of a word lands on in A register rho, and the
+// matching B multiplier 2^(7-p) (-1 for p = 7).
+__host__ __device__ constexpr int bin_p(int rho) { return rho == 2 || rho == 5 ? 5 : (rho == 0 || rho == 3 || rho == 6 ? 6 : 7); }
+__host__ __device__ constexpr int bin_bmul(int rho) { return bin_p(rho) == 5 ? 4 : (bin_p(rho) == 6 ? 2 : -1); }
+
 struct Layout {
-    int frag_off, colf_off, stage_off, red_off, bar_off, total, stages;
+    int frag_off, colf_off, cfix_off, stage_off, red_off, bar_off, total, stages;
 };
 
 // Shared-memory layout for a call (host and device compute the same thing).
-template <int FMT, int CS>
+template <int FMT, int CS, int ROWS>
 __host__ __device__ inline Layout make_layout(int G, int stages)
 {
     Layout L;
     L.frag_off = 0;
     L.colf_off = CS * G * 1024;
-    L.stage_off = (L.colf_off + 2 * CS * G * 4 + 1023) / 1024 * 1024;   // one factor per token slot
-    L.red_off = L.stage_off + stages * StageCfg<FMT>::kBytes;
-    L.bar_off = L.red_off + kTiles * 16 * CS * 8 * 4;
+    L.cfix_off = L.colf_off + 2 * CS * G * 4;                           // one factor per token slot
+    L.stage_off = (L.cfix_off + CS * G * 32 + 1023) / 1024 * 1024;      // accumulator inputs [cs][q][8]
+    L.red_off = L.stage_off + stages * StageCfg<FMT, ROWS>::kBytes;
+    L.bar_off = L.red_off + Geo<ROWS>::kTiles * 16 * CS * 8 * 4;
     L.total = L.bar_off + 256 + 1024;                // barriers + alignment slack
     L.stages = stages;
     return L;
@@ -110,12 +144,30 @@ struct Bars {
     int abort;
 };
 
+// 8 A registers of one binary word (kMask scheme): register rho holds, in byte b, bit 8b + rho
+// as b * 2^p (p = bin_p(rho)): registers 5, 6, 7 take bits 5, 6, 7 of each byte straight from
+// the word, registers 2, 3, 4 the same bits of the word shifted left by 3, registers 0, 1 by 6.
+// Two shifts (multiplies by values held in registers, on the FMA pipe) and eight ANDs (ALU
+// pipe) per 32 weights. mk = {8, 64, 0x20202020, 0x40404040, 0x80808080, ...}.
+__device__ __forceinline__ void expand_binary_mask(uint32_t w, const uint32_t (&mk)[9], uint32_t *a)
+{
+    const uint32_t s3 = w * mk[0], s6 = w * mk[1];
+    a[0] = s6 & mk[3];
+    a[1] = s6 & mk[4];
+    a[2] = s3 & mk[2];
+    a[3] = s3 & mk[3];
+    a[4] = s3 & mk[4];
+    a[5] = w & mk[2];
+    a[6] = w & mk[3];
+    a[7] = w & mk[4];
+}
+
 // 8 A registers (s8 +-64) of one binary word: register i holds, in byte b, bit 8b + i
 // (1 -> +64 = 0x40, 0 -> -64 = 0xC0). The shift is a multiply by mul[i] = 2^(7-i) held in a
 // register, so it issues on the FMA pipe; the LOP3 issues on the ALU pipe.
-// mul[8] = {2^7, .., 2^1, 0x80808080, 0x40404040}: the masks live in registers (they come
-// from a kernel argument), so each byte select is a single three-register LOP3.
-__device__ __forceinline__ void expand_binary(uint32_t w, const uint32_t (&mul)[9], uint32_t *a)
+// mul = {2^7, .., 2^1, 0x80808080, 0x40404040}: the masks live in registers (they come from a
+// kernel argument), so each byte select is a single three-register LOP3.
+__device__ __forceinline__ void expand_binary_pm64(uint32_t w, const uint32_t (&mul)[9], uint32_t *a)
 {
 #pragma unroll
     for (int i = 0; i < 8; i++) {
@@ -142,14 +194,17 @@ __device__ __forceinline__ void expand_ternary(uint32_t w, uint32_t *a)
 // Expand one group of this thread's two rows straight into the four MMA A operands:
 // quad[j] = {row r0 reg 2j, row r1 reg 2j, row r0 reg 2j+1, row r1 reg 2j+1}, the register
 // order mma.sync wants, so no copies are needed to form the operand tuples.
-template <int FMT>
+template <int FMT, bool MASK>
 __device__ __forceinline__ void expand_group(const uint8_t *p0, const uint8_t *p1, const uint32_t (&mul)[9],
                                              uint32_t (&quad)[4][4])
 {
     uint32_t a0[8], a1[8];
-    if (FMT == BQ_BINARY_G128) {
-        expand_binary(*reinterpret_cast<const uint32_t *>(p0), mul, a0);
-        expand_binary(*reinterpret_cast<const uint32_t *>(p1), mul, a1);
+    if (FMT == BQ_BINARY_G128 && MASK) {
+        expand_binary_mask(*reinterpret_cast<const uint32_t *>(p0), mul, a0);
+        expand_binary_mask(*reinterpret_cast<const uint32_t *>(p1), mul, a1);
+    } else if (FMT == BQ_BINARY_G128) {
+        expand_binary_pm64(*reinterpret_cast<const uint32_t *>(p0), mul, a0);
+        expand_binary_pm64(*reinterpret_cast<const uint32_t *>(p1), mul, a1);
     } else {
         const uint2 w0 = *reinterpret_cast<const uint2 *>(p0);
         const uint2 w1 = *reinterpret_cast<const uint2 *>(p1);
@@ -198,17 +253,22 @@ __device__ __forceinline__ void store_y(void *y, int yt, int64_t idx, float v)
         store_out(static_cast<__half *>(y) + idx, v);
 }
 
-// Digit fragments of token slot m (MMA columns 4m .. 4m+3: digits 0, 1, 2 and a zero column)
-// in group q, and the token's factor 2^(e-27) (the 2^(8d) of digit d is applied per block),
-// written with the shared-memory layout [cs][q][half][lane][4] u32 / [slot][G] f32. One warp;
-// lane (t, rho) builds register rho of quad-thread t. Slots m >= M (the padding of the last
-// column set) get zeros, so a quad-thread's two accumulator columns always belong to one token.
-template <int FMT, typename XT>
+// Digit fragments of token slot m (MMA columns 4m .. 4m+3) in group q, the token's factor
+// 2^(e-27) (the weight 2^(kBits d) of digit d is applied per block) and the accumulator inputs
+// of its columns (the bits of 1.5 * 2^23, minus 64 sum(d) over the group for binary), written
+// with the shared-memory layouts [cs][q][half][lane][4] u32, [slot][G] f32 and [cs][q][8] s32.
+// One warp; lane (t, rho) builds register rho of quad-thread t. Slots m >= M (the padding of
+// the last column set) get zeros, so a quad-thread's two accumulator columns always belong to
+// one token.
+template <int FMT, int CS, typename XT>
 __device__ __forceinline__ void build_token(const XT *__restrict__ x, int M, int64_t K, int G, int q, int m,
-                                            int lane, uint32_t *__restrict__ frag, float *__restrict__ colf)
+                                            int lane, uint32_t *__restrict__ frag, float *__restrict__ colf,
+                                            int *__restrict__ cfix)
 {
+    using D = Scheme<FMT, CS>;
     const int t = lane >> 3, rho = lane & 7;
-    uint32_t dw[kDigits] = {0u, 0u, 0u};
+    uint32_t dw[4] = {0u, 0u, 0u, 0u};
+    int csum[4] = {0, 0, 0, 0};
     float fac = 0.f;
     if (m < M) {
         float v[4];
@@ -224,15 +284,25 @@ __device__ __forceinline__ void build_token(const XT *__restrict__ x, int M, int
             frexpf(amax, &e);                        // amax = f 2^e, f in [0.5, 1)
             e -= 1;                                  // amax in [2^e, 2^(e+1))
         }
+        const int bmul = D::kMask ? bin_bmul(rho) : 1;
 #pragma unroll
         for (int b = 0; b < 4; b++) {
             int X = amax > 0.f ? __float2int_rn(ldexpf(v[b], 21 - e)) : 0;   // |X| < 2^22
 #pragma unroll
-            for (int d = 0; d < kDigits; d++) {
-                const int dig = ((X + 128) & 255) - 128;                     // balanced digit
-                dw[d] |= ((uint32_t)dig & 0xFFu) << (8 * b);
-                X = (X - dig) >> 8;                                          // exact
+            for (int d = 0; d < D::kCount; d++) {
+                constexpr int kHalf = 1 << (D::kBits - 1), kMask = (1 << D::kBits) - 1;
+                const int dig = ((X + kHalf) & kMask) - kHalf;               // balanced digit
+                dw[d] |= ((uint32_t)(dig * bmul) & 0xFFu) << (8 * b);
+                csum[d] += dig;
+                X = (X - dig) >> D::kBits;                                   // exact
             }
+        }
+        if (D::kMask) {
+#pragma unroll
+            for (int d = 0; d < 4; d++)
+#pragma unroll
+                for (int o = 16; o; o >>= 1)
+                    csum[d] += __shfl_xor_sync(0xffffffffu, csum[d], o);
         }
         fac = amax > 0.f ? ldexpf(1.f, e - 27) : 0.f;                       // 2^(e-21) / 64
     }
@@ -240,7 +310,9 @@ __device__ __forceinline__ void build_token(const XT *__restrict__ x, int M, int
     for (int d = 0; d < kColsPerTok; d++) {
         const int c = m * kColsPerTok + d;
         const int cs = c >> 3, ln = 4 * (c & 7) + t;
-        frag[(((cs * G + q) * 2 + (rho >> 2)) * 32 + ln) * 4 + (rho & 3)] = d < kDigits ? dw[d] : 0u;
+        frag[(((cs * G + q) * 2 + (rho >> 2)) * 32 + ln) * 4 + (rho & 3)] = d < D::kCount ? dw[d] : 0u;
+        if (lane == 0)
+            cfix[(cs * G + q) * 8 + (c & 7)] = kMagic - (D::kMask ? 64 * csum[d] : 0);
     }
     if (lane == 0)
         colf[m * G + q] = fac;
@@ -253,7 +325,8 @@ constexpr int kPrepThreads = 256;
 template <int FMT, int CS, typename XT>
 __global__ void __launch_bounds__(kPrepThreads)
 gemv_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint32_t *__restrict__ frag,
-                 float *__restrict__ colf, unsigned int *__restrict__ counters, int n_counters)
+                 float *__restrict__ colf, int *__restrict__ cfix, unsigned int *__restrict__ counters,
+                 int n_counters)
 {
     // the GEMV that reads these fragments may start its weight stream now
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -266,26 +339,30 @@ gemv_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint32_t *__restric
             counters[i] = 0u;
     const int item = (int)((blockIdx.x * kPrepThreads + threadIdx.x) >> 5), lane = threadIdx.x & 31;
     if (item < G * 2 * CS)
-        build_token<FMT, XT>(x, M, K, G, item / (2 * CS), item % (2 * CS), lane, frag, colf);
+        build_token<FMT, CS, XT>(x, M, K, G, item / (2 * CS), item % (2 * CS), lane, frag, colf, cfix);
 }
 
-template <int FMT, int CS>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int FMT, int CS, int ROWS>
+__global__ void __launch_bounds__(Geo<ROWS>::kThreads, 1)
 gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restrict__ scales,
                int M, int64_t N, int64_t K, void *__restrict__ y, int yt,
                float *__restrict__ part, unsigned int *__restrict__ counters,
-               const uint32_t *__restrict__ frag_g, const float *__restrict__ colf_g, int64_t U, int C,
+               const uint32_t *__restrict__ frag_g, const float *__restrict__ colf_g,
+               const int *__restrict__ cfix_g, int64_t U, int C,
                int stages, uint32_t one, unsigned int *dev_status)
 {
-    using SC = StageCfg<FMT>;
+    using SC = StageCfg<FMT, ROWS>;
+    using SCH = Scheme<FMT, CS>;
+    constexpr int kRows = ROWS, kTiles = Geo<ROWS>::kTiles, kConsumers = Geo<ROWS>::kConsumers;
     const int G = (int)(K / 128);
-    const Layout L = make_layout<FMT, CS>(G, stages);
+    const Layout L = make_layout<FMT, CS, ROWS>(G, stages);
     const int S = stages;
     extern __shared__ uint8_t smem_raw[];
     // align by an offset on the shared array itself, so every access stays a shared-memory one
     uint8_t *smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint32_t *frag_s = reinterpret_cast<uint32_t *>(smem + L.frag_off);
     float *colf_s = reinterpret_cast<float *>(smem + L.colf_off);
+    int *cfix_s = reinterpret_cast<int *>(smem + L.cfix_off);
     float *red = reinterpret_cast<float *>(smem + L.red_off);
     Bars *bars = reinterpret_cast<Bars *>(smem + L.bar_off);
     volatile int *abort = &bars->abort;
@@ -360,9 +437,9 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                 }
             }
             constexpr uint32_t kChunkBytes = SC::kGroups * 1024;
-            const uint32_t colf_bytes = (uint32_t)(2 * CS * G * 4);
-            ptx::mbar_arrive_expect_tx(&bars->frag,
-                                       (uint32_t)CS * (uint32_t)(ra1 - ra0 + rb1 - rb0) * kChunkBytes + colf_bytes);
+            const uint32_t colf_bytes = (uint32_t)(2 * CS * G * 4), cfix_bytes = (uint32_t)(CS * G * 32);
+            ptx::mbar_arrive_expect_tx(&bars->frag, (uint32_t)CS * (uint32_t)(ra1 - ra0 + rb1 - rb0) * kChunkBytes +
+                                                        colf_bytes + cfix_bytes);
 #pragma unroll
             for (int cs = 0; cs < CS; cs++) {
                 const size_t o = (size_t)cs * G * 256;
@@ -372,27 +449,38 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                     ptx::bulk_load(frag_s + o, frag_g + o, (uint32_t)(rb1 - rb0) * kChunkBytes, &bars->frag);
             }
             ptx::bulk_load(colf_s, colf_g, colf_bytes, &bars->frag);
+            ptx::bulk_load(cfix_s, cfix_g, cfix_bytes, &bars->frag);
         }
 
-        const int tile = warp & (kTiles - 1), half = warp / kTiles;   // this warp's share of the groups
+        const int tile = warp;                          // this warp's 16-row tile; it takes every group
         const int g8 = lane >> 2, t = lane & 3;
         const int r0 = tile * 16 + g8, r1 = r0 + 8;          // rows of this thread in the block
-        uint32_t mul[9];                                  // runtime values: kept in registers
+        // shift multipliers and byte masks of the binary expansion: runtime values, kept in registers
+        uint32_t mul[9];
+        if (SCH::kMask) {
+            mul[0] = one * 8u;
+            mul[1] = one * 64u;
+            mul[2] = one * 0x20202020u;
+            mul[3] = one * 0x40404040u;
+            mul[4] = one * 0x80808080u;
+            mul[5] = mul[6] = mul[7] = mul[8] = 0u;
+        } else {
 #pragma unroll
-        for (int i = 0; i < 7; i++)
-            mul[i] = one << (7 - i);
-        mul[7] = one * 0x80808080u;
-        mul[8] = one * 0x40404040u;
-        const int m0 = (int)(one - 1u) + kMagic;      // the accumulators start at 1.5 * 2^23 (as float bits)
+            for (int i = 0; i < 7; i++)
+                mul[i] = one << (7 - i);
+            mul[7] = one * 0x80808080u;
+            mul[8] = one * 0x40404040u;
+        }
+        const int m0 = (int)(one - 1u) + kMagic;        // constant accumulator input (not kMask)
         const int magic[4] = {m0, m0, m0, m0};
-        // this warp takes groups [half GH, (half + 1) GH) of every stage, two at a time
-        constexpr int GH = SC::kGroups / kHalves;
+        // the stage's groups, GP at a time
+        constexpr int GH = SC::kGroups;
         // byte offsets of this thread's packed word(s) of each of those groups in rows r0 / r1
         // (128-byte rows, 128B swizzle: 16-byte chunk j of row r sits at j ^ (r & 7))
         int woff[GH][2];
 #pragma unroll
         for (int h = 0; h < GH; h++) {
-            const int q = half * GH + h;
+            const int q = h;
             const int j = FMT == BQ_BINARY_G128 ? q : 2 * q + (t >> 1);          // 16-byte chunk
             const int within = FMT == BQ_BINARY_G128 ? 4 * t : 8 * (t & 1);
             woff[h][0] = r0 * 128 + ((j ^ (r0 & 7)) << 4) + within;
@@ -409,8 +497,8 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
             ScaleRows sr;
             sr.v0 = n0 < N;
             sr.v1 = n1 < N;
-            sr.p0 = scales + (sr.v0 ? n0 : 0) * G + half * GH;
-            sr.p1 = scales + (sr.v1 ? n1 : 0) * G + half * GH;
+            sr.p0 = scales + (sr.v0 ? n0 : 0) * G;
+            sr.p1 = scales + (sr.v1 ? n1 : 0) * G;
             return sr;
         };
         auto load_scales = [&](const ScaleRows &sr, int c_, uint32_t (&o0)[GH / 2], uint32_t (&o1)[GH / 2]) {
@@ -433,8 +521,9 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
         // per-stage bases: digit fragments [cs][q][half][lane][4] (q stride 256 words, cs
         // stride 256 G), factors [slot][G] (slot 2 cs + t/2)
         const int fstride = G * 256, cstride = 2 * G;
-        const uint32_t *frag_lane = frag_s + lane * 4 + half * GH * 256;
-        const float *colf_tok = colf_s + (t >> 1) * G + half * GH;
+        const uint32_t *frag_lane = frag_s + lane * 4;
+        const float *colf_tok = colf_s + (t >> 1) * G;
+        const int *cfix_lane = cfix_s + 2 * t;          // [cs][q][8]: this thread's columns 2t, 2t+1
         uint32_t nx0[GH / 2], nx1[GH / 2];
         ScaleRows rows = scale_rows(u0 / C);
         load_scales(rows, (int)(u0 % C), nx0, nx1);
@@ -473,16 +562,17 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                     break;                          // still meet the partner warp below
                 const uint32_t *fb = frag_lane + c * (SC::kGroups * 256);
                 const float *cb = colf_tok + c * SC::kGroups;
+                const int *xb = cfix_lane + c * (SC::kGroups * 8);
                 // groups expanded at once: four independent MMA chains at one column set, two
                 // per column set beyond (fewer live A registers where there are more chains)
-                constexpr int GPW = CS >= 2 ? 2 : kGP;
+                constexpr int GPW = CS >= 2 || ROWS > 128 ? 2 : 4;
                 constexpr int GP = GH < GPW ? GH : GPW;
 #pragma unroll
                 for (int h0 = 0; h0 < GH; h0 += GP) {          // GP groups at a time
                     uint32_t A[GP][4][4];                       // [group][mma][a0..a3]
 #pragma unroll
                     for (int h = 0; h < GP; h++)
-                        expand_group<FMT>(stage + woff[h0 + h][0], stage + woff[h0 + h][1], mul, A[h]);
+                        expand_group<FMT, SCH::kMask>(stage + woff[h0 + h][0], stage + woff[h0 + h][1], mul, A[h]);
                     if (h0 + GP == GH) {
                         __syncwarp();
                         if (lane == 0)
@@ -496,7 +586,15 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                             const uint32_t *fq = fb + cs * fstride + (h0 + h) * 256;
                             const uint4 bA = *reinterpret_cast<const uint4 *>(fq);
                             const uint4 bB = *reinterpret_cast<const uint4 *>(fq + 128);
-                            mma_s8_first(d[h], A[h][0][0], A[h][0][1], A[h][0][2], A[h][0][3], bA.x, bA.y, magic);
+                            // accumulator input of columns 2t, 2t+1 (both rows): 1.5 * 2^23 as float
+                            // bits, minus 64 sum(d) for binary
+                            if (SCH::kMask) {
+                                const int2 cc = *reinterpret_cast<const int2 *>(xb + cs * G * 8 + (h0 + h) * 8);
+                                const int cin[4] = {cc.x, cc.y, cc.x, cc.y};
+                                mma_s8_first(d[h], A[h][0][0], A[h][0][1], A[h][0][2], A[h][0][3], bA.x, bA.y, cin);
+                            } else {
+                                mma_s8_first(d[h], A[h][0][0], A[h][0][1], A[h][0][2], A[h][0][3], bA.x, bA.y, magic);
+                            }
                             mma_s8(d[h], A[h][1][0], A[h][1][1], A[h][1][2], A[h][1][3], bA.z, bA.w);
                             mma_s8(d[h], A[h][2][0], A[h][2][1], A[h][2][2], A[h][2][3], bB.x, bB.y);
                             mma_s8(d[h], A[h][3][0], A[h][3][1], A[h][3][2], A[h][3][3], bB.z, bB.w);
@@ -530,43 +628,19 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                 }
             }
 
-            // ---- the two warps of a tile meet: half 1 hands its sums to half 0 through a slot
-            // (barrier 1: written; barrier 2: read), then half 0 adds the digits and writes.
+            // ---- the warp's accumulators go through its slot, where the digit columns of a
+            // token (held by neighbouring quad-threads) are combined
             float *slot = red + (tile * 16) * (CS * 8);   // [16 rows][CS*8]
-            if (kHalves == 1) {
 #pragma unroll
-                for (int cs = 0; cs < CS; cs++) {
-                    slot[g8 * (CS * 8) + cs * 8 + 2 * t] = acc[cs][0];
-                    slot[g8 * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][1];
-                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t] = acc[cs][2];
-                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][3];
-                }
-                __syncwarp();
-                if (!ok || *abort)
-                    break;
-            } else if (half == 1) {
-#pragma unroll
-                for (int cs = 0; cs < CS; cs++) {
-                    slot[g8 * (CS * 8) + cs * 8 + 2 * t] = acc[cs][0];
-                    slot[g8 * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][1];
-                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t] = acc[cs][2];
-                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][3];
-                }
+            for (int cs = 0; cs < CS; cs++) {
+                slot[g8 * (CS * 8) + cs * 8 + 2 * t] = acc[cs][0];
+                slot[g8 * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][1];
+                slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t] = acc[cs][2];
+                slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t + 1] = acc[cs][3];
             }
-            if (kHalves == 2)
-                asm volatile("bar.sync %0, 64;" ::"r"(2 + tile) : "memory");   // id 1 is the prologue barrier
+            __syncwarp();
             if (!ok || *abort)
-                break;                                      // both warps of the tile stop here
-            if (kHalves == 2 && half == 0) {
-#pragma unroll
-                for (int cs = 0; cs < CS; cs++) {
-                    slot[g8 * (CS * 8) + cs * 8 + 2 * t] += acc[cs][0];
-                    slot[g8 * (CS * 8) + cs * 8 + 2 * t + 1] += acc[cs][1];
-                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t] += acc[cs][2];
-                    slot[(g8 + 8) * (CS * 8) + cs * 8 + 2 * t + 1] += acc[cs][3];
-                }
-                __syncwarp();
-            }
+                break;
             // the tile's 16 M (row, token) sums, element e = lane + 32 i (16 M <= 128)
             float fin[4];
 #pragma unroll
@@ -575,15 +649,10 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                 float v = 0.f;
                 if (e < 16 * M) {
 #pragma unroll
-                    for (int dg = kDigits - 1; dg >= 0; dg--)                // digit d weighs 256^d
-                        v = fmaf(v, 256.f, slot[rr * (CS * 8) + m * kColsPerTok + dg]);
+                    for (int dg = SCH::kCount - 1; dg >= 0; dg--)            // digit d weighs 2^(kBits d)
+                        v = fmaf(v, (float)(1 << SCH::kBits), slot[rr * (CS * 8) + m * kColsPerTok + dg]);
                 }
                 fin[i] = v;
-            }
-            if (kHalves == 2) {
-                asm volatile("bar.sync %0, 64;" ::"r"(2 + tile) : "memory");   // the slot is free again
-                if (half == 1)
-                    continue;
             }
             const int64_t row0 = rb * kRows + tile * 16;
             const bool whole = c_lo == 0 && c_hi == C;
@@ -610,15 +679,17 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
             }
             if (!whole) {
                 // the last of the nseg warps that own these 16 rows sums the partials in
-                // segment order; the counters were zeroed by this call's prep kernel
-                __threadfence();
+                // segment order; the counters were zeroed by this call's prep kernel. The warp
+                // barrier orders every lane's partial stores before lane 0's release-add; lane
+                // 0's acquire and the next warp barrier order the other segments' partials
+                // before this warp's loads.
                 __syncwarp();
                 int last = 0;
                 if (lane == 0)
-                    last = atomicAdd(counters + i_first * kTiles + tile, 1u) == (unsigned)(nseg - 1);
+                    last = ptx::atom_add_acq_rel_gpu(counters + i_first * kTiles + tile, 1u) == (unsigned)(nseg - 1);
                 last = __shfl_sync(0xffffffffu, last, 0);
                 if (last) {
-                    __threadfence();
+                    __syncwarp();
                     for (int e = lane; e < 16 * M; e += 32) {
                         const int rr = e / M, m = e % M;
                         float v = 0.f;
@@ -676,7 +747,7 @@ int sm_count()
 struct Plan {
     int CS, stages, grid;
     int64_t NB, C, U;
-    size_t part_bytes, counter_bytes, frag_bytes, colf_bytes;
+    size_t part_bytes, counter_bytes, frag_bytes, colf_bytes, cfix_bytes;
     int n_counters;
 };
 
@@ -684,7 +755,7 @@ template <int FMT, int CS>
 int plan_stages(int G)
 {
     for (int s = kMaxStages; s >= 2; s--)
-        if (make_layout<FMT, CS>(G, s).total <= kSmemLimit)
+        if (make_layout<FMT, CS, rows_for(FMT, CS)>(G, s).total <= kSmemLimit)
             return s;
     return 0;
 }
@@ -704,20 +775,22 @@ Plan make_plan(int M, int fmt, int64_t N, int64_t K)
     p.CS = (M * kColsPerTok + 7) / 8;
     const int G = (int)(K / 128);
     p.stages = stages_for(fmt, p.CS, G);
-    p.NB = (N + kRows - 1) / kRows;
+    const int rows = rows_for(fmt, p.CS);
+    p.NB = (N + rows - 1) / rows;
     p.C = K / (fmt == BQ_BINARY_G128 ? 1024 : 512);
     p.U = p.NB * p.C;
     const int64_t sms = sm_count();
     p.grid = (int)(p.U < sms ? p.U : sms);
-    // partial sums: two 128-row slots per CTA (its first and last block, the only ones it
+    // partial sums: two block-sized slots per CTA (its first and last block, the only ones it
     // may share); one counter per tile of the split block each CTA opens
     auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
-    p.part_bytes = al((size_t)p.grid * 2 * kRows * M * 4);
-    p.n_counters = p.grid * kTiles;
+    p.part_bytes = al((size_t)p.grid * 2 * rows * M * 4);
+    p.n_counters = p.grid * (rows / 16);
     p.counter_bytes = al((size_t)p.n_counters * 4);
     // the digit fragments and factors the prep kernel writes (the shared-memory images)
     p.frag_bytes = al((size_t)p.CS * G * 1024);
     p.colf_bytes = al((size_t)2 * p.CS * G * 4);
+    p.cfix_bytes = al((size_t)p.CS * G * 32);
     return p;
 }
 
@@ -732,12 +805,14 @@ cudaError_t launch_tc_t(const GemvArgs &a, const Plan &pl, cudaStream_t s)
     unsigned int *counters = reinterpret_cast<unsigned int *>(ws + pl.part_bytes);
     uint32_t *frag = reinterpret_cast<uint32_t *>(ws + pl.part_bytes + pl.counter_bytes);
     float *colf = reinterpret_cast<float *>(ws + pl.part_bytes + pl.counter_bytes + pl.frag_bytes);
+    int *cfix = reinterpret_cast<int *>(ws + pl.part_bytes + pl.counter_bytes + pl.frag_bytes + pl.colf_bytes);
 
     CUtensorMap mw;
     const cuuint64_t wpr = (cuuint64_t)(FMT == BQ_BINARY_G128 ? a.K / 32 : a.K / 16);
     cuuint64_t wdims[2] = {wpr, (cuuint64_t)a.N};
     cuuint64_t wstr[1] = {wpr * 4};
-    cuuint32_t wbox[2] = {32, (cuuint32_t)kRows};        // 128 bytes x 128 rows
+    constexpr int ROWS = rows_for(FMT, CS);
+    cuuint32_t wbox[2] = {32, (cuuint32_t)ROWS};         // 128 bytes x ROWS rows
     cuuint32_t est[2] = {1, 1};
     CUresult r = enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(a.words), wdims, wstr, wbox, est,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -745,8 +820,8 @@ cudaError_t launch_tc_t(const GemvArgs &a, const Plan &pl, cudaStream_t s)
     if (r != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     const cuuint64_t G = (cuuint64_t)(a.K / 128);
-    const int smem = make_layout<FMT, CS>((int)G, pl.stages).total;
-    auto kern = gemv_tc_kernel<FMT, CS>;
+    const int smem = make_layout<FMT, CS, ROWS>((int)G, pl.stages).total;
+    auto kern = gemv_tc_kernel<FMT, CS, ROWS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return e;
@@ -763,17 +838,17 @@ cudaError_t launch_tc_t(const GemvArgs &a, const Plan &pl, cudaStream_t s)
     pcfg.attrs = attr;
     pcfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&pcfg, gemv_prep_kernel<FMT, CS, XT>, static_cast<const XT *>(a.x), a.M, a.K, frag, colf,
-                           counters, pl.n_counters);
+                           cfix, counters, pl.n_counters);
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(Geo<ROWS>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mw, reinterpret_cast<const uint16_t *>(a.scales), a.M, a.N, a.K, a.y, a.yt, part, counters, frag, colf, pl.U, (int)pl.C, pl.stages, 1u,
+    return cudaLaunchKernelEx(&cfg, kern, mw, reinterpret_cast<const uint16_t *>(a.scales), a.M, a.N, a.K, a.y, a.yt, part, counters, frag, colf, cfix, pl.U, (int)pl.C, pl.stages, 1u,
                               a.dev_status);
 }
 
@@ -802,7 +877,7 @@ bool gemv_tc_supported(int M, int fmt, int64_t K)
 size_t gemv_tc_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
 {
     Plan p = make_plan(M, fmt, N, K);
-    return p.part_bytes + p.counter_bytes + p.frag_bytes + p.colf_bytes;
+    return p.part_bytes + p.counter_bytes + p.frag_bytes + p.colf_bytes + p.cfix_bytes;
 }
 
 cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s)
@@ -821,15 +896,17 @@ cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s)
 // The workspace this kernel needs is at most two 128-row slots of M <= 8 fp32 partial sums
 // per CTA, one counter per 16-row tile per CTA (the grid is at most one CTA per SM), and the
 // digit fragments and factors, which fit in shared memory. This array holds that for grids of
-// up to kStaticMaxCtas CTAs (1.55 MiB). Nothing in it needs an initial value: each call's
+// up to kStaticMaxCtas CTAs (1.56 MB). Nothing in it needs an initial value: each call's
 // prep kernel zeroes the counters before the GEMV uses them.
 constexpr int kStaticMaxCtas = 160;
-constexpr size_t kStaticPartBytes = (size_t)kStaticMaxCtas * 2 * kRows * 8 * sizeof(float);
-constexpr size_t kStaticCounterBytes = ((size_t)kStaticMaxCtas * kTiles * 4 + 255) & ~size_t(255);
+// (rows x M of a slot: 128 x 8 at two to four column sets, 192 x 2 at one)
+constexpr size_t kStaticPartBytes = (size_t)kStaticMaxCtas * 2 * 1024 * sizeof(float);
+constexpr size_t kStaticCounterBytes = ((size_t)kStaticMaxCtas * kMaxTiles * 4 + 255) & ~size_t(255);
 constexpr size_t kStaticFragBytes = (size_t)kSmemLimit;        // the fragments fit in shared memory
 constexpr size_t kStaticColfBytes = ((size_t)kSmemLimit / 128 + 255) & ~size_t(255);
+constexpr size_t kStaticCfixBytes = ((size_t)kSmemLimit / 32 + 255) & ~size_t(255);
 static __device__ __align__(256) unsigned char
-    g_gemv_scratch[kStaticPartBytes + kStaticCounterBytes + kStaticFragBytes + kStaticColfBytes];
+    g_gemv_scratch[kStaticPartBytes + kStaticCounterBytes + kStaticFragBytes + kStaticColfBytes + kStaticCfixBytes];
 
 cudaError_t gemv_static_scratch(void **ptr, size_t *bytes)
 {

@@ -118,6 +118,18 @@ __device__ __forceinline__ bool mbar_wait_bounded_sleep(uint64_t *bar, uint32_t 
     }
 }
 
+// ---------------------------------------------------------------- global atomics
+
+// atomicAdd with acquire-release semantics at GPU scope: the caller's earlier writes (and those
+// it has observed, e.g. through a warp barrier) are visible before the add, and writes released
+// by earlier adders are visible after it.
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int *p, unsigned int v)
+{
+    unsigned int old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // ---------------------------------------------------------------- TMA (tensor, no multicast)
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
