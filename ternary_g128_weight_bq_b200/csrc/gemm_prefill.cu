@@ -11,16 +11,18 @@
 // One CTA computes a 128 (weight rows) x BN (tokens) tile of Y^T:
 //   * warp 0, one lane: TMA loads of the X tile [BN tokens x 64 k] per k-block into a ring
 //     of shared-memory stages (128-byte swizzle, zero fill past M); warp 0 also owns TMEM.
-//   * warps 2-5 (128 threads, one weight row each): read the row's packed bits and its group
-//     scale straight from global memory, expand each 8-weight chunk to +-s (binary) or
-//     {-s, 0, +s} (ternary) in the operand type through a 256-entry sign-mask table, and
-//     store the 128 x 64 A tile in the same swizzled layout. The scale is folded into the
-//     operand, so a group needs no separate rescaling: +-s is exact in fp16 and rounded to
-//     nearest even in bf16 (x's type decides).
+//   * warps 2-9 (256 threads, two per weight row, each taking half of a k-block): read the
+//     row's packed bits and its group scale straight from global memory, expand each 8-weight
+//     chunk to +-s (binary) or {-s, 0, +s} (ternary) in the operand type through a 256-entry
+//     sign-mask table, and store the 128 x 64 A tile in the same swizzled layout. The scale is
+//     folded into the operand, so a group needs no separate rescaling: +-s is exact in fp16 and
+//     rounded to nearest even in bf16 (x's type decides). Per-CTA cycle counters showed the MMA
+//     issuer waiting on this step for more than half of its loop with four warps, one per row.
 //   * warp 1, one lane: issues 4 tcgen05.mma (128 x BN x 16) per k-block into a TMEM
 //     accumulator and commits each stage back to the producers.
-//   * warps 2-5 then read the accumulator with tcgen05.ld (lane = weight row, column =
-//     token) and store Y with one coalesced 32-row segment per token.
+//   * warps 2-9 then read the accumulator with tcgen05.ld (lane = weight row, column =
+//     token; the two warps of a lane quarter take alternate 32-token blocks) and store Y with
+//     one coalesced 32-row segment per token.
 // The expanded weights exist only in shared memory. Every mbarrier wait is bounded: after
 // 2 s the kernel records kDevErrTimeout, lets its copies and MMAs drain, frees TMEM and
 // returns.
@@ -34,7 +36,8 @@ namespace {
 
 constexpr int kBM = 128;              // weight rows per tile (MMA M)
 constexpr int kBK = 64;               // k per stage: one 128-byte swizzle row of 16-bit values
-constexpr int kThreads = 192;         // 6 warps
+constexpr int kDequantWarps = 8;      // two per weight row: each expands half of a k-block
+constexpr int kThreads = (2 + kDequantWarps) * 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 template <int BN> struct Cfg {
@@ -105,7 +108,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; s++) {
             ptx::mbar_init(&bars->full_x[s], 1);
-            ptx::mbar_init(&bars->full_a[s], 4);
+            ptx::mbar_init(&bars->full_a[s], kDequantWarps);
             ptx::mbar_init(&bars->empty[s], 1);
         }
         ptx::mbar_init(&bars->acc_full, 1);
@@ -120,7 +123,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
     }
     if (warp >= 2) {
         // sign-mask table: entry b describes the 8 (binary) or 4 (ternary) weights of byte b
-        for (int b = threadIdx.x - 64; b < 256; b += 128) {
+        for (int b = threadIdx.x - 64; b < 256; b += kDequantWarps * 32) {
             uint32_t e[4];
             if (FMT == BQ_BINARY_G128) {
                 for (int i = 0; i < 4; i++) {
@@ -155,7 +158,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
             for (int kb = 0; kb < KB; kb++) {
                 const int s = kb % S;
                 const uint32_t ph = (kb / S) & 1;
-                if (!ptx::mbar_wait_bounded(&bars->empty[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
+                if (!ptx::mbar_wait_bounded_sleep(&bars->empty[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
                     break;
                 ptx::mbar_arrive_expect_tx(&bars->full_x[s], C::kXBytes);
                 ptx::tma_load_2d(xs + s * C::kXBytes, &tmap_x, &bars->full_x[s], kb * kBK, (int32_t)m0);
@@ -200,35 +203,38 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         }
     } else {
         // ------------------------------------------------------------ dequant, then epilogue
-        const int r = threadIdx.x - 64;                      // weight row within the tile
+        // warp 2 + 4 h + j, lane l: row 32 j + l of the tile, half h of every k-block (chunks
+        // 4h .. 4h+3 of 8 weights: one binary word or two ternary words)
+        const int hk = (warp - 2) >> 2;
+        const int r = 32 * ((warp - 2) & 3) + lane;          // weight row within the tile
         const int64_t n = n0 + r;
         const bool row_ok = n < N;
         const int64_t G = K / 128;
-        constexpr int WPB = FMT == BQ_BINARY_G128 ? 2 : 4;   // words per k-block
-        const uint32_t *wrow = words + (row_ok ? n : 0) * (K / 32 * (FMT == BQ_BINARY_G128 ? 1 : 2));
+        constexpr int WPT = FMT == BQ_BINARY_G128 ? 1 : 2;   // words per thread per k-block
+        const uint32_t *wrow = words + (row_ok ? n : 0) * (K / 32 * (FMT == BQ_BINARY_G128 ? 1 : 2)) + hk * WPT;
         const uint16_t *srow = scales + (row_ok ? n : 0) * G;
         uint8_t *arow_base = as + r * 128;
         const int sw = r & 7;
 
         constexpr int kAhead = 4;                           // k-blocks of bits loaded ahead
-        uint4 wq[kAhead];
+        uint2 wq[kAhead];
         uint16_t sq[kAhead];
+        auto load_kb = [&](int kb_, uint2 &wv_, uint16_t &sv_) {
+            if (WPT == 1)
+                wv_ = make_uint2(__ldg(wrow + (size_t)kb_ * 2), 0u);
+            else
+                wv_ = __ldg(reinterpret_cast<const uint2 *>(wrow + (size_t)kb_ * 4));
+            sv_ = __ldg(srow + kb_ / 2);
+        };
 #pragma unroll
         for (int i = 0; i < kAhead; i++) {
-            wq[i] = make_uint4(0, 0, 0, 0);
+            wq[i] = make_uint2(0, 0);
             sq[i] = 0;
-            if (row_ok && i < KB) {
-                if (WPB == 2) {
-                    uint2 v = __ldg(reinterpret_cast<const uint2 *>(wrow) + i);
-                    wq[i] = make_uint4(v.x, v.y, 0, 0);
-                } else {
-                    wq[i] = __ldg(reinterpret_cast<const uint4 *>(wrow) + i);
-                }
-                sq[i] = __ldg(srow + i / 2);
-            }
+            if (row_ok && i < KB)
+                load_kb(i, wq[i], sq[i]);
         }
         for (int kb = 0; kb < KB; kb++) {
-            const uint4 wv = wq[0];
+            const uint2 wv = wq[0];
             const uint16_t sv = sq[0];
 #pragma unroll
             for (int i = 0; i < kAhead - 1; i++) {
@@ -236,16 +242,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
                 sq[i] = sq[i + 1];
             }
             const int nk = kb + kAhead;
-            wq[kAhead - 1] = make_uint4(0, 0, 0, 0);
-            if (row_ok && nk < KB) {
-                if (WPB == 2) {
-                    uint2 v = __ldg(reinterpret_cast<const uint2 *>(wrow) + nk);
-                    wq[kAhead - 1] = make_uint4(v.x, v.y, 0, 0);
-                } else {
-                    wq[kAhead - 1] = __ldg(reinterpret_cast<const uint4 *>(wrow) + nk);
-                }
-                sq[kAhead - 1] = __ldg(srow + nk / 2);
-            }
+            wq[kAhead - 1] = make_uint2(0, 0);
+            if (row_ok && nk < KB)
+                load_kb(nk, wq[kAhead - 1], sq[kAhead - 1]);
 
             const int s = kb % S;
             const uint32_t ph = (kb / S) & 1;
@@ -253,16 +252,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
                 break;
             uint8_t *arow = arow_base + s * C::kABytes;
             const uint32_t s2 = row_ok ? scale_pair(sv, BF16) : 0u;
-            const uint32_t wds[4] = {wv.x, wv.y, wv.z, wv.w};
+            const uint32_t wds[2] = {wv.x, wv.y};
 #pragma unroll
-            for (int c = 0; c < 8; c++) {                    // 8 chunks of 8 weights (16 B each)
+            for (int cl = 0; cl < 4; cl++) {                 // this thread's 4 chunks of 8 weights
+                const int c = 4 * hk + cl;                   // chunk within the k-block (16 B of A)
                 uint4 o;
                 if (FMT == BQ_BINARY_G128) {
-                    const uint32_t byte = (wds[c >> 2] >> (8 * (c & 3))) & 0xFFu;
+                    const uint32_t byte = (wds[0] >> (8 * cl)) & 0xFFu;
                     const uint4 e = lut[byte];
                     o = make_uint4(s2 ^ e.x, s2 ^ e.y, s2 ^ e.z, s2 ^ e.w);
                 } else {
-                    const uint32_t half16 = (wds[c >> 1] >> (16 * (c & 1))) & 0xFFFFu;
+                    const uint32_t half16 = (wds[cl >> 1] >> (16 * (cl & 1))) & 0xFFFFu;
                     const uint4 e0 = lut[half16 & 0xFFu], e1 = lut[half16 >> 8];
                     o = make_uint4((s2 & e0.x) ^ e0.z, (s2 & e0.y) ^ e0.w, (s2 & e1.x) ^ e1.z, (s2 & e1.y) ^ e1.w);
                 }
@@ -282,8 +282,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
             const int quad = warp & 3;                       // TMEM lanes 32*quad .. +31
             const int64_t nrow = n0 + quad * 32 + lane;
             const bool nok = nrow < N;
+            // the two warps of a lane quarter take alternate 32-token column blocks
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 32; cc++) {
+            for (int cc = hk; cc < BN / 32; cc += 2) {
                 uint32_t v[32];
                 ptx::tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(quad * 32) << 16) + cc * 32, v);
                 ptx::tmem_wait_ld();

@@ -690,17 +690,40 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__res
                 last = __shfl_sync(0xffffffffu, last, 0);
                 if (last) {
                     __syncwarp();
-                    for (int e = lane; e < 16 * M; e += 32) {
-                        const int rr = e / M, m = e % M;
-                        float v = 0.f;
-                        for (int sg = 0; sg < nseg; sg++) {         // fixed order: deterministic
+                    // element e = lane + 32 q of the tile's [16 rows][M] sums; the partials of
+                    // eight segments are loaded at once (independent loads, one round trip),
+                    // then added in segment order, so the result does not depend on timing
+                    constexpr int QN = CS;                          // 16 M <= 32 CS elements
+                    float v[QN];
+#pragma unroll
+                    for (int q = 0; q < QN; q++)
+                        v[q] = 0.f;
+                    for (int sg0 = 0; sg0 < nseg; sg0 += 8) {
+                        float pv[8][QN];
+#pragma unroll
+                        for (int j = 0; j < 8; j++) {
+                            const int sg = sg0 + j;
                             const int64_t i = i_first + sg;
                             const int slot_i = sg == 0 && i * U / Pn != x0 ? 1 : 0;
-                            v += __ldcg(part + ((i * 2 + slot_i) * kRows + tile * 16 + rr) * M + m);
+                            const float *pp = part + ((i * 2 + slot_i) * kRows + tile * 16) * M;
+#pragma unroll
+                            for (int q = 0; q < QN; q++) {
+                                const int e = lane + 32 * q;
+                                pv[j][q] = sg < nseg && e < 16 * M ? __ldcg(pp + e) : 0.f;
+                            }
                         }
+#pragma unroll
+                        for (int j = 0; j < 8; j++)
+#pragma unroll
+                            for (int q = 0; q < QN; q++)
+                                v[q] += pv[j][q];
+                    }
+#pragma unroll
+                    for (int q = 0; q < QN; q++) {
+                        const int e = lane + 32 * q, rr = e / M, m = e % M;
                         const int64_t n = row0 + rr;
-                        if (n < N)
-                            store_y<float>(y, yt, (int64_t)m * N + n, v);
+                        if (e < 16 * M && n < N)
+                            store_y<float>(y, yt, (int64_t)m * N + n, v[q]);
                     }
                 }
             }
