@@ -172,15 +172,22 @@ cudaError_t launch_gemv_simt(const GemvArgs &a, cudaStream_t s)
 // their counters); the SIMT kernel needs none.
 size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
 {
+    if (gemv_tmem_supported(M, fmt, K))
+        return gemv_tmem_workspace_bytes(M, N, K);
     if (!gemv_tc_supported(M, fmt, K))
         return 0;
     return gemv_tc_workspace_bytes(M, fmt, N, K);
 }
 
-// K a multiple of 1024 (and its digit fragments fit in shared memory): the integer
-// tensor-core kernel; otherwise the SIMT kernel. One launch either way.
+// Binary with 5 <= M <= 8 and K a multiple of 1024: the tcgen05 kernel (gemv_tmem.cu); other
+// shapes with K a multiple of 1024 whose digit fragments fit in shared memory: the mma.sync
+// kernel (gemv_tc.cu); otherwise the SIMT kernel.
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches)
 {
+    if (gemv_tmem_supported(a.M, a.fmt, a.K)) {
+        *launches = 2;                               // fragment prep + the GEMV
+        return launch_gemv_tmem(a, s);
+    }
     if (gemv_tc_supported(a.M, a.fmt, a.K)) {
         *launches = 2;                               // fragment prep + the GEMV
         return launch_gemv_tc(a, s);

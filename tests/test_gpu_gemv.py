@@ -134,10 +134,12 @@ def test_api_errors_on_device():
 
 # ---- tensor-core path (K a multiple of 1024): fp8 pieces of x, stream-K split ----------
 
-@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("xdt", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("N,K", [(1, 1024), (127, 2048), (129, 1024), (1000, 3072)])
 def test_tensor_path_ragged_all_outputs(orc, M, xdt, N, K):
+    """All outputs of ragged shapes on the tensor-core kernels: mma.sync for M <= 4, tcgen05
+    (sign operand in tensor memory) for binary M >= 5."""
     run_binary(orc, 400 + M, N, K, M, xdt=xdt)
 
 
@@ -147,10 +149,12 @@ def test_tensor_path_ternary(orc, M, N, K):
     run_ternary(orc, 500 + M, N, K, M)
 
 
-def test_tensor_path_wide_dynamic_range(orc):
-    """x spanning 40 binades inside each group: the e4m3 pieces stay within the bound."""
+@pytest.mark.parametrize("M", [3, 8])
+def test_tensor_path_wide_dynamic_range(orc, M):
+    """x spanning 40 binades inside each group: the integer digits of x (22 bits below the
+    group maximum) stay within the bound. M = 3 runs the mma.sync kernel, M = 8 the tcgen05 one."""
     m = bq()
-    N, K, M = 300, 2048, 3
+    N, K = 300, 2048
     x = synth.activations(7, M, K, dtype=torch.float32)
     mag = torch.tensor([2.0 ** (-30 + (k % 41)) for k in range(K)])
     x = (x * mag).to(torch.bfloat16)
@@ -162,9 +166,10 @@ def test_tensor_path_wide_dynamic_range(orc):
     assert_within_bound(y, y_ref, bound, "wide range")
 
 
-def test_tensor_path_zero_and_tiny_groups(orc):
+@pytest.mark.parametrize("M", [2, 6])
+def test_tensor_path_zero_and_tiny_groups(orc, M):
     m = bq()
-    N, K, M = 200, 1024, 2
+    N, K = 200, 1024
     x = synth.activations(8, M, K).float()
     x[0, :128] = 0.0                                   # an all-zero group
     x[1, 128:256] = 1e-30                              # a group of tiny values
