@@ -367,15 +367,27 @@ def e2e_gemv(bq, device, steps, warmup, stream):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 5)}
 
 
-def traffic_record(kernel_src: str):
+GEMV_SOURCES = ("gemv_tc.cu", "gemv_tmem.cu")
+
+
+def gemv_source_sha() -> str:
+    """Hash of the GEMV kernel sources the bench step runs (mma.sync and tcgen05 kernels)."""
+    h = hashlib.sha256()
+    for name in GEMV_SOURCES:
+        with open(os.path.join(ROOT, "ternary_g128_weight_bq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record():
     """ncu DRAM bytes (read + write) of one bench step's launches, if taken on the current
-    kernel source (profiles/gemv_traffic.json records the source hash and the command)."""
+    kernel sources (profiles/gemv_traffic.json records the source hash and the command)."""
     p = os.path.join(ROOT, "profiles", "gemv_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f)
-    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    h = gemv_source_sha()
     if rec.get("source_sha") != h:
         return None
     return rec
@@ -522,8 +534,7 @@ def run_gpu(args):
             e2e["value"] = round(world * step_bytes / 1e9 / (e2e_ms / 1e3), 1)
 
     if rank == 0:
-        gemv_src = os.path.join(ROOT, "ternary_g128_weight_bq_b200", "csrc", "gemv_tc.cu")
-        tr = traffic_record(gemv_src)
+        tr = traffic_record()
         achieved = step_bytes / 1e9 / (ms_total / args.steps / 1e3)
         cpu = None
         if not args.quick:
@@ -553,8 +564,9 @@ def run_gpu(args):
                 "traffic_unit": "DRAM bytes per step (the twelve launches of six GEMVs), one ncu capture",
                 "bytes_per_step": step_bytes,
                 "peak_source": f"{peaks['source']} (HBM copy, burst)",
-                "kernel": "bq gemv: gemv_prep_kernel + gemv_tc_kernel per GEMV, six GEMVs per step; "
-                          "achieved = algorithmic bytes per step / device time per step",
+                "kernel": "bq gemv: a prep kernel + gemv_tc_kernel (mma.sync, M <= 4) or gemv_tmem_kernel "
+                          "(tcgen05, M = 8) per GEMV, six GEMVs per step; achieved = algorithmic bytes "
+                          "per step / device time per step",
             },
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -59,10 +59,10 @@ bool gemv_tc_supported(int M, int fmt, int64_t K);
 size_t gemv_tc_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
 cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s);
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches);
-// tcgen05 path with the sign operand in tensor memory (gemv_tmem.cu): binary, 5 <= M <= 8,
-// K a multiple of 1024
+// tcgen05 path with the sign operand in tensor memory (gemv_tmem.cu): binary with 5 <= M <= 8,
+// ternary with any M <= 8; K a multiple of 1024
 bool gemv_tmem_supported(int M, int fmt, int64_t K);
-size_t gemv_tmem_workspace_bytes(int M, int64_t N, int64_t K);
+size_t gemv_tmem_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
 cudaError_t launch_gemv_tmem(const GemvArgs &a, cudaStream_t s);
 // Device address and size of the fixed scratch array of bq_gemv_noalloc on the current
 // device (gemv_tc.cu); resolved once per device.

@@ -173,15 +173,15 @@ cudaError_t launch_gemv_simt(const GemvArgs &a, cudaStream_t s)
 size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
 {
     if (gemv_tmem_supported(M, fmt, K))
-        return gemv_tmem_workspace_bytes(M, N, K);
+        return gemv_tmem_workspace_bytes(M, fmt, N, K);
     if (!gemv_tc_supported(M, fmt, K))
         return 0;
     return gemv_tc_workspace_bytes(M, fmt, N, K);
 }
 
-// Binary with 5 <= M <= 8 and K a multiple of 1024: the tcgen05 kernel (gemv_tmem.cu); other
-// shapes with K a multiple of 1024 whose digit fragments fit in shared memory: the mma.sync
-// kernel (gemv_tc.cu); otherwise the SIMT kernel.
+// K a multiple of 1024: the tcgen05 kernel (gemv_tmem.cu) for binary with 5 <= M <= 8 and for
+// ternary, the mma.sync kernel (gemv_tc.cu) for binary with M <= 4; otherwise (or when the
+// digit fragments do not fit in shared memory) the SIMT kernel.
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches)
 {
     if (gemv_tmem_supported(a.M, a.fmt, a.K)) {

@@ -1,33 +1,37 @@
-// gemv_tmem.cu -- decode GEMV for 5 <= M <= 8 token rows on packed binary-g128 weights, on the
-// fifth-generation tensor cores (tcgen05 kind::i8) with the sign operand in tensor memory.
+// gemv_tmem.cu -- decode GEMV for 5 <= M <= 8 token rows on packed binary-g128 and ternary-g128
+// weights, on the fifth-generation tensor cores (tcgen05 kind::i8) with the weight operand in
+// tensor memory.
 //
 // y[m][n] = sum_g s[n][g] * sum_{k in g} (2 b[n][k] - 1) x[m][k]: model card
 // "prism-ml/Bonsai-27B-mlx-1bit", sections "Weight representation: Binary g128" and "CUDA
 // (NVIDIA GPUs)"; the decode workload of section "Cross-platform throughput".
 //
 // Per CTA, a ring of TMA stages of 128 rows x 128 bytes of packed words (1024 k), and:
-//   * 4 expander warps: each thread takes one weight row, turns the sign bits of each group
-//     (four words) into s8 values b * 2^p (two shifts and eight ANDs per word) and writes them
-//     with tcgen05.st into a 128-lane x 32-column A tile in tensor memory: four groups per
-//     buffer, two or three buffers;
+//   * 4 expander warps: each thread takes one weight row and turns each group into s8 values:
+//     binary sign bits into b * 2^p (two shifts and eight ANDs per word), ternary codes into
+//     {-64, 0, +64} (PRMT through a byte table, four codes per instruction). It writes them with
+//     tcgen05.st into a 128-lane x 32-column A tile in tensor memory: four groups per buffer,
+//     two buffers;
 //   * 1 MMA warp: per group, 4 tcgen05.mma kind::i8 (M 128, N 32, K 32), A from tensor memory
 //     and the x digits (B) from shared memory, into one of two half-stage accumulator buffers;
 //   * 8 readout warps, two per lane quarter, each taking half of the groups: tcgen05.ld of the
 //     row's accumulators, then the digit weights, the -64 sum(X) correction, the group scale
 //     and the x factor, summed in fp32 per row and token (the pair meets once per block);
 //   * 1 TMA producer warp.
-// x enters as four balanced base-64 digits per (token, group) of X = round(x 2^(21-e)), each
-// digit multiplied by 2^(7-p) (negated for p = 7) to match the sign byte's position p. Each
-// product is then 128 b d, and sum_d 64^d D_d - 64 sum(X) = 64 sum((2b - 1) X). A prep kernel
+// Binary: x enters as four balanced base-64 digits per (token, group) of X = round(x 2^(21-e)),
+// each digit multiplied by 2^(7-p) (negated for p = 7) to match the sign byte's position p. Each
+// product is then 128 b d, and sum_d 64^d D_d - 64 sum(X) = 64 sum((2b - 1) X). Ternary: three
+// balanced base-256 digits and a zero column, products 64 (c - 1) d. A prep kernel
 // builds the B tiles, the factors 2^(e-27) and sum(X) once per call. The work is split
 // stream-K over (128-row block, 1024-k stage) units, with the same split-block partial sums
 // and counters as gemv_tc.cu.
 //
 // Why only M >= 5. Per-warp clock counters measured one issuing thread taking about 74 cycles
-// per tcgen05.mma at N = 8 (M <= 2) and about 41 at N = 32. A 128 x 32 sign tile (4096 weights)
-// per instruction then caps M = 1 well below the mma.sync kernel of gemv_tc.cu (LM head 129 us
-// against 73 us). At M = 8 the mma.sync kernel is itself tensor-bound (32 MMA columns per
-// group), and this kernel is faster: N = 20480, K = 5120: 24.0 us against 26.4 us.
+// per tcgen05.mma at N = 8 (M <= 2) and about 41 at N = 32. A 128 x 32 weight tile (4096
+// weights) per instruction then caps M = 1 well below the mma.sync kernel of gemv_tc.cu (binary
+// LM head 129 us against 73 us; ternary N = 248320: 145 us against 110 us). At M = 8 the
+// mma.sync kernel is itself tensor-bound (32 MMA columns per group), and this kernel is faster:
+// N = 20480, K = 5120: binary 24.0 us against 26.4 us, ternary 25.1 us against 26.6 us.
 #include <cuda.h>
 
 #include "bq_internal.cuh"
@@ -38,7 +42,11 @@ namespace {
 
 constexpr int kRows = 128;
 constexpr int kStageBytes = kRows * 128;
-constexpr int kGroups = 8;                   // groups per stage
+// a stage is 128 bytes of packed words per row: 8 binary groups or 4 ternary groups
+template <int FMT> struct TCfg {
+    static constexpr int kGroups = FMT == BQ_BINARY_G128 ? 8 : 4;
+    static constexpr int kHalves = kGroups / 4;       // 4-group half stages (the A buffer unit)
+};
 constexpr int kExpWarps = 4, kOutWarps = 8;
 constexpr int kThreads = (2 + kExpWarps + kOutWarps) * 32;
 constexpr int kMaxABuf = 3;            // sign-operand buffers of 4 groups (128 columns) each
@@ -96,16 +104,32 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t ta, uint32_t (&r)[8]) { pt
 __device__ __forceinline__ void tmem_ld_cols(uint32_t ta, uint32_t (&r)[16]) { ptx::tmem_ld_32x32b_x16(ta, r); }
 __device__ __forceinline__ void tmem_ld_cols(uint32_t ta, uint32_t (&r)[32]) { ptx::tmem_ld_32x32b_x32(ta, r); }
 
+// 4 s8 registers of one ternary word (16 codes) through a PRMT byte table: code 0 -> -64, 1 -> 0,
+// 2 -> +64, 3 (never written by the pack calls) -> 0. Register j, byte b holds code i(j, b):
+// j = 0: 2b, 1: 8 + 2b, 2: 2b + 1, 3: 9 + 2b.
+__device__ __forceinline__ void expand_ternary4(uint32_t w, uint32_t *a)
+{
+    const uint32_t table = 0x004000C0u;
+    const uint32_t e = w & 0x33333333u, o = (w >> 2) & 0x33333333u;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a[0]) : "r"(table), "r"(e));
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a[1]) : "r"(table), "r"(e >> 16));
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a[2]) : "r"(table), "r"(o));
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(a[3]) : "r"(table), "r"(o >> 16));
+}
+
 // Warp-uniform bounded wait (every lane observes the phase).
 __device__ __forceinline__ bool wwait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err)
 {
     return __all_sync(0xffffffffu, ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, kWaitLimitNs));
 }
 
-// B tiles, factors and sum(X) of (group q, token slot m), one warp; lane L = 8 w + rho holds
-// k = 32 w + 8 b + rho (b = 0..3), which sits at byte 4 L + b of the group's 128-byte B row
-// (the byte position of that weight in the A tile written by expand_mask / tcgen05.st).
-template <int N, typename XT>
+// B tiles, factors and sum(X) of (group q, token slot m), one warp. Lane L fills bytes 4 L + b
+// (b = 0..3) of the group's 128-byte B rows, i.e. tensor-memory column L of the A tile:
+//   binary (expand_mask, L = 8 w + rho): k = 32 w + 8 b + rho; four base-64 digits, each
+//     times 2^(7 - p(rho)), and sum(X) for the -64 sum(X) correction;
+//   ternary (expand_ternary4, L = 4 w + j): k = 16 w + i(j, b); three base-256 digits and a
+//     zero column (the codes enter as {-64, 0, +64}, so no correction).
+template <int FMT, int N, typename XT>
 __global__ void __launch_bounds__(256)
 gemv_tmem_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint8_t *__restrict__ btile, float *__restrict__ fx,
                unsigned int *__restrict__ counters, int n_counters)
@@ -121,7 +145,15 @@ gemv_tmem_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint8_t *__res
     if (item >= G * kSlots)
         return;
     const int q = item / kSlots, m = item % kSlots;
-    const int w = lane >> 3, rho = lane & 7;
+    constexpr bool kBin = FMT == BQ_BINARY_G128;
+    constexpr int kBits = kBin ? 6 : 8, kDig = kBin ? 4 : 3;
+    const int w = kBin ? lane >> 3 : lane >> 2, rho = kBin ? lane & 7 : lane & 3;
+    auto kidx = [&](int b) {
+        if (kBin)
+            return 32 * w + 8 * b + rho;
+        const int i = rho == 0 ? 2 * b : rho == 1 ? 8 + 2 * b : rho == 2 ? 2 * b + 1 : 9 + 2 * b;
+        return 16 * w + i;
+    };
     uint32_t dw[4] = {0u, 0u, 0u, 0u};
     int xs = 0;
     float fac = 0.f;
@@ -129,7 +161,7 @@ gemv_tmem_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint8_t *__res
         float v[4];
 #pragma unroll
         for (int b = 0; b < 4; b++)
-            v[b] = load_x(x + (int64_t)m * K + 128 * q + 32 * w + 8 * b + rho);
+            v[b] = load_x(x + (int64_t)m * K + 128 * q + kidx(b));
         float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
         for (int o = 16; o; o >>= 1)
@@ -139,16 +171,17 @@ gemv_tmem_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint8_t *__res
             frexpf(amax, &e);
             e -= 1;
         }
-        const int bmul = bin_bmul(rho);
+        const int bmul = kBin ? bin_bmul(rho) : 1;
 #pragma unroll
         for (int b = 0; b < 4; b++) {
             int X = amax > 0.f ? __float2int_rn(ldexpf(v[b], 21 - e)) : 0;
-            xs += X;
+            xs += kBin ? X : 0;
 #pragma unroll
-            for (int d = 0; d < 4; d++) {
-                const int dig = ((X + 32) & 63) - 32;
+            for (int d = 0; d < kDig; d++) {
+                constexpr int kHalf = 1 << (kBits - 1), kMask = (1 << kBits) - 1;
+                const int dig = ((X + kHalf) & kMask) - kHalf;
                 dw[d] |= ((uint32_t)(dig * bmul) & 0xFFu) << (8 * b);
-                X = (X - dig) >> 6;
+                X = (X - dig) >> kBits;
             }
         }
 #pragma unroll
@@ -179,7 +212,7 @@ __device__ __forceinline__ void store_y(void *y, int yt, int64_t idx, float v)
         store_out(static_cast<__half *>(y) + idx, v);
 }
 
-template <int N>
+template <int FMT, int N>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_tmem_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restrict__ scales, int M,
                int64_t Nr, int64_t K, void *__restrict__ y, int yt, float *__restrict__ part,
@@ -188,6 +221,8 @@ gemv_tmem_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__r
                unsigned int *dev_status)
 {
     constexpr int kSlots = N / 4;
+    constexpr int kGroups = TCfg<FMT>::kGroups, kHalves = TCfg<FMT>::kHalves;
+    constexpr bool kBin = FMT == BQ_BINARY_G128;
     const int G = (int)(K / 128);
     const Layout L = make_layout<N>(G, stages);
     const int S = stages;
@@ -297,7 +332,7 @@ gemv_tmem_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__r
             int64_t hs = 0;
             for (int64_t u = u0; ok && u < u1; u++) {
                 const int c = (int)(u % C);
-                for (int h = 0; ok && h < 2; h++, hs++) {
+                for (int h = 0; ok && h < kHalves; h++, hs++) {
                     const int ab = (int)(hs % NA), db = (int)(hs & 1);
                     ok = ptx::mbar_wait_bounded(&bars->afull[ab], (uint32_t)((hs / NA) & 1), abort, err,
                                                 kDevErrTimeout, kWaitLimitNs) &&
@@ -340,7 +375,7 @@ gemv_tmem_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__r
             if (!ok)
                 break;
             const uint8_t *stage = smem + L.stage_off + s * kStageBytes + r * 128;
-            for (int h = 0; h < 2; h++, hs++) {
+            for (int h = 0; h < kHalves; h++, hs++) {
                 const int ab = (int)(hs % NA);
                 ok = wwait(&bars->afree[ab], (uint32_t)(((hs / NA) & 1) ^ 1), abort, err);
                 if (!ok)
@@ -349,12 +384,25 @@ gemv_tmem_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__r
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
                     const int qs = 4 * h + i;
-                    const uint4 wv = *reinterpret_cast<const uint4 *>(stage + ((qs ^ (r & 7)) << 4));
                     uint32_t a[32];
-                    expand_mask(wv.x, mk, a);
-                    expand_mask(wv.y, mk, a + 8);
-                    expand_mask(wv.z, mk, a + 16);
-                    expand_mask(wv.w, mk, a + 24);
+                    if (kBin) {                                  // 4 words: 16-byte chunk qs
+                        const uint4 wv = *reinterpret_cast<const uint4 *>(stage + ((qs ^ (r & 7)) << 4));
+                        expand_mask(wv.x, mk, a);
+                        expand_mask(wv.y, mk, a + 8);
+                        expand_mask(wv.z, mk, a + 16);
+                        expand_mask(wv.w, mk, a + 24);
+                    } else {                                     // 8 words: chunks 2 qs, 2 qs + 1
+                        const uint4 w0 = *reinterpret_cast<const uint4 *>(stage + (((2 * qs) ^ (r & 7)) << 4));
+                        const uint4 w1 = *reinterpret_cast<const uint4 *>(stage + (((2 * qs + 1) ^ (r & 7)) << 4));
+                        expand_ternary4(w0.x, a);
+                        expand_ternary4(w0.y, a + 4);
+                        expand_ternary4(w0.z, a + 8);
+                        expand_ternary4(w0.w, a + 12);
+                        expand_ternary4(w1.x, a + 16);
+                        expand_ternary4(w1.y, a + 20);
+                        expand_ternary4(w1.z, a + 24);
+                        expand_ternary4(w1.w, a + 28);
+                    }
                     ptx::tmem_st_32x32b_x32(a_base + ((uint32_t)(32 * qd) << 16) + 128 * ab + 32 * i, a);
                 }
                 ptx::tmem_wait_st();
@@ -391,11 +439,16 @@ gemv_tmem_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__r
             for (int m = 0; m < kSlots; m++)
                 acc[m] = 0.f;
             for (int c = c_lo; ok && c < c_hi; c++) {
-                const uint4 sv = nok ? __ldg(reinterpret_cast<const uint4 *>(scales + n * G + kGroups * c))
-                                     : make_uint4(0, 0, 0, 0);
-                const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+                uint32_t sw[4] = {0u, 0u, 0u, 0u};
+                if (nok && kBin) {
+                    const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(scales + n * G + kGroups * c));
+                    sw[0] = sv.x; sw[1] = sv.y; sw[2] = sv.z; sw[3] = sv.w;
+                } else if (nok) {
+                    const uint2 sv = __ldg(reinterpret_cast<const uint2 *>(scales + n * G + kGroups * c));
+                    sw[0] = sv.x; sw[1] = sv.y;
+                }
 #pragma unroll
-                for (int h = 0; h < 2; h++, hs++) {
+                for (int h = 0; h < kHalves; h++, hs++) {
                     const int db = (int)(hs & 1);
                     ok = wwait(&bars->dfull[db], (uint32_t)((hs >> 1) & 1), abort, err);
                     if (!ok)
@@ -417,11 +470,13 @@ gemv_tmem_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__r
 #pragma unroll
                             for (int m = 0; m < kSlots; m++) {
                                 const uint32_t *dm = dv + N * gl + 4 * m;
+                                constexpr float kW = kBin ? 64.f : 256.f;    // digit weight
                                 float v = (float)(int)dm[3];
-                                v = fmaf(v, 64.f, (float)(int)dm[2]);
-                                v = fmaf(v, 64.f, (float)(int)dm[1]);
-                                v = fmaf(v, 64.f, (float)(int)dm[0]);
-                                v = fmaf(-64.f, xq[m * G + q], v);
+                                v = fmaf(v, kW, (float)(int)dm[2]);
+                                v = fmaf(v, kW, (float)(int)dm[1]);
+                                v = fmaf(v, kW, (float)(int)dm[0]);
+                                if (kBin)
+                                    v = fmaf(-64.f, xq[m * G + q], v);
                                 acc[m] = fmaf(sg * fq[m * G + q], v, acc[m]);
                             }
                         }
@@ -546,7 +601,14 @@ int sm_count_tmem()
     return n;
 }
 
-int n_cols(int M) { (void)M; return 32; }   // 8 token slots x 4 digits
+// accumulator columns: 4 per token slot (four binary digits, or three ternary ones and a zero);
+// this kernel runs for M >= 5 only, so always 8 slots
+int n_cols(int fmt, int M)
+{
+    (void)fmt;
+    (void)M;
+    return 32;
+}
 
 template <int N>
 int plan_stages_tmem(int G)
@@ -557,8 +619,9 @@ int plan_stages_tmem(int G)
     return 0;
 }
 
-int stages_tmem(int M, int G)
+int stages_tmem(int fmt, int M, int G)
 {
+    (void)fmt;
     (void)M;
     return plan_stages_tmem<32>(G);
 }
@@ -570,14 +633,14 @@ struct PlanTmem {
     int n_counters;
 };
 
-PlanTmem make_plan_tmem(int M, int64_t Nr, int64_t K)
+PlanTmem make_plan_tmem(int M, int fmt, int64_t Nr, int64_t K)
 {
     PlanTmem p;
-    p.N = n_cols(M);
+    p.N = n_cols(fmt, M);
     const int G = (int)(K / 128);
-    p.stages = stages_tmem(M, G);
+    p.stages = stages_tmem(fmt, M, G);
     p.NB = (Nr + kRows - 1) / kRows;
-    p.C = K / 1024;
+    p.C = K / (fmt == BQ_BINARY_G128 ? 1024 : 512);   // stages of 128 bytes per row
     p.U = p.NB * p.C;
     const int64_t sms = sm_count_tmem();
     p.grid = (int)(p.U < sms ? p.U : sms);
@@ -590,7 +653,7 @@ PlanTmem make_plan_tmem(int M, int64_t Nr, int64_t K)
     return p;
 }
 
-template <int N, typename XT>
+template <int FMT, int N, typename XT>
 cudaError_t launch_tmem_t(const GemvArgs &a, const PlanTmem &pl, cudaStream_t s)
 {
     EncodeTiledFn enc = encode_fn_tmem();
@@ -602,10 +665,10 @@ cudaError_t launch_tmem_t(const GemvArgs &a, const PlanTmem &pl, cudaStream_t s)
     uint8_t *btile = ws + pl.part_bytes + pl.counter_bytes;
     float *fx = reinterpret_cast<float *>(ws + pl.part_bytes + pl.counter_bytes + pl.b_bytes);
     CUtensorMap mw;
-    const cuuint64_t wpr = (cuuint64_t)(a.K / 32);
+    const cuuint64_t wpr = (cuuint64_t)(FMT == BQ_BINARY_G128 ? a.K / 32 : a.K / 16);
     cuuint64_t wdims[2] = {wpr, (cuuint64_t)a.N};
     cuuint64_t wstr[1] = {wpr * 4};
-    cuuint32_t wbox[2] = {32, (cuuint32_t)kRows};
+    cuuint32_t wbox[2] = {32, (cuuint32_t)kRows};        // 128 bytes x 128 rows
     cuuint32_t est[2] = {1, 1};
     CUresult r = enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(a.words), wdims, wstr, wbox, est,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -614,7 +677,7 @@ cudaError_t launch_tmem_t(const GemvArgs &a, const PlanTmem &pl, cudaStream_t s)
         return cudaErrorInvalidValue;
     const int G = (int)(a.K / 128);
     const int smem = make_layout<N>(G, pl.stages).total;
-    auto kern = gemv_tmem_kernel<N>;
+    auto kern = gemv_tmem_kernel<FMT, N>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return e;
@@ -628,8 +691,8 @@ cudaError_t launch_tmem_t(const GemvArgs &a, const PlanTmem &pl, cudaStream_t s)
     pcfg.stream = s;
     pcfg.attrs = attr;
     pcfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&pcfg, gemv_tmem_prep_kernel<N, XT>, static_cast<const XT *>(a.x), a.M, a.K, btile, fx, counters,
-                           pl.n_counters);
+    e = cudaLaunchKernelEx(&pcfg, gemv_tmem_prep_kernel<FMT, N, XT>, static_cast<const XT *>(a.x), a.M, a.K, btile, fx,
+                           counters, pl.n_counters);
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
@@ -644,25 +707,41 @@ cudaError_t launch_tmem_t(const GemvArgs &a, const PlanTmem &pl, cudaStream_t s)
                               1u, a.dev_status);
 }
 
-}  // namespace
-
-bool gemv_tmem_supported(int M, int fmt, int64_t K)
+template <int FMT, typename XT>
+cudaError_t launch_tmem_n(const GemvArgs &a, const PlanTmem &pl, cudaStream_t s)
 {
-    if (fmt != BQ_BINARY_G128 || M < 5 || M > 8 || K % 1024 != 0)
-        return false;
-    return stages_tmem(M, (int)(K / 128)) >= 2;
+    return launch_tmem_t<FMT, 32, XT>(a, pl, s);
 }
 
-size_t gemv_tmem_workspace_bytes(int M, int64_t N, int64_t K)
+}  // namespace
+
+// 5 <= M <= 8 (binary or ternary), K a multiple of 1024 and the B tiles of all of K in shared
+// memory next to at least two stages. Below M = 5 the mma.sync kernel of gemv_tc.cu is faster:
+// ternary N = 20480, K = 5120: 18.1 us against 19.6 (M = 1), 21.3 against 22.3 (M = 4), while
+// M = 8 is 25.1 here against 26.6 there.
+bool gemv_tmem_supported(int M, int fmt, int64_t K)
 {
-    PlanTmem p = make_plan_tmem(M, N, K);
+    if (M < 5 || M > 8 || K % 1024 != 0)
+        return false;
+    if (fmt != BQ_BINARY_G128 && fmt != BQ_TERNARY_G128)
+        return false;
+    return stages_tmem(fmt, M, (int)(K / 128)) >= 2;
+}
+
+size_t gemv_tmem_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
+{
+    PlanTmem p = make_plan_tmem(M, fmt, N, K);
     return p.part_bytes + p.counter_bytes + p.b_bytes + p.fx_bytes;
 }
 
 cudaError_t launch_gemv_tmem(const GemvArgs &a, cudaStream_t s)
 {
-    PlanTmem pl = make_plan_tmem(a.M, a.N, a.K);
-    return a.xt == BQ_F16 ? launch_tmem_t<32, __half>(a, pl, s) : launch_tmem_t<32, __nv_bfloat16>(a, pl, s);
+    PlanTmem pl = make_plan_tmem(a.M, a.fmt, a.N, a.K);
+    if (a.fmt == BQ_BINARY_G128)
+        return a.xt == BQ_F16 ? launch_tmem_n<BQ_BINARY_G128, __half>(a, pl, s)
+                              : launch_tmem_n<BQ_BINARY_G128, __nv_bfloat16>(a, pl, s);
+    return a.xt == BQ_F16 ? launch_tmem_n<BQ_TERNARY_G128, __half>(a, pl, s)
+                          : launch_tmem_n<BQ_TERNARY_G128, __nv_bfloat16>(a, pl, s);
 }
 
 }  // namespace bq
