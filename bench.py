@@ -459,7 +459,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     o = OracleSample(max_rows=512)
-    budget = 150.0 / max(1, args.steps + args.warmup)
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)
     rows = o.rows_for(budget)
     for _ in range(args.warmup):
         o.run(rows)
@@ -633,6 +633,8 @@ def main():
     ap.add_argument("--impl", choices=["bq", "reference"], default="bq")
     ap.add_argument("--quick", action="store_true", help="headline number only")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="total CPU time budget of --impl reference (split over warm-up and steps)")
     ap.add_argument("--case", choices=["gemv", "prefill", "embed"],
                     help="time one workload alone (for profiling) instead of the benchmark")
     ap.add_argument("--fmt", choices=["binary", "ternary"], default="binary")
