@@ -14,12 +14,15 @@
 //   * warps 2-9 (256 threads, two per weight row, each taking half of a k-block): read the
 //     row's packed bits and its group scale straight from global memory, expand each 8-weight
 //     chunk to +-s (binary) or {-s, 0, +s} (ternary) in the operand type through a 256-entry
-//     sign-mask table, and store the 128 x 64 A tile in the same swizzled layout. The scale is
-//     folded into the operand, so a group needs no separate rescaling: +-s is exact in fp16 and
-//     rounded to nearest even in bf16 (x's type decides). Per-CTA cycle counters showed the MMA
-//     issuer waiting on this step for more than half of its loop with four warps, one per row.
-//   * warp 1, one lane: issues 4 tcgen05.mma (128 x BN x 16) per k-block into a TMEM
-//     accumulator and commits each stage back to the producers.
+//     sign-mask table, and write the 128 x 64 A tile with tcgen05.st straight into tensor
+//     memory (a ring of A stages next to the accumulator), so no shared memory, no proxy
+//     fence, and more shared memory for the X ring. The scale is folded into the operand, so a
+//     group needs no separate rescaling: +-s is exact in fp16 and rounded to nearest even in
+//     bf16 (x's type decides). Per-CTA cycle counters showed the MMA issuer waiting on this
+//     step for more than half of its loop with four warps, one per row, writing shared memory.
+//   * warp 1, one lane: issues 4 tcgen05.mma (128 x BN x 16, A from tensor memory, X from
+//     shared memory) per k-block into the TMEM accumulator and commits each stage back to the
+//     producers.
 //   * warps 2-9 then read the accumulator with tcgen05.ld (lane = weight row, column =
 //     token; the two warps of a lane quarter take alternate 32-token blocks) and store Y with
 //     one coalesced 32-row segment per token.
@@ -40,20 +43,27 @@ constexpr int kDequantWarps = 8;      // two per weight row: each expands half o
 constexpr int kThreads = (2 + kDequantWarps) * 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// X tiles come by TMA into a shared-memory ring; A tiles (the +-s operand) are written by the
+// dequant warps straight into tensor memory, next to the accumulator: D in columns [0, BN),
+// A stage a in columns BN + 32 a (64 k of 16-bit values = 32 columns per lane).
 template <int BN> struct Cfg {
-    static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+    static constexpr int kXStages = BN == 256 ? 6 : 8;
+    static constexpr int kAStages = BN == 256 ? 6 : 8;
     static constexpr int kXBytes = BN * 128;          // X stage: BN rows x 128 B
-    static constexpr int kABytes = kBM * 128;         // A stage: 128 rows x 128 B
     static constexpr int kLutBytes = 256 * 16;
-    static constexpr int kBarOffset = kStages * (kXBytes + kABytes) + kLutBytes;
-    static constexpr int kSmem = kBarOffset + 256 + 1024;   // barriers + alignment slack
-    static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+    static constexpr int kBarOffset = kXStages * kXBytes + kLutBytes;
+    // barriers + alignment slack; at least 116 KB so that one CTA holds the SM (and all 512
+    // tensor-memory columns)
+    static constexpr int kSmemUsed = kBarOffset + 512 + 1024;
+    static constexpr int kSmem = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
+    static constexpr uint32_t kTmemCols = 512;
 };
 
 struct Bars {
     uint64_t full_x[8];
+    uint64_t empty_x[8];
     uint64_t full_a[8];
-    uint64_t empty[8];
+    uint64_t empty_a[8];
     uint64_t acc_full;
     uint64_t drain;
     uint32_t tmem_base;
@@ -89,12 +99,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
                int yt, unsigned int *dev_status)
 {
     using C = Cfg<BN>;
-    constexpr int S = C::kStages;
+    constexpr int SX = C::kXStages, SA = C::kAStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *xs = smem;                                         // S x kXBytes
-    uint8_t *as = smem + S * C::kXBytes;                        // S x kABytes
-    uint4 *lut = reinterpret_cast<uint4 *>(smem + S * (C::kXBytes + C::kABytes));
+    uint8_t *xs = smem;                                         // SX x kXBytes
+    uint4 *lut = reinterpret_cast<uint4 *>(smem + SX * C::kXBytes);
     Bars *bars = reinterpret_cast<Bars *>(smem + C::kBarOffset);
     volatile int *abort = &bars->abort;
     unsigned int *err = dev_status + kSlotErrBits;
@@ -106,10 +115,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
 
     // ---------------------------------------------------------------- set-up
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; s++) {
+        for (int s = 0; s < SX; s++) {
             ptx::mbar_init(&bars->full_x[s], 1);
+            ptx::mbar_init(&bars->empty_x[s], 1);
+        }
+        for (int s = 0; s < SA; s++) {
             ptx::mbar_init(&bars->full_a[s], kDequantWarps);
-            ptx::mbar_init(&bars->empty[s], 1);
+            ptx::mbar_init(&bars->empty_a[s], 1);
         }
         ptx::mbar_init(&bars->acc_full, 1);
         ptx::mbar_init(&bars->drain, 1);
@@ -156,18 +168,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         if (lane == 0) {
             int issued = 0;
             for (int kb = 0; kb < KB; kb++) {
-                const int s = kb % S;
-                const uint32_t ph = (kb / S) & 1;
-                if (!ptx::mbar_wait_bounded_sleep(&bars->empty[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
+                const int s = kb % SX;
+                const uint32_t ph = (kb / SX) & 1;
+                if (!ptx::mbar_wait_bounded_sleep(&bars->empty_x[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
                     break;
                 ptx::mbar_arrive_expect_tx(&bars->full_x[s], C::kXBytes);
                 ptx::tma_load_2d(xs + s * C::kXBytes, &tmap_x, &bars->full_x[s], kb * kBK, (int32_t)m0);
                 issued++;
             }
             // no copy may still be in flight when the CTA exits
-            for (int kb = issued > S ? issued - S : 0; kb < issued; kb++) {
+            for (int kb = issued > SX ? issued - SX : 0; kb < issued; kb++) {
                 volatile int no_abort = 0;
-                ptx::mbar_wait_bounded(&bars->full_x[kb % S], (kb / S) & 1, &no_abort, err, kDevErrTimeout,
+                ptx::mbar_wait_bounded(&bars->full_x[kb % SX], (kb / SX) & 1, &no_abort, err, kDevErrTimeout,
                                        kWaitLimitNs);
             }
         }
@@ -177,19 +189,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
             constexpr uint32_t idesc = ptx::umma_idesc_f16(BF16 ? 1u : 0u, kBM, BN);
             int issued = 0;
             for (int kb = 0; kb < KB; kb++) {
-                const int s = kb % S;
-                const uint32_t ph = (kb / S) & 1;
-                if (!ptx::mbar_wait_bounded(&bars->full_x[s], ph, abort, err, kDevErrTimeout, kWaitLimitNs))
+                const int sx = kb % SX, sa = kb % SA;
+                if (!ptx::mbar_wait_bounded(&bars->full_x[sx], (kb / SX) & 1, abort, err, kDevErrTimeout, kWaitLimitNs))
                     break;
-                if (!ptx::mbar_wait_bounded(&bars->full_a[s], ph, abort, err, kDevErrTimeout, kWaitLimitNs))
+                if (!ptx::mbar_wait_bounded(&bars->full_a[sa], (kb / SA) & 1, abort, err, kDevErrTimeout, kWaitLimitNs))
                     break;
                 ptx::tc_fence_after();
-                const uint64_t adesc = ptx::sw128_kmajor_desc(ptx::smem_u32(as + s * C::kABytes));
-                const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(xs + s * C::kXBytes));
+                const uint32_t a_tmem = tmem_d + BN + 32 * sa;
+                const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(xs + sx * C::kXBytes));
 #pragma unroll
-                for (int k = 0; k < kBK / 16; k++)   // advance 16 elements = 32 B inside the swizzle row
-                    ptx::umma_f16(tmem_d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
-                ptx::umma_commit(&bars->empty[s]);
+                for (int k = 0; k < kBK / 16; k++)   // K step k: 16 elements = 8 A columns, 32 B of the X rows
+                    ptx::umma_f16_ts(tmem_d, a_tmem + 8 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+                ptx::umma_commit(&bars->empty_x[sx]);   // both slots are free once these MMAs finish
+                ptx::umma_commit(&bars->empty_a[sa]);
                 issued++;
             }
             if (issued == KB) {
@@ -203,18 +215,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         }
     } else {
         // ------------------------------------------------------------ dequant, then epilogue
-        // warp 2 + 4 h + j, lane l: row 32 j + l of the tile, half h of every k-block (chunks
-        // 4h .. 4h+3 of 8 weights: one binary word or two ternary words)
+        // warp w = 2 + 4 h + j, lane l: row 32 (w % 4) + l of the tile (a warp reaches only its
+        // own quarter of the tensor-memory lanes), half h of every k-block (chunks 4h .. 4h+3 of
+        // 8 weights: one binary word or two ternary words)
         const int hk = (warp - 2) >> 2;
-        const int r = 32 * ((warp - 2) & 3) + lane;          // weight row within the tile
+        const int r = 32 * (warp & 3) + lane;                // weight row within the tile
         const int64_t n = n0 + r;
         const bool row_ok = n < N;
         const int64_t G = K / 128;
         constexpr int WPT = FMT == BQ_BINARY_G128 ? 1 : 2;   // words per thread per k-block
         const uint32_t *wrow = words + (row_ok ? n : 0) * (K / 32 * (FMT == BQ_BINARY_G128 ? 1 : 2)) + hk * WPT;
         const uint16_t *srow = scales + (row_ok ? n : 0) * G;
-        uint8_t *arow_base = as + r * 128;
-        const int sw = r & 7;
+        // this thread's row in tensor memory: lane r (the warp's lane quarter), columns 16 hk ..
+        const uint32_t arow_tmem = tmem_d + ((uint32_t)(32 * (warp & 3)) << 16) + BN + 16 * hk;
 
         constexpr int kAhead = 4;                           // k-blocks of bits loaded ahead
         uint2 wq[kAhead];
@@ -246,16 +259,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
             if (row_ok && nk < KB)
                 load_kb(nk, wq[kAhead - 1], sq[kAhead - 1]);
 
-            const int s = kb % S;
-            const uint32_t ph = (kb / S) & 1;
-            if (!warp_wait(&bars->empty[s], ph ^ 1, abort, err))
+            const int s = kb % SA;
+            const uint32_t ph = (kb / SA) & 1;
+            if (!warp_wait(&bars->empty_a[s], ph ^ 1, abort, err))
                 break;
-            uint8_t *arow = arow_base + s * C::kABytes;
+            ptx::tc_fence_after();
             const uint32_t s2 = row_ok ? scale_pair(sv, BF16) : 0u;
             const uint32_t wds[2] = {wv.x, wv.y};
+            uint32_t av[16];                                 // 32 weights: 2 per 32-bit column
 #pragma unroll
             for (int cl = 0; cl < 4; cl++) {                 // this thread's 4 chunks of 8 weights
-                const int c = 4 * hk + cl;                   // chunk within the k-block (16 B of A)
                 uint4 o;
                 if (FMT == BQ_BINARY_G128) {
                     const uint32_t byte = (wds[0] >> (8 * cl)) & 0xFFu;
@@ -268,9 +281,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
                 }
                 if (!row_ok)
                     o = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4 *>(arow + ((c ^ sw) << 4)) = o;
+                av[4 * cl] = o.x;
+                av[4 * cl + 1] = o.y;
+                av[4 * cl + 2] = o.z;
+                av[4 * cl + 3] = o.w;
             }
-            ptx::fence_proxy_async_smem();
+            ptx::tmem_st_32x32b_x16(arow_tmem + 32 * s, av);
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 ptx::mbar_arrive(&bars->full_a[s]);
