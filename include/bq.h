@@ -177,7 +177,11 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
  *   x  [M][K], xt = BQ_F16 or BQ_BF16. The scale is applied inside the operand, rounded to
  *      x's type (exact for BQ_F16; bf16 keeps 8 of the scale's 11 significant bits).
  *   y  [M][N], yt = BQ_F32, BQ_BF16 or BQ_F16.
- *   workspace: at least bq_gemm_prefill_workspace_bytes(M, w) bytes (currently 0).
+ *   workspace: at least bq_gemm_prefill_workspace_bytes(M, w) bytes, 16-byte aligned (may be
+ *      NULL when that size is 0). It holds fp32 partial sums when the last wave of output tiles
+ *      would leave most SMs idle and its tiles are split along K instead (for example M = 512,
+ *      N = 20480: 18.9 MB). Contents need not be initialised; calls that share a workspace
+ *      must be ordered on one stream.
  */
 bq_status bq_gemm_prefill(const void *x, bq_dtype xt, int64_t M, const bq_weight *w,
                           void *y, bq_dtype yt, void *workspace, size_t ws_bytes,

@@ -317,11 +317,13 @@ bq_status bq_gemm_prefill(const void *x, bq_dtype xt, int64_t M, const bq_weight
     size_t need = prefill_workspace_bytes(M, w->fmt, w->N, w->K);
     if (need && (!workspace || ws_bytes < need))
         return set_error(BQ_ERR_WORKSPACE, "gemm_prefill: workspace needs %zu bytes", need);
+    if (workspace && !aligned16(workspace))
+        return set_error(BQ_ERR_ALIGNMENT, "gemm_prefill: workspace must be 16-byte aligned");
     unsigned int *status = device_status(&st);
     if (!status)
         return st;
     PrefillArgs a{x, (int)xt, M, (int)w->fmt, w->N, w->K, w->words,
-                  reinterpret_cast<const __half *>(w->scales), y, (int)yt, status};
+                  reinterpret_cast<const __half *>(w->scales), y, (int)yt, need ? workspace : nullptr, status};
     unsigned launches = 0;
     cudaError_t e = launch_prefill(a, stream, &launches);
     if (e != cudaSuccess)

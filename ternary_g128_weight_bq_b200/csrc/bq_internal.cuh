@@ -78,6 +78,7 @@ struct PrefillArgs {
     const __half *scales;
     void *y;
     int yt;
+    void *workspace;          // fp32 partials of split tail tiles (prefill_workspace_bytes)
     unsigned int *dev_status;
 };
 size_t prefill_workspace_bytes(int64_t M, int fmt, int64_t N, int64_t K);

@@ -26,7 +26,9 @@
 //   * warps 2-9 then read the accumulator with tcgen05.ld (lane = weight row, column =
 //     token; the two warps of a lane quarter take alternate 32-token blocks) and store Y with
 //     one coalesced 32-row segment per token.
-// The expanded weights exist only in shared memory. Every mbarrier wait is bounded: after
+// Tiles fill whole waves of one tile per CTA; a short last wave is split along K over the idle
+// SMs (fp32 partials in the workspace, added in split order by prefill_reduce_kernel).
+// The expanded weights exist only on chip. Every mbarrier wait is bounded: after
 // 2 s the kernel records kDevErrTimeout, lets its copies and MMAs drain, frees TMEM and
 // returns.
 #include <cuda.h>
@@ -96,7 +98,7 @@ template <int FMT, int BN, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__restrict__ words,
                const uint16_t *__restrict__ scales, int64_t M, int64_t N, int64_t K, void *__restrict__ y,
-               int yt, unsigned int *dev_status)
+               int yt, int tiles_m, int tile0, int splits, float *__restrict__ part, unsigned int *dev_status)
 {
     using C = Cfg<BN>;
     constexpr int SX = C::kXStages, SA = C::kAStages;
@@ -109,9 +111,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
     unsigned int *err = dev_status + kSlotErrBits;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m0 = (int64_t)blockIdx.x * BN;
-    const int64_t n0 = (int64_t)blockIdx.y * kBM;
-    const int KB = (int)(K / kBK);
+    // CTA b takes tile tile0 + b / splits (token tile = tile % tiles_m, row block = tile /
+    // tiles_m) and k-blocks [kb0, kb1) of it: all of K unless the tile is split
+    const int tile = tile0 + (int)blockIdx.x / splits, split = (int)blockIdx.x % splits;
+    const int64_t m0 = (int64_t)(tile % tiles_m) * BN;
+    const int64_t n0 = (int64_t)(tile / tiles_m) * kBM;
+    const int KBall = (int)(K / kBK);
+    const int kb0 = (int)((int64_t)split * KBall / splits), kb1 = (int)((int64_t)(split + 1) * KBall / splits);
+    const int KB = kb1 - kb0;                                   // k-blocks of this CTA
 
     // ---------------------------------------------------------------- set-up
     if (threadIdx.x == 0) {
@@ -173,7 +180,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
                 if (!ptx::mbar_wait_bounded_sleep(&bars->empty_x[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
                     break;
                 ptx::mbar_arrive_expect_tx(&bars->full_x[s], C::kXBytes);
-                ptx::tma_load_2d(xs + s * C::kXBytes, &tmap_x, &bars->full_x[s], kb * kBK, (int32_t)m0);
+                ptx::tma_load_2d(xs + s * C::kXBytes, &tmap_x, &bars->full_x[s], (kb0 + kb) * kBK, (int32_t)m0);
                 issued++;
             }
             // no copy may still be in flight when the CTA exits
@@ -232,12 +239,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         constexpr int kAhead = 4;                           // k-blocks of bits loaded ahead
         uint2 wq[kAhead];
         uint16_t sq[kAhead];
-        auto load_kb = [&](int kb_, uint2 &wv_, uint16_t &sv_) {
+        auto load_kb = [&](int kbl, uint2 &wv_, uint16_t &sv_) {   // kbl: k-block of this CTA
+            const int kbg = kb0 + kbl;
             if (WPT == 1)
-                wv_ = make_uint2(__ldg(wrow + (size_t)kb_ * 2), 0u);
+                wv_ = make_uint2(__ldg(wrow + (size_t)kbg * 2), 0u);
             else
-                wv_ = __ldg(reinterpret_cast<const uint2 *>(wrow + (size_t)kb_ * 4));
-            sv_ = __ldg(srow + kb_ / 2);
+                wv_ = __ldg(reinterpret_cast<const uint2 *>(wrow + (size_t)kbg * 4));
+            sv_ = __ldg(srow + kbg / 2);
         };
 #pragma unroll
         for (int i = 0; i < kAhead; i++) {
@@ -307,6 +315,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
                 ptx::tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(quad * 32) << 16) + cc * 32, v);
                 ptx::tmem_wait_ld();
                 const int64_t mbase = m0 + cc * 32;
+                if (splits > 1) {
+                    // fp32 partial of this split: [tail tile][split][BN tokens][128 rows]
+                    float *pt = part + (((size_t)(tile - tile0) * splits + split) * BN + cc * 32) * kBM + quad * 32 + lane;
+#pragma unroll
+                    for (int j = 0; j < 32; j++)
+                        pt[(size_t)j * kBM] = __uint_as_float(v[j]);
+                    continue;
+                }
                 if (!nok)
                     continue;
 #pragma unroll
@@ -334,6 +350,75 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         ptx::tmem_dealloc(tmem_d, C::kTmemCols);
     }
 }
+
+// Y for the tiles that were split along K: the fp32 partials of each output added in split
+// order (so the result does not depend on timing), then rounded once to the output type.
+template <int BN>
+__global__ void __launch_bounds__(256)
+prefill_reduce_kernel(const float *__restrict__ part, int tiles, int splits, int tiles_m, int tile0, int64_t M,
+                      int64_t N, void *__restrict__ y, int yt)
+{
+    const int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x;   // (tail tile, token, row)
+    if (idx >= (int64_t)tiles * BN * kBM)
+        return;
+    const int t = (int)(idx / (BN * kBM)), mr = (int)(idx % (BN * kBM));
+    const int ml = mr / kBM, rl = mr % kBM;
+    const int tile = tile0 + t;
+    const int64_t m = (int64_t)(tile % tiles_m) * BN + ml, n = (int64_t)(tile / tiles_m) * kBM + rl;
+    if (m >= M || n >= N)
+        return;
+    const float *p = part + (size_t)t * splits * BN * kBM + mr;
+    float v = 0.f;
+    for (int sp = 0; sp < splits; sp++)
+        v += p[(size_t)sp * BN * kBM];
+    if (yt == BQ_F32)
+        store_out(static_cast<float *>(y) + m * N + n, v);
+    else if (yt == BQ_BF16)
+        store_out(static_cast<__nv_bfloat16 *>(y) + m * N + n, v);
+    else
+        store_out(static_cast<__half *>(y) + m * N + n, v);
+}
+
+int sm_count_pf()
+{
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+// Tile schedule: whole waves of one tile per CTA; when the last wave would be short (at most
+// half the SMs), its tiles are split along K over the idle SMs instead, and a reduce kernel
+// adds the splits. M = 512, N = 20480 at BN = 256: 320 tiles = 2 waves of 148 + 24 tiles,
+// which become 24 x 6 split CTAs instead of a third, mostly empty wave.
+struct PfPlan {
+    int tiles_m, tiles, full, tail, splits;
+};
+
+PfPlan pf_plan(int64_t M, int64_t N, int64_t K, int BN)
+{
+    PfPlan p;
+    p.tiles_m = (int)((M + BN - 1) / BN);
+    p.tiles = p.tiles_m * (int)((N + kBM - 1) / kBM);
+    const int sms = sm_count_pf();
+    const int waves = p.tiles / sms;
+    p.tail = p.tiles - waves * sms;
+    p.splits = 1;
+    if (waves >= 1 && p.tail > 0 && p.tail <= sms / 2) {
+        p.splits = sms / p.tail < 8 ? sms / p.tail : 8;
+        const int kblocks = (int)(K / kBK);          // every split gets at least 4 k-blocks
+        if (p.splits > kblocks / 4)
+            p.splits = kblocks / 4;
+        if (p.splits < 2)
+            p.splits = 1;
+    }
+    if (p.splits == 1)
+        p.tail = 0;
+    p.full = p.tiles - p.tail;
+    return p;
+}
+
+int bn_for(int64_t M) { return M <= 64 ? 64 : (M <= 128 ? 128 : 256); }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
@@ -374,33 +459,48 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmem);
     if (e != cudaSuccess)
         return e;
-    dim3 grid((unsigned)((a.M + BN - 1) / BN), (unsigned)((a.N + kBM - 1) / kBM));
-    kern<<<grid, kThreads, Cfg<BN>::kSmem, s>>>(map, a.words, reinterpret_cast<const uint16_t *>(a.scales), a.M,
-                                                a.N, a.K, a.y, a.yt, a.dev_status);
+    const PfPlan pl = pf_plan(a.M, a.N, a.K, BN);
+    const uint16_t *sc = reinterpret_cast<const uint16_t *>(a.scales);
+    float *part = static_cast<float *>(a.workspace);
+    kern<<<pl.full, kThreads, Cfg<BN>::kSmem, s>>>(map, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m, 0, 1,
+                                                   part, a.dev_status);
+    if (pl.tail > 0) {
+        kern<<<pl.tail * pl.splits, kThreads, Cfg<BN>::kSmem, s>>>(map, a.words, sc, a.M, a.N, a.K, a.y, a.yt,
+                                                                   pl.tiles_m, pl.full, pl.splits, part,
+                                                                   a.dev_status);
+        const int64_t n_out = (int64_t)pl.tail * BN * kBM;
+        prefill_reduce_kernel<BN><<<(unsigned)((n_out + 255) / 256), 256, 0, s>>>(
+            part, pl.tail, pl.splits, pl.tiles_m, pl.full, a.M, a.N, a.y, a.yt);
+    }
     return cudaGetLastError();
 }
 
 template <int FMT, bool BF16>
 cudaError_t launch_bn(const PrefillArgs &a, cudaStream_t s)
 {
-    if (a.M <= 64)
+    const int bn = bn_for(a.M);
+    if (bn == 64)
         return launch_t<FMT, 64, BF16>(a, s);
-    if (a.M <= 128)
+    if (bn == 128)
         return launch_t<FMT, 128, BF16>(a, s);
     return launch_t<FMT, 256, BF16>(a, s);
 }
 
 }  // namespace
 
+// fp32 partials of the split tail tiles (0 when the tiles fill whole waves or the last wave
+// is more than half full)
 size_t prefill_workspace_bytes(int64_t M, int fmt, int64_t N, int64_t K)
 {
-    (void)M; (void)fmt; (void)N; (void)K;
-    return 0;
+    (void)fmt;
+    const int bn = bn_for(M);
+    const PfPlan pl = pf_plan(M, N, K, bn);
+    return (size_t)pl.tail * pl.splits * bn * kBM * sizeof(float);
 }
 
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s, unsigned *launches)
 {
-    *launches = 1;
+    *launches = pf_plan(a.M, a.N, a.K, bn_for(a.M)).tail > 0 ? 3 : 1;
     const bool bf16 = a.xt == BQ_BF16;
     if (a.fmt == BQ_BINARY_G128)
         return bf16 ? launch_bn<BQ_BINARY_G128, true>(a, s) : launch_bn<BQ_BINARY_G128, false>(a, s);

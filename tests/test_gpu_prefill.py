@@ -61,6 +61,17 @@ def test_prefill_m512_k5120_n20480_sampled(orc, fmt):
     check(orc, fmt, 0, 512, 20480, 5120, rows=sample_rows(20480, 96, 5))
 
 
+@pytest.mark.parametrize("fmt,M", [(oracle.BINARY, 128), (oracle.TERNARY, 77)])
+def test_prefill_split_tail_rows(orc, fmt, M):
+    """160 tiles of 128 rows on 148 SMs: the 12 tiles past the full wave are split along K
+    (8 splits) and their fp32 partials added in order by a reduce pass. Every row of those
+    tiles is checked, plus a sample of the whole-K tiles."""
+    N, K = 20480, 2048
+    tail_rows = np.arange(148 * 128, N)
+    rows = np.unique(np.concatenate([tail_rows, sample_rows(148 * 128, 64, 7)]))
+    check(orc, fmt, 21, M, N, K, rows=rows)
+
+
 def test_prefill_fp16_is_exact_scale(orc):
     """With fp16 x the +-s operand is exact: the error is fp32 accumulation only."""
     r = check(orc, oracle.BINARY, 11, 256, 512, 2048, xdt=torch.float16)
