@@ -12,14 +12,16 @@
 //   * warp 0, one lane: TMA loads of the X tile [BN tokens x 64 k] per k-block into a ring
 //     of shared-memory stages (128-byte swizzle, zero fill past M); warp 0 also owns TMEM.
 //   * warps 2-9 (256 threads, two per weight row, each taking half of a k-block): read the
-//     row's packed bits and its group scale straight from global memory, expand each 8-weight
-//     chunk to +-s (binary) or {-s, 0, +s} (ternary) in the operand type through a 256-entry
-//     sign-mask table, and write the 128 x 64 A tile with tcgen05.st straight into tensor
-//     memory (a ring of A stages next to the accumulator), so no shared memory, no proxy
-//     fence, and more shared memory for the X ring. The scale is folded into the operand, so a
+//     row's packed bits and its group scale straight from global memory, expand every pair of
+//     weights to +-s (binary) or {-s, 0, +s} (ternary) in the operand type with a few integer
+//     or packed 16-bit float operations (expand_pairs), and write the 128 x 64 A tile with
+//     tcgen05.st straight into tensor memory (a ring of A stages next to the accumulator), so
+//     A needs no shared memory and no proxy fence. The scale is folded into the operand, so a
 //     group needs no separate rescaling: +-s is exact in fp16 and rounded to nearest even in
 //     bf16 (x's type decides). Per-CTA cycle counters showed the MMA issuer waiting on this
-//     step for more than half of its loop with four warps, one per row, writing shared memory.
+//     step for more than half of its loop while it wrote shared memory; with a 256-entry
+//     sign-mask table in shared memory the table's bank-conflicted lookups still held the
+//     load/store pipe at about 64% busy, next to the X tiles that the tensor cores read there.
 //   * warp 1, one lane: issues 4 tcgen05.mma (128 x BN x 16, A from tensor memory, X from
 //     shared memory) per k-block into the TMEM accumulator and commits each stage back to the
 //     producers.
@@ -27,7 +29,10 @@
 //     token; the two warps of a lane quarter take alternate 32-token blocks) and store Y with
 //     one coalesced 32-row segment per token.
 // Tiles fill whole waves of one tile per CTA; a short last wave is split along K over the idle
-// SMs (fp32 partials in the workspace, added in split order by prefill_reduce_kernel).
+// SMs (fp32 partials in the workspace, added in split order by prefill_reduce_kernel). The
+// split grid and the reduce are programmatic dependent launches: the split CTAs take SMs as
+// the whole-tile grid frees them, and each dependent grid completes only after its
+// predecessor, so the stream order seen by later work is unchanged.
 // The expanded weights exist only on chip. Every mbarrier wait is bounded: after
 // 2 s the kernel records kDevErrTimeout, lets its copies and MMAs drain, frees TMEM and
 // returns.
@@ -41,7 +46,9 @@ namespace {
 
 constexpr int kBM = 128;              // weight rows per tile (MMA M)
 constexpr int kBK = 64;               // k per stage: one 128-byte swizzle row of 16-bit values
-constexpr int kDequantWarps = 8;      // two per weight row: each expands half of a k-block
+constexpr int kDequantWarps = 8;      // kParts per weight row: each expands 1/kParts of a k-block
+                                      // (16 warps, four per row, measured slower)
+constexpr int kParts = kDequantWarps / 4;
 constexpr int kThreads = (2 + kDequantWarps) * 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -52,8 +59,7 @@ template <int BN> struct Cfg {
     static constexpr int kXStages = BN == 256 ? 6 : 8;
     static constexpr int kAStages = BN == 256 ? 6 : 8;
     static constexpr int kXBytes = BN * 128;          // X stage: BN rows x 128 B
-    static constexpr int kLutBytes = 256 * 16;
-    static constexpr int kBarOffset = kXStages * kXBytes + kLutBytes;
+    static constexpr int kBarOffset = kXStages * kXBytes;
     // barriers + alignment slack; at least 116 KB so that one CTA holds the SM (and all 512
     // tensor-memory columns)
     static constexpr int kSmemUsed = kBarOffset + 512 + 1024;
@@ -86,6 +92,58 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
+// Column c of a thread's A slice holds weights 2c (low half) and 2c+1 (high half) as +-s or
+// {-s, 0, +s} in the operand type; s2 is s in both halves. Plain ALU work, no table: the
+// shared-memory pipe stays with the X tiles that the tensor cores read.
+//   binary: the two sign bits of a pair are moved to bits 15 and 31 (a set bit means -s) and
+//     XORed into s2; for a 16-bit slice the odd bits are first lifted by 15, so that one shift
+//     per pair puts both in place.
+//   ternary: the two codes of a pair go to the low bits of the two halves of a 16-bit float
+//     whose exponent makes one unit of the last place 1 (1024 in fp16, 128 in bf16), then
+//     (1024 + c) - 1025 = c - 1 and (c - 1) * s are both exact. A code 3 (never written by the
+//     pack calls) gives +2s.
+template <int FMT, bool BF16, int COLS>
+__device__ __forceinline__ void expand_pairs(uint2 wv, uint32_t s2, uint32_t (&av)[COLS])
+{
+    if (FMT == BQ_BINARY_G128) {
+        const uint32_t nw = ~wv.x;
+#pragma unroll
+        for (int hh = 0; hh < COLS / 8; hh++) {
+            const uint32_t x = nw >> (16 * hh);
+            const uint32_t d = (x & 0x5555u) | ((x & 0xAAAAu) << 15);
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                av[8 * hh + j] = s2 ^ ((d << (15 - 2 * j)) & 0x80008000u);
+        }
+    } else {
+        constexpr uint32_t kMagic = BF16 ? 0x43004300u : 0x64006400u;      // 128 | 1024
+        constexpr uint32_t kMagic1 = BF16 ? 0x43014301u : 0x64016401u;     // 129 | 1025
+#pragma unroll
+        for (int wi = 0; wi < COLS / 8; wi++) {
+            const uint32_t w = wi ? wv.y : wv.x;
+            const uint32_t e = w & 0x33333333u, o = (w >> 2) & 0x33333333u;   // even / odd weights
+            const uint32_t p[2] = {__byte_perm(e, o, 0x5410), __byte_perm(e, o, 0x7632)};
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const uint32_t h = ((p[j >> 2] >> (4 * (j & 3))) & 0x00030003u) | kMagic;
+                uint32_t r;
+                if (BF16) {
+                    __nv_bfloat162 v = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&h),
+                                               *reinterpret_cast<const __nv_bfloat162 *>(&kMagic1));
+                    v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162 *>(&s2));
+                    r = *reinterpret_cast<const uint32_t *>(&v);
+                } else {
+                    __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&h),
+                                        *reinterpret_cast<const __half2 *>(&kMagic1));
+                    v = __hmul2(v, *reinterpret_cast<const __half2 *>(&s2));
+                    r = *reinterpret_cast<const uint32_t *>(&v);
+                }
+                av[8 * wi + j] = r;
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ uint32_t scale_pair(uint16_t s_f16, bool bf16)
 {
     uint16_t h = s_f16;
@@ -105,7 +163,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *xs = smem;                                         // SX x kXBytes
-    uint4 *lut = reinterpret_cast<uint4 *>(smem + SX * C::kXBytes);
     Bars *bars = reinterpret_cast<Bars *>(smem + C::kBarOffset);
     volatile int *abort = &bars->abort;
     unsigned int *err = dev_status + kSlotErrBits;
@@ -140,35 +197,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         ptx::tmem_alloc(&bars->tmem_base, C::kTmemCols);
         ptx::tmem_relinquish();
     }
-    if (warp >= 2) {
-        // sign-mask table: entry b describes the 8 (binary) or 4 (ternary) weights of byte b
-        for (int b = threadIdx.x - 64; b < 256; b += kDequantWarps * 32) {
-            uint32_t e[4];
-            if (FMT == BQ_BINARY_G128) {
-                for (int i = 0; i < 4; i++) {
-                    uint32_t lo = ((b >> (2 * i)) & 1) ? 0u : 0x8000u;        // bit 0 -> -s
-                    uint32_t hi = ((b >> (2 * i + 1)) & 1) ? 0u : 0x80000000u;
-                    e[i] = lo | hi;
-                }
-            } else {
-                uint32_t keep[2] = {0, 0}, sign[2] = {0, 0};
-                for (int i = 0; i < 4; i++) {
-                    uint32_t c = (b >> (2 * i)) & 3u;                        // 0:-1 1:0 2:+1 3:invalid
-                    uint32_t sh = 16 * (i & 1);
-                    if (c == 0u || c == 2u)
-                        keep[i >> 1] |= 0xFFFFu << sh;
-                    if (c == 0u)
-                        sign[i >> 1] |= 0x8000u << sh;
-                }
-                e[0] = keep[0]; e[1] = keep[1]; e[2] = sign[0]; e[3] = sign[1];
-            }
-            lut[b] = make_uint4(e[0], e[1], e[2], e[3]);
-        }
-    }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_d = bars->tmem_base;
+    // the split-tail launch that follows reads only X and the weights, never this grid's
+    // output, so it may start on each SM as soon as a CTA of this grid leaves it
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -225,16 +260,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         // warp w = 2 + 4 h + j, lane l: row 32 (w % 4) + l of the tile (a warp reaches only its
         // own quarter of the tensor-memory lanes), half h of every k-block (chunks 4h .. 4h+3 of
         // 8 weights: one binary word or two ternary words)
-        const int hk = (warp - 2) >> 2;
+        const int hk = (warp - 2) >> 2;                     // part of the k-block, 0 .. kParts-1
         const int r = 32 * (warp & 3) + lane;                // weight row within the tile
         const int64_t n = n0 + r;
         const bool row_ok = n < N;
         const int64_t G = K / 128;
-        constexpr int WPT = FMT == BQ_BINARY_G128 ? 1 : 2;   // words per thread per k-block
-        const uint32_t *wrow = words + (row_ok ? n : 0) * (K / 32 * (FMT == BQ_BINARY_G128 ? 1 : 2)) + hk * WPT;
+        constexpr int kWts = kBK / kParts;                   // weights per thread per k-block
+        constexpr int kChunks = kWts / 8, kCols = kWts / 2;  // 8-weight chunks, 32-bit TMEM columns
+        constexpr int kBitsPerW = FMT == BQ_BINARY_G128 ? 1 : 2;
+        constexpr int WPT = (kWts * kBitsPerW + 31) / 32;    // words per thread per k-block (1 or 2)
+        // the thread's first bit: word hk * kWts * bits / 32 of the k-block, shifted by the rest
+        const int bitpos = hk * kWts * kBitsPerW;
+        const int bshift = bitpos & 31;
+        const uint32_t *wrow = words + (row_ok ? n : 0) * (K / 32 * kBitsPerW) + (bitpos >> 5);
         const uint16_t *srow = scales + (row_ok ? n : 0) * G;
         // this thread's row in tensor memory: lane r (the warp's lane quarter), columns 16 hk ..
-        const uint32_t arow_tmem = tmem_d + ((uint32_t)(32 * (warp & 3)) << 16) + BN + 16 * hk;
+        const uint32_t arow_tmem = tmem_d + ((uint32_t)(32 * (warp & 3)) << 16) + BN + kCols * hk;
 
         constexpr int kAhead = 4;                           // k-blocks of bits loaded ahead
         uint2 wq[kAhead];
@@ -242,7 +283,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         auto load_kb = [&](int kbl, uint2 &wv_, uint16_t &sv_) {   // kbl: k-block of this CTA
             const int kbg = kb0 + kbl;
             if (WPT == 1)
-                wv_ = make_uint2(__ldg(wrow + (size_t)kbg * 2), 0u);
+                wv_ = make_uint2(__ldg(wrow + (size_t)kbg * 2 * kBitsPerW) >> bshift, 0u);
             else
                 wv_ = __ldg(reinterpret_cast<const uint2 *>(wrow + (size_t)kbg * 4));
             sv_ = __ldg(srow + kbg / 2);
@@ -273,28 +314,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
                 break;
             ptx::tc_fence_after();
             const uint32_t s2 = row_ok ? scale_pair(sv, BF16) : 0u;
-            const uint32_t wds[2] = {wv.x, wv.y};
-            uint32_t av[16];                                 // 32 weights: 2 per 32-bit column
+            uint32_t av[kCols];                              // 2 weights per 32-bit column
+            expand_pairs<FMT, BF16, kCols>(wv, s2, av);
+            if (!row_ok) {
 #pragma unroll
-            for (int cl = 0; cl < 4; cl++) {                 // this thread's 4 chunks of 8 weights
-                uint4 o;
-                if (FMT == BQ_BINARY_G128) {
-                    const uint32_t byte = (wds[0] >> (8 * cl)) & 0xFFu;
-                    const uint4 e = lut[byte];
-                    o = make_uint4(s2 ^ e.x, s2 ^ e.y, s2 ^ e.z, s2 ^ e.w);
-                } else {
-                    const uint32_t half16 = (wds[cl >> 1] >> (16 * (cl & 1))) & 0xFFFFu;
-                    const uint4 e0 = lut[half16 & 0xFFu], e1 = lut[half16 >> 8];
-                    o = make_uint4((s2 & e0.x) ^ e0.z, (s2 & e0.y) ^ e0.w, (s2 & e1.x) ^ e1.z, (s2 & e1.y) ^ e1.w);
-                }
-                if (!row_ok)
-                    o = make_uint4(0, 0, 0, 0);
-                av[4 * cl] = o.x;
-                av[4 * cl + 1] = o.y;
-                av[4 * cl + 2] = o.z;
-                av[4 * cl + 3] = o.w;
+                for (int c = 0; c < kCols; c++)
+                    av[c] = 0u;
             }
-            ptx::tmem_st_32x32b_x16(arow_tmem + 32 * s, av);
+            if constexpr (kCols == 16)
+                ptx::tmem_st_32x32b_x16(arow_tmem + 32 * s, *reinterpret_cast<const uint32_t(*)[16]>(av));
+            else
+                ptx::tmem_st_32x32b_x8(arow_tmem + 32 * s, *reinterpret_cast<const uint32_t(*)[8]>(av));
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -308,9 +338,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
             const int quad = warp & 3;                       // TMEM lanes 32*quad .. +31
             const int64_t nrow = n0 + quad * 32 + lane;
             const bool nok = nrow < N;
-            // the two warps of a lane quarter take alternate 32-token column blocks
+            // the kParts warps of a lane quarter take alternate 32-token column blocks
 #pragma unroll 1
-            for (int cc = hk; cc < BN / 32; cc += 2) {
+            for (int cc = hk; cc < BN / 32; cc += kParts) {
                 uint32_t v[32];
                 ptx::tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(quad * 32) << 16) + cc * 32, v);
                 ptx::tmem_wait_ld();
@@ -349,6 +379,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_d, C::kTmemCols);
     }
+    // launched as a dependent of the whole-tile grid, this grid completes only after that one
+    // has, so work queued behind it on the stream sees both (a no-op for an ordinary launch)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Y for the tiles that were split along K: the fp32 partials of each output added in split
@@ -358,6 +391,9 @@ __global__ void __launch_bounds__(256)
 prefill_reduce_kernel(const float *__restrict__ part, int tiles, int splits, int tiles_m, int tile0, int64_t M,
                       int64_t N, void *__restrict__ y, int yt)
 {
+    // launched as a dependent of the split grid: wait until that grid (and through it the
+    // whole-tile grid) has completed and its partials are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x;   // (tail tile, token, row)
     if (idx >= (int64_t)tiles * BN * kBM)
         return;
@@ -465,12 +501,35 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
     kern<<<pl.full, kThreads, Cfg<BN>::kSmem, s>>>(map, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m, 0, 1,
                                                    part, a.dev_status);
     if (pl.tail > 0) {
-        kern<<<pl.tail * pl.splits, kThreads, Cfg<BN>::kSmem, s>>>(map, a.words, sc, a.M, a.N, a.K, a.y, a.yt,
-                                                                   pl.tiles_m, pl.full, pl.splits, part,
-                                                                   a.dev_status);
+        // programmatic dependent launches: the tail CTAs take the SMs the whole-tile grid
+        // frees without waiting for all of it (the predecessor of the whole-tile grid, which
+        // may write X, is already complete when that grid runs), and the reduce is resident
+        // before the tail grid ends, waiting on it in griddepcontrol.wait
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(pl.tail * pl.splits));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = Cfg<BN>::kSmem;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, map, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m, pl.full, pl.splits,
+                               part, a.dev_status);
+        if (e != cudaSuccess)
+            return e;
         const int64_t n_out = (int64_t)pl.tail * BN * kBM;
-        prefill_reduce_kernel<BN><<<(unsigned)((n_out + 255) / 256), 256, 0, s>>>(
-            part, pl.tail, pl.splits, pl.tiles_m, pl.full, a.M, a.N, a.y, a.yt);
+        cudaLaunchConfig_t rcfg = {};
+        rcfg.gridDim = dim3((unsigned)((n_out + 255) / 256));
+        rcfg.blockDim = dim3(256);
+        rcfg.stream = s;
+        rcfg.attrs = attr;
+        rcfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&rcfg, prefill_reduce_kernel<BN>, (const float *)part, pl.tail, pl.splits, pl.tiles_m,
+                               pl.full, a.M, a.N, a.y, a.yt);
+        if (e != cudaSuccess)
+            return e;
     }
     return cudaGetLastError();
 }
