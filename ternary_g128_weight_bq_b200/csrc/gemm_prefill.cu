@@ -26,8 +26,10 @@
 //     shared memory) per k-block into the TMEM accumulator and commits each stage back to the
 //     producers.
 //   * warps 2-9 then read the accumulator with tcgen05.ld (lane = weight row, column =
-//     token; the two warps of a lane quarter take alternate 32-token blocks) and store Y with
-//     one coalesced 32-row segment per token.
+//     token; the two warps of a lane quarter take alternate 32-token blocks), convert to the
+//     output type into a [BN tokens][128 rows] tile in the (now idle) X ring, and one thread
+//     writes the tile with a TMA tensor store that clips at M and N. When a row of Y is not a
+//     whole number of 16-byte units, each warp stores its 32-row segments directly instead.
 // Tiles fill whole waves of one tile per CTA; a short last wave is split along K over the idle
 // SMs (fp32 partials in the workspace, added in split order by prefill_reduce_kernel). The
 // split grid and the reduce are programmatic dependent launches: the split CTAs take SMs as
@@ -37,6 +39,8 @@
 // 2 s the kernel records kDevErrTimeout, lets its copies and MMAs drain, frees TMEM and
 // returns.
 #include <cuda.h>
+
+#include <cstring>
 
 #include "bq_internal.cuh"
 #include "sm100_ptx.cuh"
@@ -65,6 +69,8 @@ template <int BN> struct Cfg {
     static constexpr int kSmemUsed = kBarOffset + 512 + 1024;
     static constexpr int kSmem = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
     static constexpr uint32_t kTmemCols = 512;
+    // the epilogue stages a [BN][128] output tile (at most fp32) in the X ring
+    static_assert(BN * kBM * 4 <= kXStages * kXBytes, "output staging tile exceeds the X ring");
 };
 
 struct Bars {
@@ -76,6 +82,7 @@ struct Bars {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    int staged;   // epilogue warps whose slice of the output tile is in shared memory
 };
 
 // Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast, then every lane
@@ -154,7 +161,8 @@ __device__ __forceinline__ uint32_t scale_pair(uint16_t s_f16, bool bf16)
 
 template <int FMT, int BN, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__restrict__ words,
+prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_y, int y_tma,
+               const uint32_t *__restrict__ words,
                const uint16_t *__restrict__ scales, int64_t M, int64_t N, int64_t K, void *__restrict__ y,
                int yt, int tiles_m, int tile0, int splits, float *__restrict__ part, unsigned int *dev_status)
 {
@@ -190,6 +198,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         ptx::mbar_init(&bars->acc_full, 1);
         ptx::mbar_init(&bars->drain, 1);
         bars->abort = 0;
+        bars->staged = 0;
         ptx::fence_barrier_init();
         ptx::tma_prefetch_desc(&tmap_x);
     }
@@ -266,7 +275,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         const bool row_ok = n < N;
         const int64_t G = K / 128;
         constexpr int kWts = kBK / kParts;                   // weights per thread per k-block
-        constexpr int kChunks = kWts / 8, kCols = kWts / 2;  // 8-weight chunks, 32-bit TMEM columns
+        constexpr int kCols = kWts / 2;                      // 32-bit TMEM columns per thread
         constexpr int kBitsPerW = FMT == BQ_BINARY_G128 ? 1 : 2;
         constexpr int WPT = (kWts * kBitsPerW + 31) / 32;    // words per thread per k-block (1 or 2)
         // the thread's first bit: word hk * kWts * bits / 32 of the k-block, shifted by the rest
@@ -333,6 +342,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
         }
 
         // ------------------------------------------------------------ epilogue
+        // Whole tiles whose output rows are 16-byte aligned go through shared memory (the X ring,
+        // idle once the last MMA has completed) and leave as one TMA tile store: [BN tokens][128
+        // rows] in the output type, clipped by the tensor map at M and N. Otherwise each warp
+        // stores its 32-row segments directly; split tiles store fp32 partials.
+        const bool staged_out = splits == 1 && y_tma;
         if (warp_wait(&bars->acc_full, 0, abort, err)) {
             ptx::tc_fence_after();
             const int quad = warp & 3;                       // TMEM lanes 32*quad .. +31
@@ -353,6 +367,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
                         pt[(size_t)j * kBM] = __uint_as_float(v[j]);
                     continue;
                 }
+                if (staged_out) {
+                    const int e0 = (cc * 32) * kBM + quad * 32 + lane;   // token cc*32, this row
+#pragma unroll
+                    for (int j = 0; j < 32; j++) {
+                        const float f = __uint_as_float(v[j]);
+                        if (yt == BQ_F32)
+                            store_out(reinterpret_cast<float *>(xs) + e0 + j * kBM, f);
+                        else if (yt == BQ_BF16)
+                            store_out(reinterpret_cast<__nv_bfloat16 *>(xs) + e0 + j * kBM, f);
+                        else
+                            store_out(reinterpret_cast<__half *>(xs) + e0 + j * kBM, f);
+                    }
+                    continue;
+                }
                 if (!nok)
                     continue;
 #pragma unroll
@@ -368,6 +396,21 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__res
                             store_out(static_cast<__half *>(y) + m * N + nrow, f);
                     }
                 }
+            }
+            if (staged_out) {
+                ptx::fence_proxy_async_smem();               // the tile store reads these writes
+                __syncwarp();
+                if (lane == 0)
+                    atomicAdd(&bars->staged, 1);
+            }
+        }
+        if (staged_out) {
+            // every epilogue warp passes here once, whatever its waits returned
+            asm volatile("bar.sync 1, %0;" ::"n"(kDequantWarps * 32) : "memory");
+            if (threadIdx.x == 64 && *reinterpret_cast<volatile int *>(&bars->staged) == kDequantWarps) {
+                ptx::tma_store_2d(&tmap_y, xs, (int32_t)n0, (int32_t)m0);
+                ptx::bulk_commit_group();
+                ptx::bulk_wait_all();
             }
         }
     }
@@ -491,6 +534,23 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    // Y as [M][N] in the output type, stored in [BN tokens][128 rows] boxes; usable when a row
+    // of Y is a whole number of 16-byte units (the tensor map's stride rule)
+    CUtensorMap map_y;
+    std::memset(&map_y, 0, sizeof(map_y));
+    const int esize = a.yt == BQ_F32 ? 4 : 2;
+    int y_tma = 0;
+    if ((a.N * esize) % 16 == 0) {
+        cuuint64_t ydims[2] = {(cuuint64_t)a.N, (cuuint64_t)a.M};
+        cuuint64_t ystrides[1] = {(cuuint64_t)a.N * esize};
+        cuuint32_t ybox[2] = {(cuuint32_t)kBM, (cuuint32_t)BN};
+        const CUtensorMapDataType yd = a.yt == BQ_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                       : a.yt == BQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+        y_tma = enc(&map_y, yd, 2, a.y, ydims, ystrides, ybox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
     auto kern = prefill_kernel<FMT, BN, BF16>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmem);
     if (e != cudaSuccess)
@@ -498,8 +558,8 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
     const PfPlan pl = pf_plan(a.M, a.N, a.K, BN);
     const uint16_t *sc = reinterpret_cast<const uint16_t *>(a.scales);
     float *part = static_cast<float *>(a.workspace);
-    kern<<<pl.full, kThreads, Cfg<BN>::kSmem, s>>>(map, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m, 0, 1,
-                                                   part, a.dev_status);
+    kern<<<pl.full, kThreads, Cfg<BN>::kSmem, s>>>(map, map_y, y_tma, a.words, sc, a.M, a.N, a.K, a.y, a.yt,
+                                                   pl.tiles_m, 0, 1, part, a.dev_status);
     if (pl.tail > 0) {
         // programmatic dependent launches: the tail CTAs take the SMs the whole-tile grid
         // frees without waiting for all of it (the predecessor of the whole-tile grid, which
@@ -515,8 +575,8 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
         cfg.stream = s;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, kern, map, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m, pl.full, pl.splits,
-                               part, a.dev_status);
+        e = cudaLaunchKernelEx(&cfg, kern, map, map_y, y_tma, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m,
+                               pl.full, pl.splits, part, a.dev_status);
         if (e != cudaSuccess)
             return e;
         const int64_t n_out = (int64_t)pl.tail * BN * kBM;

@@ -56,6 +56,15 @@ def test_prefill_dtypes(orc, xdt, ydt):
     check(orc, oracle.BINARY, 9, 200, 256, 1024, xdt=xdt, ydt=ydt)
 
 
+@pytest.mark.parametrize("N,ydt", [(1000, torch.bfloat16), (1000, torch.float16), (300, torch.bfloat16),
+                                   (129, torch.float32), (392, torch.float32)])
+def test_prefill_output_store_paths(orc, N, ydt):
+    """Rows of Y that are a whole number of 16-byte units leave each tile as one tensor-map
+    store clipped at M and N (N = 1000, 392); other widths take per-row stores (N = 300 in a
+    16-bit type, N = 129 in fp32). Ragged M = 77 clips the token side of the box."""
+    check(orc, oracle.BINARY, 31, 77, N, 512, ydt=ydt)
+
+
 @pytest.mark.parametrize("fmt", [oracle.BINARY, oracle.TERNARY])
 def test_prefill_m512_k5120_n20480_sampled(orc, fmt):
     check(orc, fmt, 0, 512, 20480, 5120, rows=sample_rows(20480, 96, 5))
