@@ -170,9 +170,10 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
 /*
  * Prefill GEMM: the same product for M up to 512 token rows (larger M is accepted),
  * Y[M][N] = X[M][K] * W^T with W the dequantised +-s (binary) or {-s, 0, +s} (ternary)
- * matrix. The packed tiles are unpacked into shared memory next to the tensor cores
- * (tcgen05, accumulation in fp32 in tensor memory); no expanded copy is written to device
- * memory. The pp512 (512-token prompt, compute-bound) workload of the model card's section
+ * matrix. The packed bits are expanded on chip, straight into tensor memory, as the A
+ * operand of the tensor cores (tcgen05, accumulation in fp32 in tensor memory); no expanded
+ * copy is written to device memory. One call is one kernel launch, or three when the tail of
+ * the output tiles is split along K (the split grid and a reduce pass). The pp512 (512-token prompt, compute-bound) workload of the model card's section
  * "Cross-platform throughput" and of the Ternary Bonsai 27B article's throughput table.
  *   x  [M][K], xt = BQ_F16 or BQ_BF16. The scale is applied inside the operand, rounded to
  *      x's type (exact for BQ_F16; bf16 keeps 8 of the scale's 11 significant bits).
