@@ -84,10 +84,10 @@ def test_prefill_split_tail_rows(orc, fmt, M):
 @pytest.mark.parametrize("fmt", [oracle.BINARY, oracle.TERNARY])
 def test_prefill_m512_split_tail_rows(orc, fmt):
     """M = 512 at BN = 256: 320 tiles of 128 rows on 148 SMs, the 24 past the second full
-    wave split along K and reduced. Every row of the last 4096 (which hold all split tiles)
-    is checked, plus a sample of the whole-K rows."""
+    wave (rows 18944 .. 20479, both token tiles) split along K and reduced. Every one of
+    those rows is checked, plus a sample of the whole-K rows."""
     N, K = 20480, 2048
-    tail_rows = np.arange(N - 16 * 256, N)
+    tail_rows = np.arange(148 * 128, N)
     rows = np.unique(np.concatenate([tail_rows, sample_rows(N - 16 * 256, 64, 8)]))
     check(orc, fmt, 23, 512, N, K, rows=rows)
 
