@@ -337,7 +337,7 @@ def full_depth_step(bq, device, stream, peaks):
 
 def stage_step_io(layer, device, pin):
     """One device buffer for the six x of a step and one for the six y, with the GEMV operands
-    as views into them, plus host twins made by `pin` (pinned memory on a GPU machine), so a step
+    as views into them, plus host twins made by `pin` (pinned host memory in the bench), so a step
     moves its inputs and its results with one copy each way. Returns (x_dev, y_dev, x_host,
     y_host, [(w, x_view, y_view)]). Every view starts at a multiple of 16 bytes."""
     nx = [x.numel() for (_, x, _) in layer]
