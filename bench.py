@@ -392,7 +392,7 @@ def e2e_gemv(bq, device, steps, warmup, stream):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 5)}
 
 
-GEMV_SOURCES = ("gemv_tc.cu", "gemv_tmem.cu")
+GEMV_SOURCES = ("gemv_rows.cu", "gemv_mma.cuh")
 
 
 def gemv_source_sha() -> str:

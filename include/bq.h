@@ -130,12 +130,19 @@ bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStr
  * Model card "prism-ml/Bonsai-27B-mlx-1bit", sections "Weight representation: Binary g128"
  * and "CUDA (NVIDIA GPUs)"; the decode (tg128) workload of section "Cross-platform
  * throughput".
- *   x          [M][K], xt = BQ_F16 or BQ_BF16
+ *   x          [M][K], xt = BQ_F16 or BQ_BF16. A token row that holds an infinity or a NaN
+ *              gets non-finite outputs (NaN where K is a multiple of 1024, where the kernels
+ *              carry x as integer digits per group; +-inf or NaN otherwise).
  *   M          1..8
  *   y          [M][N], yt = BQ_F32, BQ_BF16 or BQ_F16 (fp32 accumulation, rounded once)
  *   workspace  device scratch of at least bq_gemv_workspace_bytes(M, w) bytes (may be
- *              NULL when that size is 0); its contents need not be initialised and are
- *              left undefined. Calls that share a workspace must be ordered on one stream.
+ *              NULL when that size is 0): the digit fragments of x that a prep kernel writes
+ *              once per call (1 KB per 128 inputs and per two tokens, plus factors). Its
+ *              contents need not be initialised and are left undefined. Calls that share a
+ *              workspace must be ordered on one stream.
+ * Launches: two kernels (the prep and the GEMV, both programmatic dependent launches) when K
+ * is a multiple of 1024 and the fragments fit in shared memory (K <= 5120 at M = 8, K <= 20480
+ * at M = 1); otherwise one SIMT kernel.
  */
 bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w,
                   void *y, bq_dtype yt, void *workspace, size_t ws_bytes, cudaStream_t stream);
@@ -153,9 +160,10 @@ size_t bq_gemv_workspace_bytes(int64_t M, const bq_weight *w);
  *   - a decode loop that must not call cudaMalloc or cudaFree between steps, since those
  *     calls can synchronise the device and stall the queued work;
  *   - plain C hosts that do not want to size, own and free a buffer per weight shape.
- * Limit: the array is 1.56 MB per device, enough for every M <= 8 and every K on a device
- * with up to 160 SMs; a shape that needs more returns BQ_ERR_WORKSPACE with the two sizes in
- * bq_last_error(), and bq_gemv with a workspace then serves it.
+ * Limit: the array is 256 KB per device. It holds the digit fragments of x that this GEMV
+ * keeps in scratch, which by construction fit in one CTA's shared memory, so every shape the
+ * tensor-core path takes fits; a shape that needs more returns BQ_ERR_WORKSPACE with the two
+ * sizes in bq_last_error(), and bq_gemv with a workspace then serves it.
  * Set-up: the first call on each device (with that device current) resolves the array's
  * address; make that first call before any stream capture. Later calls do no set-up.
  * Sharing: all calls on a device share the one array. Nothing in it needs an initial value
@@ -172,17 +180,26 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
  * Y[M][N] = X[M][K] * W^T with W the dequantised +-s (binary) or {-s, 0, +s} (ternary)
  * matrix. The packed bits are expanded on chip, straight into tensor memory, as the A
  * operand of the tensor cores (tcgen05, accumulation in fp32 in tensor memory); no expanded
- * copy is written to device memory. One call is one kernel launch, or three when the tail of
- * the output tiles is split along K (the split grid and a reduce pass). The pp512 (512-token prompt, compute-bound) workload of the model card's section
- * "Cross-platform throughput" and of the Ternary Bonsai 27B article's throughput table.
- *   x  [M][K], xt = BQ_F16 or BQ_BF16. The scale is applied inside the operand, rounded to
- *      x's type (exact for BQ_F16; bf16 keeps 8 of the scale's 11 significant bits).
+ * copy is written to device memory. The pp512 (512-token prompt, compute-bound) workload of
+ * the model card's section "Cross-platform throughput" and of the Ternary Bonsai 27B
+ * article's throughput table.
+ *   x  [M][K], xt = BQ_F16 or BQ_BF16. The tensor-core operands are always fp16: the weight
+ *      operand is +-s (or 0) in fp16, which holds every fp16 scale exactly. fp16 x is used as
+ *      it is. bf16 x is first copied into the workspace as fp16 x * 2^e, with one power of two
+ *      per token row that puts the row's largest finite |x| in [2^14, 2^15); the fp32 results
+ *      are multiplied by 2^-e (exact). Every bf16 element within a factor 2^31 of its row's
+ *      largest magnitude is carried exactly; smaller ones are rounded to fp16's subnormal
+ *      spacing, an error of at most 2^-39 of the row's largest magnitude. Infinities and NaNs
+ *      stay non-finite.
  *   y  [M][N], yt = BQ_F32, BQ_BF16 or BQ_F16.
- *   workspace: at least bq_gemm_prefill_workspace_bytes(M, w) bytes, 16-byte aligned (may be
- *      NULL when that size is 0). It holds fp32 partial sums when the last wave of output tiles
- *      would leave most SMs idle and its tiles are split along K instead (for example M = 512,
- *      N = 20480: 18.9 MB). Contents need not be initialised; calls that share a workspace
- *      must be ordered on one stream.
+ *   workspace: at least bq_gemm_prefill_workspace_bytes(M, w) bytes, 16-byte aligned. It holds
+ *      the fp16 copy of bf16 x (M*K*2 bytes, reserved for either x type) with its M factors,
+ *      and fp32 partial sums when the last wave of output tiles would leave most SMs idle and
+ *      its tiles are split along K instead (for example M = 512, N = 20480: 18.9 MB of
+ *      partials). Contents need not be initialised; calls that share a workspace must be
+ *      ordered on one stream.
+ * Launches: one kernel, plus the conversion pass for bf16 x, plus two (the split grid and a
+ * reduce pass) when the tail of the output tiles is split along K.
  */
 bq_status bq_gemm_prefill(const void *x, bq_dtype xt, int64_t M, const bq_weight *w,
                           void *y, bq_dtype yt, void *workspace, size_t ws_bytes,

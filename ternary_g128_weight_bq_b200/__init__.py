@@ -98,6 +98,34 @@ def _dev(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _same_device(name: str, t: torch.Tensor, ref: torch.Tensor):
+    if t.device != ref.device:
+        raise ValueError(f"{name} is on {t.device}, expected {ref.device}")
+
+
+def _out(out, shape, dtype, x: torch.Tensor, w) -> torch.Tensor:
+    """The caller's output tensor, checked (shape, dtype, device), or a new one."""
+    if out is None:
+        return torch.empty(shape, dtype=dtype, device=x.device)
+    _dev(out, "out")
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"out must have shape {tuple(shape)}, got {tuple(out.shape)}")
+    if out.dtype not in _DTYPE:
+        raise ValueError(f"out dtype {out.dtype} is not supported")
+    _same_device("out", out, x)
+    return out
+
+
+def _operands(x: torch.Tensor, w) -> None:
+    _dev(x, "x")
+    if x.dim() != 2 or x.shape[1] != w.K:
+        raise ValueError(f"x must be [M, {w.K}]")
+    if x.dtype not in _DTYPE:
+        raise ValueError(f"x dtype {x.dtype} is not supported")
+    _same_device("weight words", w.words, x)
+    _same_device("weight scales", w.scales, x)
+
+
 @dataclass
 class BQWeight:
     """A packed weight matrix held in device memory.
@@ -184,20 +212,20 @@ def gemv_workspace_bytes(M: int, w: BQWeight) -> int:
 def gemv(x: torch.Tensor, w: BQWeight, out_dtype=torch.float32, out: torch.Tensor = None,
          workspace: torch.Tensor = None) -> torch.Tensor:
     """Decode GEMV: y[M, N] = x[M, K] @ W^T for M <= 8 (fp32 accumulation)."""
-    _dev(x, "x")
-    if x.dim() != 2 or x.shape[1] != w.K:
-        raise ValueError(f"x must be [M, {w.K}]")
+    _operands(x, w)
     M = x.shape[0]
-    if out is None:
-        out = torch.empty((M, w.N), dtype=out_dtype, device=x.device)
-    _dev(out, "out")
+    out = _out(out, (M, w.N), out_dtype, x, w)
     need = gemv_workspace_bytes(M, w)
+    if workspace is not None:
+        _dev(workspace, "workspace")
+        _same_device("workspace", workspace, x)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(lib().bq_gemv(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(), _DTYPE[out.dtype],
-                         ws_ptr, ws_bytes, _stream(x.device)))
+    with torch.cuda.device(x.device):
+        _check(lib().bq_gemv(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(), _DTYPE[out.dtype],
+                             ws_ptr, ws_bytes, _stream(x.device)))
     return out
 
 
@@ -205,33 +233,36 @@ def gemv_noalloc(x: torch.Tensor, w: BQWeight, out_dtype=torch.float32,
                  out: torch.Tensor = None) -> torch.Tensor:
     """gemv with the library's fixed scratch array instead of a workspace (no device
     allocation inside the call; calls on one device must not overlap)."""
-    _dev(x, "x")
-    if x.dim() != 2 or x.shape[1] != w.K:
-        raise ValueError(f"x must be [M, {w.K}]")
+    _operands(x, w)
     M = x.shape[0]
-    if out is None:
-        out = torch.empty((M, w.N), dtype=out_dtype, device=x.device)
-    _dev(out, "out")
-    _check(lib().bq_gemv_noalloc(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(),
-                                 _DTYPE[out.dtype], _stream(x.device)))
+    out = _out(out, (M, w.N), out_dtype, x, w)
+    with torch.cuda.device(x.device):
+        _check(lib().bq_gemv_noalloc(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(),
+                                     _DTYPE[out.dtype], _stream(x.device)))
     return out
 
 
+def prefill_workspace_bytes(M: int, w: BQWeight) -> int:
+    return int(lib().bq_gemm_prefill_workspace_bytes(M, w.c))
+
+
 def gemm_prefill(x: torch.Tensor, w: BQWeight, out_dtype=torch.float32,
-                 out: torch.Tensor = None) -> torch.Tensor:
+                 out: torch.Tensor = None, workspace: torch.Tensor = None) -> torch.Tensor:
     """Prefill GEMM: Y[M, N] = X[M, K] @ W^T on the tensor cores (fp32 accumulation)."""
-    _dev(x, "x")
-    if x.dim() != 2 or x.shape[1] != w.K:
-        raise ValueError(f"x must be [M, {w.K}]")
+    _operands(x, w)
     M = x.shape[0]
-    if out is None:
-        out = torch.empty((M, w.N), dtype=out_dtype, device=x.device)
-    _dev(out, "out")
-    need = int(lib().bq_gemm_prefill_workspace_bytes(M, w.c))
-    ws = torch.empty(need, dtype=torch.uint8, device=x.device) if need else None
-    _check(lib().bq_gemm_prefill(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(),
-                                 _DTYPE[out.dtype], ws.data_ptr() if ws is not None else None,
-                                 need, _stream(x.device)))
+    out = _out(out, (M, w.N), out_dtype, x, w)
+    need = prefill_workspace_bytes(M, w)
+    if workspace is not None:
+        _dev(workspace, "workspace")
+        _same_device("workspace", workspace, x)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(x.device):
+        _check(lib().bq_gemm_prefill(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(),
+                                     _DTYPE[out.dtype], ws_ptr, ws_bytes, _stream(x.device)))
     return out
 
 
@@ -242,11 +273,12 @@ def embed_gather(ids: torch.Tensor, w: BQWeight, out_dtype=torch.bfloat16,
     if ids.dtype != torch.int32 or ids.dim() != 1:
         raise ValueError("ids must be int32 [T]")
     T = ids.shape[0]
-    if out is None:
-        out = torch.empty((T, w.K), dtype=out_dtype, device=ids.device)
-    _dev(out, "out")
-    _check(lib().bq_embed_gather(ids.data_ptr(), T, w.c, out.data_ptr(), _DTYPE[out.dtype],
-                                 _stream(ids.device)))
+    _same_device("weight words", w.words, ids)
+    _same_device("weight scales", w.scales, ids)
+    out = _out(out, (T, w.K), out_dtype, ids, w)
+    with torch.cuda.device(ids.device):
+        _check(lib().bq_embed_gather(ids.data_ptr(), T, w.c, out.data_ptr(), _DTYPE[out.dtype],
+                                     _stream(ids.device)))
     return out
 
 

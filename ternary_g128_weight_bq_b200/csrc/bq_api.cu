@@ -4,6 +4,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "bq_internal.cuh"
 
 namespace bq {
@@ -35,6 +37,11 @@ bq_status check_launch(const char *what)
 }
 
 static constexpr int kMaxDevices = 64;
+// Per-device cache of the architecture check and of the status array's device address,
+// filled on the first call on each device under g_status_mu (host threads may make their
+// first calls concurrently). The addresses belong to the device's primary context: after a
+// cudaDeviceReset the library must be reloaded.
+static std::mutex g_status_mu;
 static unsigned int *g_status_ptr[kMaxDevices];
 static bool g_checked_arch[kMaxDevices];
 
@@ -46,6 +53,7 @@ unsigned int *device_status(bq_status *st)
         *st = set_error(BQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
         return nullptr;
     }
+    std::lock_guard<std::mutex> lock(g_status_mu);
     if (!g_checked_arch[dev]) {
         int major = 0, minor = 0;
         cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);

@@ -54,18 +54,14 @@ struct GemvArgs {
     unsigned int *dev_status;
 };
 size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
-// integer tensor-core path (gemv_tc.cu): K a multiple of 1024
-bool gemv_tc_supported(int M, int fmt, int64_t K);
-size_t gemv_tc_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
-cudaError_t launch_gemv_tc(const GemvArgs &a, cudaStream_t s);
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches);
-// tcgen05 path with the sign operand in tensor memory (gemv_tmem.cu): binary with 5 <= M <= 8,
-// ternary with any M <= 8; K a multiple of 1024
-bool gemv_tmem_supported(int M, int fmt, int64_t K);
-size_t gemv_tmem_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
-cudaError_t launch_gemv_tmem(const GemvArgs &a, cudaStream_t s);
+// integer tensor-core path, whole output rows per CTA (gemv_rows.cu): K a multiple of 1024 and
+// the digit fragments of all of K in shared memory
+bool gemv_rows_supported(int M, int fmt, int64_t N, int64_t K);
+size_t gemv_rows_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
+cudaError_t launch_gemv_rows(const GemvArgs &a, cudaStream_t s, unsigned *launches);
 // Device address and size of the fixed scratch array of bq_gemv_noalloc on the current
-// device (gemv_tc.cu); resolved once per device.
+// device (gemv_rows.cu); resolved once per device.
 cudaError_t gemv_static_scratch(void **ptr, size_t *bytes);
 
 struct PrefillArgs {

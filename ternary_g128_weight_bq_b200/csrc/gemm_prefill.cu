@@ -17,8 +17,10 @@
 //     or packed 16-bit float operations (expand_pairs), and write the 128 x 64 A tile with
 //     tcgen05.st straight into tensor memory (a ring of A stages next to the accumulator), so
 //     A needs no shared memory and no proxy fence. The scale is folded into the operand, so a
-//     group needs no separate rescaling: +-s is exact in fp16 and rounded to nearest even in
-//     bf16 (x's type decides). Per-CTA cycle counters showed the MMA issuer waiting on this
+//     group needs no separate rescaling. The operand type is always fp16, where +-s is exact
+//     (an fp16 scale has 11 significant bits; bf16 would keep 8, a relative error of up to
+//     2^-8 per weight, about twice the 2e-3 sum|x s| tolerance when every term errs the same
+//     way). Per-CTA cycle counters showed the MMA issuer waiting on this
 //     step for more than half of its loop while it wrote shared memory; with a 256-entry
 //     sign-mask table in shared memory the table's bank-conflicted lookups still held the
 //     load/store pipe at about 64% busy, next to the X tiles that the tensor cores read there.
@@ -30,6 +32,12 @@
 //     output type into a [BN tokens][128 rows] tile in the (now idle) X ring, and one thread
 //     writes the tile with a TMA tensor store that clips at M and N. When a row of Y is not a
 //     whole number of 16-byte units, each warp stores its 32-row segments directly instead.
+// bf16 x: a conversion pass (prefill_x16_kernel) first writes x * 2^e_m as fp16 into the
+// workspace, e_m a power of two per token row that puts the row's largest finite magnitude in
+// [2^14, 2^15). A bf16 value has 8 significant bits, so every element within 2^31 of its row's
+// largest magnitude is exact in fp16; smaller ones round to fp16's subnormal spacing (error at
+// most 2^-39 of the row's largest magnitude). The epilogue (and the split-tail reduce)
+// multiplies each token's fp32 result by 2^-e_m, which is exact.
 // Tiles fill whole waves of one tile per CTA; a short last wave is split along K over the idle
 // SMs (fp32 partials in the workspace, added in split order by prefill_reduce_kernel). The
 // split grid and the reduce are programmatic dependent launches: the split CTAs take SMs as
@@ -100,16 +108,15 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // Column c of a thread's A slice holds weights 2c (low half) and 2c+1 (high half) as +-s or
-// {-s, 0, +s} in the operand type; s2 is s in both halves. Plain ALU work, no table: the
-// shared-memory pipe stays with the X tiles that the tensor cores read.
+// {-s, 0, +s} in fp16; s2 is s in both halves. Plain ALU work, no table: the shared-memory
+// pipe stays with the X tiles that the tensor cores read.
 //   binary: the two sign bits of a pair are moved to bits 15 and 31 (a set bit means -s) and
 //     XORed into s2; for a 16-bit slice the odd bits are first lifted by 15, so that one shift
 //     per pair puts both in place.
-//   ternary: the two codes of a pair go to the low bits of the two halves of a 16-bit float
-//     whose exponent makes one unit of the last place 1 (1024 in fp16, 128 in bf16), then
-//     (1024 + c) - 1025 = c - 1 and (c - 1) * s are both exact. A code 3 (never written by the
-//     pack calls) gives +2s.
-template <int FMT, bool BF16, int COLS>
+//   ternary: the two codes of a pair go to the low bits of the two halves of the fp16 value
+//     1024, where one unit of the last place is 1; then (1024 + c) - 1025 = c - 1 and
+//     (c - 1) * s are both exact. A code 3 (never written by the pack calls) gives +2s.
+template <int FMT, int COLS>
 __device__ __forceinline__ void expand_pairs(uint2 wv, uint32_t s2, uint32_t (&av)[COLS])
 {
     if (FMT == BQ_BINARY_G128) {
@@ -123,8 +130,8 @@ __device__ __forceinline__ void expand_pairs(uint2 wv, uint32_t s2, uint32_t (&a
                 av[8 * hh + j] = s2 ^ ((d << (15 - 2 * j)) & 0x80008000u);
         }
     } else {
-        constexpr uint32_t kMagic = BF16 ? 0x43004300u : 0x64006400u;      // 128 | 1024
-        constexpr uint32_t kMagic1 = BF16 ? 0x43014301u : 0x64016401u;     // 129 | 1025
+        constexpr uint32_t kMagic = 0x64006400u;                           // 1024 | 1024
+        constexpr uint32_t kMagic1 = 0x64016401u;                          // 1025 | 1025
 #pragma unroll
         for (int wi = 0; wi < COLS / 8; wi++) {
             const uint32_t w = wi ? wv.y : wv.x;
@@ -133,38 +140,106 @@ __device__ __forceinline__ void expand_pairs(uint2 wv, uint32_t s2, uint32_t (&a
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 const uint32_t h = ((p[j >> 2] >> (4 * (j & 3))) & 0x00030003u) | kMagic;
-                uint32_t r;
-                if (BF16) {
-                    __nv_bfloat162 v = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&h),
-                                               *reinterpret_cast<const __nv_bfloat162 *>(&kMagic1));
-                    v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162 *>(&s2));
-                    r = *reinterpret_cast<const uint32_t *>(&v);
-                } else {
-                    __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&h),
-                                        *reinterpret_cast<const __half2 *>(&kMagic1));
-                    v = __hmul2(v, *reinterpret_cast<const __half2 *>(&s2));
-                    r = *reinterpret_cast<const uint32_t *>(&v);
-                }
-                av[8 * wi + j] = r;
+                __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&h),
+                                    *reinterpret_cast<const __half2 *>(&kMagic1));
+                v = __hmul2(v, *reinterpret_cast<const __half2 *>(&s2));
+                av[8 * wi + j] = *reinterpret_cast<const uint32_t *>(&v);
             }
         }
     }
 }
 
-__device__ __forceinline__ uint32_t scale_pair(uint16_t s_f16, bool bf16)
+__device__ __forceinline__ uint32_t scale_pair(uint16_t s_f16) { return (uint32_t)s_f16 | ((uint32_t)s_f16 << 16); }
+
+// bf16 x -> fp16 x * 2^e_m, one block per token row m: e_m puts the row's largest finite
+// magnitude in [2^14, 2^15) (e_m = 0 for a row with no finite non-zero value), and tok_fac[m]
+// = 2^-e_m undoes it on the fp32 results. Non-finite values stay non-finite. K is a multiple
+// of 128, so every thread moves whole 16-byte chunks of 8 values.
+constexpr int kX16Threads = 256;
+
+__global__ void __launch_bounds__(kX16Threads)
+prefill_x16_kernel(const __nv_bfloat16 *__restrict__ x, int64_t K, __half *__restrict__ x16,
+                   float *__restrict__ tok_fac)
 {
-    uint16_t h = s_f16;
-    if (bf16)
-        h = __bfloat16_as_ushort(__float2bfloat16_rn(__half2float(__ushort_as_half(s_f16))));
-    return (uint32_t)h | ((uint32_t)h << 16);
+    // the GEMM grid may set itself up meanwhile; it waits for this grid before reading x16
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ float wmax[kX16Threads / 32];
+    const int64_t m = blockIdx.x;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + m * K);
+    uint4 *dst = reinterpret_cast<uint4 *>(x16 + m * K);
+    const int chunks = (int)(K / 8);
+    // rows up to kHeld chunks per thread (K <= 8192) are read once and kept in registers
+    constexpr int kHeld = 4;
+    uint4 held[kHeld];
+    float amax = 0.f;
+    auto absmax = [&](const uint4 &v) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+            if (isfinite(f.x))
+                amax = fmaxf(amax, fabsf(f.x));
+            if (isfinite(f.y))
+                amax = fmaxf(amax, fabsf(f.y));
+        }
+    };
+#pragma unroll
+    for (int j = 0; j < kHeld; j++) {
+        const int c = threadIdx.x + j * kX16Threads;
+        held[j] = c < chunks ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < kHeld; j++)
+        absmax(held[j]);
+    for (int c = threadIdx.x + kHeld * kX16Threads; c < chunks; c += kX16Threads)
+        absmax(__ldg(src + c));
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0)
+        wmax[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = wmax[0];
+#pragma unroll
+    for (int i = 1; i < kX16Threads / 32; i++)
+        amax = fmaxf(amax, wmax[i]);
+    int e = 0;
+    if (amax > 0.f) {
+        int ex;
+        frexpf(amax, &ex);                 // amax = f 2^ex, f in [0.5, 1)
+        e = 15 - ex;                       // amax 2^e in [2^14, 2^15)
+    }
+    auto convert = [&](const uint4 &v) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+            const __half2 h = __halves2half2(__float2half_rn(ldexpf(f.x, e)), __float2half_rn(ldexpf(f.y, e)));
+            o[i] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        return make_uint4(o[0], o[1], o[2], o[3]);
+    };
+#pragma unroll
+    for (int j = 0; j < kHeld; j++) {
+        const int c = threadIdx.x + j * kX16Threads;
+        if (c < chunks)
+            dst[c] = convert(held[j]);
+    }
+    for (int c = threadIdx.x + kHeld * kX16Threads; c < chunks; c += kX16Threads)
+        dst[c] = convert(__ldg(src + c));
+    if (threadIdx.x == 0)
+        tok_fac[m] = ldexpf(1.f, -e);      // exact: -e is in [-147, 113]
 }
 
-template <int FMT, int BN, bool BF16>
+// tok_fac: the per-token factor 2^-e_m of bf16 x (NULL for fp16 x, which is used as it is).
+template <int FMT, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_y, int y_tma,
                const uint32_t *__restrict__ words,
                const uint16_t *__restrict__ scales, int64_t M, int64_t N, int64_t K, void *__restrict__ y,
-               int yt, int tiles_m, int tile0, int splits, float *__restrict__ part, unsigned int *dev_status)
+               int yt, int tiles_m, int tile0, int splits, float *__restrict__ part,
+               const float *__restrict__ tok_fac, unsigned int *dev_status)
 {
     using C = Cfg<BN>;
     constexpr int SX = C::kXStages, SA = C::kAStages;
@@ -210,13 +285,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_d = bars->tmem_base;
-    // the split-tail launch that follows reads only X and the weights, never this grid's
-    // output, so it may start on each SM as soon as a CTA of this grid leaves it
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // The split-tail grid (and, after it, the reduce) reads only X and the weights, never this
+    // grid's output, so it may start on each SM as soon as a CTA of this grid leaves it. The
+    // whole-tile grid of a bf16-x call is itself a dependent of the conversion pass: there only
+    // the TMA producer (which reads x16) and the epilogue (tok_fac) wait for that pass, and the
+    // producer lets the split-tail grid launch only after its wait, so that grid, which never
+    // waits for its own predecessor, also starts after the conversion. The dequant warps read
+    // only the weights and start at once. (griddepcontrol.wait is a no-op for an ordinary
+    // launch.)
+    if (splits > 1)
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            if (splits == 1) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+            }
             int issued = 0;
             for (int kb = 0; kb < KB; kb++) {
                 const int s = kb % SX;
@@ -237,7 +323,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = ptx::umma_idesc_f16(BF16 ? 1u : 0u, kBM, BN);
+            constexpr uint32_t idesc = ptx::umma_idesc_f16(0u, kBM, BN);   // fp16 x fp16 -> fp32
             int issued = 0;
             for (int kb = 0; kb < KB; kb++) {
                 const int sx = kb % SX, sa = kb % SA;
@@ -322,9 +408,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             if (!warp_wait(&bars->empty_a[s], ph ^ 1, abort, err))
                 break;
             ptx::tc_fence_after();
-            const uint32_t s2 = row_ok ? scale_pair(sv, BF16) : 0u;
+            const uint32_t s2 = row_ok ? scale_pair(sv) : 0u;
             uint32_t av[kCols];                              // 2 weights per 32-bit column
-            expand_pairs<FMT, BF16, kCols>(wv, s2, av);
+            expand_pairs<FMT, kCols>(wv, s2, av);
             if (!row_ok) {
 #pragma unroll
                 for (int c = 0; c < kCols; c++)
@@ -347,6 +433,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         // rows] in the output type, clipped by the tensor map at M and N. Otherwise each warp
         // stores its 32-row segments directly; split tiles store fp32 partials.
         const bool staged_out = splits == 1 && y_tma;
+        if (tok_fac && splits == 1)
+            asm volatile("griddepcontrol.wait;" ::: "memory");   // tok_fac comes from the conversion pass
         if (warp_wait(&bars->acc_full, 0, abort, err)) {
             ptx::tc_fence_after();
             const int quad = warp & 3;                       // TMEM lanes 32*quad .. +31
@@ -359,6 +447,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 ptx::tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(quad * 32) << 16) + cc * 32, v);
                 ptx::tmem_wait_ld();
                 const int64_t mbase = m0 + cc * 32;
+                if (tok_fac && splits == 1) {
+                    // undo the per-token power of two of bf16 x (exact); split partials are
+                    // scaled by the reduce pass
+#pragma unroll
+                    for (int j = 0; j < 32; j++) {
+                        const int64_t m = mbase + j < M ? mbase + j : M - 1;
+                        v[j] = __float_as_uint(__uint_as_float(v[j]) * __ldg(tok_fac + m));
+                    }
+                }
                 if (splits > 1) {
                     // fp32 partial of this split: [tail tile][split][BN tokens][128 rows]
                     float *pt = part + (((size_t)(tile - tile0) * splits + split) * BN + cc * 32) * kBM + quad * 32 + lane;
@@ -432,7 +529,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 template <int BN>
 __global__ void __launch_bounds__(256)
 prefill_reduce_kernel(const float *__restrict__ part, int tiles, int splits, int tiles_m, int tile0, int64_t M,
-                      int64_t N, void *__restrict__ y, int yt)
+                      int64_t N, void *__restrict__ y, int yt, const float *__restrict__ tok_fac)
 {
     // launched as a dependent of the split grid: wait until that grid (and through it the
     // whole-tile grid) has completed and its partials are visible
@@ -450,6 +547,8 @@ prefill_reduce_kernel(const float *__restrict__ part, int tiles, int splits, int
     float v = 0.f;
     for (int sp = 0; sp < splits; sp++)
         v += p[(size_t)sp * BN * kBM];
+    if (tok_fac)
+        v *= tok_fac[m];                                   // exact power of two (bf16 x)
     if (yt == BQ_F32)
         store_out(static_cast<float *>(y) + m * N + n, v);
     else if (yt == BQ_BF16)
@@ -517,20 +616,44 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-template <int FMT, int BN, bool BF16>
+// Workspace: [fp32 partials of the split tail tiles][fp16 x16 [M][K]][tok_fac [M]], each
+// 256-byte aligned. The x16 part serves bf16 x only; it is reserved for either x type so
+// that the size does not depend on x's type.
+struct PfWs {
+    size_t part, x16, fac, total;
+};
+
+PfWs pf_ws(int64_t M, int64_t N, int64_t K)
+{
+    auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
+    const int bn = bn_for(M);
+    const PfPlan pl = pf_plan(M, N, K, bn);
+    PfWs w;
+    w.part = 0;
+    w.x16 = al((size_t)pl.tail * pl.splits * bn * kBM * sizeof(float));
+    w.fac = w.x16 + al((size_t)M * (size_t)K * 2);
+    w.total = w.fac + al((size_t)M * sizeof(float));
+    return w;
+}
+
+template <int FMT, int BN>
 cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc)
         return cudaErrorNotSupported;
+    const PfWs ws = pf_ws(a.M, a.N, a.K);
+    uint8_t *wsb = static_cast<uint8_t *>(a.workspace);
+    const bool bf16 = a.xt == BQ_BF16;
+    const void *xop = bf16 ? static_cast<const void *>(wsb + ws.x16) : a.x;
+    float *tok_fac = bf16 ? reinterpret_cast<float *>(wsb + ws.fac) : nullptr;
     CUtensorMap map;
     cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
     cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
     cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BN};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&map, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                     const_cast<void *>(a.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(xop), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
@@ -551,23 +674,47 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     }
-    auto kern = prefill_kernel<FMT, BN, BF16>;
+    auto kern = prefill_kernel<FMT, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmem);
     if (e != cudaSuccess)
         return e;
     const PfPlan pl = pf_plan(a.M, a.N, a.K, BN);
     const uint16_t *sc = reinterpret_cast<const uint16_t *>(a.scales);
-    float *part = static_cast<float *>(a.workspace);
-    kern<<<pl.full, kThreads, Cfg<BN>::kSmem, s>>>(map, map_y, y_tma, a.words, sc, a.M, a.N, a.K, a.y, a.yt,
-                                                   pl.tiles_m, 0, 1, part, a.dev_status);
+    float *part = reinterpret_cast<float *>(wsb + ws.part);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (bf16) {
+        // conversion pass (an ordinary launch: x may be the previous kernel's output), then the
+        // whole-tile grid as its programmatic dependent: the GEMM CTAs allocate tensor memory
+        // and set up their barriers while the conversion runs, and wait for it in
+        // griddepcontrol.wait
+        prefill_x16_kernel<<<(unsigned)a.M, kX16Threads, 0, s>>>(static_cast<const __nv_bfloat16 *>(a.x), a.K,
+                                                                 reinterpret_cast<__half *>(wsb + ws.x16), tok_fac);
+        e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+        cudaLaunchConfig_t wcfg = {};
+        wcfg.gridDim = dim3((unsigned)pl.full);
+        wcfg.blockDim = dim3(kThreads);
+        wcfg.dynamicSmemBytes = Cfg<BN>::kSmem;
+        wcfg.stream = s;
+        wcfg.attrs = attr;
+        wcfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&wcfg, kern, map, map_y, y_tma, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m, 0,
+                               1, part, (const float *)tok_fac, a.dev_status);
+    } else {
+        kern<<<pl.full, kThreads, Cfg<BN>::kSmem, s>>>(map, map_y, y_tma, a.words, sc, a.M, a.N, a.K, a.y, a.yt,
+                                                       pl.tiles_m, 0, 1, part, (const float *)nullptr, a.dev_status);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess)
+        return e;
     if (pl.tail > 0) {
         // programmatic dependent launches: the tail CTAs take the SMs the whole-tile grid
-        // frees without waiting for all of it (the predecessor of the whole-tile grid, which
-        // may write X, is already complete when that grid runs), and the reduce is resident
-        // before the tail grid ends, waiting on it in griddepcontrol.wait
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        // frees without waiting for all of it (the whole-tile grid lets them launch only after
+        // its own predecessors, including the conversion pass, are complete), and the reduce is
+        // resident before the tail grid ends, waiting on it in griddepcontrol.wait
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(pl.tail * pl.splits));
         cfg.blockDim = dim3(kThreads);
@@ -576,7 +723,7 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, kern, map, map_y, y_tma, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m,
-                               pl.full, pl.splits, part, a.dev_status);
+                               pl.full, pl.splits, part, (const float *)tok_fac, a.dev_status);
         if (e != cudaSuccess)
             return e;
         const int64_t n_out = (int64_t)pl.tail * BN * kBM;
@@ -587,43 +734,40 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
         rcfg.attrs = attr;
         rcfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&rcfg, prefill_reduce_kernel<BN>, (const float *)part, pl.tail, pl.splits, pl.tiles_m,
-                               pl.full, a.M, a.N, a.y, a.yt);
+                               pl.full, a.M, a.N, a.y, a.yt, (const float *)tok_fac);
         if (e != cudaSuccess)
             return e;
     }
     return cudaGetLastError();
 }
 
-template <int FMT, bool BF16>
+template <int FMT>
 cudaError_t launch_bn(const PrefillArgs &a, cudaStream_t s)
 {
     const int bn = bn_for(a.M);
     if (bn == 64)
-        return launch_t<FMT, 64, BF16>(a, s);
+        return launch_t<FMT, 64>(a, s);
     if (bn == 128)
-        return launch_t<FMT, 128, BF16>(a, s);
-    return launch_t<FMT, 256, BF16>(a, s);
+        return launch_t<FMT, 128>(a, s);
+    return launch_t<FMT, 256>(a, s);
 }
 
 }  // namespace
 
-// fp32 partials of the split tail tiles (0 when the tiles fill whole waves or the last wave
-// is more than half full)
+// fp32 partials of the split tail tiles (none when the tiles fill whole waves or the last wave
+// is more than half full), the fp16 copy of bf16 x and its per-token factors
 size_t prefill_workspace_bytes(int64_t M, int fmt, int64_t N, int64_t K)
 {
     (void)fmt;
-    const int bn = bn_for(M);
-    const PfPlan pl = pf_plan(M, N, K, bn);
-    return (size_t)pl.tail * pl.splits * bn * kBM * sizeof(float);
+    return pf_ws(M, N, K).total;
 }
 
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s, unsigned *launches)
 {
-    *launches = pf_plan(a.M, a.N, a.K, bn_for(a.M)).tail > 0 ? 3 : 1;
-    const bool bf16 = a.xt == BQ_BF16;
+    *launches = (pf_plan(a.M, a.N, a.K, bn_for(a.M)).tail > 0 ? 3 : 1) + (a.xt == BQ_BF16 ? 1 : 0);
     if (a.fmt == BQ_BINARY_G128)
-        return bf16 ? launch_bn<BQ_BINARY_G128, true>(a, s) : launch_bn<BQ_BINARY_G128, false>(a, s);
-    return bf16 ? launch_bn<BQ_TERNARY_G128, true>(a, s) : launch_bn<BQ_TERNARY_G128, false>(a, s);
+        return launch_bn<BQ_BINARY_G128>(a, s);
+    return launch_bn<BQ_TERNARY_G128>(a, s);
 }
 
 }  // namespace bq

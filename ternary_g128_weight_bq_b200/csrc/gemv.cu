@@ -12,7 +12,7 @@
 //     groups (128 B contiguous), so a warp's load touches 4 full 128-byte lines.
 //   * the activations are staged once per block into shared memory as fp32 when they fit
 //     (M*K*4 <= 200 KB), else read from global memory (L1/L2-resident).
-// This kernel serves the shapes the tensor-core kernel (gemv_tc.cu) does not take: K not a
+// This kernel serves the shapes the tensor-core kernel (gemv_rows.cu) does not take: K not a
 // multiple of 1024, or digit fragments too large for shared memory.
 #include "bq_internal.cuh"
 
@@ -90,11 +90,12 @@ gemv_simt_kernel(const XT *__restrict__ x, int64_t K, const uint32_t *__restrict
                 for (int i = 0; i < 8; i++) {
 #pragma unroll 4
                     for (int b = 0; b < 16; b++) {
-                        const uint32_t c = (w[i] >> (2 * b)) & 3u;   // 0 -> -x, 1 -> 0, 2 -> +x
+                        const uint32_t c = (w[i] >> (2 * b)) & 3u;   // 0 -> -x, 1 -> 0 * x, 2 -> +x
 #pragma unroll
                         for (int m = 0; m < M; m++) {
                             float xv = xs[xg + m * K + i * 16 + b];
-                            part[m] += c == 2u ? xv : (c == 0u ? -xv : 0.f);
+                            // a zero weight still multiplies x, so an infinity or NaN in x gives NaN
+                            part[m] += c == 2u ? xv : (c == 0u ? -xv : 0.f * xv);
                         }
                     }
                 }
@@ -168,30 +169,18 @@ cudaError_t launch_gemv_simt(const GemvArgs &a, cudaStream_t s)
                           : launch_simt_m<BQ_TERNARY_G128, __nv_bfloat16>(a, s);
 }
 
-// Workspace of the tensor-core path (partial sums of row blocks split between CTAs and
-// their counters); the SIMT kernel needs none.
+// Workspace of the tensor-core path (the digit fragments of x); the SIMT kernel needs none.
 size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
 {
-    if (gemv_tmem_supported(M, fmt, K))
-        return gemv_tmem_workspace_bytes(M, fmt, N, K);
-    if (!gemv_tc_supported(M, fmt, K))
-        return 0;
-    return gemv_tc_workspace_bytes(M, fmt, N, K);
+    return gemv_rows_supported(M, fmt, N, K) ? gemv_rows_workspace_bytes(M, fmt, N, K) : 0;
 }
 
-// K a multiple of 1024: the tcgen05 kernel (gemv_tmem.cu) for binary with 5 <= M <= 8 and for
-// ternary, the mma.sync kernel (gemv_tc.cu) for binary with M <= 4; otherwise (or when the
-// digit fragments do not fit in shared memory) the SIMT kernel.
+// K a multiple of 1024 and the fragments in shared memory: the integer tensor-core kernel
+// (gemv_rows.cu); otherwise the SIMT kernel.
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches)
 {
-    if (gemv_tmem_supported(a.M, a.fmt, a.K)) {
-        *launches = 2;                               // fragment prep + the GEMV
-        return launch_gemv_tmem(a, s);
-    }
-    if (gemv_tc_supported(a.M, a.fmt, a.K)) {
-        *launches = 2;                               // fragment prep + the GEMV
-        return launch_gemv_tc(a, s);
-    }
+    if (gemv_rows_supported(a.M, a.fmt, a.N, a.K))
+        return launch_gemv_rows(a, s, launches);
     *launches = 1;
     return launch_gemv_simt(a, s);
 }

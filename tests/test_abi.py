@@ -96,3 +96,32 @@ def test_validation_before_any_cuda_call(libbq):
     assert libbq.bq_embed_gather(16, -1, W(_weight()), 16, 1, None) == 2
     msg = libbq.bq_last_error()
     assert b"T=-1" in msg
+
+
+def _symbol_size(name: str) -> int:
+    out = subprocess.run(["nm", "-S", "-C", bq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    for line in out.splitlines():
+        parts = line.split()
+        if len(parts) >= 4 and parts[-1] == name:
+            return int(parts[1], 16)
+    raise AssertionError(f"{name} not found")
+
+
+def test_noalloc_array_covers_every_supported_shape(libbq):
+    """bq_gemv_noalloc serves a shape from the library's fixed array only when the workspace
+    bq_gemv would need fits in it. That array must hold every shape the GEMV kernels take on a
+    148-SM B200 (without a GPU the library plans for 148 SMs): every M, both formats, K up to
+    64K, N up to 2^22. The array's size is read from the library's symbol table."""
+    cap = _symbol_size("bq::g_gemv_scratch")
+    assert 64 << 10 <= cap <= 4 << 20
+    worst = 0
+    for fmt in (bq.BINARY_G128, bq.TERNARY_G128):
+        for M in range(1, 9):
+            for K in (128, 1024, 2048, 4096, 5120, 6144, 8192, 16384, 20480, 65536):
+                for N in (1, 129, 5120, 20480, 248320, 1 << 22):
+                    w = bq._Weight(fmt, N, K, 16, 16)
+                    need = int(libbq.bq_gemv_workspace_bytes(M, ctypes.byref(w)))
+                    worst = max(worst, need)
+                    assert need <= cap, (fmt, M, K, N, need, cap)
+    assert worst > 0

@@ -132,14 +132,14 @@ def test_api_errors_on_device():
     torch.cuda.synchronize()
 
 
-# ---- tensor-core path (K a multiple of 1024): fp8 pieces of x, stream-K split ----------
+# ---- tensor-core path (K a multiple of 1024): x as integer digits, whole rows per CTA ------
 
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("xdt", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("N,K", [(1, 1024), (127, 2048), (129, 1024), (1000, 3072)])
 def test_tensor_path_ragged_all_outputs(orc, M, xdt, N, K):
-    """All outputs of ragged shapes on the tensor-core kernels: mma.sync for M <= 4, tcgen05
-    (sign operand in tensor memory) for binary M >= 5."""
+    """All outputs of ragged shapes on the integer tensor-core kernel, every M (one to four
+    column sets), tile counts that leave partial tile-groups, both x types."""
     run_binary(orc, 400 + M, N, K, M, xdt=xdt)
 
 
@@ -152,7 +152,7 @@ def test_tensor_path_ternary(orc, M, N, K):
 @pytest.mark.parametrize("M", [3, 8])
 def test_tensor_path_wide_dynamic_range(orc, M):
     """x spanning 40 binades inside each group: the integer digits of x (22 bits below the
-    group maximum) stay within the bound. M = 3 runs the mma.sync kernel, M = 8 the tcgen05 one."""
+    group maximum) stay within the bound, at two and at four column sets."""
     m = bq()
     N, K = 300, 2048
     x = synth.activations(7, M, K, dtype=torch.float32)
@@ -183,7 +183,8 @@ def test_tensor_path_zero_and_tiny_groups(orc, M):
 
 
 def test_tensor_path_deterministic():
-    """Split blocks are summed in a fixed order: repeated calls give identical bits."""
+    """The eight per-group sums of every output are added in a fixed order: repeated calls
+    give identical bits."""
     m = bq()
     x, words, s = binary_inputs(9, 5120, 5120, 8)
     w = m.BQWeight(m.BINARY_G128, 5120, 5120, words.cuda(), s.cuda())
@@ -193,15 +194,76 @@ def test_tensor_path_deterministic():
         assert torch.equal(m.gemv(xd, w), y1)
 
 
-def test_workspace_too_small_is_rejected():
+def test_workspace_sizes():
+    """The tensor-core path keeps the digit fragments of x in the workspace (written once per
+    call by the prep kernel; 1 KB per group and column set, plus factors and accumulator
+    inputs), the SIMT path needs none, and a workspace that is too small is rejected before
+    anything is launched."""
     m = bq()
-    x, words, s = binary_inputs(10, 256, 1024, 2)
+    x, words, s = binary_inputs(10, 256, 1024, 4)
     w = m.BQWeight(m.BINARY_G128, 256, 1024, words.cuda(), s.cuda())
-    need = m.gemv_workspace_bytes(2, w)
+    assert m.gemv_workspace_bytes(1, w) >= 8 * 1024
+    w640 = m.BQWeight(m.BINARY_G128, 256, 640, synth.binary_words(10, 256, 640).cuda(),
+                      synth.scales(10, 256, 5).cuda())
+    assert m.gemv_workspace_bytes(4, w640) == 0
+    need = m.gemv_workspace_bytes(4, w)
     assert need > 0
-    y = torch.empty((2, 256), dtype=torch.float32, device="cuda")
+    y = torch.empty((4, 256), dtype=torch.float32, device="cuda")
     ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
     with pytest.raises(m.BQError) as e:
-        m._check(m.lib().bq_gemv(x.cuda().data_ptr(), 1, 2, w.c, y.data_ptr(), 2, ws.data_ptr(),
+        m._check(m.lib().bq_gemv(x.cuda().data_ptr(), 1, 4, w.c, y.data_ptr(), 2, ws.data_ptr(),
                                  need - 256, m._stream()))
     assert e.value.status_name == "BQ_ERR_WORKSPACE"
+
+
+@pytest.mark.parametrize("M,K,kernel", [(3, 2048, "tensor-core"), (6, 2048, "tensor-core"), (3, 640, "simt")])
+@pytest.mark.parametrize("fmt", [oracle.BINARY, oracle.TERNARY])
+def test_nonfinite_x_propagates(orc, M, K, kernel, fmt):
+    """An infinity or NaN in x makes every output of that token non-finite, as in the oracle
+    (the tensor-core kernel gives NaN: the digit prep marks the group's factor NaN); tokens
+    with finite x are unaffected. K = 2048 runs the integer tensor-core kernel (two and four
+    column sets), K = 640 the SIMT kernel."""
+    m = bq()
+    N = 700
+    s = synth.scales(5, N, K // 128)
+    if fmt == oracle.BINARY:
+        words = synth.binary_words(5, N, K)
+        w = m.BQWeight(m.BINARY_G128, N, K, words.cuda(), s.cuda())
+        words_np = words.numpy()
+    else:
+        q = ternary_q(5, N, K)
+        w = m.pack_ternary_g128(q.cuda(), s.cuda())
+        st, words_np, _ = orc.pack(oracle.TERNARY, q.numpy(), s.numpy())
+        assert st == oracle.OK
+    x = synth.activations(6, M, K)
+    x[0, 17] = float("nan")
+    x[1, K - 1] = float("inf")
+    x[2, 300] = float("-inf")
+    y = m.gemv(x.cuda(), w).double().cpu().numpy()
+    torch.cuda.synchronize()
+    y_ref, bound = orc.gemv(fmt, x, oracle.X_BF16, words_np, s, K)
+    for t in range(3):
+        assert not np.isfinite(y_ref[t]).any(), "the oracle's outputs of that token are non-finite"
+        assert not np.isfinite(y[t]).any(), f"{kernel}: token {t} has finite outputs"
+    err = np.abs(y[3:] - y_ref[3:])
+    assert np.all(err <= bound[3:]), f"{kernel}: finite tokens, max err/bound {np.max(err / bound[3:]):.3g}"
+
+
+def test_binding_rejects_wrong_out_shape():
+    """The binding checks a caller's out tensor (shape, dtype, device) before anything is
+    launched: a smaller out would otherwise receive out-of-bounds writes."""
+    m = bq()
+    N, K = 64, 1024
+    x, words, s = binary_inputs(2, N, K, 3)
+    w = m.BQWeight(m.BINARY_G128, N, K, words.cuda(), s.cuda())
+    xd = x.cuda()
+    for bad in (torch.empty((3, N - 1), device="cuda"), torch.empty((2, N), device="cuda"),
+                torch.empty((3, N), dtype=torch.int32, device="cuda"), torch.empty((3, N))):
+        with pytest.raises(ValueError):
+            m.gemv(xd, w, out=bad)
+        with pytest.raises(ValueError):
+            m.gemv_noalloc(xd, w, out=bad)
+        with pytest.raises(ValueError):
+            m.gemm_prefill(xd, w, out=bad)
+    with pytest.raises(ValueError):
+        m.gemv(x, w)                                            # x on the host

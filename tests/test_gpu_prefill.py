@@ -106,3 +106,70 @@ def test_prefill_matches_gemv(orc):
     a = m.gemm_prefill(x, w)
     b = m.gemv(x, w)
     assert torch.allclose(a, b, rtol=1e-4, atol=1e-4)
+
+
+# ---------------------------------------------------------------------------------------
+# bf16 x with scales that bf16 cannot hold: the +-s operand must stay exact
+# ---------------------------------------------------------------------------------------
+
+from tests.adversarial import (adversarial_binary, adversarial_ternary_q, positive_bf16_x,  # noqa: E402
+                               wide_range_bf16_x)
+
+
+def check_adversarial(orc, fmt, M, N, K, x, rows=None):
+    m = bq()
+    if fmt == oracle.BINARY:
+        words, s = adversarial_binary(N, K)
+        w = m.BQWeight(m.BINARY_G128, N, K, words.cuda(), s.cuda())
+        words_np = words.numpy()
+    else:
+        q, s = adversarial_ternary_q(N, K)
+        w = m.pack_ternary_g128(q.cuda(), s.cuda())
+        st, words_np, _ = orc.pack(oracle.TERNARY, q.numpy(), s.numpy())
+        assert st == oracle.OK
+        assert np.array_equal(w.words.cpu().numpy().view(np.uint32), words_np)
+    y = m.gemm_prefill(x.cuda(), w, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    m.get_device_error()
+    y_ref, bound = orc.gemv(fmt, x, oracle.X_BF16, words_np, s, K, rows=rows)
+    yg = y if rows is None else y[:, torch.from_numpy(rows).cuda()]
+    return assert_within_bound(yg, y_ref, bound, f"adversarial prefill fmt={fmt} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("fmt", [oracle.BINARY, oracle.TERNARY])
+@pytest.mark.parametrize("M", [77, 512])
+def test_prefill_bf16_tie_scales_all_outputs(orc, fmt, M):
+    """Scales on bf16 rounding ties in many binades (0x3C04 = 1.00390625 rounds to 1.0 in
+    bf16, a 2^-8 relative error), groups of all-ones / all-zeros bits (or all +1 / all -1
+    ternary codes) and strictly positive bf16 x, so that every term of a group would err the
+    same way if the scale were rounded to bf16: about 1.95x the bound. With the exact fp16
+    operand only fp32 accumulation error is left. Every output is checked."""
+    K, N = 1024, 256
+    r = check_adversarial(orc, fmt, M, N, K, positive_bf16_x(40 + M, M, K))
+    print(f"max err/bound = {r:.4g}")
+    assert r < 0.1
+
+
+@pytest.mark.parametrize("fmt", [oracle.BINARY, oracle.TERNARY])
+def test_prefill_bf16_tie_scales_split_tail(orc, fmt):
+    """The same adversarial inputs through the split tail: M = 512, N = 10240, K = 1024 is 160
+    tiles on 148 SMs; the 12 tiles past the full wave (rows 9472 .. 10239, both token tiles)
+    are split along K and reduced, where the per-token factor is applied by the reduce pass.
+    Every row of those tiles and a sample of the others are checked."""
+    M, N, K = 512, 10240, 1024
+    rows = np.unique(np.concatenate([np.arange(74 * 128, N), sample_rows(74 * 128, 64, 9)]))
+    r = check_adversarial(orc, fmt, M, N, K, positive_bf16_x(51, M, K), rows=rows)
+    assert r < 0.1
+
+
+@pytest.mark.parametrize("M,N", [(130, 384), (512, 10240)])
+def test_prefill_bf16_wide_range_tokens(orc, M, N):
+    """Token rows whose magnitudes span 2^-100 .. 2^100 (two binades per token): each row
+    gets its own power-of-two factor, so a factor applied to the wrong token, or one lost in
+    the split-tail reduce (M = 512, N = 10240: rows 9472 .. 10239 are split along K), shows
+    up at once. Rows of all zeros give zeros."""
+    K = 1024
+    rows = None if N < 1000 else np.unique(np.concatenate([np.arange(74 * 128, N),
+                                                           sample_rows(74 * 128, 32, 10)]))
+    r = check_adversarial(orc, oracle.BINARY, M, N, K, wide_range_bf16_x(60, M, K), rows=rows)
+    assert r < 0.1

@@ -1,9 +1,9 @@
 """bq_gemv_noalloc (the decode GEMV with the library's fixed scratch array) against bq_gemv
 with a caller workspace, through the C ABI. Two calls in a row per shape, each within the
 GEMV tolerance max|y - y_ws| <= 2e-3 * sum_k |x s| of the workspace call's result (the same
-kernel and the same fixed summation order, so the outputs are also bit-identical). The
-shapes split row blocks between CTAs, so the partial sums and counters in the array are used.
-Collected last, so it also runs after every other test has used the library."""
+kernel and the same fixed summation order, so the outputs are also bit-identical). On these
+shapes the prep kernel writes the digit fragments of x into the array and the GEMV reads them
+back from it. Collected last, so it also runs after every other test has used the library."""
 
 import numpy as np
 import pytest
@@ -33,7 +33,7 @@ def _bound(orc, fmt, x, words, s, K, rows):
 
 
 @pytest.mark.parametrize("fmt,N,K,M", [
-    (0, 20480, 5120, 8),      # 160 row blocks x 5 stages over the SMs: split blocks at M = 8
+    (0, 20480, 5120, 8),      # four column sets: the largest fragment set at K = 5120
     (0, 248320, 5120, 1),     # the LM head
     (1, 20480, 5120, 4),      # ternary
     (0, 1000, 640, 3),        # K not a multiple of 1024: the kernel that needs no scratch
