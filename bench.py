@@ -188,6 +188,8 @@ def capture_step_graphs(bq, sets, stream):
 
 
 def time_graphs(graphs, steps, warmup, stream, dist, device):
+    """Device ms of exactly `steps` steps after `warmup` untimed ones, bracketed by a barrier and
+    a synchronize on both sides."""
     for i in range(warmup):
         graphs[i % len(graphs)].replay()
     torch.cuda.synchronize()
@@ -204,6 +206,17 @@ def time_graphs(graphs, steps, warmup, stream, dist, device):
     torch.cuda.synchronize()
     barrier(dist, device)
     return start.elapsed_time(end)
+
+
+def time_regions(graphs, steps, warmup, stream, dist, device, min_seconds=1.0, max_regions=2000):
+    """The timed region (exactly `steps` steps) repeated R times, so that a clock sampler running
+    alongside sees the GPU under load; R is the same on every rank. Returns (the median region's
+    ms, every region's ms)."""
+    first = time_graphs(graphs, steps, warmup, stream, dist, device)
+    R = max(1, min(max_regions, math.ceil(min_seconds * 1e3 / max(first, 1e-3))))
+    R = int(reduce_max(float(R), dist, device))
+    times = [time_graphs(graphs, steps, 0, stream, dist, device) for _ in range(R)]
+    return statistics.median(times), times
 
 
 def time_single(fn, reps, warmup, stream):
@@ -238,65 +251,285 @@ def per_config_breakdown(bq, sets, stream):
     return out
 
 
-def extra_workloads(bq, device, stream, peaks):
-    """LM head, ternary GEMV, embedding gather, prefill (when available): one line each."""
-    res = {}
-    # LM head: M=1, K=5120, N=248320 (179 MB > L2 on its own)
-    N = 248320
-    w = bq.BQWeight(bq.BINARY_G128, N, K_HEAD, synth.binary_words(0, N, K_HEAD, device=device),
-                    synth.scales(0, N, K_HEAD // 128).to(device))
-    x = synth.activations(0, 1, K_HEAD).to(device)
+# --------------------------------------------------------------------------------------
+# every configuration of the benchmark: device time, roofline fraction, the CPU oracle's time
+# on the host cores beside it, and a sampled oracle check of the same outputs
+# --------------------------------------------------------------------------------------
+
+class OracleBench:
+    """The CPU oracle (plain C, fp64) timed on the host cores on bounded samples of a workload,
+    and used to check sampled outputs of the GPU runs (outside every timed region)."""
+
+    def __init__(self, budget_s: float = 1.5):
+        import oracle
+        self.o = oracle
+        self.orc = oracle.default()
+        self.cores = os.cpu_count() or 1
+        self.budget = budget_s
+
+    def time_items(self, work, n_items: int, threads: int):
+        """Seconds for n items of `work(lo, hi)` (item indices taken modulo n_items) on `threads`
+        threads, with n sized to about the budget (one item is timed first). Returns (seconds, n)."""
+        import concurrent.futures as cf
+        t0 = time.perf_counter()
+        work(0, 1)
+        one = max(time.perf_counter() - t0, 1e-6)
+        n = max(threads, int(self.budget * threads / one))
+        chunks = []
+        for i in range(threads):                       # each thread's share, in passes over the items
+            lo, hi = n * i // threads, n * (i + 1) // threads
+            while hi > lo:
+                a = lo % n_items
+                b = min(n_items, a + (hi - lo))
+                chunks.append((a, b))
+                lo += b - a
+        t0 = time.perf_counter()
+        with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(lambda c: work(*c), chunks))
+        return time.perf_counter() - t0, n
+
+    def gemv_timing(self, fmt, x, xt, words, scales, K, bytes_per_row, x_bytes, one_core: bool):
+        """Oracle GB/s on the rows of `words` (host arrays), all cores (and one core)."""
+        def work(lo, hi):
+            self.orc.gemv(fmt, x, xt, words[lo:hi], scales[lo:hi], K)
+        res = {}
+        for label, th in (("all_cores", self.cores), ("one_core", 1)) if one_core else (("all_cores", self.cores),):
+            dt, n = self.time_items(work, len(words), th)
+            res[label] = {"GBps": round((n * bytes_per_row + x_bytes) / 1e9 / dt, 4), "cores": th,
+                          "sample": f"{n} rows x all K (passes over {len(words)} distinct rows), {dt:.3f} s"}
+        return res
+
+    def max_ratio(self, fmt, x, xt, words, scales, K, y_rows):
+        """max |y - y_ref| / (2e-3 sum |x s|) over the given rows (y_rows [M, R] from the GPU)."""
+        y_ref, bound = self.orc.gemv(fmt, x, xt, words, scales, K)
+        import numpy as np
+        err = np.abs(y_rows.astype(np.float64) - y_ref)
+        return float(np.max(err / np.maximum(bound, 1e-300)))
+
+
+def _host_binary(seed, rows, K, row0=0):
+    return (synth.binary_words(seed, rows, K, row0=row0).numpy(),
+            synth.scales(seed, rows, K // 128, row0=row0).numpy())
+
+
+def _host_ternary(ob, seed, rows, K, row0=0):
+    q = synth.random_ternary(seed, synth.TID_TERNARY, (rows, K), row0=row0)
+    s = synth.scales(seed, rows, K // 128, row0=row0)
+    st, words, s_out = ob.orc.pack(ob.o.TERNARY, q.numpy(), s.numpy())
+    assert st == ob.o.OK
+    return words, s_out
+
+
+def _gemv_entry(name, N, K, M, fmt_bits, ms, peaks, extra=None):
+    gb = gemv_bytes(N, K, M, fmt_bits) / 1e9
+    gbs = gb / (ms / 1e3)
+    e = {"workload": name, "N": N, "K": K, "M": M, "us": round(ms * 1e3, 2), "GBps": round(gbs, 1),
+         "bound": "hbm", "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"]}
+    if extra:
+        e.update(extra)
+    return e
+
+
+def _rotating_gemv_ms(bq, mats, x, y, ws, stream, reps=20):
+    """Device ms of one call over a CUDA graph of back-to-back calls that rotate through `mats`
+    (weight copies together larger than L2)."""
+    g = torch.cuda.CUDAGraph()
+    for w in mats:
+        bq.gemv(x, w, out=y, workspace=ws)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(reps):
+            bq.gemv(x, mats[i % len(mats)], out=y, workspace=ws)
+    ms = time_single(g.replay, 10, 3, stream) / reps
+    del g
+    return ms
+
+
+def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
+    """One entry per benchmark configuration (BASELINE's five, in order)."""
+    import numpy as np
+    l2 = l2_bytes(device)
+    out = []
+    o = ob.o
+
+    # ---- config 1: binary GEMV, M=1, K=N=1024, x fp16, seed 0 (L2-resident: reported in us)
+    N, K = 1024, 1024
+    w = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(0, N, K, device=device),
+                    synth.scales(0, N, K // 128, device=device))
+    x = synth.activations(0, 1, K, dtype=torch.float16)
+    xd = x.to(device)
     y = torch.empty((1, N), dtype=torch.float32, device=device)
-    ms = time_single(lambda: bq.gemv(x, w, out=y), 50, 5, stream)
-    res["lm_head_gemv"] = {"N": N, "K": K_HEAD, "M": 1, "us": round(ms * 1e3, 2),
-                           "GBps": round(gemv_bytes(N, K_HEAD, 1) / 1e9 / (ms / 1e3), 1)}
-    # embedding gather: 4096 ids over the same matrix, bf16 out
-    ids = synth.random_ids(0, synth.TID_IDS, 4096, N).to(device)
-    out = torch.empty((4096, K_HEAD), dtype=torch.bfloat16, device=device)
-    ms = time_single(lambda: bq.embed_gather(ids, w, out=out), 50, 5, stream)
-    eb = 4096 * (K_HEAD // 8 + K_HEAD // 64 + K_HEAD * 2) + 4096 * 4
-    res["embed_gather"] = {"T": 4096, "K": K_HEAD, "us": round(ms * 1e3, 2),
-                           "GBps": round(eb / 1e9 / (ms / 1e3), 1)}
-    del w, ids, out
-    # ternary GEMV: N=20480, K=5120, M=1 (rotating 12 copies: 334 MB)
-    tsets = []
-    for c in range(12):
-        q = synth.random_ternary(c, synth.TID_TERNARY, (20480, K_HEAD)).to(device)
-        tw = bq.pack_ternary_g128(q, synth.scales(c, 20480, K_HEAD // 128).to(device))
-        tsets.append(tw)
-        del q
-    x = synth.activations(0, 1, K_HEAD).to(device)
-    y = torch.empty((1, 20480), dtype=torch.float32, device=device)
+    ws = torch.empty(max(bq.gemv_workspace_bytes(1, w), 16), dtype=torch.uint8, device=device)
+    ms = _rotating_gemv_ms(bq, [w], xd, y, ws, stream, reps=50)
+    bq.gemv(xd, w, out=y, workspace=ws)
+    words, sc = _host_binary(0, N, K)
+    ratio = ob.max_ratio(o.BINARY, x, o.X_F16, words, sc, K, y.cpu().numpy())
+    e = _gemv_entry("config 1: binary g128 GEMV, M=1, K=N=1024, x fp16, seed 0 (all 1024 outputs checked)",
+                    N, K, 1, 1, ms, peaks,
+                    {"timing": "graph of 50 back-to-back calls on the same weights (147 KB: L2-resident)",
+                     "parity": {"max_err_over_bound": round(ratio, 5), "outputs": N}})
+    e["oracle"] = ob.gemv_timing(o.BINARY, x, o.X_F16, words, sc, K, K // 8 + K // 64, 2 * K, True)
+    out.append(e)
+    del w, y, ws
+
+    # ---- config 2: the headline GEMVs (K=5120, N in {5120, 20480}, M in {1, 4, 8}); the
+    # device times are the breakdown's (rotating weight copies); parity on copy 0
+    shapes = []
+    for j, (N, M) in enumerate(GEMV_SHAPES):
+        K = K_HEAD
+        bd = breakdown[j] if breakdown else None
+        w = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(0, N, K, device=device),
+                        synth.scales(0, N, K // 128, device=device))
+        x = synth.activations(0, M, K)
+        y = bq.gemv(x.to(device), w)
+        rows = 256
+        words, sc = _host_binary(0, rows, K)
+        ratio = ob.max_ratio(o.BINARY, x, o.X_BF16, words, sc, K, y[:, :rows].cpu().numpy())
+        ent = {"N": N, "M": M, "parity": {"max_err_over_bound": round(ratio, 5), "rows": rows}}
+        if bd:
+            ent.update({"us": bd["us"], "GBps": bd["GBps"], "frac": round(bd["GBps"] / peaks["hbm_gbs"], 4)})
+        ent["oracle"] = ob.gemv_timing(o.BINARY, x, o.X_BF16, *_host_binary(0, 4096, K), K,
+                                       K // 8 + K // 64, 2 * M * K, N <= 5120)
+        shapes.append(ent)
+        del w, y
+    out.append({"workload": "config 2: binary g128 decode GEMV, K=5120, N in {5120, 20480}, M in {1, 4, 8} "
+                            "(the headline step; one entry per GEMV, each timed alone over rotating copies)",
+                "bound": "hbm", "peak": peaks["hbm_gbs"], "gemvs": shapes})
+
+    # ---- config 3: LM head (M=1, K=5120, N=248320) and the embedding gather of 4096 ids
+    N, K = 248320, K_HEAD
+    w = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(0, N, K, device=device),
+                    synth.scales(0, N, K // 128, device=device))
+    x = synth.activations(0, 1, K)
+    xd = x.to(device)
+    y = torch.empty((1, N), dtype=torch.float32, device=device)
+    ws = torch.empty(max(bq.gemv_workspace_bytes(1, w), 16), dtype=torch.uint8, device=device)
+    ms = _rotating_gemv_ms(bq, [w], xd, y, ws, stream, reps=20)
+    rows = 512
+    words, sc = _host_binary(0, rows, K, row0=N - rows)
+    ratio = ob.max_ratio(o.BINARY, x, o.X_BF16, words, sc, K, y[:, N - rows:].cpu().numpy())
+    e = _gemv_entry("config 3a: LM-head GEMV, binary g128, M=1, K=5120, N=248320", N, K, 1, 1, ms, peaks,
+                    {"timing": "graph of 20 back-to-back calls (179 MB of weights per call, above L2)",
+                     "parity": {"max_err_over_bound": round(ratio, 5), "rows": rows}})
+    e["oracle"] = ob.gemv_timing(o.BINARY, x, o.X_BF16, *_host_binary(0, 4096, K), K, K // 8 + K // 64,
+                                 2 * K, False)
+    out.append(e)
+    # embedding gather: output buffers rotate (together above L2), so the writes reach HBM
+    T = 4096
+    ids = synth.random_ids(0, synth.TID_IDS, T, N)
+    idd = ids.to(device)
+    nbuf = max(2, math.ceil(2.5 * l2 / (T * K * 2)))
+    outs = [torch.empty((T, K), dtype=torch.bfloat16, device=device) for _ in range(nbuf)]
     it = [0]
 
-    def tstep():
-        bq.gemv(x, tsets[it[0] % len(tsets)], out=y)
+    def gather():
+        bq.embed_gather(idd, w, out=outs[it[0] % nbuf])
         it[0] += 1
-    ms = time_single(tstep, 48, 4, stream)
-    res["ternary_gemv"] = {"N": 20480, "K": K_HEAD, "M": 1, "us": round(ms * 1e3, 2),
-                           "GBps": round(gemv_bytes(20480, K_HEAD, 1, 2) / 1e9 / (ms / 1e3), 1)}
-    del tsets
-    res["full_depth_decode_step"] = full_depth_step(bq, device, stream, peaks)
-    # prefill GEMM: M=512, K=5120, N=20480 binary and ternary
-    try:
-        for fmt_name in ("binary", "ternary"):
-            if fmt_name == "binary":
-                pw = bq.BQWeight(bq.BINARY_G128, 20480, K_HEAD,
-                                 synth.binary_words(0, 20480, K_HEAD, device=device),
-                                 synth.scales(0, 20480, K_HEAD // 128).to(device))
-            else:
-                q = synth.random_ternary(0, synth.TID_TERNARY, (20480, K_HEAD)).to(device)
-                pw = bq.pack_ternary_g128(q, synth.scales(0, 20480, K_HEAD // 128).to(device))
-            X = synth.activations(0, 512, K_HEAD).to(device)
-            Y = torch.empty((512, 20480), dtype=torch.bfloat16, device=device)
-            ms = time_single(lambda: bq.gemm_prefill(X, pw, out=Y), 20, 3, stream)
-            tf = 2 * 512 * 20480 * K_HEAD / (ms / 1e3) / 1e12
-            res[f"prefill_{fmt_name}"] = {"M": 512, "N": 20480, "K": K_HEAD, "us": round(ms * 1e3, 1),
-                                          "TFLOPs": round(tf, 1),
-                                          "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 3)}
-    except Exception as e:  # reported, not hidden: the line says why there is no number
-        res["prefill"] = {"error": str(e).splitlines()[0][:200]}
-    return res
+    ms = time_single(gather, 5 * nbuf, nbuf, stream)
+    eb = T * (K // 8 + K // 64 + K * 2) + T * 4
+    # bit-exact check of the ids that fall in the first 4096 rows (host words of those rows only)
+    R = 4096
+    words, sc = _host_binary(0, R, K)
+    sel = (ids < R).nonzero().flatten()
+    ref, bad = ob.orc.embed(o.BINARY, ids[sel].numpy(), words, sc, K)
+    got = outs[(it[0] - 1) % nbuf][sel.to(device)].view(torch.int16).cpu().numpy().view(np.uint16)
+    exact = bool(np.array_equal(got, ob.orc.to_bf16_bits(ref))) and bad == 0
+
+    def ework(lo, hi):
+        ob.orc.embed(o.BINARY, (ids[lo:hi] % R).numpy(), words, sc, K)
+    dt, n = ob.time_items(ework, T, ob.cores)
+    gbs = eb / 1e9 / (ms / 1e3)
+    out.append({"workload": "config 3b: embedding gather, 4096 ids uniform in [0, 248320), K=5120, bf16 out",
+                "us": round(ms * 1e3, 2), "GBps": round(gbs, 1), "bound": "hbm",
+                "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"],
+                "timing": f"{nbuf} output buffers rotated ({nbuf * T * K * 2 / 1e6:.0f} MB vs {l2 / 1e6:.0f} MB L2)",
+                "parity": {"bit_exact": exact, "ids_checked": int(len(sel))},
+                "oracle": {"all_cores": {"GBps": round(n / T * eb / 1e9 / dt, 4), "cores": ob.cores,
+                                         "sample": f"{n} ids (rows of a 4096-row slice), {dt:.3f} s"}}})
+    del w, y, ws, outs
+
+    # ---- config 4: ternary GEMV (N=20480, K=5120, M=1) and ternary prefill (M=512)
+    N, K = 20480, K_HEAD
+    copies = max(2, math.ceil(2.5 * l2 / gemv_bytes(N, K, 1, 2)))
+    tmats = []
+    for c in range(copies):
+        q = synth.random_ternary(c, synth.TID_TERNARY, (N, K), device=device)
+        tmats.append(bq.pack_ternary_g128(q, synth.scales(c, N, K // 128, device=device)))
+        del q
+    x = synth.activations(0, 1, K)
+    xd = x.to(device)
+    y = torch.empty((1, N), dtype=torch.float32, device=device)
+    ws = torch.empty(max(bq.gemv_workspace_bytes(1, tmats[0]), 16), dtype=torch.uint8, device=device)
+    ms = _rotating_gemv_ms(bq, tmats, xd, y, ws, stream, reps=2 * copies)
+    bq.gemv(xd, tmats[0], out=y, workspace=ws)
+    rows = 256
+    words, sc = _host_ternary(ob, 0, rows, K)
+    ratio = ob.max_ratio(o.TERNARY, x, o.X_BF16, words, sc, K, y[:, :rows].cpu().numpy())
+    e = _gemv_entry("config 4a: ternary g128 GEMV, M=1, K=5120, N=20480", N, K, 1, 2, ms, peaks,
+                    {"timing": f"graph of back-to-back calls rotating {copies} weight copies (above L2)",
+                     "parity": {"max_err_over_bound": round(ratio, 5), "rows": rows}})
+    e["oracle"] = ob.gemv_timing(o.TERNARY, x, o.X_BF16, *_host_ternary(ob, 0, 2048, K), K,
+                                 K // 4 + K // 64, 2 * K, False)
+    out.append(e)
+    del tmats, y, ws
+    out.append(prefill_report(bq, device, stream, peaks, ob, "ternary", l2))
+
+    # ---- config 5: binary prefill (M=512) and the full-depth decode step
+    out.append(prefill_report(bq, device, stream, peaks, ob, "binary", l2))
+    out.append(full_depth_step(bq, device, stream, peaks, ob))
+    torch.cuda.empty_cache()
+    return out
+
+
+def prefill_report(bq, device, stream, peaks, ob, fmt_name, l2):
+    """M=512, K=5120, N=20480 prefill GEMM, bf16 x and out; sets of (weights, x, y) rotate so
+    that they are together larger than L2."""
+    M, N, K = 512, 20480, K_HEAD
+    o = ob.o
+    per_set = gemv_bytes(N, K, 0, 1 if fmt_name == "binary" else 2) + M * K * 2 + M * N * 2
+    nset = max(2, math.ceil(1.5 * l2 / per_set))
+    sets = []
+    for c in range(nset):
+        if fmt_name == "binary":
+            pw = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(c, N, K, device=device),
+                             synth.scales(c, N, K // 128, device=device))
+        else:
+            q = synth.random_ternary(c, synth.TID_TERNARY, (N, K), device=device)
+            pw = bq.pack_ternary_g128(q, synth.scales(c, N, K // 128, device=device))
+            del q
+        sets.append((pw, synth.activations(c, M, K).to(device),
+                     torch.empty((M, N), dtype=torch.bfloat16, device=device)))
+    ws = torch.empty(max(bq.prefill_workspace_bytes(M, sets[0][0]), 16), dtype=torch.uint8, device=device)
+    it = [0]
+
+    def call():
+        pw, X, Y = sets[it[0] % nset]
+        bq.gemm_prefill(X, pw, out=Y, workspace=ws)
+        it[0] += 1
+    ms = time_single(call, 4 * nset, nset, stream)
+    tf = 2 * M * N * K / (ms / 1e3) / 1e12
+    # parity: rows 0..63 of set 0 against the oracle, all 512 tokens
+    pw, X, Y = sets[0]
+    bq.gemm_prefill(X, pw, out=Y, workspace=ws)
+    x = synth.activations(0, M, K)
+    rows = 64
+    fmt = o.BINARY if fmt_name == "binary" else o.TERNARY
+    words, sc = _host_binary(0, rows, K) if fmt_name == "binary" else _host_ternary(ob, 0, rows, K)
+    ratio = ob.max_ratio(fmt, x, o.X_BF16, words, sc, K, Y[:, :rows].float().cpu().numpy())
+
+    def work(lo, hi):
+        ob.orc.gemv(fmt, x, o.X_BF16, words[lo:hi], sc[lo:hi], K)
+    dt, n = ob.time_items(work, rows, ob.cores)
+    del sets, ws
+    return {"workload": f"config {'5a' if fmt_name == 'binary' else '4b'}: {fmt_name} g128 prefill GEMM, "
+                        "M=512, K=5120, N=20480, x and y bf16",
+            "us": round(ms * 1e3, 1), "TFLOPs": round(tf, 1), "bound": "tensor",
+            "frac": round(tf / peaks["bf16_tflops"], 4), "peak": peaks["bf16_tflops"],
+            "timing": f"back-to-back calls rotating {nset} sets of weights, x and y "
+                      f"({nset * per_set / 1e6:.0f} MB vs {l2 / 1e6:.0f} MB L2)",
+            "parity": {"max_err_over_bound": round(ratio, 5), "rows": rows, "tokens": M},
+            "oracle": {"all_cores": {"GFLOPs": round(2 * M * n * K / dt / 1e9, 3), "cores": ob.cores,
+                                     "sample": f"{n} weight rows x 512 tokens x K, {dt:.3f} s"}}}
 
 
 # the 64 blocks of the full-depth decode step: (N, K) of each block's four binary GEMVs
@@ -304,35 +537,61 @@ FULL_DEPTH_BLOCK = [(9120, 5120), (5120, 5120), (40960, 5120), (5120, 20480)]
 FULL_DEPTH_BLOCKS = 64
 
 
-def full_depth_step(bq, device, stream, peaks):
+def full_depth_step(bq, device, stream, peaks, ob=None):
     """One decode token through all 64 blocks: 256 binary GEMVs at M = 1 (24.8e9 weights,
-    3.49 GB, every block's weights distinct), replayed as one CUDA graph."""
+    3.49 GB, every block's weights distinct), replayed as one CUDA graph. Each call is ordered
+    after the previous one on the stream, as the layers of a decode step are."""
     mats = []
     for b in range(FULL_DEPTH_BLOCKS):
         for j, (N, K) in enumerate(FULL_DEPTH_BLOCK):
             seed = 1000 + 4 * b + j
             mats.append(bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(seed, N, K, device=device),
                                     synth.scales(seed, N, K // 128, device=device)))
-    xs = {K: synth.activations(0, 1, K).to(device) for K in (5120, 20480)}
-    ys = {N: torch.empty((1, N), dtype=torch.float32, device=device) for (N, _) in FULL_DEPTH_BLOCK}
+    xh = {K: synth.activations(0, 1, K) for K in (5120, 20480)}
+    xs = {K: v.to(device) for K, v in xh.items()}
+    ys = {(N, K): torch.empty((1, N), dtype=torch.float32, device=device) for (N, K) in FULL_DEPTH_BLOCK}
     ws_bytes = max(bq.gemv_workspace_bytes(1, w) for w in mats[:4])
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
     total = sum(gemv_bytes(w.N, w.K, 1) for w in mats)
     with torch.cuda.stream(stream):
         for w in mats[:4]:
-            bq.gemv(xs[w.K], w, out=ys[w.N], workspace=ws)
+            bq.gemv(xs[w.K], w, out=ys[(w.N, w.K)], workspace=ws)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for w in mats:
-                bq.gemv(xs[w.K], w, out=ys[w.N], workspace=ws)
+                bq.gemv(xs[w.K], w, out=ys[(w.N, w.K)], workspace=ws)
         ms = time_single(g.replay, 20, 3, stream)
+    gbs = total / 1e9 / (ms / 1e3)
+    res = {"workload": "config 5b: full-depth decode step, 64 blocks x {9120x5120, 5120x5120, 40960x5120, "
+                       "5120x20480} binary GEMVs at M=1 (24.8e9 weights)",
+           "blocks": FULL_DEPTH_BLOCKS, "gemvs": 4 * FULL_DEPTH_BLOCKS, "bytes": total,
+           "us": round(ms * 1e3, 1), "tokens_per_s": round(1e3 / ms, 1), "GBps": round(gbs, 1),
+           "bound": "hbm", "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"],
+           "timing": "one CUDA graph of the 256 calls, 3.49 GB of distinct weights per step"}
+    if ob is not None:
+        # the last block's four outputs (held in ys after the graph) against the oracle
+        o = ob.o
+        ratios = []
+        g.replay()
+        torch.cuda.synchronize()
+        for j, (N, K) in enumerate(FULL_DEPTH_BLOCK):
+            seed = 1000 + 4 * (FULL_DEPTH_BLOCKS - 1) + j
+            words, sc = _host_binary(seed, 64, K)
+            ratios.append(ob.max_ratio(o.BINARY, xh[K], o.X_BF16, words, sc, K, ys[(N, K)][:, :64].cpu().numpy()))
+        res["parity"] = {"max_err_over_bound": round(max(ratios), 5), "rows": "64 of each of the last block's 4 GEMVs"}
+        timing = {}
+        for (N, K) in FULL_DEPTH_BLOCK:
+            words, sc = _host_binary(1000, 1024, K)
+            t = ob.gemv_timing(o.BINARY, xh[K], o.X_BF16, words, sc, K, K // 8 + K // 64, 2 * K, False)
+            timing[f"{N}x{K}"] = t["all_cores"]["GBps"]
+        gb_o = sum(timing.values()) / len(timing)
+        res["oracle"] = {"all_cores": {"GBps": round(gb_o, 4), "cores": ob.cores,
+                                       "tokens_per_s": round(gb_o * 1e9 / total, 6),
+                                       "sample": "up to 1024 rows of each block shape, mean GB/s of the four"}}
     del g, mats
     torch.cuda.empty_cache()
-    gbs = total / 1e9 / (ms / 1e3)
-    return {"blocks": FULL_DEPTH_BLOCKS, "gemvs": 4 * FULL_DEPTH_BLOCKS, "bytes": total,
-            "us": round(ms * 1e3, 1), "tokens_per_s": round(1e3 / ms, 1), "GBps": round(gbs, 1),
-            "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4)}
+    return res
 
 
 def stage_step_io(layer, device, pin):
@@ -535,13 +794,13 @@ def run_gpu(args):
         graphs, launches = capture_step_graphs(bq, sets, stream)
         torch.cuda.synchronize()
         clocks = ClockSampler(local) if rank == 0 else None
-        ms_total = time_graphs(graphs, args.steps, args.warmup, stream, dist, device)
+        ms_total, region_ms = time_regions(graphs, args.steps, args.warmup, stream, dist, device)
         clk = clocks.stop() if clocks else None
     ms_step = reduce_max(ms_total / args.steps, dist, device)
     value = world * step_bytes / 1e9 / (ms_step / 1e3)
     launches_timed = sum(launches[i % len(graphs)] for i in range(args.steps))
 
-    extras = {}
+    extras = None
     breakdown = None
     e2e = None
     if rank == 0 and not args.quick:
@@ -556,7 +815,10 @@ def run_gpu(args):
             except Exception as ex:   # keep the kernel-timed line; say why e2e is missing
                 e2e = {"error": str(ex).splitlines()[0][:200]}
             if rank == 0:
-                extras = extra_workloads(bq, device, stream, peaks)
+                try:
+                    extras = config_reports(bq, device, stream, peaks, OracleBench(), breakdown)
+                except Exception as ex:   # keep the headline line; say why the configs are missing
+                    extras = {"error": str(ex).splitlines()[0][:300]}
         if e2e is not None and "ms_per_step" in e2e:
             e2e_ms = reduce_max(e2e["ms_per_step"], dist, device)
             e2e["value"] = round(world * step_bytes / 1e9 / (e2e_ms / 1e3), 1)
@@ -582,26 +844,28 @@ def run_gpu(args):
                       f"({copies * step_bytes / 1e6:.0f} MB vs {l2 / 1e6:.0f} MB L2)",
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                 "bytes_per_step": step_bytes,
-                "timing": "CUDA graph per step (six launches), CUDA events on the launch stream",
+                "timing": f"CUDA graph per step (six GEMV calls, each ordered after the previous), CUDA "
+                          f"events on the launch stream; value from the median of {len(region_ms)} timed "
+                          f"regions of {args.steps} steps (min {min(region_ms) / args.steps:.5f}, max "
+                          f"{max(region_ms) / args.steps:.5f} ms per step)",
             },
             "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 1),
             "roofline": {
                 "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": tr["dram_bytes_per_step"] if tr else None,
-                "traffic_unit": "DRAM bytes per step (the twelve launches of six GEMVs), one ncu capture",
+                "traffic_unit": "DRAM bytes per step (the twelve launches of six GEMV calls), one ncu capture",
                 "bytes_per_step": step_bytes,
                 "peak_source": f"{peaks['source']} (HBM copy, burst)",
-                "kernel": "bq gemv: a prep kernel + gemv_tc_kernel (mma.sync, M <= 4) or gemv_tmem_kernel "
-                          "(tcgen05, M = 8) per GEMV, six GEMVs per step; achieved = algorithmic bytes "
-                          "per step / device time per step",
+                "kernel": "bq gemv: gemv_rows_prep_kernel (x digits) + gemv_rows_kernel (mma.sync s8, whole "
+                          "output rows per CTA) per GEMV call, six calls per step; achieved = algorithmic "
+                          "bytes per step / device time per step",
             },
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_timed,
             "clocks": clk,
-            "breakdown": breakdown,
-            "extras": extras,
+            "configs": extras,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

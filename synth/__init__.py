@@ -93,10 +93,12 @@ def random_signs(seed: int, tid: int, shape, device="cpu") -> torch.Tensor:
     return ((u >> 31) * 2 - 1).to(torch.int8).reshape(shape)
 
 
-def random_ternary(seed: int, tid: int, shape, device="cpu") -> torch.Tensor:
-    """int8 values in {-1, 0, +1}, each with probability 1/3 (Lemire multiply-shift)."""
+def random_ternary(seed: int, tid: int, shape, device="cpu", row0: int = 0) -> torch.Tensor:
+    """int8 values in {-1, 0, +1}, each with probability 1/3 (Lemire multiply-shift); with row0,
+    rows [row0, row0 + shape[0]) of a matrix whose rows have shape[1] elements."""
     n = math.prod(shape)
-    u = u32_stream(seed, tid, 0, n, device)
+    start = row0 * (n // shape[0]) if row0 else 0
+    u = u32_stream(seed, tid, start, n, device)
     return (((u * 3) >> 32) - 1).to(torch.int8).reshape(shape)
 
 

@@ -455,7 +455,8 @@ int rows_total_rt(int fmt, int CS, int G, int TB, int S)
 
 // Tiles per tile-group: as many as a CTA owns, up to 4 per warp group; two warp groups (16
 // consumer warps) at one column set when a CTA owns at least 8 tiles, where the stream is long
-// and more warps hide more latency. Stages: as many as fit, preferring (with one warp group) a
+// and more warps hide more latency (on the 248320-row LM head 8 warps measured 58% slower than
+// 16; 24 warps, at 80 registers a thread, 5% slower). Stages: as many as fit, preferring (with one warp group) a
 // footprint that lets two CTAs share an SM, so that the next call's CTA can become resident and
 // prefetch while this one runs; 0 stages if even three do not fit.
 RPlan rows_plan(int M, int fmt, int64_t N, int64_t K)
