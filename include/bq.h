@@ -227,6 +227,27 @@ bq_status bq_embed_gather(const int32_t *ids, int64_t T, const bq_weight *w, voi
  */
 bq_status bq_get_device_error(cudaStream_t stream);
 
+/*
+ * Test hooks for the failure paths (not for production use; process-wide, any thread).
+ *
+ * bq_debug_set_wait_limit_ns: the pipeline waits of the GEMV and prefill kernels (a stage of
+ * weights or x to arrive, a slot to free, the accumulator to complete) give up after `ns`
+ * nanoseconds instead of the built-in 2 s; 0 restores 2 s. Below 1000 ns (finer than the
+ * device timer) a wait gives up at its first poll that finds the phase incomplete, which makes
+ * a timeout certain on any call that waits for a copy. A wait that gives up records
+ * BQ_ERR_TIMEOUT in the device error word (see bq_get_device_error); the kernel then skips its
+ * remaining work, waits (2 s at most) for its copies and MMAs in flight, frees its tensor
+ * memory and returns, and that call's outputs are undefined. Later calls are unaffected.
+ *
+ * bq_debug_fail_next_launches: the next `count` compute calls (pack, unpack, gemv,
+ * gemv_noalloc, gemm_prefill, embed_gather) that pass argument validation return BQ_ERR_CUDA
+ * ("injected launch failure") without launching anything, as if their launch had failed.
+ * BQ_FAULT=launch or BQ_FAULT=launch:<count> in the environment sets the same when the library
+ * is loaded. 0 cancels.
+ */
+void bq_debug_set_wait_limit_ns(uint64_t ns);
+void bq_debug_fail_next_launches(int count);
+
 #ifdef __cplusplus
 }
 #endif

@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
             "bq_gemm_prefill_workspace_bytes": ([I64, W], ctypes.c_size_t),
             "bq_embed_gather": ([P, I64, W, P, I, P], I),
             "bq_get_device_error": ([P], I),
+            "bq_debug_set_wait_limit_ns": ([ctypes.c_uint64], None),
+            "bq_debug_fail_next_launches": ([I], None),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -286,3 +288,14 @@ def get_device_error():
     """Synchronise the current stream and raise BQError if a device-side condition was
     recorded (an out-of-range embedding id, a bounded wait that gave up)."""
     _check(lib().bq_get_device_error(_stream()))
+
+
+def debug_set_wait_limit_ns(ns: int):
+    """Test hook: the kernels' pipeline waits give up after `ns` ns (0: the built-in 2 s); a
+    wait that gives up is reported by get_device_error() as BQ_ERR_TIMEOUT."""
+    lib().bq_debug_set_wait_limit_ns(int(ns))
+
+
+def debug_fail_next_launches(count: int):
+    """Test hook: the next `count` compute calls fail with BQ_ERR_CUDA before launching."""
+    lib().bq_debug_fail_next_launches(int(count))

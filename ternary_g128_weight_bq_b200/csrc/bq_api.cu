@@ -2,6 +2,7 @@
 // codes and the per-device error word.
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -16,6 +17,36 @@ __device__ unsigned int g_status[4];
 
 static thread_local char t_msg[512] = "no error";
 static unsigned long long g_launches = 0;
+
+// Test hooks (bq_debug_*): a shorter limit for the kernels' pipeline waits, and a number of
+// compute calls that fail as if their launch had failed. BQ_FAULT=launch[:count] in the
+// environment sets the latter when the library is loaded.
+static uint64_t g_wait_ns = 0;
+static int g_fail_launches = 0;
+
+static int fault_from_env()
+{
+    const char *f = getenv("BQ_FAULT");
+    if (!f || strncmp(f, "launch", 6) != 0)
+        return 0;
+    return f[6] == ':' ? atoi(f + 7) : 1;
+}
+[[maybe_unused]] static const int g_env_fault = (__atomic_store_n(&g_fail_launches, fault_from_env(), __ATOMIC_RELAXED), 0);
+
+uint64_t pipeline_wait_ns()
+{
+    const uint64_t v = __atomic_load_n(&g_wait_ns, __ATOMIC_RELAXED);
+    return v ? v : kWaitLimitDefaultNs;
+}
+
+bool take_injected_launch_failure()
+{
+    int n = __atomic_load_n(&g_fail_launches, __ATOMIC_RELAXED);
+    while (n > 0)
+        if (__atomic_compare_exchange_n(&g_fail_launches, &n, n - 1, false, __ATOMIC_RELAXED, __ATOMIC_RELAXED))
+            return true;
+    return false;
+}
 
 void note_launches(unsigned n) { __atomic_fetch_add(&g_launches, (unsigned long long)n, __ATOMIC_RELAXED); }
 
@@ -146,6 +177,8 @@ static bq_status pack_common(int fmt, const int8_t *q, const uint16_t *s_in, int
         return set_error(BQ_ERR_SHAPE, "pack: N=%lld K=%lld invalid", (long long)N, (long long)K);
     if (!aligned16(q) || !aligned16(words))
         return set_error(BQ_ERR_ALIGNMENT, "pack: q and words must be 16-byte aligned");
+    if (take_injected_launch_failure())
+        return set_error(BQ_ERR_CUDA, "%s: injected launch failure (test hook)", "pack");
     bq_status st;
     unsigned int *status = device_status(&st);
     if (!status)
@@ -194,6 +227,8 @@ bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStr
         return set_error(BQ_ERR_INVALID_ARG, "unpack: q is NULL");
     if (!aligned16(q))
         return set_error(BQ_ERR_ALIGNMENT, "unpack: q must be 16-byte aligned");
+    if (take_injected_launch_failure())
+        return set_error(BQ_ERR_CUDA, "%s: injected launch failure (test hook)", "unpack");
     unsigned int *status = device_status(&st);
     if (!status)
         return st;
@@ -255,11 +290,14 @@ bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, voi
                          workspace ? ws_bytes : (size_t)0);
     if (workspace && !aligned16(workspace))
         return set_error(BQ_ERR_ALIGNMENT, "gemv: workspace must be 16-byte aligned");
+    if (take_injected_launch_failure())
+        return set_error(BQ_ERR_CUDA, "%s: injected launch failure (test hook)", "gemv");
     unsigned int *status = device_status(&st);
     if (!status)
         return st;
     GemvArgs a{x, (int)xt, (int)M, (int)w->fmt, w->N, w->K, w->words,
-               reinterpret_cast<const __half *>(w->scales), y, (int)yt, workspace, ws_bytes, status};
+               reinterpret_cast<const __half *>(w->scales), y, (int)yt, workspace, ws_bytes, status,
+               pipeline_wait_ns()};
     unsigned launches = 0;
     cudaError_t e = launch_gemv(a, stream, &launches);
     if (e != cudaSuccess)
@@ -278,6 +316,8 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
         return st;
     if (M < 1 || M > 8)
         return set_error(BQ_ERR_SHAPE, "gemv_noalloc: M=%lld, need 1 <= M <= 8", (long long)M);
+    if (take_injected_launch_failure())
+        return set_error(BQ_ERR_CUDA, "%s: injected launch failure (test hook)", "gemv_noalloc");
     unsigned int *status = device_status(&st);
     if (!status)
         return st;
@@ -296,7 +336,7 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
                              need, cap);
     }
     GemvArgs a{x, (int)xt, (int)M, (int)w->fmt, w->N, w->K, w->words,
-               reinterpret_cast<const __half *>(w->scales), y, (int)yt, scratch, cap, status};
+               reinterpret_cast<const __half *>(w->scales), y, (int)yt, scratch, cap, status, pipeline_wait_ns()};
     unsigned launches = 0;
     cudaError_t e = launch_gemv(a, stream, &launches);
     if (e != cudaSuccess)
@@ -327,11 +367,14 @@ bq_status bq_gemm_prefill(const void *x, bq_dtype xt, int64_t M, const bq_weight
         return set_error(BQ_ERR_WORKSPACE, "gemm_prefill: workspace needs %zu bytes", need);
     if (workspace && !aligned16(workspace))
         return set_error(BQ_ERR_ALIGNMENT, "gemm_prefill: workspace must be 16-byte aligned");
+    if (take_injected_launch_failure())
+        return set_error(BQ_ERR_CUDA, "%s: injected launch failure (test hook)", "gemm_prefill");
     unsigned int *status = device_status(&st);
     if (!status)
         return st;
     PrefillArgs a{x, (int)xt, M, (int)w->fmt, w->N, w->K, w->words,
-                  reinterpret_cast<const __half *>(w->scales), y, (int)yt, need ? workspace : nullptr, status};
+                  reinterpret_cast<const __half *>(w->scales), y, (int)yt, need ? workspace : nullptr, status,
+                  pipeline_wait_ns()};
     unsigned launches = 0;
     cudaError_t e = launch_prefill(a, stream, &launches);
     if (e != cudaSuccess)
@@ -354,6 +397,8 @@ bq_status bq_embed_gather(const int32_t *ids, int64_t T, const bq_weight *w, voi
         return set_error(BQ_ERR_DTYPE, "embed_gather: out must be BQ_F32, BQ_BF16 or BQ_F16");
     if (!aligned16(out))
         return set_error(BQ_ERR_ALIGNMENT, "embed_gather: out must be 16-byte aligned");
+    if (take_injected_launch_failure())
+        return set_error(BQ_ERR_CUDA, "%s: injected launch failure (test hook)", "embed_gather");
     unsigned int *status = device_status(&st);
     if (!status)
         return st;
@@ -365,6 +410,13 @@ bq_status bq_embed_gather(const int32_t *ids, int64_t T, const bq_weight *w, voi
         return set_error(BQ_ERR_CUDA, "embed_gather launch: %s", cudaGetErrorString(e));
     note_launches(1);
     return BQ_OK;
+}
+
+void bq_debug_set_wait_limit_ns(uint64_t ns) { __atomic_store_n(&g_wait_ns, ns, __ATOMIC_RELAXED); }
+
+void bq_debug_fail_next_launches(int count)
+{
+    __atomic_store_n(&g_fail_launches, count > 0 ? count : 0, __ATOMIC_RELAXED);
 }
 
 bq_status bq_get_device_error(cudaStream_t stream)

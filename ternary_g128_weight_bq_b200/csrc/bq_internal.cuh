@@ -24,6 +24,14 @@ unsigned int *device_status(bq_status *st);
 
 bq_status set_error(bq_status st, const char *fmt, ...);
 
+// Limit of a bounded device-side wait: 2 s. Pipeline waits use the (test-only) shorter limit set
+// by bq_debug_set_wait_limit_ns when there is one; the waits that drain copies and MMAs before a
+// kernel exits always use this one.
+constexpr uint64_t kWaitLimitDefaultNs = 2000000000ull;
+uint64_t pipeline_wait_ns();
+// True (once per injected failure) when a test asked the next launches to fail.
+bool take_injected_launch_failure();
+
 // Count of kernel launches enqueued by the library (instrumentation for benchmarks).
 void note_launches(unsigned n);
 bq_status check_launch(const char *what);
@@ -52,6 +60,7 @@ struct GemvArgs {
     void *workspace;
     size_t ws_bytes;
     unsigned int *dev_status;
+    uint64_t wait_ns;         // limit of the kernels' pipeline waits (bq_debug_set_wait_limit_ns)
 };
 size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches);
@@ -76,6 +85,7 @@ struct PrefillArgs {
     int yt;
     void *workspace;          // fp32 partials of split tail tiles (prefill_workspace_bytes)
     unsigned int *dev_status;
+    uint64_t wait_ns;         // limit of the kernels' pipeline waits (bq_debug_set_wait_limit_ns)
 };
 size_t prefill_workspace_bytes(int64_t M, int fmt, int64_t N, int64_t K);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s, unsigned *launches);

@@ -43,9 +43,9 @@
 // split grid and the reduce are programmatic dependent launches: the split CTAs take SMs as
 // the whole-tile grid frees them, and each dependent grid completes only after its
 // predecessor, so the stream order seen by later work is unchanged.
-// The expanded weights exist only on chip. Every mbarrier wait is bounded: after
-// 2 s the kernel records kDevErrTimeout, lets its copies and MMAs drain, frees TMEM and
-// returns.
+// The expanded weights exist only on chip. Every mbarrier wait is bounded: after 2 s (or the
+// shorter test limit of bq_debug_set_wait_limit_ns, for the pipeline waits) the kernel records
+// kDevErrTimeout, lets its copies and MMAs drain (those waits keep 2 s), frees TMEM and returns.
 #include <cuda.h>
 
 #include <cstring>
@@ -62,7 +62,7 @@ constexpr int kDequantWarps = 8;      // kParts per weight row: each expands 1/k
                                       // (16 warps, four per row, measured slower)
 constexpr int kParts = kDequantWarps / 4;
 constexpr int kThreads = (2 + kDequantWarps) * 32;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kWaitLimitNs = kWaitLimitDefaultNs;   // drain waits before exit
 
 // X tiles come by TMA into a shared-memory ring; A tiles (the +-s operand) are written by the
 // dequant warps straight into tensor memory, next to the accumulator: D in columns [0, BN),
@@ -96,14 +96,15 @@ struct Bars {
 // Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast, then every lane
 // observes the (already completed) phase itself so that it acquires the producer's writes.
 // All lanes return the same value, so later warp-collective instructions stay converged.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err)
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err,
+                                          uint64_t limit)
 {
     bool ok = true;
     if ((threadIdx.x & 31) == 0)
-        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, kWaitLimitNs);
+        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, limit);
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok)
-        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, kWaitLimitNs);
+        ok = ptx::mbar_wait_bounded(bar, parity, abort, err, kDevErrTimeout, limit);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -150,6 +151,21 @@ __device__ __forceinline__ void expand_pairs(uint2 wv, uint32_t s2, uint32_t (&a
 }
 
 __device__ __forceinline__ uint32_t scale_pair(uint16_t s_f16) { return (uint32_t)s_f16 | ((uint32_t)s_f16 << 16); }
+
+// floor(log2 a) of a finite a > 0, from its bits (subnormals included).
+__device__ __forceinline__ int ilog2_pos(float a)
+{
+    const uint32_t u = __float_as_uint(a);
+    return u >= 0x00800000u ? (int)(u >> 23) - 127 : -118 - (int)__clz(u);
+}
+
+// 2^k as a float for k in [-149, 127] (exact; subnormal below -126), 0 below.
+__device__ __forceinline__ float pow2_float(int k)
+{
+    if (k >= -126)
+        return __uint_as_float((uint32_t)(k + 127) << 23);
+    return k >= -149 ? __uint_as_float(1u << (k + 149)) : 0.f;
+}
 
 // bf16 x -> fp16 x * 2^e_m, one block per token row m: e_m puts the row's largest finite
 // magnitude in [2^14, 2^15) (e_m = 0 for a row with no finite non-zero value), and tok_fac[m]
@@ -203,19 +219,17 @@ prefill_x16_kernel(const __nv_bfloat16 *__restrict__ x, int64_t K, __half *__res
 #pragma unroll
     for (int i = 1; i < kX16Threads / 32; i++)
         amax = fmaxf(amax, wmax[i]);
-    int e = 0;
-    if (amax > 0.f) {
-        int ex;
-        frexpf(amax, &ex);                 // amax = f 2^ex, f in [0.5, 1)
-        e = 15 - ex;                       // amax 2^e in [2^14, 2^15)
-    }
+    // e = 14 - floor(log2 amax) puts amax 2^e in [2^14, 2^15); the factor 2^e is applied as two
+    // exact power-of-two multiplies (e reaches 147 for the smallest bf16 subnormal)
+    const int e = amax > 0.f ? 14 - ilog2_pos(amax) : 0;
+    const float f1 = pow2_float(e < 127 ? e : 127), f2 = pow2_float(e > 127 ? e - 127 : 0);
     auto convert = [&](const uint4 &v) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t o[4];
 #pragma unroll
         for (int i = 0; i < 4; i++) {
             const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
-            const __half2 h = __halves2half2(__float2half_rn(ldexpf(f.x, e)), __float2half_rn(ldexpf(f.y, e)));
+            const __half2 h = __floats2half2_rn(f.x * f1 * f2, f.y * f1 * f2);
             o[i] = *reinterpret_cast<const uint32_t *>(&h);
         }
         return make_uint4(o[0], o[1], o[2], o[3]);
@@ -229,7 +243,7 @@ prefill_x16_kernel(const __nv_bfloat16 *__restrict__ x, int64_t K, __half *__res
     for (int c = threadIdx.x + kHeld * kX16Threads; c < chunks; c += kX16Threads)
         dst[c] = convert(__ldg(src + c));
     if (threadIdx.x == 0)
-        tok_fac[m] = ldexpf(1.f, -e);      // exact: -e is in [-147, 113]
+        tok_fac[m] = pow2_float(-e);       // exact: -e is in [-147, 113]
 }
 
 // tok_fac: the per-token factor 2^-e_m of bf16 x (NULL for fp16 x, which is used as it is).
@@ -239,7 +253,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                const uint32_t *__restrict__ words,
                const uint16_t *__restrict__ scales, int64_t M, int64_t N, int64_t K, void *__restrict__ y,
                int yt, int tiles_m, int tile0, int splits, float *__restrict__ part,
-               const float *__restrict__ tok_fac, unsigned int *dev_status)
+               const float *__restrict__ tok_fac, unsigned int *dev_status, uint64_t wait_ns)
 {
     using C = Cfg<BN>;
     constexpr int SX = C::kXStages, SA = C::kAStages;
@@ -307,7 +321,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             for (int kb = 0; kb < KB; kb++) {
                 const int s = kb % SX;
                 const uint32_t ph = (kb / SX) & 1;
-                if (!ptx::mbar_wait_bounded_sleep(&bars->empty_x[s], ph ^ 1, abort, err, kDevErrTimeout, kWaitLimitNs))
+                if (!ptx::mbar_wait_bounded_sleep(&bars->empty_x[s], ph ^ 1, abort, err, kDevErrTimeout, wait_ns))
                     break;
                 ptx::mbar_arrive_expect_tx(&bars->full_x[s], C::kXBytes);
                 ptx::tma_load_2d(xs + s * C::kXBytes, &tmap_x, &bars->full_x[s], (kb0 + kb) * kBK, (int32_t)m0);
@@ -327,9 +341,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             int issued = 0;
             for (int kb = 0; kb < KB; kb++) {
                 const int sx = kb % SX, sa = kb % SA;
-                if (!ptx::mbar_wait_bounded(&bars->full_x[sx], (kb / SX) & 1, abort, err, kDevErrTimeout, kWaitLimitNs))
+                if (!ptx::mbar_wait_bounded(&bars->full_x[sx], (kb / SX) & 1, abort, err, kDevErrTimeout, wait_ns))
                     break;
-                if (!ptx::mbar_wait_bounded(&bars->full_a[sa], (kb / SA) & 1, abort, err, kDevErrTimeout, kWaitLimitNs))
+                if (!ptx::mbar_wait_bounded(&bars->full_a[sa], (kb / SA) & 1, abort, err, kDevErrTimeout, wait_ns))
                     break;
                 ptx::tc_fence_after();
                 const uint32_t a_tmem = tmem_d + BN + 32 * sa;
@@ -405,7 +419,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 
             const int s = kb % SA;
             const uint32_t ph = (kb / SA) & 1;
-            if (!warp_wait(&bars->empty_a[s], ph ^ 1, abort, err))
+            if (!warp_wait(&bars->empty_a[s], ph ^ 1, abort, err, wait_ns))
                 break;
             ptx::tc_fence_after();
             const uint32_t s2 = row_ok ? scale_pair(sv) : 0u;
@@ -435,7 +449,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         const bool staged_out = splits == 1 && y_tma;
         if (tok_fac && splits == 1)
             asm volatile("griddepcontrol.wait;" ::: "memory");   // tok_fac comes from the conversion pass
-        if (warp_wait(&bars->acc_full, 0, abort, err)) {
+        if (warp_wait(&bars->acc_full, 0, abort, err, wait_ns)) {
             ptx::tc_fence_after();
             const int quad = warp & 3;                       // TMEM lanes 32*quad .. +31
             const int64_t nrow = n0 + quad * 32 + lane;
@@ -702,10 +716,11 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
         wcfg.attrs = attr;
         wcfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&wcfg, kern, map, map_y, y_tma, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m, 0,
-                               1, part, (const float *)tok_fac, a.dev_status);
+                               1, part, (const float *)tok_fac, a.dev_status, a.wait_ns);
     } else {
         kern<<<pl.full, kThreads, Cfg<BN>::kSmem, s>>>(map, map_y, y_tma, a.words, sc, a.M, a.N, a.K, a.y, a.yt,
-                                                       pl.tiles_m, 0, 1, part, (const float *)nullptr, a.dev_status);
+                                                       pl.tiles_m, 0, 1, part, (const float *)nullptr, a.dev_status,
+                                                       a.wait_ns);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess)
@@ -723,7 +738,7 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, kern, map, map_y, y_tma, a.words, sc, a.M, a.N, a.K, a.y, a.yt, pl.tiles_m,
-                               pl.full, pl.splits, part, (const float *)tok_fac, a.dev_status);
+                               pl.full, pl.splits, part, (const float *)tok_fac, a.dev_status, a.wait_ns);
         if (e != cudaSuccess)
             return e;
         const int64_t n_out = (int64_t)pl.tail * BN * kBM;

@@ -17,6 +17,10 @@
 // below the ~160 binary weights per SM clock that HBM delivers; mma.sync takes its operands from
 // registers and peaks at ~240.
 //
+// Every wait is bounded: a pipeline wait that gives up (after 2 s, or the shorter test limit of
+// bq_debug_set_wait_limit_ns) records kDevErrTimeout and makes the CTA skip its remaining work;
+// the producer still waits (2 s at most) for its copies in flight before the CTA exits.
+//
 // What this file decides is the work split and the latency of a call:
 //   * Rows. The N outputs are 16-row tiles; CTA b owns tiles [b T / P, (b+1) T / P) over all of
 //     K, so no output is split between CTAs: no partial sums in device memory, no counters, no
@@ -54,7 +58,7 @@ constexpr int kWarpTiles = 4;                 // 16-row tiles a warp takes per s
 constexpr int kMaxStages = 8;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kSmemPair = 113 * 1024;         // two CTAs fit on one SM below this
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kWaitLimitNs = kWaitLimitDefaultNs;   // drain waits before exit
 
 template <int FMT> struct RCfg {
     static constexpr int kBoxes = FMT == BQ_BINARY_G128 ? 1 : 2;   // 128-byte boxes per tile per slice
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__((WG * kGroupWarps + 1) * 32, CS == 1 && WG == 
 gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s, int M,
                  int64_t N, int64_t K, void *__restrict__ y, int yt, int T, int TB, int S,
                  const uint32_t *__restrict__ frag_g, const float *__restrict__ colf_g, const int *__restrict__ cfix_g,
-                 uint32_t one, unsigned int *dev_status)
+                 uint32_t one, unsigned int *dev_status, uint64_t wait_ns)
 {
     using SCH = Scheme<FMT, CS>;
     constexpr int kConsumers = WG * kGroupWarps;
@@ -248,7 +252,7 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
                 for (int c = 0; c < C; c++, it++) {
                     // a free slot: the producer sleeps in the wait, leaving the issue slots to the consumers
                     if (!ptx::mbar_wait_bounded_sleep(&bars->empty[s], ph ^ 1, abort, err, kDevErrTimeout,
-                                                      kWaitLimitNs)) {
+                                                      wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -289,7 +293,7 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
             ptx::bulk_load(cfix_s, cfix_g, xb, &bars->frag);
         }
         bool ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&bars->frag, 0, abort, err, kDevErrTimeout,
-                                                                 kWaitLimitNs));
+                                                                 wait_ns));
 
         Lane ln;
         if (SCH::kMask) {
@@ -340,7 +344,7 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
             for (int c = 0; c < C; c++) {
                 if (ok)
                     ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&bars->full[s], ph, abort, err,
-                                                                        kDevErrTimeout, kWaitLimitNs));
+                                                                        kDevErrTimeout, wait_ns));
                 if (ok) {
                     const uint8_t *st = ring + s * L.stage_bytes;
                     const int q = 8 * c + w;                    // this warp's group
@@ -558,7 +562,7 @@ cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, mw, ms, a.M, a.N, a.K, a.y, a.yt, pl.T, pl.TB, pl.S, (const uint32_t *)frag,
-                              (const float *)colf, (const int *)cfix, 1u, a.dev_status);
+                              (const float *)colf, (const int *)cfix, 1u, a.dev_status, a.wait_ns);
 }
 
 template <int FMT, typename XT>

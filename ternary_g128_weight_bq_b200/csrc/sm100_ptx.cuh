@@ -56,6 +56,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// A limit below this gives up at the first poll that finds the phase incomplete (a test mode:
+// the device timer is coarser than such limits, and try_wait may itself block until the phase
+// completes).
+constexpr uint64_t kImmediateLimitNs = 1000;
+
 // As mbar_try_wait, but the thread may sleep up to `hint_ns` for the phase to complete instead
 // of returning at once: for waiters that are not on the critical path (a producer waiting for a
 // free slot), so that they do not take issue slots from the warps that compute.
@@ -79,6 +98,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
                                                   unsigned int *err, unsigned int timeout_bit,
                                                   uint64_t limit_ns)
 {
+    if (limit_ns < kImmediateLimitNs) {
+        if (mbar_test_wait(bar, parity))
+            return true;
+        atomicOr(err, timeout_bit);
+        *abort = 1;
+        return false;
+    }
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer_ns();
@@ -102,6 +128,8 @@ __device__ __forceinline__ bool mbar_wait_bounded_sleep(uint64_t *bar, uint32_t 
                                                         unsigned int *err, unsigned int timeout_bit,
                                                         uint64_t limit_ns)
 {
+    if (limit_ns < kImmediateLimitNs)
+        return mbar_wait_bounded(bar, parity, abort, err, timeout_bit, limit_ns);
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer_ns();

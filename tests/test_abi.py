@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -125,3 +126,52 @@ def test_noalloc_array_covers_every_supported_shape(libbq):
                     worst = max(worst, need)
                     assert need <= cap, (fmt, M, K, N, need, cap)
     assert worst > 0
+
+
+def _gemv_call(libbq):
+    """bq_gemv with valid-looking arguments (aligned fake pointers): validation passes."""
+    w = bq._Weight(bq.BINARY_G128, 256, 1024, 1 << 20, 1 << 21)
+    return libbq.bq_gemv(1 << 22, 1, 1, ctypes.byref(w), 1 << 23, 2, 1 << 24, 1 << 20, None)
+
+
+def test_injected_launch_failure(libbq):
+    """bq_debug_fail_next_launches(n): the next n calls that pass validation return
+    BQ_ERR_CUDA with the injected-failure message and launch nothing; invalid arguments are
+    still reported as such first."""
+    libbq.bq_debug_fail_next_launches(2)
+    try:
+        w = bq._Weight(bq.BINARY_G128, 256, 1000, 1 << 20, 1 << 21)          # K not a multiple of 128
+        assert libbq.bq_gemv(1 << 22, 1, 1, ctypes.byref(w), 1 << 23, 2, None, 0, None) == 2
+        for _ in range(2):
+            assert _gemv_call(libbq) == 6
+            assert b"injected launch failure" in libbq.bq_last_error()
+        st = _gemv_call(libbq)                                                # back to the real path
+        assert b"injected" not in libbq.bq_last_error()
+        if not torch_cuda_available():
+            assert st == 6                                                    # no device here
+    finally:
+        libbq.bq_debug_fail_next_launches(0)
+
+
+def torch_cuda_available():
+    import torch
+    return torch.cuda.is_available()
+
+
+def test_fault_injection_from_environment(tmp_path):
+    """BQ_FAULT=launch:2 makes the first two compute calls of a fresh process fail as injected."""
+    code = (
+        "import ctypes, sys\n"
+        f"sys.path.insert(0, {ROOT!r})\n"
+        "import ternary_g128_weight_bq_b200 as bq\n"
+        "L = bq.lib()\n"
+        "w = bq._Weight(0, 256, 1024, 1 << 20, 1 << 21)\n"
+        "out = []\n"
+        "for _ in range(3):\n"
+        "    L.bq_gemv(1 << 22, 1, 1, ctypes.byref(w), 1 << 23, 2, 1 << 24, 1 << 20, None)\n"
+        "    out.append(b'injected' in L.bq_last_error())\n"
+        "print(out)\n")
+    env = dict(os.environ, BQ_FAULT="launch:2")
+    p = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, timeout=120)
+    assert p.returncode == 0, p.stderr
+    assert p.stdout.strip().splitlines()[-1] == "[True, True, False]"
