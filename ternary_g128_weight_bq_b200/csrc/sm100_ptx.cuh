@@ -240,7 +240,7 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, ui
         : "memory");
 }
 
-// 32 lanes x 16 consecutive 32-bit columns: thread i writes r[0..15] to lane (base + i).
+// 32 lanes x 8 consecutive 32-bit columns: thread i writes r[0..7] to lane (base + i).
 __device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8])
 {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
