@@ -22,6 +22,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 BINARY = 0
 TERNARY = 1
+TERNARY_B3 = 2
 X_F16 = 0
 X_BF16 = 1
 OK = 0
@@ -79,6 +80,18 @@ def _u32(a) -> np.ndarray:
     return a.view(np.uint32)
 
 
+def _weights(fmt: int, a) -> np.ndarray:
+    """Packed weights as the oracle reads them: uint32 words, or bytes for base-3."""
+    if fmt != TERNARY_B3:
+        return _u32(a)
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().contiguous().numpy()
+    a = np.ascontiguousarray(a)
+    if a.dtype not in (np.uint8, np.int8):
+        raise TypeError(f"expected bytes, got {a.dtype}")
+    return a.view(np.uint8)
+
+
 def _i8(a) -> np.ndarray:
     if hasattr(a, "detach"):
         a = a.detach().cpu().contiguous().numpy()
@@ -106,10 +119,12 @@ class Oracle:
         L.bqo_f64_to_f16.restype = ctypes.c_uint16
         L.bqo_words_per_row.argtypes = [ctypes.c_int, I64]
         L.bqo_words_per_row.restype = I64
-        for f in (L.bqo_pack_binary_g128, L.bqo_pack_ternary_g128):
+        L.bqo_row_bytes.argtypes = [ctypes.c_int, I64]
+        L.bqo_row_bytes.restype = I64
+        for f in (L.bqo_pack_binary_g128, L.bqo_pack_ternary_g128, L.bqo_pack_ternary_b3):
             f.argtypes = [P, P, I64, I64, P, P]
             f.restype = ctypes.c_int
-        for f in (L.bqo_unpack_binary_g128, L.bqo_unpack_ternary_g128):
+        for f in (L.bqo_unpack_binary_g128, L.bqo_unpack_ternary_g128, L.bqo_unpack_ternary_b3):
             f.argtypes = [P, I64, I64, P]
             f.restype = I64
         L.bqo_weight.argtypes = [ctypes.c_int, P, P, I64, I64, I64]
@@ -128,31 +143,40 @@ class Oracle:
     def words_per_row(self, fmt: int, K: int) -> int:
         return int(self.L.bqo_words_per_row(fmt, K))
 
+    def row_bytes(self, fmt: int, K: int) -> int:
+        return int(self.L.bqo_row_bytes(fmt, K))
+
     def pack(self, fmt: int, q, s):
-        """(q int8[N,K], s fp16[N,K/128]) -> (status, words uint32[N,W], s_out uint16)."""
+        """(q int8[N,K], s fp16[N,K/128]) -> (status, packed, s_out uint16); packed is
+        uint32[N, W] for the binary and 2-bit formats and uint8[N, 26 K/128] for base-3."""
         q = _i8(q)
         s = _bits16(s)
         N, K = q.shape
-        W = self.words_per_row(fmt, K)
-        if W < 0:
+        RB = self.row_bytes(fmt, K)
+        if RB < 0:
             return ERR_SHAPE, None, None
-        words = np.zeros((N, W), dtype=np.uint32)
+        if fmt == TERNARY_B3:
+            words = np.zeros((N, RB), dtype=np.uint8)
+        else:
+            words = np.zeros((N, RB // 4), dtype=np.uint32)
         s_out = np.zeros((N, K // 128), dtype=np.uint16)
-        f = self.L.bqo_pack_binary_g128 if fmt == BINARY else self.L.bqo_pack_ternary_g128
+        f = {BINARY: self.L.bqo_pack_binary_g128, TERNARY: self.L.bqo_pack_ternary_g128,
+             TERNARY_B3: self.L.bqo_pack_ternary_b3}[fmt]
         st = f(_p(q), _p(s), N, K, _p(words), _p(s_out))
         return st, words, s_out
 
     def unpack(self, fmt: int, words, K: int):
-        """words[N, W] -> (q int8[N, K], number of invalid codes)."""
-        w = _u32(words)
+        """packed[N, ...] -> (q int8[N, K], number of invalid codes or bytes)."""
+        w = _weights(fmt, words)
         N = w.shape[0]
         q = np.zeros((N, K), dtype=np.int8)
-        f = self.L.bqo_unpack_binary_g128 if fmt == BINARY else self.L.bqo_unpack_ternary_g128
+        f = {BINARY: self.L.bqo_unpack_binary_g128, TERNARY: self.L.bqo_unpack_ternary_g128,
+             TERNARY_B3: self.L.bqo_unpack_ternary_b3}[fmt]
         bad = f(_p(w), N, K, _p(q))
         return q, int(bad)
 
     def dequant(self, fmt: int, words, scales, K: int) -> np.ndarray:
-        w = _u32(words)
+        w = _weights(fmt, words)
         s = _bits16(scales)
         N = w.shape[0]
         out = np.zeros((N, K), dtype=np.float64)
@@ -165,7 +189,7 @@ class Oracle:
         """y[M, R] and bound[M, R] in fp64 for the selected rows (all rows by default)."""
         xb = _bits16(x)
         M = xb.shape[0]
-        w = _u32(words)
+        w = _weights(fmt, words)
         s = _bits16(scales)
         N = w.shape[0]
         r = (np.arange(N, dtype=np.int64) if rows is None
@@ -181,7 +205,7 @@ class Oracle:
     def embed(self, fmt: int, ids, words, scales, K: int):
         """(out fp64[T, K], number of out-of-range ids)."""
         i = np.ascontiguousarray(ids.numpy() if hasattr(ids, "numpy") else ids, dtype=np.int32)
-        w = _u32(words)
+        w = _weights(fmt, words)
         s = _bits16(scales)
         out = np.zeros((len(i), K), dtype=np.float64)
         bad = self.L.bqo_embed(fmt, _p(i), len(i), _p(w), _p(s), w.shape[0], K, _p(out))

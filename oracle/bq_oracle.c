@@ -35,6 +35,8 @@
  *   - Ternary codes are 2-bit fields, LSB-first: bits 2*(k % 16)..2*(k % 16)+1 of word
  *     (k / 16) hold code c with value c - 1 (0 -> -1, 1 -> 0, 2 -> +1); c = 3 is invalid.
  *   - Scales are IEEE binary16 [N, K/128]; x is binary16 or bfloat16 [M, K].
+ *   - Base-3 ternary storage (BQO_TERNARY_B3): see the section "Ternary g128 in base-3
+ *     storage" below for the byte layout, which the pages leave open.
  *   - The tolerance bound of an output is 2e-3 * sum_k |x[m,k] * s[n, k/128]|; for
  *     ternary weights the scale counts even where the code is 0.
  */
@@ -144,6 +146,19 @@ int64_t bqo_words_per_row(int fmt, int64_t K)
     return -1;
 }
 
+int64_t bqo_row_bytes(int fmt, int64_t K)
+{
+    if (K <= 0 || K % 128)
+        return -1;
+    if (fmt == BQO_BINARY)
+        return K / 8;
+    if (fmt == BQO_TERNARY)
+        return K / 4;
+    if (fmt == BQO_TERNARY_B3)
+        return 26 * (K / 128);    /* 26 bytes per group of 128 */
+    return -1;
+}
+
 /* ---------------------------------------------------------------------------------------
  * Pack / unpack: loop over every k and set or read its bit (binary) or 2-bit field
  * (ternary). [card] "Weight representation: Binary g128"; [tern] 2-bit storage.
@@ -227,8 +242,123 @@ int64_t bqo_unpack_ternary_g128(const uint32_t *words, int64_t N, int64_t K, int
 }
 
 /* ---------------------------------------------------------------------------------------
+ * Ternary g128 in base-3 storage (BQO_TERNARY_B3).
+ * [tern] "局限性与未来发展": the deployed ternary model keeps 2-bit codes (7.2 GB) while the
+ * information is 1.71 bits per weight (5.9 GB), and native ternary kernels are still to
+ * come; [agent] "两种硬件对应的运行点" gives the same 1.71 bits per weight and 5.9 GB. The
+ * pages give no base-3 layout; this is the library's reading:
+ *   - The codes c = value + 1 in {0, 1, 2} of a group of 128 are stored in 26 bytes:
+ *     bytes 0..23 hold five codes each (positions 5j .. 5j+4 of the group), bytes 24 and
+ *     25 four codes each (positions 120..123 and 124..127).
+ *   - A byte holding n codes c_0 .. c_{n-1} (c_0 at the lowest position) stores
+ *     ceil(256 v / 3^n), v = sum_p c_p 3^(n-1-p): the codes read as a base-3 number,
+ *     first code most significant, kept as the fraction v / 3^n in 8-bit fixed point
+ *     rounded up. v is floor(byte * 3^n / 256).
+ *   - A row is a run of blocks of 8 groups (the last block may hold fewer, nb). A block
+ *     stores the 24 five-code bytes of each of its groups first (group i of the block at
+ *     byte 24 i) and then the two four-code bytes of each (group i at 24 nb + 2 i). A row
+ *     is 26 K / 128 bytes; with the fp16 scale, (26 * 8 + 16) / 128 = 1.75 bits per weight.
+ *   - 243 of the 256 byte values are written for five codes and 81 for four; any other
+ *     value is invalid (the pack never writes it; the unpack counts it).
+ * ------------------------------------------------------------------------------------- */
+
+static const int64_t kPow3[6] = {1, 3, 9, 27, 81, 243};
+
+/* Byte j (0..25) of a group holds b3_count(j) codes starting at position b3_first(j). */
+static int b3_count(int j) { return j < 24 ? 5 : 4; }
+static int b3_first(int j) { return j < 24 ? 5 * j : 120 + 4 * (j - 24); }
+
+/* The byte of a group that holds position kk (0..127). */
+static int b3_byte_of(int kk) { return kk < 120 ? kk / 5 : 24 + (kk - 120) / 4; }
+
+/* Offset, within a row of G groups, of byte j of group g. */
+static int64_t b3_byte_offset(int64_t G, int64_t g, int j)
+{
+    int64_t first = 8 * (g / 8);                      /* first group of g's block */
+    int64_t nb = G - first < 8 ? G - first : 8;       /* groups in that block */
+    if (j < 24)
+        return 26 * first + 24 * (g - first) + j;
+    return 26 * first + 24 * nb + 2 * (g - first) + (j - 24);
+}
+
+static uint8_t b3_encode(int64_t v, int n)
+{
+    return (uint8_t)((256 * v + kPow3[n] - 1) / kPow3[n]);   /* ceil(256 v / 3^n) */
+}
+
+/* v of a stored byte holding n codes; *valid says whether the encoding writes that byte. */
+static int64_t b3_decode(uint8_t byte, int n, int *valid)
+{
+    int64_t v = ((int64_t)byte * kPow3[n]) / 256;
+    *valid = b3_encode(v, n) == byte;
+    return v;
+}
+
+/* Code p (0 = first, the most significant digit) of the n codes with value v. */
+static int b3_code(int64_t v, int n, int p)
+{
+    return (int)((v / kPow3[n - 1 - p]) % 3);
+}
+
+int bqo_pack_ternary_b3(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                        uint8_t *bytes, uint16_t *s_out)
+{
+    int64_t RB = bqo_row_bytes(BQO_TERNARY_B3, K);
+    if (RB < 0 || N < 0)
+        return BQO_ERR_SHAPE;
+    int64_t G = K / 128;
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t g = 0; g < G; g++)
+            for (int j = 0; j < 26; j++) {
+                int cnt = b3_count(j);
+                int64_t v = 0;
+                for (int p = 0; p < cnt; p++) {
+                    int8_t w = q[n * K + 128 * g + b3_first(j) + p];
+                    if (w < -1 || w > 1)
+                        return BQO_ERR_CODE;
+                    v = 3 * v + (w + 1);                 /* first code most significant */
+                }
+                bytes[n * RB + b3_byte_offset(G, g, j)] = b3_encode(v, cnt);
+            }
+    for (int64_t i = 0; i < N * G; i++)
+        s_out[i] = s_in[i];
+    return BQO_OK;
+}
+
+/* Returns the number of invalid bytes; the q of their codes is set to 0. */
+int64_t bqo_unpack_ternary_b3(const uint8_t *bytes, int64_t N, int64_t K, int8_t *q)
+{
+    int64_t RB = bqo_row_bytes(BQO_TERNARY_B3, K);
+    if (RB < 0 || N < 0)
+        return -1;
+    int64_t G = K / 128, bad = 0;
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t g = 0; g < G; g++)
+            for (int j = 0; j < 26; j++) {
+                int cnt = b3_count(j), valid;
+                int64_t v = b3_decode(bytes[n * RB + b3_byte_offset(G, g, j)], cnt, &valid);
+                if (!valid)
+                    bad++;
+                for (int p = 0; p < cnt; p++)
+                    q[n * K + 128 * g + b3_first(j) + p] = valid ? (int8_t)(b3_code(v, cnt, p) - 1) : 0;
+            }
+    return bad;
+}
+
+/* Code of weight (n, k) of a base-3 matrix, or -1 if its byte is invalid. */
+static int b3_code_at(const uint8_t *bytes, int64_t K, int64_t n, int64_t k)
+{
+    int64_t G = K / 128;
+    int kk = (int)(k % 128);
+    int j = b3_byte_of(kk), cnt = b3_count(j), valid;
+    int64_t v = b3_decode(bytes[n * 26 * G + b3_byte_offset(G, k / 128, j)], cnt, &valid);
+    return valid ? b3_code(v, cnt, kk - b3_first(j)) : -1;
+}
+
+/* ---------------------------------------------------------------------------------------
  * Dequantised weight W[n, k] = s[n, k/128] * (2b - 1)   (binary, [card])
- *                            = s[n, k/128] * (c - 1)    (ternary, [tern])
+ *                            = s[n, k/128] * (c - 1)    (ternary, either storage, [tern])
+ * The weight buffer is uint32 words for the binary and 2-bit formats and bytes for base-3.
  * ------------------------------------------------------------------------------------- */
 
 double bqo_weight(int fmt, const uint32_t *words, const uint16_t *scales, int64_t K,
@@ -239,6 +369,10 @@ double bqo_weight(int fmt, const uint32_t *words, const uint16_t *scales, int64_
         uint32_t bit = (words[n * (K / 32) + k / 32] >> (k % 32)) & 1u;
         return bit ? s : -s;
     }
+    if (fmt == BQO_TERNARY_B3) {
+        int c = b3_code_at((const uint8_t *)words, K, n, k);
+        return c < 0 ? NAN : s * (double)(c - 1);
+    }
     uint32_t code = (words[n * (K / 16) + k / 16] >> (2 * (k % 16))) & 3u;
     if (code == 3)
         return NAN;
@@ -248,7 +382,7 @@ double bqo_weight(int fmt, const uint32_t *words, const uint16_t *scales, int64_
 int bqo_dequant(int fmt, const uint32_t *words, const uint16_t *scales, int64_t N, int64_t K,
                 double *Wd)
 {
-    if (bqo_words_per_row(fmt, K) < 0 || N < 0)
+    if (bqo_row_bytes(fmt, K) < 0 || N < 0)
         return BQO_ERR_SHAPE;
     for (int64_t n = 0; n < N; n++)
         for (int64_t k = 0; k < K; k++)
@@ -272,7 +406,7 @@ int bqo_gemv_rows(int fmt, const uint16_t *x, int xt, int64_t M, int64_t K,
                   const uint32_t *words, const uint16_t *scales, int64_t N,
                   const int64_t *rows, int64_t R, double *y, double *bound)
 {
-    if (bqo_words_per_row(fmt, K) < 0 || M < 0 || N < 0 || R < 0)
+    if (bqo_row_bytes(fmt, K) < 0 || M < 0 || N < 0 || R < 0)
         return BQO_ERR_SHAPE;
     for (int64_t r = 0; r < R; r++) {
         int64_t n = rows[r];
@@ -301,7 +435,7 @@ int bqo_gemv_rows(int fmt, const uint16_t *x, int xt, int64_t M, int64_t K,
 int64_t bqo_embed(int fmt, const int32_t *ids, int64_t T, const uint32_t *words,
                   const uint16_t *scales, int64_t N, int64_t K, double *out)
 {
-    if (bqo_words_per_row(fmt, K) < 0 || T < 0 || N < 0)
+    if (bqo_row_bytes(fmt, K) < 0 || T < 0 || N < 0)
         return -1;
     int64_t bad = 0;
     for (int64_t t = 0; t < T; t++) {

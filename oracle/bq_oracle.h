@@ -12,7 +12,7 @@
 extern "C" {
 #endif
 
-enum { BQO_BINARY = 0, BQO_TERNARY = 1 };
+enum { BQO_BINARY = 0, BQO_TERNARY = 1, BQO_TERNARY_B3 = 2 };
 enum { BQO_X_F16 = 0, BQO_X_BF16 = 1 };
 enum { BQO_OK = 0, BQO_ERR_SHAPE = 1, BQO_ERR_CODE = 2 };
 
@@ -23,6 +23,7 @@ uint16_t bqo_f64_to_f16(double v);
 void bqo_f64_to_bf16_array(const double *v, int64_t n, uint16_t *out);
 
 int64_t bqo_words_per_row(int fmt, int64_t K);
+int64_t bqo_row_bytes(int fmt, int64_t K);
 
 int bqo_pack_binary_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
                          uint32_t *words, uint16_t *s_out);
@@ -30,6 +31,9 @@ int bqo_pack_ternary_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int6
                           uint32_t *words, uint16_t *s_out);
 int64_t bqo_unpack_binary_g128(const uint32_t *words, int64_t N, int64_t K, int8_t *q);
 int64_t bqo_unpack_ternary_g128(const uint32_t *words, int64_t N, int64_t K, int8_t *q);
+int bqo_pack_ternary_b3(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                        uint8_t *bytes, uint16_t *s_out);
+int64_t bqo_unpack_ternary_b3(const uint8_t *bytes, int64_t N, int64_t K, int8_t *q);
 
 double bqo_weight(int fmt, const uint32_t *words, const uint16_t *scales, int64_t K,
                   int64_t n, int64_t k);

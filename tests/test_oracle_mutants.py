@@ -57,6 +57,22 @@ MUTANTS = {
         "out[t * K + k] = bqo_weight(fmt, words, scales, K, t % N, k);"),
     "mlx_bias_sign": (
         "uint16_t bias = bqo_f64_to_f16(-s);", "uint16_t bias = bqo_f64_to_f16(s);"),
+    "b3_codes_lsb_first": (
+        "int8_t w = q[n * K + 128 * g + b3_first(j) + p];",
+        "int8_t w = q[n * K + 128 * g + b3_first(j) + (cnt - 1 - p)];"),
+    "b3_encode_floor": (
+        "return (uint8_t)((256 * v + kPow3[n] - 1) / kPow3[n]);",
+        "return (uint8_t)((256 * v) / kPow3[n]);"),
+    "b3_four_code_bytes_in_group": (
+        "return 26 * first + 24 * nb + 2 * (g - first) + (j - 24);",
+        "return 26 * first + 26 * (g - first) + j;"),
+    "b3_digit_order": (
+        "return (int)((v / kPow3[n - 1 - p]) % 3);", "return (int)((v / kPow3[p]) % 3);"),
+    "b3_every_byte_valid": (
+        "*valid = b3_encode(v, n) == byte;", "*valid = 1;"),
+    "b3_decode_rounds": (
+        "int64_t v = ((int64_t)byte * kPow3[n]) / 256;",
+        "int64_t v = ((int64_t)byte * kPow3[n] + 128) / 256;"),
     "sum_skips_last_k": (
         "for (int64_t k = 0; k < K; k++) {\n                double xv",
         "for (int64_t k = 0; k < K - 1; k++) {\n                double xv"),

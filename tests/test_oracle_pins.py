@@ -18,7 +18,7 @@ import oracle
 import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
-B, T = oracle.BINARY, oracle.TERNARY
+B, T, T3 = oracle.BINARY, oracle.TERNARY, oracle.TERNARY_B3
 
 
 def _golden(name):
@@ -164,6 +164,104 @@ def pin_invalid_codes(o):
     assert bad == 1 and q[0, 35] == 0
     assert np.isnan(o.dequant(T, words, np.ones((1, 1), np.float16), K)[0, 35])
     assert o.words_per_row(B, 100) == -1 and o.words_per_row(T, 0) == -1
+
+
+# --------------------------------------------------------------------------------------
+# Base-3 ternary storage
+# --------------------------------------------------------------------------------------
+
+def pin_b3_examples(o):
+    """Hand-derived bytes (tests/golden/b3_examples.json) for the base-3 layout."""
+    for ex in _golden("b3_examples.json")["cases"]:
+        K = ex["K"]
+        q = np.full((1, K), ex["default"], np.int8)
+        for k, v in ex["values_at"].items():
+            q[0, int(k)] = v
+        st, b, _ = o.pack(T3, q, np.ones((1, K // 128), np.float16))
+        assert st == oracle.OK and b.shape == (1, 26 * K // 128)
+        if "all_bytes" in ex:
+            expect = np.array(ex["all_bytes"], np.uint8)
+        else:
+            expect = np.zeros(26 * K // 128, np.uint8)
+            for off, v in ex["nonzero_bytes"].items():
+                expect[int(off)] = v
+        assert np.array_equal(b[0], expect), ex["why"]
+        back, bad = o.unpack(T3, b, K)
+        assert bad == 0 and np.array_equal(back, q)
+
+
+def pin_b3_byte_values(o):
+    """Every one of the 256 byte values at every byte position: exactly 3^5 = 243 values
+    decode as five codes and 3^4 = 81 as four (each v written once), and a valid byte's
+    codes are the base-3 digits of floor(byte * 3^n / 256), first digit most significant."""
+    K = 128
+    rows = np.repeat(np.arange(256, dtype=np.uint8)[:, None], 26, axis=1)
+    q, _ = o.unpack(T3, rows, K)
+    valid5, valid4 = set(), set()
+    for byte in range(256):
+        _, bad = o.unpack(T3, rows[byte:byte + 1], K)
+        assert bad in (0, 2, 24, 26)
+        if bad in (0, 2):
+            valid5.add(byte)
+            v = byte * 243 // 256
+            digits = [(v // 3 ** (4 - p)) % 3 - 1 for p in range(5)]
+            assert list(q[byte, :5]) == digits and list(q[byte, 115:120]) == digits
+        if bad in (0, 24):
+            valid4.add(byte)
+            v = byte * 81 // 256
+            digits = [(v // 3 ** (3 - p)) % 3 - 1 for p in range(4)]
+            assert list(q[byte, 120:124]) == digits and list(q[byte, 124:128]) == digits
+    assert len(valid5) == 243 and len(valid4) == 81
+    assert sorted(valid5) == sorted({-(-256 * v // 243) for v in range(243)})
+    assert sorted(valid4) == sorted({-(-256 * v // 81) for v in range(81)})
+    # an invalid byte: its codes unpack as 0 and its weights are NaN
+    bad_byte = min(set(range(256)) - valid5)
+    one = np.zeros((1, 26), np.uint8)
+    one[0, 3] = bad_byte
+    qq, bad = o.unpack(T3, one, K)
+    assert bad == 1 and np.all(qq[0, 15:20] == 0)
+    w = o.dequant(T3, one, np.ones((1, 1), np.float16), K)
+    assert np.all(np.isnan(w[0, 15:20])) and not np.any(np.isnan(w[0, :15]))
+
+
+def pin_b3_equals_2bit(o):
+    """Base-3 storage holds the same ternary weights as the (separately pinned) 2-bit
+    storage: dequant, GEMV (fp64, k ascending, so bit for bit) and embedding agree; the
+    round trip gives back the codes, over ragged block counts."""
+    for N, K, M in ((5, 128, 2), (4, 1024, 1), (3, 1280, 3), (2, 2176, 8)):
+        q = synth.random_ternary(19, 2, (N, K)).numpy()
+        s = synth.scales(19, N, K // 128).numpy()
+        st3, b3, s3 = o.pack(T3, q, s)
+        st2, w2, s2 = o.pack(T, q, s)
+        assert st3 == st2 == oracle.OK and np.array_equal(s3, s2)
+        back, bad = o.unpack(T3, b3, K)
+        assert bad == 0 and np.array_equal(back, q)
+        assert np.array_equal(o.dequant(T3, b3, s3, K), o.dequant(T, w2, s2, K))
+        assert np.array_equal(o.dequant(T3, b3, s3, K), _dense(q, s))
+        xb = synth.activations(20, M, K, dtype=torch.bfloat16)
+        y3, b_3 = o.gemv(T3, xb, oracle.X_BF16, b3, s3, K)
+        y2, b_2 = o.gemv(T, xb, oracle.X_BF16, w2, s2, K)
+        assert np.array_equal(y3, y2) and np.array_equal(b_3, b_2)
+        ids = np.array([N - 1, 0, N, -3], np.int32)
+        e3, bad3 = o.embed(T3, ids, b3, s3, K)
+        e2, bad2 = o.embed(T, ids, w2, s2, K)
+        assert bad3 == bad2 == 2 and np.array_equal(e3, e2)
+    for badv in (2, -2, 5):
+        q = np.zeros((1, 256), np.int8)
+        q[0, 200] = badv
+        assert o.pack(T3, q, np.ones((1, 2), np.float16))[0] == oracle.ERR_CODE
+    assert o.row_bytes(T3, 128) == 26 and o.row_bytes(T3, 5120) == 1040 and o.row_bytes(T3, 100) == -1
+
+
+def pin_b3_bits_per_weight(o):
+    """Stored size from the oracle's buffers: 26 bytes + one fp16 scale per 128 weights is
+    1.75 bits per weight, between the pages' 1.71 (log2 3 + 16/128) and the 2.125 of the
+    2-bit storage."""
+    g = _golden("pages_figures.json")
+    bpw3 = _stored_bpw(o, T3, K=1152)
+    assert bpw3 == 1.75
+    assert g["ternary_true_bits_per_weight"]["value"] < bpw3 < _stored_bpw(o, T)
+    assert math.log2(3) + 16 / 128 < bpw3
 
 
 # --------------------------------------------------------------------------------------
@@ -381,3 +479,7 @@ def test_bf16_x(orc): pin_bf16_x(orc)
 def test_embed(orc): pin_embed(orc)
 def test_bits_per_weight(orc): pin_bits_per_weight(orc)
 def test_mlx_identity(orc): pin_mlx_identity(orc)
+def test_b3_examples(orc): pin_b3_examples(orc)
+def test_b3_byte_values(orc): pin_b3_byte_values(orc)
+def test_b3_equals_2bit(orc): pin_b3_equals_2bit(orc)
+def test_b3_bits_per_weight(orc): pin_b3_bits_per_weight(orc)
