@@ -27,6 +27,17 @@
  *     2*(k % 16) .. 2*(k % 16)+1 of word (k / 16); code 0 -> -1, 1 -> 0, 2 -> +1, and code 3
  *     is invalid (never written by the pack calls; results of the compute calls are
  *     undefined where it occurs; bq_unpack_g128 reports it). One group is 8 words.
+ *   - Ternary, base-3 storage (BQ_TERNARY_B3_G128; the article says the 2-bit storage is
+ *     what ships today while the information is 1.71 bits per weight and native ternary
+ *     kernels are in development): bytes[N][26 K/128]. Codes c = value + 1; bytes 0..23 of a
+ *     group hold five codes each (group positions 5j .. 5j+4), bytes 24 and 25 four each
+ *     (120..123, 124..127); a byte holding n codes stores ceil(256 v / 3^n), v the codes
+ *     as a base-3 number with the first code most significant. A row is a run of blocks of
+ *     8 groups (the last may hold fewer, nb): the 24 five-code bytes of each group of the
+ *     block (group i at 24 i), then the two four-code bytes of each (at 24 nb + 2 i). With
+ *     the scale this is 1.75 bits per weight. Byte values no v produces (13 of 256 for five
+ *     codes, 175 for four) are invalid: never written by the pack call, undefined in the
+ *     compute calls, reported by bq_unpack_g128.
  *   - Scales: IEEE binary16 scales[N][K/128].
  *   - Activations x[M][K] and outputs y[M][N] are dense row-major.
  *
@@ -68,14 +79,15 @@ typedef enum {
 
 typedef enum { BQ_F16 = 0, BQ_BF16 = 1, BQ_F32 = 2 } bq_dtype;
 
-typedef enum { BQ_BINARY_G128 = 0, BQ_TERNARY_G128 = 1 } bq_format;
+typedef enum { BQ_BINARY_G128 = 0, BQ_TERNARY_G128 = 1, BQ_TERNARY_B3_G128 = 2 } bq_format;
 
 /* Non-owning view of a packed weight matrix (device memory). */
 typedef struct {
     bq_format fmt;
     int64_t N;                /* output rows, >= 1 */
     int64_t K;                /* inputs per row, a positive multiple of 128 */
-    const uint32_t *words;    /* [N][K/32] (binary) or [N][K/16] (ternary) */
+    const uint32_t *words;    /* [N][K/32] (binary), [N][K/16] (ternary), or the bytes
+                                 [N][26 K/128] of the base-3 storage */
     const uint16_t *scales;   /* fp16 [N][K/128] */
 } bq_weight;
 
@@ -92,9 +104,13 @@ const char *bq_last_error(void);
  * all threads); instrumentation for benchmarks. */
 unsigned long long bq_kernel_launches(void);
 
-/* Number of uint32 words in a packed matrix: N*K/32 (binary) or N*K/16 (ternary);
- * 0 if the arguments are invalid. Scales always take N*K/128 fp16 values. */
+/* Number of uint32 words in a packed matrix: N*K/32 (binary), N*K/16 (ternary) or the
+ * base-3 bytes rounded up to whole words; 0 if the arguments are invalid. Scales always take
+ * N*K/128 fp16 values. */
 size_t bq_packed_words(bq_format fmt, int64_t N, int64_t K);
+
+/* Bytes of a packed matrix: N*K/8, N*K/4, or N*26*K/128 (base-3); 0 if invalid. */
+size_t bq_packed_bytes(bq_format fmt, int64_t N, int64_t K);
 
 /*
  * Pack already-quantised weights into the binary-g128 format.
@@ -118,9 +134,19 @@ bq_status bq_pack_ternary_g128(const int8_t *q, const uint16_t *s_in, int64_t N,
                                uint32_t *words, uint16_t *s_out, cudaStream_t stream);
 
 /*
+ * Pack already-quantised ternary weights (q in {-1, 0, +1}) into the base-3 storage
+ * described at the top of this file, bytes [N][26 K/128] (16-byte aligned). Ternary Bonsai
+ * 27B article (wmrh.cn), section "局限性与未来发展" (1.71 bits per weight in principle;
+ * native ternary kernels in development). Synchronous, like the other pack calls; returns
+ * BQ_ERR_INVALID_CODE if any q is outside {-1, 0, +1}.
+ */
+bq_status bq_pack_ternary_b3_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
+                                  uint8_t *bytes, uint16_t *s_out, cudaStream_t stream);
+
+/*
  * Inverse of the pack calls: q int8 [N][K] and, if s_out is not NULL, a copy of the
- * scales. SYNCHRONOUS. Returns BQ_ERR_INVALID_CODE if a ternary code 3 is found (its q is
- * written as 0).
+ * scales. SYNCHRONOUS. Returns BQ_ERR_INVALID_CODE if a ternary code 3, or an invalid base-3
+ * byte, is found (the q of its codes is written as 0).
  */
 bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStream_t stream);
 

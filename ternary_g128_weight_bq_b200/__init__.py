@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libbq.so")
 
 BINARY_G128 = 0
 TERNARY_G128 = 1
+TERNARY_B3_G128 = 2      # ternary codes in base-3 bytes (26 per group of 128): 1.75 bits/weight
 
 _DTYPE = {torch.float16: 0, torch.bfloat16: 1, torch.float32: 2}
 
@@ -63,8 +64,10 @@ def lib() -> ctypes.CDLL:
             "bq_last_error": ([], ctypes.c_char_p),
             "bq_kernel_launches": ([], ctypes.c_ulonglong),
             "bq_packed_words": ([I, I64, I64], ctypes.c_size_t),
+            "bq_packed_bytes": ([I, I64, I64], ctypes.c_size_t),
             "bq_pack_binary_g128": ([P, P, I64, I64, P, P, P], I),
             "bq_pack_ternary_g128": ([P, P, I64, I64, P, P, P], I),
+            "bq_pack_ternary_b3_g128": ([P, P, I64, I64, P, P, P], I),
             "bq_unpack_g128": ([W, P, P, P], I),
             "bq_gemv": ([P, I, I64, W, P, I, P, ctypes.c_size_t, P], I),
             "bq_gemv_workspace_bytes": ([I64, W], ctypes.c_size_t),
@@ -132,7 +135,8 @@ def _operands(x: torch.Tensor, w) -> None:
 class BQWeight:
     """A packed weight matrix held in device memory.
 
-    words: int32 [N, K/32] (binary) or [N, K/16] (ternary), the uint32 bit patterns.
+    words: int32 [N, K/32] (binary) or [N, K/16] (ternary), the uint32 bit patterns, or
+        uint8 [N, 26 K/128] (ternary in base-3 bytes).
     scales: float16 [N, K/128].
     """
     fmt: int
@@ -144,9 +148,9 @@ class BQWeight:
     def __post_init__(self):
         _dev(self.words, "words")
         _dev(self.scales, "scales")
-        wpr = self.K // (32 if self.fmt == BINARY_G128 else 16)
-        if tuple(self.words.shape) != (self.N, wpr) or self.words.dtype != torch.int32:
-            raise ValueError(f"words must be int32 [{self.N}, {wpr}]")
+        shape, dtype = _packed_shape(self.fmt, self.N, self.K)
+        if tuple(self.words.shape) != shape or self.words.dtype != dtype:
+            raise ValueError(f"words must be {dtype} {list(shape)}")
         if tuple(self.scales.shape) != (self.N, self.K // 128) or self.scales.dtype != torch.float16:
             raise ValueError(f"scales must be float16 [{self.N}, {self.K // 128}]")
         self._c = _Weight(self.fmt, self.N, self.K, self.words.data_ptr(), self.scales.data_ptr())
@@ -157,7 +161,16 @@ class BQWeight:
 
     @property
     def nbytes(self) -> int:
-        return self.words.numel() * 4 + self.scales.numel() * 2
+        return self.words.numel() * self.words.element_size() + self.scales.numel() * 2
+
+
+def _packed_shape(fmt: int, N: int, K: int):
+    """Shape and dtype of the packed-weight tensor of a format."""
+    if fmt == TERNARY_B3_G128:
+        return (N, 26 * (K // 128)), torch.uint8
+    if fmt in (BINARY_G128, TERNARY_G128):
+        return (N, K // (32 if fmt == BINARY_G128 else 16)), torch.int32
+    raise ValueError(f"unknown format {fmt}")
 
 
 def version() -> str:
@@ -173,6 +186,10 @@ def packed_words(fmt: int, N: int, K: int) -> int:
     return int(lib().bq_packed_words(fmt, N, K))
 
 
+def packed_bytes(fmt: int, N: int, K: int) -> int:
+    return int(lib().bq_packed_bytes(fmt, N, K))
+
+
 def _pack(fn, fmt, q, s):
     _dev(q, "q")
     _dev(s, "s")
@@ -181,8 +198,8 @@ def _pack(fn, fmt, q, s):
     N, K = q.shape
     if s.dtype != torch.float16:
         raise ValueError("s must be float16 [N, K/128]")
-    wpr = max(K // (32 if fmt == BINARY_G128 else 16), 1)
-    words = torch.empty((N, wpr), dtype=torch.int32, device=q.device)
+    shape, dtype = _packed_shape(fmt, N, max(K, 128))
+    words = torch.empty(shape, dtype=dtype, device=q.device)
     s_out = torch.empty((N, max(K // 128, 1)), dtype=torch.float16, device=q.device)
     _check(fn(q.data_ptr(), s.data_ptr(), N, K, words.data_ptr(), s_out.data_ptr(),
               _stream(q.device)))
@@ -197,6 +214,12 @@ def pack_binary_g128(q: torch.Tensor, s: torch.Tensor) -> BQWeight:
 def pack_ternary_g128(q: torch.Tensor, s: torch.Tensor) -> BQWeight:
     """Pack int8 q in {-1, 0, +1} [N, K] and fp16 scales (synchronous; validates q)."""
     return _pack(lib().bq_pack_ternary_g128, TERNARY_G128, q, s)
+
+
+def pack_ternary_b3_g128(q: torch.Tensor, s: torch.Tensor) -> BQWeight:
+    """Pack int8 q in {-1, 0, +1} [N, K] into base-3 bytes (26 per group of 128) and fp16
+    scales (synchronous; validates q)."""
+    return _pack(lib().bq_pack_ternary_b3_g128, TERNARY_B3_G128, q, s)
 
 
 def unpack_g128(w: BQWeight):

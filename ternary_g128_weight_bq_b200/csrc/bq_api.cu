@@ -113,7 +113,7 @@ static bq_status validate_weight(const bq_weight *w)
 {
     if (!w)
         return set_error(BQ_ERR_INVALID_ARG, "weight view is NULL");
-    if (w->fmt != BQ_BINARY_G128 && w->fmt != BQ_TERNARY_G128)
+    if (w->fmt != BQ_BINARY_G128 && w->fmt != BQ_TERNARY_G128 && w->fmt != BQ_TERNARY_B3_G128)
         return set_error(BQ_ERR_INVALID_ARG, "unknown format %d", (int)w->fmt);
     if (w->N < 1 || w->K < 128 || w->K % 128)
         return set_error(BQ_ERR_SHAPE, "N=%lld K=%lld: need N >= 1 and K a positive multiple of 128",
@@ -165,11 +165,22 @@ size_t bq_packed_words(bq_format fmt, int64_t N, int64_t K)
         return (size_t)N * (size_t)(K / 32);
     if (fmt == BQ_TERNARY_G128)
         return (size_t)N * (size_t)(K / 16);
+    if (fmt == BQ_TERNARY_B3_G128)
+        return (bq_packed_bytes(fmt, N, K) + 3) / 4;
     return 0;
 }
 
+size_t bq_packed_bytes(bq_format fmt, int64_t N, int64_t K)
+{
+    if (N < 1 || K < 128 || K % 128)
+        return 0;
+    if (fmt == BQ_TERNARY_B3_G128)
+        return (size_t)N * (size_t)(26 * (K / 128));
+    return 4 * bq_packed_words(fmt, N, K);
+}
+
 static bq_status pack_common(int fmt, const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K,
-                             uint32_t *words, uint16_t *s_out, cudaStream_t stream)
+                             void *words, uint16_t *s_out, cudaStream_t stream)
 {
     if (!q || !s_in || !words || !s_out)
         return set_error(BQ_ERR_INVALID_ARG, "pack: NULL pointer");
@@ -186,8 +197,9 @@ static bq_status pack_common(int fmt, const int8_t *q, const uint16_t *s_in, int
     unsigned int *cnt = status + kSlotInvalidCount;
     cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(unsigned int), stream);
     if (e == cudaSuccess)
-        e = fmt == BQ_BINARY_G128 ? launch_pack_binary(q, N, K, words, cnt, stream)
-                                  : launch_pack_ternary(q, N, K, words, cnt, stream);
+        e = fmt == BQ_BINARY_G128    ? launch_pack_binary(q, N, K, static_cast<uint32_t *>(words), cnt, stream)
+            : fmt == BQ_TERNARY_G128 ? launch_pack_ternary(q, N, K, static_cast<uint32_t *>(words), cnt, stream)
+                                     : launch_pack_b3(q, N, K, static_cast<uint8_t *>(words), cnt, stream);
     if (e == cudaSuccess)
         note_launches(1);
     if (e == cudaSuccess && s_out != s_in)
@@ -216,6 +228,12 @@ bq_status bq_pack_ternary_g128(const int8_t *q, const uint16_t *s_in, int64_t N,
                                uint32_t *words, uint16_t *s_out, cudaStream_t stream)
 {
     return pack_common(BQ_TERNARY_G128, q, s_in, N, K, words, s_out, stream);
+}
+
+bq_status bq_pack_ternary_b3_g128(const int8_t *q, const uint16_t *s_in, int64_t N, int64_t K, uint8_t *bytes,
+                                  uint16_t *s_out, cudaStream_t stream)
+{
+    return pack_common(BQ_TERNARY_B3_G128, q, s_in, N, K, bytes, s_out, stream);
 }
 
 bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStream_t stream)
@@ -249,8 +267,9 @@ bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStr
     if (e != cudaSuccess)
         return set_error(BQ_ERR_CUDA, "unpack: %s", cudaGetErrorString(e));
     if (host_cnt)
-        return set_error(BQ_ERR_INVALID_CODE, "unpack: %u ternary fields hold the invalid code 3",
-                         host_cnt);
+        return set_error(BQ_ERR_INVALID_CODE, "unpack: %u %s", host_cnt,
+                         w->fmt == BQ_TERNARY_B3_G128 ? "bytes hold a value the base-3 encoding never writes"
+                                                      : "ternary fields hold the invalid code 3");
     return BQ_OK;
 }
 
@@ -360,6 +379,8 @@ bq_status bq_gemm_prefill(const void *x, bq_dtype xt, int64_t M, const bq_weight
         return st;
     if ((st = validate_xy("gemm_prefill", x, xt, y, yt)) != BQ_OK)
         return st;
+    if (w->fmt == BQ_TERNARY_B3_G128)
+        return set_error(BQ_ERR_UNSUPPORTED, "gemm_prefill: the base-3 storage has no prefill kernel");
     if (M < 1 || M > (int64_t(1) << 24))
         return set_error(BQ_ERR_SHAPE, "gemm_prefill: M=%lld out of range", (long long)M);
     size_t need = prefill_workspace_bytes(M, w->fmt, w->N, w->K);

@@ -44,6 +44,8 @@ cudaError_t launch_pack_binary(const int8_t *q, int64_t N, int64_t K, uint32_t *
                                unsigned int *invalid_count, cudaStream_t s);
 cudaError_t launch_pack_ternary(const int8_t *q, int64_t N, int64_t K, uint32_t *words,
                                 unsigned int *invalid_count, cudaStream_t s);
+cudaError_t launch_pack_b3(const int8_t *q, int64_t N, int64_t K, uint8_t *bytes, unsigned int *invalid_count,
+                           cudaStream_t s);
 cudaError_t launch_unpack(int fmt, const uint32_t *words, int64_t N, int64_t K, int8_t *q,
                           unsigned int *invalid_count, cudaStream_t s);
 

@@ -8,9 +8,12 @@
 // One warp per token row. The row is cut into 8-weight chunks (one byte of a binary word,
 // half of a ternary word); lane l takes chunks l, l + 32, ..., so each warp store covers one
 // contiguous 512-byte (bf16/fp16) or 1 KB (fp32) span of the output row. The packed bytes of
-// four chunks are loaded before any is expanded, so their loads overlap.
+// four chunks are loaded before any is expanded, so their loads overlap. Base-3 rows (b3.cuh) are
+// turned into the 2-bit codes of a chunk on load (its 8 codes sit in 2 or 3 bytes) and expanded
+// like ternary ones.
 #include <type_traits>
 
+#include "b3.cuh"
 #include "bq_internal.cuh"
 
 namespace bq {
@@ -36,11 +39,30 @@ template <> struct Pack8<float> {
 // The 8 codes of chunk q of a packed row (binary: byte q % 4 of word q / 4; ternary: 16-bit
 // half q % 2 of word q / 2), as the low 8 or 16 bits.
 template <int FMT>
-__device__ __forceinline__ uint32_t load_chunk(const uint32_t *__restrict__ row, int64_t q)
+__device__ __forceinline__ uint32_t load_chunk(const uint32_t *__restrict__ row, int64_t q, int64_t G)
 {
     if (FMT == BQ_BINARY_G128)
         return (__ldg(row + (q >> 2)) >> (8 * (q & 3))) & 0xFFu;
-    return (__ldg(row + (q >> 1)) >> (16 * (q & 1))) & 0xFFFFu;
+    if (FMT == BQ_TERNARY_G128)
+        return (__ldg(row + (q >> 1)) >> (16 * (q & 1))) & 0xFFFFu;
+    // base-3: positions 8 (q % 16) .. + 7 of group q / 16; a byte the encoding never writes
+    // gives code 1 (a zero weight)
+    const uint8_t *rb = reinterpret_cast<const uint8_t *>(row);
+    const int64_t g = q >> 4;
+    const int kk0 = 8 * (int)(q & 15);
+    uint32_t codes = 0, byte = 0;
+    int jprev = -1;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const int kk = kk0 + i, j = b3::byte_of(kk);
+        if (j != jprev) {
+            byte = __ldg(rb + b3::byte_offset(G, g, j));
+            jprev = j;
+        }
+        const int c = b3::code(byte, b3::count(j), kk - b3::first(j));
+        codes |= (uint32_t)(c < 0 ? 1 : c) << (2 * i);
+    }
+    return codes;
 }
 
 // Value of weight i (0..7) of a chunk: +s / -s (binary bit 1 / 0), +s / 0 / -s (ternary code
@@ -70,8 +92,12 @@ embed_kernel(const int32_t *__restrict__ ids, int64_t T, const uint32_t *__restr
     const bool valid = id >= 0 && id < N;
     if (!valid && lane == 0)
         atomicOr(dev_status + kSlotErrBits, kDevErrInvalidId);
-    constexpr int KPW = FMT == BQ_BINARY_G128 ? 32 : 16;      // weights per word
-    const uint32_t *row = words + (valid ? id : 0) * (K / KPW);
+    constexpr int KPW = FMT == BQ_BINARY_G128 ? 32 : 16;      // weights per word (2-bit or binary)
+    const int64_t G = K / 128;
+    const uint32_t *row = FMT == BQ_TERNARY_B3_G128
+        ? reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(words) +
+                                             (valid ? id : 0) * (b3::kGroupBytes * G))
+        : words + (valid ? id : 0) * (K / KPW);
     const __half *srow = scales + (valid ? id : 0) * (K / 128);
     OT *orow = out + t * K;
     const int64_t nq = K / 8;                                  // 8-weight chunks in the row
@@ -84,7 +110,7 @@ embed_kernel(const int32_t *__restrict__ ids, int64_t T, const uint32_t *__restr
             codes[j] = 0u;
             s[j] = 0.f;
             if (valid && q < nq) {
-                codes[j] = load_chunk<FMT>(row, q);
+                codes[j] = load_chunk<FMT>(row, q, G);
                 s[j] = __half2float(srow[q >> 4]);             // 16 chunks per group of 128
             }
         }
@@ -133,7 +159,7 @@ cudaError_t launch_embed(int fmt, const int32_t *ids, int64_t T, const uint32_t 
         else
             embed_kernel<BQ_BINARY_G128, float><<<blocks, block, 0, s>>>(
                 ids, T, words, scales, N, K, static_cast<float *>(out), dev_status);
-    } else {
+    } else if (fmt == BQ_TERNARY_G128) {
         if (ot == BQ_BF16)
             embed_kernel<BQ_TERNARY_G128, __nv_bfloat16><<<blocks, block, 0, s>>>(
                 ids, T, words, scales, N, K, static_cast<__nv_bfloat16 *>(out), dev_status);
@@ -142,6 +168,16 @@ cudaError_t launch_embed(int fmt, const int32_t *ids, int64_t T, const uint32_t 
                 ids, T, words, scales, N, K, static_cast<__half *>(out), dev_status);
         else
             embed_kernel<BQ_TERNARY_G128, float><<<blocks, block, 0, s>>>(
+                ids, T, words, scales, N, K, static_cast<float *>(out), dev_status);
+    } else {
+        if (ot == BQ_BF16)
+            embed_kernel<BQ_TERNARY_B3_G128, __nv_bfloat16><<<blocks, block, 0, s>>>(
+                ids, T, words, scales, N, K, static_cast<__nv_bfloat16 *>(out), dev_status);
+        else if (ot == BQ_F16)
+            embed_kernel<BQ_TERNARY_B3_G128, __half><<<blocks, block, 0, s>>>(
+                ids, T, words, scales, N, K, static_cast<__half *>(out), dev_status);
+        else
+            embed_kernel<BQ_TERNARY_B3_G128, float><<<blocks, block, 0, s>>>(
                 ids, T, words, scales, N, K, static_cast<float *>(out), dev_status);
     }
     return cudaGetLastError();

@@ -1,4 +1,5 @@
-// gemv.cu -- decode GEMV on packed binary-g128 / ternary-g128 weights, M <= 8 token rows.
+// gemv.cu -- decode GEMV on packed binary-g128 / ternary-g128 weights (2-bit or base-3
+// storage), M <= 8 token rows.
 //
 // y[m][n] = sum_g s[n][g] * sum_{k in g} v[n][k] * x[m][k],  v = 2b - 1 (binary) or c - 1
 // (ternary). Model card "prism-ml/Bonsai-27B-mlx-1bit", sections "Weight representation:
@@ -14,6 +15,7 @@
 //     (M*K*4 <= 200 KB), else read from global memory (L1/L2-resident).
 // This kernel serves the shapes the tensor-core kernel (gemv_rows.cu) does not take: K not a
 // multiple of 1024, or digit fragments too large for shared memory.
+#include "b3.cuh"
 #include "bq_internal.cuh"
 
 namespace bq {
@@ -57,14 +59,17 @@ gemv_simt_kernel(const XT *__restrict__ x, int64_t K, const uint32_t *__restrict
         acc[m] = 0.f;
 
     if (n < N) {
-        constexpr int WPG = FMT == BQ_BINARY_G128 ? 4 : 8;     // words per group
+        constexpr int WPG = FMT == BQ_BINARY_G128 ? 4 : 8;     // words per group (not base-3)
         const uint32_t *wrow = words + n * G * WPG;
+        const uint8_t *brow = reinterpret_cast<const uint8_t *>(words) + n * G * b3::kGroupBytes;
         for (int64_t g = j; g < G; g += 8) {
             uint32_t w[WPG];
+            if (FMT != BQ_TERNARY_B3_G128) {
 #pragma unroll
-            for (int i = 0; i < WPG; i += 4) {
-                uint4 v = __ldg(reinterpret_cast<const uint4 *>(wrow + g * WPG + i));
-                w[i] = v.x; w[i + 1] = v.y; w[i + 2] = v.z; w[i + 3] = v.w;
+                for (int i = 0; i < WPG; i += 4) {
+                    uint4 v = __ldg(reinterpret_cast<const uint4 *>(wrow + g * WPG + i));
+                    w[i] = v.x; w[i + 1] = v.y; w[i + 2] = v.z; w[i + 3] = v.w;
+                }
             }
             const float s = __half2float(scales[n * G + g]);
             float part[M];
@@ -82,6 +87,27 @@ gemv_simt_kernel(const XT *__restrict__ x, int64_t K, const uint32_t *__restrict
                         for (int m = 0; m < M; m++) {
                             float xv = xs[xg + m * K + i * 32 + b];
                             part[m] += on ? xv : -xv;
+                        }
+                    }
+                }
+            } else if (FMT == BQ_TERNARY_B3_G128) {
+                // byte jb holds codes first(jb) .. first(jb) + count(jb) - 1 of the group;
+                // code p is F_{p+1} - 3 F_p with F_i = floor(q 3^i / 256)
+                for (int jb = 0; jb < b3::kGroupBytes; jb++) {
+                    const uint32_t qb = __ldg(brow + b3::byte_offset(G, g, jb));
+                    const int cnt = b3::count(jb), k0 = b3::first(jb);
+                    uint32_t fprev = 0;
+#pragma unroll
+                    for (int p = 0; p < 5; p++) {
+                        if (p < cnt) {
+                            const uint32_t f = (qb * b3::pow3(p + 1)) >> 8;
+                            const uint32_t c = f - 3u * fprev;
+                            fprev = f;
+#pragma unroll
+                            for (int m = 0; m < M; m++) {
+                                float xv = xs[xg + m * K + k0 + p];
+                                part[m] += c == 2u ? xv : (c == 0u ? -xv : 0.f * xv);
+                            }
                         }
                     }
                 }
@@ -165,6 +191,9 @@ cudaError_t launch_gemv_simt(const GemvArgs &a, cudaStream_t s)
     if (a.fmt == BQ_BINARY_G128)
         return a.xt == BQ_F16 ? launch_simt_m<BQ_BINARY_G128, __half>(a, s)
                               : launch_simt_m<BQ_BINARY_G128, __nv_bfloat16>(a, s);
+    if (a.fmt == BQ_TERNARY_B3_G128)
+        return a.xt == BQ_F16 ? launch_simt_m<BQ_TERNARY_B3_G128, __half>(a, s)
+                              : launch_simt_m<BQ_TERNARY_B3_G128, __nv_bfloat16>(a, s);
     return a.xt == BQ_F16 ? launch_simt_m<BQ_TERNARY_G128, __half>(a, s)
                           : launch_simt_m<BQ_TERNARY_G128, __nv_bfloat16>(a, s);
 }

@@ -13,8 +13,15 @@
 // tolerance. The int32 column sums are exact (each starts at the bits of 1.5 * 2^23, so one
 // fp32 subtraction turns it into a float without rounding); the group scale times 2^(e-27) is
 // applied once per group in fp32, and the digit weights once per output.
+//
+// Base-3 storage (b3.cuh) uses the same MMA with u8 weight operands: for a byte q holding n codes,
+// F_i = floor(q 3^i / 256) (i = 1 .. n) is the number formed by its first i codes, so
+// sum_p x_p c_p = sum_i F_i (x_{i-1} - 3 x_i) (x_n = 0 past the last code): the A operand is
+// F_i (0..242, one IMAD per two bytes and a PRMT per four values) and the x side carries the
+// combinations x_{i-1} - 3 x_i, built once per call by the prep kernel.
 #pragma once
 
+#include "b3.cuh"
 #include "bq_internal.cuh"
 
 namespace bq {
@@ -45,11 +52,57 @@ __device__ __forceinline__ int k_local(int t, int rho, int b)
 //     a per-(group, column) value.
 //   otherwise (ternary): three balanced base-256 digits and a zero column; the codes enter as
 //     {-64, 0, +64} (one PRMT per four codes); the accumulator input is a constant.
+//   base-3: three balanced base-256 digits of the level combinations and a zero column; the
+//     weights enter as u8 F values; the accumulator input of a column is minus the group's sum of
+//     that digit of x (it turns codes c into c - 1), a per-(group, column) value as for binary.
 template <int FMT, int CS> struct Scheme {
     static constexpr bool kMask = FMT == BQ_BINARY_G128;
+    static constexpr bool kB3 = FMT == BQ_TERNARY_B3_G128;
+    static constexpr bool kColFix = kMask || kB3;          // accumulator input per (group, column)
     static constexpr int kCount = kMask ? 4 : 3;
     static constexpr int kBits = kMask ? 6 : 8;
 };
+
+// Base-3: byte j and level i (1 .. count(j)) that A-operand slot (t, rho, b) holds. Quad-thread
+// t of a group owns five-code bytes 4t .. 4t+3 (registers 0..4 = levels 1..5, byte b = byte 4t+b),
+// five-code bytes 16+2t, 17+2t (registers 5, 6, 7: levels 1-2, 3-4, 5, two bytes each) and levels
+// 1-2 (t even) or 3-4 (t odd) of four-code byte 24 + t/2 (bytes 2, 3 of register 7).
+__host__ __device__ constexpr int b3_slot_byte(int t, int rho, int b)
+{
+    return rho < 5 ? 4 * t + b : (rho < 7 || b < 2) ? 16 + 2 * t + (b & 1) : 24 + (t >> 1);
+}
+__host__ __device__ constexpr int b3_slot_level(int t, int rho, int b)
+{
+    return rho < 5 ? rho + 1 : (rho < 7 || b < 2) ? 2 * (rho - 5) + 1 + (b >> 1) : 2 * (t & 1) + 1 + (b - 2);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// 8 A registers of one row of a base-3 group for quad-thread t: w = its five-code bytes
+// 4t..4t+3, h = bytes 16+2t, 17+2t in the low half, tb = its four-code byte, mt = 3^l1 + 2^16 3^l2
+// for that byte's two levels. Bytes go to 16-bit lanes, so a multiply by 3^i gives the level-i
+// values of two bytes at once in bits 8..15 and 24..31 (q 3^i < 2^16), and a PRMT takes four.
+__device__ __forceinline__ void expand_b3(uint32_t w, uint32_t h, uint32_t tb, uint32_t mt, uint32_t *a)
+{
+    uint32_t pa = prmt(w, 0u, 0x4140u), pb = prmt(w, 0u, 0x4342u), pc = prmt(h, 0u, 0x4140u);
+    uint32_t c[6];
+    c[0] = pc;
+#pragma unroll
+    for (int i = 1; i <= 5; i++) {
+        pa *= 3u;
+        pb *= 3u;
+        c[i] = c[i - 1] * 3u;
+        a[i - 1] = prmt(pa, pb, 0x7531u);        // level i of bytes 4t .. 4t+3
+    }
+    a[5] = prmt(c[1], c[2], 0x7531u);
+    a[6] = prmt(c[3], c[4], 0x7531u);
+    a[7] = prmt(c[5], tb * mt, 0x7531u);
+}
 
 // Binary: bit position p that bit (8b + rho) of a word lands on in A register rho, and the
 // matching B multiplier 2^(7-p) (-1 for p = 7).
@@ -114,6 +167,39 @@ __device__ __forceinline__ void expand_group(const uint8_t *p0, const uint8_t *p
         quad[j][2] = a0[2 * j + 1];
         quad[j][3] = a1[2 * j + 1];
     }
+}
+
+// m16n8k32 with u8 A (base-3 F values) or s8 A, s8 B, s32 accumulators.
+template <bool U8>
+__device__ __forceinline__ void mma_i8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                       uint32_t b1)
+{
+    if (U8)
+        asm volatile(
+            "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    else
+        asm volatile(
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <bool U8>
+__device__ __forceinline__ void mma_i8_first(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1, const int (&c)[4])
+{
+    if (U8)
+        asm volatile(
+            "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
+            : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]), "r"(c[2]), "r"(c[3]));
+    else
+        asm volatile(
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
+            : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]), "r"(c[2]), "r"(c[3]));
 }
 
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -238,6 +324,81 @@ __device__ __forceinline__ void build_items(const XT *__restrict__ x, int M, int
             if (lane == 0)
                 colf[m * G + q] = fac;
         }
+    }
+}
+
+// Base-3: the digit fragments, factor and accumulator inputs of one (group, token) item, with the
+// layouts of build_items. Lane (t, rho) builds register rho of quad-thread t: slot b holds level i
+// of byte j, whose x value is X[k] - 3 X[k+1] (k = first(j) + i - 1, i < count(j)) or X[k] (last
+// level), X = round(x 2^(19-e)) with e = floor(log2 max|x|) over the group, so |X| <= 2^20 and
+// each value (<= 2^22) has three balanced base-256 digits. The lane also converts positions
+// 4 lane .. 4 lane + 3 for the group's maximum and for the sums of the digits of X over the group,
+// which the accumulator inputs subtract (codes c become c - 1). Every X of a position is the same
+// rounding of the same product wherever it is formed. The column sums stay exact integers: at most
+// 128 * (24 * 358 + 2 * 116) + 128 * 128 < 2^21 in magnitude.
+template <int CS, typename XT>
+__device__ __forceinline__ void build_item_b3(const XT *__restrict__ x, int M, int64_t K, int G, int item, int lane,
+                                              uint32_t *__restrict__ frag, float *__restrict__ colf,
+                                              int *__restrict__ cfix)
+{
+    const int t = lane >> 3, rho = lane & 7;
+    const bool live = item < G * M;
+    const int q = live ? item / M : 0, m = live ? item % M : 0;
+    const XT *xg = x + (int64_t)m * K + 128 * q;
+    float pv[4], v1[4], v2[4];
+    bool two[4];
+#pragma unroll
+    for (int b = 0; b < 4; b++) {
+        const int j = b3_slot_byte(t, rho, b), i = b3_slot_level(t, rho, b);
+        const int k1 = b3::first(j) + i - 1;
+        two[b] = i < b3::count(j);
+        pv[b] = live ? load_x(xg + 4 * lane + b) : 0.f;
+        v1[b] = live ? load_x(xg + k1) : 0.f;
+        v2[b] = live && two[b] ? load_x(xg + k1 + 1) : 0.f;
+    }
+    float amax = fmaxf(fmaxf(fabsf(pv[0]), fabsf(pv[1])), fmaxf(fabsf(pv[2]), fabsf(pv[3])));
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+    const bool bad = __any_sync(0xffffffffu, !(isfinite(pv[0]) && isfinite(pv[1]) && isfinite(pv[2]) &&
+                                               isfinite(pv[3])));
+    if (bad)
+        amax = 0.f;
+    const int e = amax > 0.f ? ilog2f(amax) : 0;
+    const int k = 19 - e;
+    const float f1 = pow2f(k < 127 ? k : 127), f2 = pow2f(k > 127 ? k - 127 : 0);
+    auto to_int = [&](float v) { return amax > 0.f ? __float2int_rn(v * f1 * f2) : 0; };
+    uint32_t dw[3] = {0u, 0u, 0u};
+    int csum[3] = {0, 0, 0};
+#pragma unroll
+    for (int b = 0; b < 4; b++) {
+        int V = to_int(v1[b]) - (two[b] ? 3 * to_int(v2[b]) : 0);
+        int P = to_int(pv[b]);
+#pragma unroll
+        for (int d = 0; d < 3; d++) {
+            const int dig = ((V + 128) & 255) - 128;
+            dw[d] |= ((uint32_t)dig & 0xFFu) << (8 * b);
+            V = (V - dig) >> 8;
+            const int pd = ((P + 128) & 255) - 128;
+            csum[d] += pd;
+            P = (P - pd) >> 8;
+        }
+    }
+#pragma unroll
+    for (int d = 0; d < 3; d++)
+        csum[d] = __reduce_add_sync(0xffffffffu, csum[d]);
+    float fac = amax > 0.f ? pow2f(e - 19) : 0.f;
+    if (bad)
+        fac = __int_as_float(0x7fffffff);
+    if (live) {
+#pragma unroll
+        for (int d = 0; d < kColsPerTok; d++) {
+            const int c = m * kColsPerTok + d;
+            const int cs = c >> 3, ln = 4 * (c & 7) + t;
+            frag[(((cs * G + q) * 2 + (rho >> 2)) * 32 + ln) * 4 + (rho & 3)] = d < 3 ? dw[d] : 0u;
+            if (lane == 0)
+                cfix[(cs * G + q) * 8 + (c & 7)] = kMagic - (d < 3 ? csum[d] : 0);
+        }
+        if (lane == 0)
+            colf[m * G + q] = fac;
     }
 }
 

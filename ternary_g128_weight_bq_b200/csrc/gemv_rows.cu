@@ -61,8 +61,11 @@ constexpr int kSmemPair = 113 * 1024;         // two CTAs fit on one SM below th
 constexpr uint64_t kWaitLimitNs = kWaitLimitDefaultNs;   // drain waits before exit
 
 template <int FMT> struct RCfg {
-    static constexpr int kBoxes = FMT == BQ_BINARY_G128 ? 1 : 2;   // 128-byte boxes per tile per slice
-    static constexpr int kTileBytes = 2048 * kBoxes;               // packed words of a tile per slice
+    static constexpr bool kB3 = FMT == BQ_TERNARY_B3_G128;
+    static constexpr int kBoxes = FMT == BQ_TERNARY_G128 ? 2 : 1;      // boxes per tile per slice
+    static constexpr int kBoxInner = kB3 ? b3::kBlockBytes : 32;      // box width: 208 bytes or 32 words
+    static constexpr int kBoxBytes = 16 * (kB3 ? b3::kBlockBytes : 128);
+    static constexpr int kTileBytes = kBoxBytes * kBoxes;             // packed weights of a tile per slice
 };
 
 struct RLayout {
@@ -106,15 +109,40 @@ gemv_rows_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint32_t *__re
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int G = (int)(K / 128);
     const int item = (int)((blockIdx.x * 256 + threadIdx.x) >> 5), lane = threadIdx.x & 31;
-    if (item < G * M)
-        build_items<FMT, CS, XT, 1>(x, M, K, G, item, 1, lane, frag, colf, cfix);
+    if (item < G * M) {
+        if (FMT == BQ_TERNARY_B3_G128)
+            build_item_b3<CS, XT>(x, M, K, G, item, lane, frag, colf, cfix);
+        else
+            build_items<FMT, CS, XT, 1>(x, M, K, G, item, 1, lane, frag, colf, cfix);
+    }
 }
 
 // Per-thread constants of the inner loop.
 struct Lane {
     uint32_t mul[9];                  // shift multipliers and byte masks of the sign expansion
     int off0, off1, soff0, soff1;     // byte offsets of this thread's words / scales in a tile
+    int offh, offt;                   // base-3: its two-byte half and four-code byte (row g8)
+    uint32_t mt;                      // base-3: 3^l1 + 2^16 3^l2, the levels of its four-code byte
 };
+
+// Base-3: the A operands of one group for this thread's rows g8 and g8 + 8 of a tile (rows are
+// 208 bytes apart in shared memory), in the register order of expand_group.
+__device__ __forceinline__ void expand_group_b3(const uint8_t *wt, const Lane &ln, uint32_t (&quad)[4][4])
+{
+    constexpr int kRow8 = 8 * b3::kBlockBytes;
+    uint32_t a0[8], a1[8];
+    expand_b3(*reinterpret_cast<const uint32_t *>(wt + ln.off0), *reinterpret_cast<const uint16_t *>(wt + ln.offh),
+              wt[ln.offt], ln.mt, a0);
+    expand_b3(*reinterpret_cast<const uint32_t *>(wt + ln.off0 + kRow8),
+              *reinterpret_cast<const uint16_t *>(wt + ln.offh + kRow8), wt[ln.offt + kRow8], ln.mt, a1);
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        quad[j][0] = a0[2 * j];
+        quad[j][1] = a1[2 * j];
+        quad[j][2] = a0[2 * j + 1];
+        quad[j][3] = a1[2 * j + 1];
+    }
+}
 
 // One slice (1024 k) of NTL tiles j0, j0 + WG, j0 + 2 WG, ... of the stage, for the warp's
 // group q: the x fragment, factors and accumulator inputs are loaded once, the tiles are
@@ -137,7 +165,7 @@ __device__ __forceinline__ void slice_tiles(const uint8_t *__restrict__ st, int 
         bA[cs] = *reinterpret_cast<const uint4 *>(fq);
         bB[cs] = *reinterpret_cast<const uint4 *>(fq + 128);
         f[cs] = colf_tok[2 * cs * G + q];
-        if (SCH::kMask)
+        if (SCH::kColFix)
             cin2[cs] = *reinterpret_cast<const int2 *>(cfix_t + (cs * G + q) * 8);
     }
     const int magic[4] = {magic_in, magic_in, magic_in, magic_in};   // constant accumulator input (not kMask)
@@ -154,7 +182,10 @@ __device__ __forceinline__ void slice_tiles(const uint8_t *__restrict__ st, int 
             if (h < np) {
                 const int j = j0 + (jl + h) * WG;              // tile of the stage
                 const uint8_t *wt = st + j * kTileBytes;
-                expand_group<FMT, SCH::kMask>(wt + ln.off0, wt + ln.off1, ln.mul, A[h]);
+                if (SCH::kB3)
+                    expand_group_b3(wt, ln, A[h]);
+                else
+                    expand_group<FMT, SCH::kMask>(wt + ln.off0, wt + ln.off1, ln.mul, A[h]);
                 const uint8_t *sp = st + j * 256;
                 s0[h] = __half2float(*reinterpret_cast<const __half *>(sp + ln.soff0));
                 s1[h] = __half2float(*reinterpret_cast<const __half *>(sp + ln.soff1));
@@ -166,15 +197,17 @@ __device__ __forceinline__ void slice_tiles(const uint8_t *__restrict__ st, int 
 #pragma unroll
             for (int h = 0; h < 2; h++) {
                 if (h < np) {
-                    if (SCH::kMask) {
+                    constexpr bool U8 = SCH::kB3;
+                    if (SCH::kColFix) {
                         const int cin[4] = {cin2[cs].x, cin2[cs].y, cin2[cs].x, cin2[cs].y};
-                        mma_s8_first(d[h], A[h][0][0], A[h][0][1], A[h][0][2], A[h][0][3], bA[cs].x, bA[cs].y, cin);
+                        mma_i8_first<U8>(d[h], A[h][0][0], A[h][0][1], A[h][0][2], A[h][0][3], bA[cs].x, bA[cs].y, cin);
                     } else {
-                        mma_s8_first(d[h], A[h][0][0], A[h][0][1], A[h][0][2], A[h][0][3], bA[cs].x, bA[cs].y, magic);
+                        mma_i8_first<U8>(d[h], A[h][0][0], A[h][0][1], A[h][0][2], A[h][0][3], bA[cs].x, bA[cs].y,
+                                         magic);
                     }
-                    mma_s8(d[h], A[h][1][0], A[h][1][1], A[h][1][2], A[h][1][3], bA[cs].z, bA[cs].w);
-                    mma_s8(d[h], A[h][2][0], A[h][2][1], A[h][2][2], A[h][2][3], bB[cs].x, bB[cs].y);
-                    mma_s8(d[h], A[h][3][0], A[h][3][1], A[h][3][2], A[h][3][3], bB[cs].z, bB[cs].w);
+                    mma_i8<U8>(d[h], A[h][1][0], A[h][1][1], A[h][1][2], A[h][1][3], bA[cs].z, bA[cs].w);
+                    mma_i8<U8>(d[h], A[h][2][0], A[h][2][1], A[h][2][2], A[h][2][3], bB[cs].x, bB[cs].y);
+                    mma_i8<U8>(d[h], A[h][3][0], A[h][3][1], A[h][3][2], A[h][3][3], bB[cs].z, bB[cs].w);
                 }
             }
 #pragma unroll
@@ -262,8 +295,8 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
                         const int32_t row = (tb + j) * 16;
 #pragma unroll
                         for (int h = 0; h < kBoxes; h++)
-                            ptx::tma_load_2d(st + j * kTileBytes + h * 2048, &tmap_w, &bars->full[s],
-                                             (c * kBoxes + h) * 32, row);
+                            ptx::tma_load_2d(st + j * kTileBytes + h * RCfg<FMT>::kBoxBytes, &tmap_w, &bars->full[s],
+                                             (c * kBoxes + h) * RCfg<FMT>::kBoxInner, row);
                         ptx::tma_load_2d(st + L.scale_off + j * 256, &tmap_s, &bars->full[s], c * 8, row);
                     }
                     if (++s == S) {
@@ -318,6 +351,17 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
         const int within = FMT == BQ_BINARY_G128 ? 4 * t : 8 * (t & 1);
         ln.off0 = (FMT == BQ_BINARY_G128 ? 0 : (w >> 2) * 2048) + g8 * 128 + ((chunk ^ g8) << 4) + within;
         ln.off1 = ln.off0 + 8 * 128;
+        ln.offh = ln.offt = 0;
+        ln.mt = 0u;
+        if (SCH::kB3) {
+            // 208-byte rows, no swizzle: five-code bytes of group w at 24 w, their thread's word at
+            // + 4t and two-byte half at + 16 + 2t; the four-code bytes of group w at 192 + 2 w
+            ln.off0 = g8 * b3::kBlockBytes + 24 * w + 4 * t;
+            ln.off1 = ln.off0 + 8 * b3::kBlockBytes;
+            ln.offh = g8 * b3::kBlockBytes + 24 * w + 16 + 2 * t;
+            ln.offt = g8 * b3::kBlockBytes + 192 + 2 * w + (t >> 1);
+            ln.mt = (t & 1) ? one * (27u + (81u << 16)) : one * (3u + (9u << 16));
+        }
         ln.soff0 = L.scale_off + g8 * 16 + 2 * w;
         ln.soff1 = ln.soff0 + 8 * 16;
         const uint32_t *frag_lane = frag_s + lane * 4;
@@ -450,6 +494,9 @@ int rows_total(int G, int TB, int S) { return rows_layout<FMT, CS>(G, TB, S).tot
 
 int rows_total_rt(int fmt, int CS, int G, int TB, int S)
 {
+    if (fmt == BQ_TERNARY_B3_G128)
+        return CS == 1 ? rows_total<BQ_TERNARY_B3_G128, 1>(G, TB, S) : CS == 2 ? rows_total<BQ_TERNARY_B3_G128, 2>(G, TB, S)
+             : CS == 3 ? rows_total<BQ_TERNARY_B3_G128, 3>(G, TB, S) : rows_total<BQ_TERNARY_B3_G128, 4>(G, TB, S);
     if (fmt == BQ_BINARY_G128)
         return CS == 1 ? rows_total<BQ_BINARY_G128, 1>(G, TB, S) : CS == 2 ? rows_total<BQ_BINARY_G128, 2>(G, TB, S)
              : CS == 3 ? rows_total<BQ_BINARY_G128, 3>(G, TB, S) : rows_total<BQ_BINARY_G128, 4>(G, TB, S);
@@ -510,15 +557,28 @@ cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s)
     if (!enc)
         return cudaErrorNotSupported;
     const cuuint64_t G = (cuuint64_t)(a.K / 128);
-    const cuuint64_t wpr = (cuuint64_t)(FMT == BQ_BINARY_G128 ? a.K / 32 : a.K / 16);
     CUtensorMap mw, ms;
-    cuuint64_t wdims[2] = {wpr, (cuuint64_t)a.N};
-    cuuint64_t wstr[1] = {wpr * 4};
-    cuuint32_t wbox[2] = {32, 16};                       // 128 bytes x 16 rows
     cuuint32_t est[2] = {1, 1};
-    CUresult r = enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(a.words), wdims, wstr, wbox, est,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r;
+    if (FMT == BQ_TERNARY_B3_G128) {
+        // bytes [N][26 G]; a box is one 208-byte block (8 groups) of 16 rows, unswizzled: at a
+        // 208-byte pitch the 8 rows a warp reads fall in distinct banks
+        const cuuint64_t rb = (cuuint64_t)b3::kGroupBytes * G;
+        cuuint64_t wdims[2] = {rb, (cuuint64_t)a.N};
+        cuuint64_t wstr[1] = {rb};
+        cuuint32_t wbox[2] = {(cuuint32_t)b3::kBlockBytes, 16};
+        r = enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t *>(a.words), wdims, wstr, wbox, est,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        const cuuint64_t wpr = (cuuint64_t)(FMT == BQ_BINARY_G128 ? a.K / 32 : a.K / 16);
+        cuuint64_t wdims[2] = {wpr, (cuuint64_t)a.N};
+        cuuint64_t wstr[1] = {wpr * 4};
+        cuuint32_t wbox[2] = {32, 16};                   // 128 bytes x 16 rows
+        r = enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(a.words), wdims, wstr, wbox, est,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     if (r != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     cuuint64_t sdims[2] = {G, (cuuint64_t)a.N};
@@ -600,6 +660,9 @@ cudaError_t launch_gemv_rows(const GemvArgs &a, cudaStream_t s, unsigned *launch
     if (a.fmt == BQ_BINARY_G128)
         return a.xt == BQ_F16 ? launch_rows_cs<BQ_BINARY_G128, __half>(a, pl, s)
                               : launch_rows_cs<BQ_BINARY_G128, __nv_bfloat16>(a, pl, s);
+    if (a.fmt == BQ_TERNARY_B3_G128)
+        return a.xt == BQ_F16 ? launch_rows_cs<BQ_TERNARY_B3_G128, __half>(a, pl, s)
+                              : launch_rows_cs<BQ_TERNARY_B3_G128, __nv_bfloat16>(a, pl, s);
     return a.xt == BQ_F16 ? launch_rows_cs<BQ_TERNARY_G128, __half>(a, pl, s)
                           : launch_rows_cs<BQ_TERNARY_G128, __nv_bfloat16>(a, pl, s);
 }

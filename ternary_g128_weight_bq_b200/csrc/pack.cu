@@ -8,7 +8,9 @@
 // These kernels are elementwise and bound by device memory: one thread builds one packed
 // word from 32 (binary) or 16 (ternary) consecutive int8 values read with 16-byte loads,
 // so each warp reads 1 KB (binary) / 512 B (ternary) of q contiguously and writes 128 B
-// of words.
+// of words. The base-3 storage (b3.cuh) takes one thread per stored byte, the 4 or 5 codes it
+// holds being consecutive q values.
+#include "b3.cuh"
 #include "bq_internal.cuh"
 
 namespace bq {
@@ -121,6 +123,54 @@ __global__ void unpack_kernel(int fmt, const uint32_t *__restrict__ words, int64
     }
 }
 
+// Base-3: thread i builds byte j = i % 26 of group (i / 26) % G of row i / (26 G).
+__global__ void pack_b3_kernel(const int8_t *__restrict__ q, int64_t N, int64_t K, uint8_t *__restrict__ bytes,
+                               unsigned int *invalid_count)
+{
+    const int64_t G = K / 128;
+    const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (i >= N * G * b3::kGroupBytes)
+        return;
+    const int j = (int)(i % b3::kGroupBytes);
+    const int64_t g = (i / b3::kGroupBytes) % G, n = i / (b3::kGroupBytes * G);
+    const int8_t *src = q + n * K + 128 * g + b3::first(j);
+    const int cnt = b3::count(j);
+    uint32_t v = 0;
+    int bad = 0;
+    for (int p = 0; p < cnt; p++) {
+        const int c = (int)__ldg(src + p) + 1;
+        bad += (unsigned)c > 2u;
+        v = 3u * v + (unsigned)(c & 3) % 3u;     // first code most significant
+    }
+    bytes[n * (b3::kGroupBytes * G) + b3::byte_offset(G, g, j)] = (uint8_t)b3::encode(v, cnt);
+    if (bad)
+        atomicAdd(invalid_count, (unsigned)bad);
+}
+
+// Inverse: the codes of one stored byte; a byte the encoding never writes gives q = 0 for its
+// codes and is counted.
+__global__ void unpack_b3_kernel(const uint8_t *__restrict__ bytes, int64_t N, int64_t K, int8_t *__restrict__ q,
+                                 unsigned int *invalid_count)
+{
+    const int64_t G = K / 128;
+    const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (i >= N * G * b3::kGroupBytes)
+        return;
+    const int j = (int)(i % b3::kGroupBytes);
+    const int64_t g = (i / b3::kGroupBytes) % G, n = i / (b3::kGroupBytes * G);
+    const uint32_t byte = __ldg(bytes + n * (b3::kGroupBytes * G) + b3::byte_offset(G, g, j));
+    int8_t *dst = q + n * K + 128 * g + b3::first(j);
+    const int cnt = b3::count(j);
+    bool bad = false;
+    for (int p = 0; p < cnt; p++) {
+        const int c = b3::code(byte, cnt, p);
+        bad |= c < 0;
+        dst[p] = (int8_t)(c < 0 ? 0 : c - 1);
+    }
+    if (bad)
+        atomicAdd(invalid_count, 1u);
+}
+
 inline unsigned blocks_for(int64_t n) { return (unsigned)((n + kThreads - 1) / kThreads); }
 
 }  // namespace
@@ -141,9 +191,23 @@ cudaError_t launch_pack_ternary(const int8_t *q, int64_t N, int64_t K, uint32_t 
     return cudaGetLastError();
 }
 
+cudaError_t launch_pack_b3(const int8_t *q, int64_t N, int64_t K, uint8_t *bytes, unsigned int *invalid_count,
+                           cudaStream_t s)
+{
+    const int64_t total = N * (K / 128) * b3::kGroupBytes;
+    pack_b3_kernel<<<blocks_for(total), kThreads, 0, s>>>(q, N, K, bytes, invalid_count);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_unpack(int fmt, const uint32_t *words, int64_t N, int64_t K, int8_t *q,
                           unsigned int *invalid_count, cudaStream_t s)
 {
+    if (fmt == BQ_TERNARY_B3_G128) {
+        const int64_t total = N * (K / 128) * b3::kGroupBytes;
+        unpack_b3_kernel<<<blocks_for(total), kThreads, 0, s>>>(reinterpret_cast<const uint8_t *>(words), N, K, q,
+                                                                invalid_count);
+        return cudaGetLastError();
+    }
     int64_t total = N * (fmt == BQ_BINARY_G128 ? K / 32 : K / 16);
     unpack_kernel<<<blocks_for(total), kThreads, 0, s>>>(fmt, words, total, q, invalid_count);
     return cudaGetLastError();
