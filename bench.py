@@ -320,6 +320,14 @@ def _host_ternary(ob, seed, rows, K, row0=0):
     return words, s_out
 
 
+def _host_ternary_b3(ob, seed, rows, K, row0=0):
+    q = synth.random_ternary(seed, synth.TID_TERNARY, (rows, K), row0=row0)
+    s = synth.scales(seed, rows, K // 128, row0=row0)
+    st, packed, s_out = ob.orc.pack(ob.o.TERNARY_B3, q.numpy(), s.numpy())
+    assert st == ob.o.OK
+    return packed, s_out
+
+
 def _gemv_entry(name, N, K, M, fmt_bits, ms, peaks, extra=None):
     gb = gemv_bytes(N, K, M, fmt_bits) / 1e9
     gbs = gb / (ms / 1e3)
@@ -471,8 +479,32 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
     e["oracle"] = ob.gemv_timing(o.TERNARY, x, o.X_BF16, *_host_ternary(ob, 0, 2048, K), K,
                                  K // 4 + K // 64, 2 * K, False)
     out.append(e)
-    del tmats, y, ws
+    del tmats
+
+    # ---- the same ternary matrix in base-3 storage (26 bytes per group: 1.625 bits per weight
+    # of codes, 1.75 with the scale), decoded inside the GEMV
+    b3_bits = 26 * 8 / 128
+    copies = max(2, math.ceil(2.5 * l2 / gemv_bytes(N, K, 1, b3_bits)))
+    bmats = []
+    for c in range(copies):
+        q = synth.random_ternary(c, synth.TID_TERNARY, (N, K), device=device)
+        bmats.append(bq.pack_ternary_b3_g128(q, synth.scales(c, N, K // 128, device=device)))
+        del q
+    ms = _rotating_gemv_ms(bq, bmats, xd, y, ws, stream, reps=2 * copies)
+    bq.gemv(xd, bmats[0], out=y, workspace=ws)
+    packed, sc = _host_ternary_b3(ob, 0, rows, K)
+    ratio = ob.max_ratio(o.TERNARY_B3, x, o.X_BF16, packed, sc, K, y[:, :rows].cpu().numpy())
+    e = _gemv_entry("ternary g128 in base-3 storage (1.75 bits/weight) GEMV, M=1, K=5120, N=20480",
+                    N, K, 1, b3_bits, ms, peaks,
+                    {"timing": f"graph of back-to-back calls rotating {copies} weight copies (above L2)",
+                     "parity": {"max_err_over_bound": round(ratio, 5), "rows": rows},
+                     "bytes_vs_2bit": round(gemv_bytes(N, K, 1, b3_bits) / gemv_bytes(N, K, 1, 2), 4)})
+    e["oracle"] = ob.gemv_timing(o.TERNARY_B3, x, o.X_BF16, *_host_ternary_b3(ob, 0, 2048, K), K,
+                                 26 * K // 128 + K // 64, 2 * K, False)
+    out.append(e)
+    del bmats, y, ws
     out.append(prefill_report(bq, device, stream, peaks, ob, "ternary", l2))
+    out.append(prefill_report(bq, device, stream, peaks, ob, "ternary_b3", l2))
 
     # ---- config 5: binary prefill (M=512) and the full-depth decode step
     out.append(prefill_report(bq, device, stream, peaks, ob, "binary", l2))
@@ -486,7 +518,8 @@ def prefill_report(bq, device, stream, peaks, ob, fmt_name, l2):
     that they are together larger than L2."""
     M, N, K = 512, 20480, K_HEAD
     o = ob.o
-    per_set = gemv_bytes(N, K, 0, 1 if fmt_name == "binary" else 2) + M * K * 2 + M * N * 2
+    bits = {"binary": 1, "ternary": 2, "ternary_b3": 26 * 8 / 128}[fmt_name]
+    per_set = gemv_bytes(N, K, 0, bits) + M * K * 2 + M * N * 2
     nset = max(2, math.ceil(1.5 * l2 / per_set))
     sets = []
     for c in range(nset):
@@ -495,7 +528,8 @@ def prefill_report(bq, device, stream, peaks, ob, fmt_name, l2):
                              synth.scales(c, N, K // 128, device=device))
         else:
             q = synth.random_ternary(c, synth.TID_TERNARY, (N, K), device=device)
-            pw = bq.pack_ternary_g128(q, synth.scales(c, N, K // 128, device=device))
+            pack = bq.pack_ternary_g128 if fmt_name == "ternary" else bq.pack_ternary_b3_g128
+            pw = pack(q, synth.scales(c, N, K // 128, device=device))
             del q
         sets.append((pw, synth.activations(c, M, K).to(device),
                      torch.empty((M, N), dtype=torch.bfloat16, device=device)))
@@ -513,16 +547,18 @@ def prefill_report(bq, device, stream, peaks, ob, fmt_name, l2):
     bq.gemm_prefill(X, pw, out=Y, workspace=ws)
     x = synth.activations(0, M, K)
     rows = 64
-    fmt = o.BINARY if fmt_name == "binary" else o.TERNARY
-    words, sc = _host_binary(0, rows, K) if fmt_name == "binary" else _host_ternary(ob, 0, rows, K)
+    fmt = {"binary": o.BINARY, "ternary": o.TERNARY, "ternary_b3": o.TERNARY_B3}[fmt_name]
+    words, sc = {"binary": lambda: _host_binary(0, rows, K), "ternary": lambda: _host_ternary(ob, 0, rows, K),
+                 "ternary_b3": lambda: _host_ternary_b3(ob, 0, rows, K)}[fmt_name]()
     ratio = ob.max_ratio(fmt, x, o.X_BF16, words, sc, K, Y[:, :rows].float().cpu().numpy())
 
     def work(lo, hi):
         ob.orc.gemv(fmt, x, o.X_BF16, words[lo:hi], sc[lo:hi], K)
     dt, n = ob.time_items(work, rows, ob.cores)
     del sets, ws
-    return {"workload": f"config {'5a' if fmt_name == 'binary' else '4b'}: {fmt_name} g128 prefill GEMM, "
-                        "M=512, K=5120, N=20480, x and y bf16",
+    name = {"binary": "config 5a: binary g128", "ternary": "config 4b: ternary g128",
+            "ternary_b3": "ternary g128 in base-3 storage (1.75 bits/weight)"}[fmt_name]
+    return {"workload": f"{name} prefill GEMM, M=512, K=5120, N=20480, x and y bf16",
             "us": round(ms * 1e3, 1), "TFLOPs": round(tf, 1), "bound": "tensor",
             "frac": round(tf / peaks["bf16_tflops"], 4), "peak": peaks["bf16_tflops"],
             "timing": f"back-to-back calls rotating {nset} sets of weights, x and y "
@@ -889,14 +925,16 @@ def run_case(args):
                                 synth.scales(0, N, K // 128, device=device))
             else:
                 q = synth.random_ternary(0, synth.TID_TERNARY, (N, K), device=device)
-                w = bq.pack_ternary_g128(q, synth.scales(0, N, K // 128, device=device))
+                pack = bq.pack_ternary_g128 if args.fmt == "ternary" else bq.pack_ternary_b3_g128
+                w = pack(q, synth.scales(0, N, K // 128, device=device))
                 del q
             x = synth.activations(0, M, K).to(device)
             if args.case == "gemv":
                 y = torch.empty((M, N), dtype=torch.float32, device=device)
                 ws = torch.empty(max(bq.gemv_workspace_bytes(M, w), 16), dtype=torch.uint8, device=device)
                 fn = lambda: bq.gemv(x, w, out=y, workspace=ws)
-                work = {"GBps": gemv_bytes(N, K, M, 1 if args.fmt == "binary" else 2) / 1e9}
+                bits = {"binary": 1, "ternary": 2, "ternary_b3": 26 * 8 / 128}[args.fmt]
+                work = {"GBps": gemv_bytes(N, K, M, bits) / 1e9}
             else:
                 y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
                 fn = lambda: bq.gemm_prefill(x, w, out=y)
@@ -929,7 +967,7 @@ def main():
                     help="total CPU time budget of --impl reference (split over warm-up and steps)")
     ap.add_argument("--case", choices=["gemv", "prefill", "embed"],
                     help="time one workload alone (for profiling) instead of the benchmark")
-    ap.add_argument("--fmt", choices=["binary", "ternary"], default="binary")
+    ap.add_argument("--fmt", choices=["binary", "ternary", "ternary_b3"], default="binary")
     ap.add_argument("--N", type=int, default=248320)
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--K", type=int, default=K_HEAD)

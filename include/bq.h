@@ -152,7 +152,7 @@ bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStr
 
 /*
  * Decode GEMV: y[m][n] = sum_g s[n][g] * sum_{k in group g} v[n][k] * x[m][k], with
- * v = 2b - 1 (binary) or c - 1 (ternary), for M <= 8 token rows.
+ * v = 2b - 1 (binary) or c - 1 (ternary, 2-bit or base-3 storage), for M <= 8 token rows.
  * Model card "prism-ml/Bonsai-27B-mlx-1bit", sections "Weight representation: Binary g128"
  * and "CUDA (NVIDIA GPUs)"; the decode (tg128) workload of section "Cross-platform
  * throughput".
@@ -168,7 +168,7 @@ bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStr
  *              workspace must be ordered on one stream.
  * Launches: two kernels (the prep and the GEMV, both programmatic dependent launches) when K
  * is a multiple of 1024 and the fragments fit in shared memory (K <= 5120 at M = 8, K <= 20480
- * at M = 1); otherwise one SIMT kernel.
+ * at M = 1); otherwise one SIMT kernel. Base-3 weights are decoded inside the same kernels.
  */
 bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w,
                   void *y, bq_dtype yt, void *workspace, size_t ws_bytes, cudaStream_t stream);
@@ -203,8 +203,8 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
 
 /*
  * Prefill GEMM: the same product for M up to 512 token rows (larger M is accepted),
- * Y[M][N] = X[M][K] * W^T with W the dequantised +-s (binary) or {-s, 0, +s} (ternary)
- * matrix. The packed bits are expanded on chip, straight into tensor memory, as the A
+ * Y[M][N] = X[M][K] * W^T with W the dequantised +-s (binary) or {-s, 0, +s} (ternary,
+ * 2-bit or base-3 storage) matrix. The packed bits are expanded on chip, straight into tensor memory, as the A
  * operand of the tensor cores (tcgen05, accumulation in fp32 in tensor memory); no expanded
  * copy is written to device memory. The pp512 (512-token prompt, compute-bound) workload of
  * the model card's section "Cross-platform throughput" and of the Ternary Bonsai 27B

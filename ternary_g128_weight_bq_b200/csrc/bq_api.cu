@@ -379,8 +379,6 @@ bq_status bq_gemm_prefill(const void *x, bq_dtype xt, int64_t M, const bq_weight
         return st;
     if ((st = validate_xy("gemm_prefill", x, xt, y, yt)) != BQ_OK)
         return st;
-    if (w->fmt == BQ_TERNARY_B3_G128)
-        return set_error(BQ_ERR_UNSUPPORTED, "gemm_prefill: the base-3 storage has no prefill kernel");
     if (M < 1 || M > (int64_t(1) << 24))
         return set_error(BQ_ERR_SHAPE, "gemm_prefill: M=%lld out of range", (long long)M);
     size_t need = prefill_workspace_bytes(M, w->fmt, w->N, w->K);

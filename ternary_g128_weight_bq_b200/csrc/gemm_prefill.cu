@@ -13,8 +13,9 @@
 //     of shared-memory stages (128-byte swizzle, zero fill past M); warp 0 also owns TMEM.
 //   * warps 2-9 (256 threads, two per weight row, each taking half of a k-block): read the
 //     row's packed bits and its group scale straight from global memory, expand every pair of
-//     weights to +-s (binary) or {-s, 0, +s} (ternary) in the operand type with a few integer
-//     or packed 16-bit float operations (expand_pairs), and write the 128 x 64 A tile with
+//     weights to +-s (binary) or {-s, 0, +s} (ternary, from 2-bit codes or base-3 bytes) in the
+//     operand type with a few integer or packed 16-bit float operations (expand_pairs,
+//     expand_pairs_b3), and write the 128 x 64 A tile with
 //     tcgen05.st straight into tensor memory (a ring of A stages next to the accumulator), so
 //     A needs no shared memory and no proxy fence. The scale is folded into the operand, so a
 //     group needs no separate rescaling. The operand type is always fp16, where +-s is exact
@@ -50,6 +51,7 @@
 
 #include <cstring>
 
+#include "b3.cuh"
 #include "bq_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -147,6 +149,53 @@ __device__ __forceinline__ void expand_pairs(uint2 wv, uint32_t s2, uint32_t (&a
                 av[8 * wi + j] = *reinterpret_cast<const uint32_t *>(&v);
             }
         }
+    }
+}
+
+// Base-3 storage (b3.cuh). A thread's 32 weights of a k-block are positions 32 V .. 32 V + 31 of
+// a group (V = 2 (k-block % 2) + its half of the k-block); they sit in the 8 group bytes
+// b3_pf_start(V) .. + 7 (for V = 3: five-code bytes 18..23 and the two four-code bytes), which
+// it loads as four 16-bit values (every such offset is even). Code p of a byte q is
+// floor(3 ((q 3^p) mod 256) / 256), so the two codes of a pair come from one multiply into
+// 16-bit lanes (two when the pair straddles two bytes), a mask, a multiply by 3 and a PRMT that
+// puts each code under the exponent bits of the fp16 value 1024; then (1024 + c) - 1025 and the
+// product with s are exact, as for the 2-bit codes.
+__host__ __device__ constexpr int b3_pf_start(int V) { return V == 0 ? 0 : V == 1 ? 6 : V == 2 ? 12 : 18; }
+
+__device__ __forceinline__ uint32_t prmt_pf(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+template <int V>
+__device__ __forceinline__ uint32_t b3_pf_byte(uint2 B, int j)
+{
+    const int i = j - b3_pf_start(V);                   // 0 .. 7
+    return prmt_pf(i < 4 ? B.x : B.y, 0u, 0x4440u + (uint32_t)(i & 3));
+}
+
+template <int V>
+__device__ __forceinline__ void expand_pairs_b3(uint2 B, uint32_t s2, uint32_t (&av)[16])
+{
+    constexpr uint32_t kMagic1 = 0x64016401u;           // 1025 | 1025
+#pragma unroll
+    for (int c = 0; c < 16; c++) {
+        const int P = 32 * V + 2 * c;                   // the pair's even position in the group
+        const int ja = b3::byte_of(P), jb = b3::byte_of(P + 1);
+        const int pa = P - b3::first(ja), pb = P + 1 - b3::first(jb);
+        const uint32_t qa = b3_pf_byte<V>(B, ja);
+        uint32_t pl;                                    // lanes: q 3^p of the two positions
+        if (ja == jb)
+            pl = qa * (b3::pow3(pa) + 65536u * b3::pow3(pb));
+        else
+            pl = b3_pf_byte<V>(B, jb) * (b3::pow3(pb) << 16) + qa * b3::pow3(pa);
+        const uint32_t r = (pl & 0x00FF00FFu) * 3u;     // code in bits 8..9 of each lane
+        const uint32_t h = prmt_pf(r, 0x64646464u, 0x4341u);   // lanes 1024 + code in fp16
+        __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&h), *reinterpret_cast<const __half2 *>(&kMagic1));
+        v = __hmul2(v, *reinterpret_cast<const __half2 *>(&s2));
+        av[c] = *reinterpret_cast<const uint32_t *>(&v);
     }
 }
 
@@ -389,9 +438,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         constexpr int kAhead = 4;                           // k-blocks of bits loaded ahead
         uint2 wq[kAhead];
         uint16_t sq[kAhead];
+        // base-3 rows: 26 G bytes each, an even number, so every 16-bit load below is aligned
+        const uint8_t *brow = reinterpret_cast<const uint8_t *>(words) + (row_ok ? n : 0) * (b3::kGroupBytes * G);
         auto load_kb = [&](int kbl, uint2 &wv_, uint16_t &sv_) {   // kbl: k-block of this CTA
             const int kbg = kb0 + kbl;
-            if (WPT == 1)
+            if (FMT == BQ_TERNARY_B3_G128) {
+                const int64_t g = kbg >> 1, f = g & ~int64_t(7);
+                const int64_t nb = G - f < 8 ? G - f : 8;
+                const int V = 2 * (kbg & 1) + hk;
+                const uint8_t *five = brow + b3::kGroupBytes * f + 24 * (g - f) + b3_pf_start(V);
+                const uint8_t *four = brow + b3::kGroupBytes * f + 24 * nb + 2 * (g - f);
+                const uint32_t h0 = __ldg(reinterpret_cast<const uint16_t *>(five));
+                const uint32_t h1 = __ldg(reinterpret_cast<const uint16_t *>(five + 2));
+                const uint32_t h2 = __ldg(reinterpret_cast<const uint16_t *>(five + 4));
+                const uint32_t h3 = __ldg(reinterpret_cast<const uint16_t *>(V == 3 ? four : five + 6));
+                wv_ = make_uint2(h0 | (h1 << 16), h2 | (h3 << 16));
+            } else if (WPT == 1)
                 wv_ = make_uint2(__ldg(wrow + (size_t)kbg * 2 * kBitsPerW) >> bshift, 0u);
             else
                 wv_ = __ldg(reinterpret_cast<const uint2 *>(wrow + (size_t)kbg * 4));
@@ -424,7 +486,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             ptx::tc_fence_after();
             const uint32_t s2 = row_ok ? scale_pair(sv) : 0u;
             uint32_t av[kCols];                              // 2 weights per 32-bit column
-            expand_pairs<FMT, kCols>(wv, s2, av);
+            if constexpr (FMT == BQ_TERNARY_B3_G128) {
+                static_assert(kCols == 16, "a base-3 part is 32 weights");
+                switch (2 * ((kb0 + kb) & 1) + hk) {
+                case 0: expand_pairs_b3<0>(wv, s2, av); break;
+                case 1: expand_pairs_b3<1>(wv, s2, av); break;
+                case 2: expand_pairs_b3<2>(wv, s2, av); break;
+                default: expand_pairs_b3<3>(wv, s2, av); break;
+                }
+            } else {
+                expand_pairs<FMT, kCols>(wv, s2, av);
+            }
             if (!row_ok) {
 #pragma unroll
                 for (int c = 0; c < kCols; c++)
@@ -782,6 +854,8 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s, unsigned *launc
     *launches = (pf_plan(a.M, a.N, a.K, bn_for(a.M)).tail > 0 ? 3 : 1) + (a.xt == BQ_BF16 ? 1 : 0);
     if (a.fmt == BQ_BINARY_G128)
         return launch_bn<BQ_BINARY_G128>(a, s);
+    if (a.fmt == BQ_TERNARY_B3_G128)
+        return launch_bn<BQ_TERNARY_B3_G128>(a, s);
     return launch_bn<BQ_TERNARY_G128>(a, s);
 }
 

@@ -210,10 +210,54 @@ def test_b3_embed(orc, ot):
         assert torch.equal(out.float(), ev)
 
 
-def test_b3_prefill_reports_unsupported():
+def run_b3_prefill(orc, seed, M, N, K, xdt=torch.bfloat16, ydt=torch.float32, rows=None, x=None):
     m = bq()
-    q = ternary_q(17, 128, 1024)
-    w = m.pack_ternary_b3_g128(q.cuda(), synth.scales(17, 128, 8).cuda())
-    with pytest.raises(m.BQError) as e:
-        m.gemm_prefill(synth.activations(17, 16, 1024).cuda(), w)
-    assert e.value.status_name == "BQ_ERR_UNSUPPORTED"
+    q = ternary_q(seed, N, K)
+    s = synth.scales(seed, N, K // 128)
+    w, ref, s_ref = _pack_both(orc, q, s)
+    if x is None:
+        x = synth.activations(seed + 1, M, K, dtype=xdt)
+    y = m.gemm_prefill(x.cuda(), w, out_dtype=ydt)
+    torch.cuda.synchronize()
+    m.get_device_error()
+    y_ref, bound = orc.gemv(T3, x, x_dtype_code(x.dtype), ref, s_ref, K, rows=rows)
+    yg = y if rows is None else y[:, torch.from_numpy(rows).cuda()]
+    return assert_within_bound(yg, y_ref, bound, f"base-3 prefill M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (17, 300, 640), (77, 1000, 256), (130, 256, 1152),
+                                   (300, 200, 2176), (512, 384, 5120)])
+def test_b3_prefill_all_outputs(orc, M, N, K):
+    """tcgen05 prefill with the base-3 operand expansion: all four 32-weight parts of a group,
+    blocks of fewer than 8 groups, split tails."""
+    run_b3_prefill(orc, 800 + M, M, N, K)
+
+
+@pytest.mark.parametrize("ydt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("xdt", [torch.float16, torch.bfloat16])
+def test_b3_prefill_dtypes(orc, xdt, ydt):
+    run_b3_prefill(orc, 18, 200, 256, 1024, xdt=xdt, ydt=ydt)
+
+
+def test_b3_prefill_m512_k5120_n20480_sampled(orc):
+    """The ternary prefill workload (M=512, K=5120, N=20480) in base-3 storage, all tokens of
+    sampled weight rows, launched as the benchmark launches it."""
+    run_b3_prefill(orc, 0, 512, 20480, 5120, rows=sample_rows(20480, 400))
+
+
+def test_b3_prefill_special_codes(orc):
+    """Rows of all -1, all 0, all +1 codes and a repeating pattern through the prefill decode."""
+    m = bq()
+    N, K, M = 128, 1024, 64
+    q = torch.empty((N, K), dtype=torch.int8)
+    q[0::4] = -1
+    q[1::4] = 0
+    q[2::4] = 1
+    q[3::4] = torch.tensor([(-1, 0, 1)[k % 3] for k in range(K)], dtype=torch.int8)
+    s = synth.scales(19, N, K // 128)
+    x = synth.activations(19, M, K)
+    w, ref, s_ref = _pack_both(orc, q, s)
+    y = m.gemm_prefill(x.cuda(), w)
+    y_ref, bound = orc.gemv(T3, x, oracle.X_BF16, ref, s_ref, K)
+    assert_within_bound(y, y_ref, bound, "prefill special codes")
+    assert torch.all(y[:, 1::4] == 0)
