@@ -135,6 +135,10 @@ class Oracle:
         L.bqo_gemv_rows.restype = ctypes.c_int
         L.bqo_embed.argtypes = [ctypes.c_int, P, I64, P, P, I64, I64, P]
         L.bqo_embed.restype = I64
+        L.bqo_topk.argtypes = [P, I64, I64, ctypes.c_int, P, P]
+        L.bqo_topk.restype = ctypes.c_int
+        L.bqo_sample_topk.argtypes = [P, P, ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_double]
+        L.bqo_sample_topk.restype = I64
         L.bqo_mlx_affine_dequant.argtypes = [ctypes.c_uint16, ctypes.c_int]
         L.bqo_mlx_affine_dequant.restype = ctypes.c_uint16
         self.L = L
@@ -210,6 +214,25 @@ class Oracle:
         out = np.zeros((len(i), K), dtype=np.float64)
         bad = self.L.bqo_embed(fmt, _p(i), len(i), _p(w), _p(s), w.shape[0], K, _p(out))
         return out, int(bad)
+
+    def topk(self, y, k: int):
+        """(idx int64[M, k], vals fp64[M, k]): the k largest of each row of y (fp64 [M, N]),
+        descending, equal values in ascending index order."""
+        y = np.ascontiguousarray(y, dtype=np.float64)
+        M, N = y.shape
+        idx = np.zeros((M, k), dtype=np.int64)
+        vals = np.zeros((M, k), dtype=np.float64)
+        st = self.L.bqo_topk(_p(y), M, N, k, _p(idx), _p(vals))
+        if st != OK:
+            raise ValueError(f"topk status {st}")
+        return idx, vals
+
+    def sample_topk(self, vals, idx, T: float, top_p: float, u: float) -> int:
+        """Token drawn from one row of top-k candidates (vals descending) with temperature T,
+        top-p and the uniform number u."""
+        v = np.ascontiguousarray(vals, dtype=np.float64)
+        i = np.ascontiguousarray(idx, dtype=np.int64)
+        return int(self.L.bqo_sample_topk(_p(v), _p(i), len(v), T, top_p, u))
 
     def to_bf16_bits(self, v) -> np.ndarray:
         """Round fp64 values to bfloat16 (ties to even); returns uint16 bits."""

@@ -453,6 +453,76 @@ int64_t bqo_embed(int fmt, const int32_t *ids, int64_t T, const uint32_t *words,
 }
 
 /* ---------------------------------------------------------------------------------------
+ * Top-k of the logits and sampling from it. [card] "Generation parameters": temperature 0.7,
+ * top-p 0.95, top-k 20 for every reported benchmark run. The pages do not state the order of
+ * the three filters; the reading taken here: the k largest logits (equal values in ascending
+ * index order) are the candidates; their probabilities are softmax(logit / T) over the k; top-p
+ * keeps the shortest leading run of candidates whose probabilities sum to at least top_p (at
+ * least one); the token is the first kept candidate whose cumulative probability, renormalised
+ * over the kept ones, exceeds u, a uniform number in [0, 1) drawn by the caller.
+ * ------------------------------------------------------------------------------------- */
+
+/* a ranks before b: larger value, or the same value and a smaller index */
+static int ranks_before(double va, int64_t ia, double vb, int64_t ib)
+{
+    return va > vb || (va == vb && ia < ib);
+}
+
+int bqo_topk(const double *y, int64_t M, int64_t N, int k, int64_t *idx, double *vals)
+{
+    if (M < 0 || N < 1 || k < 1 || k > N)
+        return BQO_ERR_SHAPE;
+    for (int64_t m = 0; m < M; m++) {
+        const double *row = y + m * N;
+        for (int j = 0; j < k; j++) {
+            /* the best entry that ranks after the (j-1)-th pick */
+            int64_t best = -1;
+            for (int64_t n = 0; n < N; n++) {
+                if (j > 0 && !ranks_before(vals[m * k + j - 1], idx[m * k + j - 1], row[n], n))
+                    continue;
+                if (best < 0 || ranks_before(row[n], n, row[best], best))
+                    best = n;
+            }
+            idx[m * k + j] = best;
+            vals[m * k + j] = row[best];
+        }
+    }
+    return BQO_OK;
+}
+
+int64_t bqo_sample_topk(const double *vals, const int64_t *idx, int k, double T, double top_p, double u)
+{
+    if (k < 1 || !(T > 0.0))
+        return -1;
+    double p[64];
+    if (k > 64)
+        return -1;
+    double z = 0.0;
+    for (int i = 0; i < k; i++) {
+        p[i] = exp((vals[i] - vals[0]) / T);      /* vals[0] is the largest: no overflow */
+        z += p[i];
+    }
+    int keep = 0;
+    double c = 0.0;
+    while (keep < k) {
+        c += p[keep] / z;
+        keep++;
+        if (c >= top_p)
+            break;
+    }
+    double kept = 0.0;
+    for (int i = 0; i < keep; i++)
+        kept += p[i];
+    double cum = 0.0;
+    for (int i = 0; i < keep; i++) {
+        cum += p[i] / kept;
+        if (cum > u)
+            return idx[i];
+    }
+    return idx[keep - 1];                           /* u just below 1 and rounding */
+}
+
+/* ---------------------------------------------------------------------------------------
  * MLX affine form ([card] "MLX packaging"): w = s_mlx * q + bias with q in {0, 1},
  * s_mlx = 2 * s and bias = -s, each stored and each operation rounded in binary16.
  * Returns the binary16 bits of w.

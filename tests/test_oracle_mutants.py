@@ -73,6 +73,14 @@ MUTANTS = {
     "b3_decode_rounds": (
         "int64_t v = ((int64_t)byte * kPow3[n]) / 256;",
         "int64_t v = ((int64_t)byte * kPow3[n] + 128) / 256;"),
+    "topk_ties_high_index_first": (
+        "return va > vb || (va == vb && ia < ib);", "return va > vb || (va == vb && ia > ib);"),
+    "sample_temperature_multiplies": (
+        "p[i] = exp((vals[i] - vals[0]) / T);", "p[i] = exp((vals[i] - vals[0]) * T);"),
+    "sample_top_p_strict": (
+        "if (c >= top_p)", "if (c > top_p)"),
+    "sample_not_renormalised": (
+        "cum += p[i] / kept;", "cum += p[i] / z;"),
     "sum_skips_last_k": (
         "for (int64_t k = 0; k < K; k++) {\n                double xv",
         "for (int64_t k = 0; k < K - 1; k++) {\n                double xv"),

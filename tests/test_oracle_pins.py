@@ -265,6 +265,62 @@ def pin_b3_bits_per_weight(o):
 
 
 # --------------------------------------------------------------------------------------
+# Top-k and sampling (model card "Generation parameters": temperature 0.7, top-p 0.95, top-k 20)
+# --------------------------------------------------------------------------------------
+
+def pin_topk_hand(o):
+    idx, vals = o.topk(np.array([[1.0, 5.0, 3.0, 5.0, -2.0], [0.0, 0.0, 0.0, -1.0, 2.0]]), 3)
+    assert idx.tolist() == [[1, 3, 2], [4, 0, 1]]
+    assert vals.tolist() == [[5.0, 5.0, 3.0], [2.0, 0.0, 0.0]]
+
+
+def pin_topk_vs_numpy(o):
+    """Against numpy's lexsort (value descending, then index ascending), with many ties."""
+    rng = np.random.default_rng(21)
+    for N, k in ((1000, 20), (37, 37), (5000, 1), (300, 32)):
+        y = np.round(rng.normal(size=(3, N)) * 4) / 4          # a few hundred distinct values
+        idx, vals = o.topk(y, k)
+        for m in range(3):
+            order = np.lexsort((np.arange(N), -y[m]))[:k]
+            assert idx[m].tolist() == order.tolist()
+            assert vals[m].tolist() == y[m, order].tolist()
+
+
+def pin_sample_hand(o):
+    """Hand-worked probabilities: logits with exact exponentials."""
+    ln2 = math.log(2.0)
+    v2, i2 = np.array([0.0, 0.0]), np.array([7, 9])
+    assert o.sample_topk(v2, i2, 1.0, 1.0, 0.49) == 7 and o.sample_topk(v2, i2, 1.0, 1.0, 0.51) == 9
+    # top-p 0.5: the first candidate alone reaches it
+    assert o.sample_topk(v2, i2, 1.0, 0.5, 0.9) == 7
+    # p proportional to 4, 2, 1: cumulative 4/7, 6/7; top-p 0.8 keeps two, renormalised 2/3, 1/3
+    v3, i3 = np.array([2 * ln2, ln2, 0.0]), np.array([30, 10, 20])
+    assert o.sample_topk(v3, i3, 1.0, 0.8, 0.62) == 30
+    assert o.sample_topk(v3, i3, 1.0, 0.8, 0.70) == 10
+    assert o.sample_topk(v3, i3, 1.0, 1.0, 0.80) == 10 and o.sample_topk(v3, i3, 1.0, 1.0, 0.90) == 20
+    # temperature 0.5 squares the ratios: 16, 4, 1 -> cumulative 16/21, 20/21
+    assert o.sample_topk(v3, i3, 0.5, 1.0, 0.75) == 30 and o.sample_topk(v3, i3, 0.5, 1.0, 0.77) == 10
+    assert o.sample_topk(v3, i3, 0.5, 1.0, 0.96) == 20
+
+
+def pin_sample_frequencies(o):
+    """Over a fine grid of u the draws follow softmax(v / T) restricted to the top-p prefix."""
+    rng = np.random.default_rng(22)
+    v = np.sort(rng.normal(size=20))[::-1] * 3
+    ids = np.arange(100, 120)
+    T, top_p = 0.7, 0.95
+    p = np.exp((v - v[0]) / T)
+    p /= p.sum()
+    keep = int(np.searchsorted(np.cumsum(p), top_p) + 1)
+    q = p[:keep] / p[:keep].sum()
+    us = (np.arange(20000) + 0.5) / 20000
+    draws = np.array([o.sample_topk(v, ids, T, top_p, u) for u in us])
+    assert set(np.unique(draws)) <= set(ids[:keep].tolist())
+    freq = np.array([np.mean(draws == ids[i]) for i in range(keep)])
+    assert np.max(np.abs(freq - q)) <= 1.5 / 20000
+
+
+# --------------------------------------------------------------------------------------
 # Mapping and closed forms
 # --------------------------------------------------------------------------------------
 
@@ -483,3 +539,7 @@ def test_b3_examples(orc): pin_b3_examples(orc)
 def test_b3_byte_values(orc): pin_b3_byte_values(orc)
 def test_b3_equals_2bit(orc): pin_b3_equals_2bit(orc)
 def test_b3_bits_per_weight(orc): pin_b3_bits_per_weight(orc)
+def test_topk_hand(orc): pin_topk_hand(orc)
+def test_topk_vs_numpy(orc): pin_topk_vs_numpy(orc)
+def test_sample_hand(orc): pin_sample_hand(orc)
+def test_sample_frequencies(orc): pin_sample_frequencies(orc)
