@@ -135,6 +135,8 @@ class Oracle:
         L.bqo_gemv_rows.restype = ctypes.c_int
         L.bqo_embed.argtypes = [ctypes.c_int, P, I64, P, P, I64, I64, P]
         L.bqo_embed.restype = I64
+        L.bqo_quantize_g128.argtypes = [ctypes.c_int, P, I64, I64, P, P]
+        L.bqo_quantize_g128.restype = ctypes.c_int
         L.bqo_topk.argtypes = [P, I64, I64, ctypes.c_int, P, P]
         L.bqo_topk.restype = ctypes.c_int
         L.bqo_sample_topk.argtypes = [P, P, ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_double]
@@ -214,6 +216,20 @@ class Oracle:
         out = np.zeros((len(i), K), dtype=np.float64)
         bad = self.L.bqo_embed(fmt, _p(i), len(i), _p(w), _p(s), w.shape[0], K, _p(out))
         return out, int(bad)
+
+    def quantize(self, fmt: int, w):
+        """Dense fp32 w [N, K] -> (q int8 [N, K], s fp16 bits uint16 [N, K/128]): the
+        least-squares binary or ternary fit of every group of 128."""
+        if hasattr(w, "detach"):
+            w = w.detach().cpu().float().numpy()
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        N, K = w.shape
+        q = np.zeros((N, K), dtype=np.int8)
+        s = np.zeros((N, K // 128), dtype=np.uint16)
+        st = self.L.bqo_quantize_g128(fmt, _p(w), N, K, _p(q), _p(s))
+        if st != OK:
+            raise ValueError(f"quantize status {st}")
+        return q, s
 
     def topk(self, y, k: int):
         """(idx int64[M, k], vals fp64[M, k]): the k largest of each row of y (fp64 [M, N]),

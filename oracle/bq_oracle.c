@@ -41,6 +41,7 @@
  *     ternary weights the scale counts even where the code is 0.
  */
 #include <math.h>
+#include <stdlib.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -520,6 +521,78 @@ int64_t bqo_sample_topk(const double *vals, const int64_t *idx, int k, double T,
             return idx[i];
     }
     return idx[keep - 1];                           /* u just below 1 and rounding */
+}
+
+/* ---------------------------------------------------------------------------------------
+ * Dense -> g128 quantiser. The pages name the format but not how q and s are obtained ([card]
+ * "Weight representation: Binary g128" points to a whitepaper that is not among them). The
+ * reading taken: the least-squares fit of each group of 128 weights w,
+ *   binary:  q = +1 where w >= 0, else -1; s = mean |w| (for fixed signs, sum (w - s q)^2 is
+ *            smallest at s = sum |w| / 128);
+ *   ternary: q and s >= 0 minimising sum (w - s q)^2 over q in {-1, 0, +1}^128: on a support of
+ *            j weights the best q is their sign and the best s their mean |w|, leaving
+ *            sum w^2 - (sum_support |w|)^2 / j; so the support is the j largest |w| (equal |w|:
+ *            lower position first) with j maximising (sum of those |w|)^2 / j, the smallest such
+ *            j on a tie, and none for a group of zeros.
+ * s is then rounded to binary16 (ties to even). Inputs are binary32.
+ * ------------------------------------------------------------------------------------- */
+
+struct absw {
+    double a;
+    int k;
+};
+
+static int absw_desc(const void *pa, const void *pb)
+{
+    const struct absw *a = pa, *b = pb;
+    if (a->a != b->a)
+        return a->a > b->a ? -1 : 1;
+    return a->k - b->k;
+}
+
+int bqo_quantize_g128(int fmt, const float *w, int64_t N, int64_t K, int8_t *q, uint16_t *s)
+{
+    if (N < 0 || K <= 0 || K % 128 || (fmt != BQO_BINARY && fmt != BQO_TERNARY && fmt != BQO_TERNARY_B3))
+        return BQO_ERR_SHAPE;
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t g = 0; g < K / 128; g++) {
+            const float *wg = w + n * K + 128 * g;
+            int8_t *qg = q + n * K + 128 * g;
+            if (fmt == BQO_BINARY) {
+                double sum = 0.0;
+                for (int k = 0; k < 128; k++) {
+                    qg[k] = wg[k] >= 0.0f ? 1 : -1;
+                    sum += fabs((double)wg[k]);
+                }
+                s[n * (K / 128) + g] = bqo_f64_to_f16(sum / 128.0);
+                continue;
+            }
+            struct absw order[128];
+            for (int k = 0; k < 128; k++) {
+                order[k].a = fabs((double)wg[k]);
+                order[k].k = k;
+                qg[k] = 0;
+            }
+            qsort(order, 128, sizeof order[0], absw_desc);
+            double best = 0.0, prefix = 0.0, best_sum = 0.0;
+            int best_j = 0;
+            for (int j = 1; j <= 128; j++) {
+                prefix += order[j - 1].a;
+                double score = prefix * prefix / j;
+                if (score > best) {
+                    best = score;
+                    best_j = j;
+                    best_sum = prefix;
+                }
+            }
+            for (int j = 0; j < best_j; j++) {
+                int k = order[j].k;
+                qg[k] = wg[k] >= 0.0f ? 1 : -1;
+            }
+            s[n * (K / 128) + g] = bqo_f64_to_f16(best_j ? best_sum / best_j : 0.0);
+        }
+    }
+    return BQO_OK;
 }
 
 /* ---------------------------------------------------------------------------------------

@@ -81,6 +81,14 @@ MUTANTS = {
         "if (c >= top_p)", "if (c > top_p)"),
     "sample_not_renormalised": (
         "cum += p[i] / kept;", "cum += p[i] / z;"),
+    "quantize_zero_group_full_support": (
+        "if (score > best) {", "if (score >= best) {"),
+    "quantize_sort_ascending": (
+        "return a->a > b->a ? -1 : 1;", "return a->a > b->a ? 1 : -1;"),
+    "quantize_binary_scale_127": (
+        "s[n * (K / 128) + g] = bqo_f64_to_f16(sum / 128.0);", "s[n * (K / 128) + g] = bqo_f64_to_f16(sum / 127.0);"),
+    "quantize_binary_zero_negative": (
+        "qg[k] = wg[k] >= 0.0f ? 1 : -1;\n                    sum +=", "qg[k] = wg[k] > 0.0f ? 1 : -1;\n                    sum +="),
     "sum_skips_last_k": (
         "for (int64_t k = 0; k < K; k++) {\n                double xv",
         "for (int64_t k = 0; k < K - 1; k++) {\n                double xv"),

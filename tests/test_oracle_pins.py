@@ -265,6 +265,75 @@ def pin_b3_bits_per_weight(o):
 
 
 # --------------------------------------------------------------------------------------
+# Dense -> g128 quantiser (least-squares fit per group; the pages do not give the method)
+# --------------------------------------------------------------------------------------
+
+def _f16(v):
+    return np.float16(v).view(np.uint16)            # numpy rounds fp64 to fp16 to nearest even
+
+
+def pin_quantize_hand(o):
+    w = np.zeros((3, 128), np.float32)
+    w[0, :3] = [3, -3, 1]                           # scores 9, 36/2, 49/3: support {0, 1}, s = 3
+    w[1, ::2], w[1, 1::2] = 2, -2
+    # row 2: all zeros
+    qt, st = o.quantize(T, w)
+    assert qt[0, :3].tolist() == [1, -1, 0] and np.all(qt[0, 3:] == 0) and st[0, 0] == _f16(3.0)
+    assert np.all(qt[1] == np.where(w[1] > 0, 1, -1)) and st[1, 0] == _f16(2.0)
+    assert np.all(qt[2] == 0) and st[2, 0] == _f16(0.0)
+    qb, sb = o.quantize(B, w)
+    assert np.all(qb == np.where(w >= 0, 1, -1))
+    assert sb[0, 0] == _f16(7 / 128) and sb[1, 0] == _f16(2.0) and sb[2, 0] == _f16(0.0)
+
+
+def pin_quantize_binary_closed_form(o):
+    rng = np.random.default_rng(31)
+    w = (rng.normal(size=(6, 640)) * 0.02).astype(np.float32)
+    q, s = o.quantize(B, w)
+    assert np.array_equal(q, np.where(w >= 0, 1, -1).astype(np.int8))
+    mean = np.abs(w.astype(np.float64)).reshape(6, 5, 128).mean(axis=2)
+    assert np.array_equal(s, _f16(mean))
+
+
+def pin_quantize_ternary_bruteforce(o):
+    """Groups with at most 10 non-zero weights: the oracle's support is the subset of them with
+    the smallest squared error, found by trying all 2^10 subsets."""
+    import itertools
+    rng = np.random.default_rng(32)
+    for trial in range(40):
+        w = np.zeros((1, 128), np.float32)
+        nz = rng.choice(128, size=int(rng.integers(1, 11)), replace=False)
+        w[0, nz] = (rng.normal(size=len(nz)) * rng.uniform(0.1, 3)).astype(np.float32)
+        q, s = o.quantize(T, w)
+        a = np.abs(w[0, nz].astype(np.float64))
+        tot = float(np.sum(w[0].astype(np.float64) ** 2))
+        best, best_set = tot, ()
+        for r in range(1, len(nz) + 1):
+            for sub in itertools.combinations(range(len(nz)), r):
+                err = tot - float(np.sum(a[list(sub)])) ** 2 / r
+                if err < best - 1e-12:
+                    best, best_set = err, sub
+        support = sorted(int(nz[i]) for i in best_set)
+        assert sorted(np.nonzero(q[0])[0].tolist()) == support
+        assert np.all(q[0, support] == np.sign(w[0, support]))
+        mean = np.mean(a[list(best_set)]) if best_set else 0.0
+        assert s[0, 0] == _f16(mean)
+
+
+def pin_quantize_invariants(o):
+    rng = np.random.default_rng(33)
+    w = (rng.normal(size=(4, 256)) * 0.05).astype(np.float32)
+    w[w == 0] = 1e-3
+    for fmt in (B, T):
+        q, s = o.quantize(fmt, w)
+        q4, s4 = o.quantize(fmt, 4 * w)
+        assert np.array_equal(q4, q)
+        assert np.array_equal(s4.view(np.float16).astype(np.float64), 4 * s.view(np.float16).astype(np.float64))
+        qn, sn = o.quantize(fmt, -w)
+        assert np.array_equal(qn, -q) and np.array_equal(sn, s)
+
+
+# --------------------------------------------------------------------------------------
 # Top-k and sampling (model card "Generation parameters": temperature 0.7, top-p 0.95, top-k 20)
 # --------------------------------------------------------------------------------------
 
@@ -539,6 +608,10 @@ def test_b3_examples(orc): pin_b3_examples(orc)
 def test_b3_byte_values(orc): pin_b3_byte_values(orc)
 def test_b3_equals_2bit(orc): pin_b3_equals_2bit(orc)
 def test_b3_bits_per_weight(orc): pin_b3_bits_per_weight(orc)
+def test_quantize_hand(orc): pin_quantize_hand(orc)
+def test_quantize_binary_closed_form(orc): pin_quantize_binary_closed_form(orc)
+def test_quantize_ternary_bruteforce(orc): pin_quantize_ternary_bruteforce(orc)
+def test_quantize_invariants(orc): pin_quantize_invariants(orc)
 def test_topk_hand(orc): pin_topk_hand(orc)
 def test_topk_vs_numpy(orc): pin_topk_vs_numpy(orc)
 def test_sample_hand(orc): pin_sample_hand(orc)
