@@ -338,6 +338,47 @@ def _gemv_entry(name, N, K, M, fmt_bits, ms, peaks, extra=None):
     return e
 
 
+def lm_head_topk_entry(bq, device, stream, peaks, ob, w, x, xd, oracle_timing):
+    """The LM head fused with top-k 20 and a draw (temperature 0.7, top-p 0.95), M = 1: one call
+    computes the 248 320 logits, keeps the 20 largest and draws a token; the logits are never
+    written. Timed like the plain LM head; checked against the oracle on the full row."""
+    import numpy as np
+    o = ob.o
+    N, K, k = w.N, w.K, 20
+    u = torch.tensor([0.37], dtype=torch.float32, device=device)
+    ws = torch.empty(bq.gemv_topk_workspace_bytes(1, w, k), dtype=torch.uint8, device=device)
+    vals = torch.empty((1, k), dtype=torch.float32, device=device)
+    idx = torch.empty((1, k), dtype=torch.int32, device=device)
+    tok = torch.empty((1,), dtype=torch.int32, device=device)
+    call = lambda: bq.gemv_topk(xd, w, k=k, u=u, temperature=0.7, top_p=0.95, workspace=ws, out=(vals, idx, tok))
+    call()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(20):
+            call()
+    ms = time_single(g.replay, 10, 3, stream) / 20
+    del g
+    call()
+    torch.cuda.synchronize()
+    # parity: the oracle's logits of the full row (all 248320), its top 20, and its draw
+    words, sc = _host_binary(0, N, K)
+    y_ref, bound = ob.orc.gemv(o.BINARY, x, o.X_BF16, words, sc, K)
+    oi, ov = ob.orc.topk(y_ref, k)
+    gi, gv = idx.cpu().numpy()[0], vals.cpu().numpy()[0].astype(np.float64)
+    same_set = set(gi.tolist()) == set(oi[0].tolist())
+    ratio = float(np.max(np.abs(gv - y_ref[0, gi]) / bound[0, gi]))
+    draw_ref = ob.orc.sample_topk(gv, gi, 0.7, 0.95, 0.37)
+    ent = _gemv_entry(f"LM head fused with top-k {k} and a draw (temperature 0.7, top-p 0.95), binary g128, "
+                      f"M=1, K=5120, N=248320", N, K, 1, 1, ms, peaks,
+                      {"timing": "graph of 20 back-to-back calls (179 MB of weights per call, above L2)",
+                       "parity": {"max_err_over_bound": round(ratio, 5), "same_set_as_oracle": same_set,
+                                  "token": int(tok.item()), "oracle_draw_on_same_candidates": draw_ref,
+                                  "rows": N}})
+    ent["oracle"] = oracle_timing
+    return ent
+
+
 def _rotating_gemv_ms(bq, mats, x, y, ws, stream, reps=20):
     """Device ms of one call over a CUDA graph of back-to-back calls that rotate through `mats`
     (weight copies together larger than L2)."""
@@ -422,6 +463,7 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
     e["oracle"] = ob.gemv_timing(o.BINARY, x, o.X_BF16, *_host_binary(0, 4096, K), K, K // 8 + K // 64,
                                  2 * K, False)
     out.append(e)
+    out.append(lm_head_topk_entry(bq, device, stream, peaks, ob, w, x, xd, e["oracle"]))
     # embedding gather: output buffers rotate (together above L2), so the writes reach HBM
     T = 4096
     ids = synth.random_ids(0, synth.TID_IDS, T, N)

@@ -202,6 +202,39 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
                           void *y, bq_dtype yt, cudaStream_t stream);
 
 /*
+ * LM head with top-k: the decode GEMV's outputs y[m][n] (as bq_gemv computes them, fp32) are
+ * not written; instead each token row's k largest are returned, and optionally a token drawn
+ * from them. Model card "prism-ml/Bonsai-27B-mlx-1bit", section "Generation parameters":
+ * top-k 20, top-p 0.95, temperature 0.7 (the pages do not give the order of the three; this
+ * call applies them as described for `tokens` below).
+ *   x, xt, M, w  as bq_gemv (M 1..8); w->K a multiple of 1024 (the tensor-core path).
+ *   k            1..32 and k <= N.
+ *   vals, idx    out, float [M][k] and int32 [M][k]: the k largest outputs of each row in
+ *                descending order (equal values: lower index first) and their row indices n.
+ *   u            NULL, or float [M] uniform numbers in [0, 1), one per token row (device).
+ *   temperature, top_p   used with u: temperature > 0, 0 < top_p <= 1.
+ *   tokens       out with u, int32 [M]: probabilities softmax(v / temperature) over the k
+ *                candidates; the shortest leading run of candidates whose probabilities sum
+ *                to at least top_p is kept; the token is the first kept candidate whose
+ *                cumulative probability, renormalised over the kept ones, exceeds u.
+ *   workspace    bq_gemv_topk_workspace_bytes(M, w, k) bytes (16-byte aligned): the digit
+ *                fragments of x, each CTA's k candidates per row and a ticket counter. Contents
+ *                need not be initialised; calls sharing a workspace must be ordered on one stream.
+ * The GEMV's CTAs each own whole rows: a CTA keeps its rows' outputs in shared memory, selects
+ * their k largest and writes them to the workspace; the last CTA to finish selects the k
+ * largest of those and writes vals, idx and tokens. x with an infinity or NaN gives an
+ * unspecified selection for that row.
+ * Errors: as bq_gemv; BQ_ERR_SHAPE for K not a multiple of 1024 or a k out of range.
+ * Launches: two kernels (the x prep and the GEMV with the selection).
+ */
+bq_status bq_gemv_topk(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, int k,
+                       float *vals, int32_t *idx, const float *u, float temperature, float top_p,
+                       int32_t *tokens, void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes bq_gemv_topk needs (0 if the shape or k is not supported). */
+size_t bq_gemv_topk_workspace_bytes(int64_t M, const bq_weight *w, int k);
+
+/*
  * Prefill GEMM: the same product for M up to 512 token rows (larger M is accepted),
  * Y[M][N] = X[M][K] * W^T with W the dequantised +-s (binary) or {-s, 0, +s} (ternary,
  * 2-bit or base-3 storage) matrix. The packed bits are expanded on chip, straight into tensor memory, as the A

@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
             "bq_gemv": ([P, I, I64, W, P, I, P, ctypes.c_size_t, P], I),
             "bq_gemv_workspace_bytes": ([I64, W], ctypes.c_size_t),
             "bq_gemv_noalloc": ([P, I, I64, W, P, I, P], I),
+            "bq_gemv_topk": ([P, I, I64, W, I, P, P, P, ctypes.c_float, ctypes.c_float, P, P, ctypes.c_size_t, P], I),
+            "bq_gemv_topk_workspace_bytes": ([I64, W, I], ctypes.c_size_t),
             "bq_gemm_prefill": ([P, I, I64, W, P, I, P, ctypes.c_size_t, P], I),
             "bq_gemm_prefill_workspace_bytes": ([I64, W], ctypes.c_size_t),
             "bq_embed_gather": ([P, I64, W, P, I, P], I),
@@ -265,6 +267,52 @@ def gemv_noalloc(x: torch.Tensor, w: BQWeight, out_dtype=torch.float32,
         _check(lib().bq_gemv_noalloc(x.data_ptr(), _DTYPE[x.dtype], M, w.c, out.data_ptr(),
                                      _DTYPE[out.dtype], _stream(x.device)))
     return out
+
+
+def gemv_topk_workspace_bytes(M: int, w: BQWeight, k: int) -> int:
+    return int(lib().bq_gemv_topk_workspace_bytes(M, w.c, k))
+
+
+def gemv_topk(x: torch.Tensor, w: BQWeight, k: int = 20, u: torch.Tensor = None, temperature: float = 0.7,
+              top_p: float = 0.95, workspace: torch.Tensor = None, out=None):
+    """The k largest outputs of x @ W^T per token row, without writing the outputs:
+    (vals fp32 [M, k] descending, idx int32 [M, k]). With u (fp32 [M] uniform numbers in [0, 1))
+    also the token drawn from them with temperature and top-p: (vals, idx, tokens int32 [M]).
+    out: optional (vals, idx[, tokens]) tensors to fill."""
+    _operands(x, w)
+    M = x.shape[0]
+    if out is None:
+        vals = torch.empty((M, k), dtype=torch.float32, device=x.device)
+        idx = torch.empty((M, k), dtype=torch.int32, device=x.device)
+        tokens = torch.empty((M,), dtype=torch.int32, device=x.device) if u is not None else None
+    else:
+        vals, idx = out[0], out[1]
+        tokens = out[2] if u is not None else None
+    for name, t, dt, shape in (("vals", vals, torch.float32, (M, k)), ("idx", idx, torch.int32, (M, k))):
+        _dev(t, name)
+        _same_device(name, t, x)
+        if t.dtype != dt or tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be {dt} {list(shape)}")
+    if u is not None:
+        _dev(u, "u")
+        _same_device("u", u, x)
+        if u.dtype != torch.float32 or tuple(u.shape) != (M,):
+            raise ValueError(f"u must be float32 [{M}]")
+        _dev(tokens, "tokens")
+        if tokens.dtype != torch.int32 or tuple(tokens.shape) != (M,):
+            raise ValueError(f"tokens must be int32 [{M}]")
+    need = gemv_topk_workspace_bytes(M, w, k)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    else:
+        _dev(workspace, "workspace")
+        _same_device("workspace", workspace, x)
+    with torch.cuda.device(x.device):
+        _check(lib().bq_gemv_topk(x.data_ptr(), _DTYPE[x.dtype], M, w.c, k, vals.data_ptr(), idx.data_ptr(),
+                                  u.data_ptr() if u is not None else None, temperature, top_p,
+                                  tokens.data_ptr() if tokens is not None else None, workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(), _stream(x.device)))
+    return (vals, idx) if u is None else (vals, idx, tokens)
 
 
 def prefill_workspace_bytes(M: int, w: BQWeight) -> int:

@@ -364,6 +364,68 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
     return BQ_OK;
 }
 
+size_t bq_gemv_topk_workspace_bytes(int64_t M, const bq_weight *w, int k)
+{
+    if (!w || M < 1 || M > 8 || w->N < 1 || w->K < 128 || w->K % 128 || k < 1 || k > 32)
+        return 0;
+    if (!gemv_rows_supported((int)M, w->fmt, w->N, w->K, k))
+        return 0;
+    return gemv_rows_workspace_bytes((int)M, w->fmt, w->N, w->K, k);
+}
+
+bq_status bq_gemv_topk(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, int k, float *vals,
+                       int32_t *idx, const float *u, float temperature, float top_p, int32_t *tokens,
+                       void *workspace, size_t ws_bytes, cudaStream_t stream)
+{
+    bq_status st = validate_weight(w);
+    if (st != BQ_OK)
+        return st;
+    if (!x || !vals || !idx)
+        return set_error(BQ_ERR_INVALID_ARG, "gemv_topk: x, vals or idx is NULL");
+    if (xt != BQ_F16 && xt != BQ_BF16)
+        return set_error(BQ_ERR_DTYPE, "gemv_topk: x must be BQ_F16 or BQ_BF16");
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(vals) & 3u) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+        return set_error(BQ_ERR_ALIGNMENT, "gemv_topk: x must be 16-byte aligned, vals and idx 4-byte aligned");
+    if (M < 1 || M > 8)
+        return set_error(BQ_ERR_SHAPE, "gemv_topk: M=%lld, need 1 <= M <= 8", (long long)M);
+    if (k < 1 || k > 32 || k > w->N)
+        return set_error(BQ_ERR_SHAPE, "gemv_topk: k=%d, need 1 <= k <= 32 and k <= N", k);
+    if (u) {
+        if (!tokens)
+            return set_error(BQ_ERR_INVALID_ARG, "gemv_topk: u given without tokens");
+        if ((reinterpret_cast<uintptr_t>(u) & 3u) || (reinterpret_cast<uintptr_t>(tokens) & 3u))
+            return set_error(BQ_ERR_ALIGNMENT, "gemv_topk: u and tokens must be 4-byte aligned");
+        if (!(temperature > 0.f) || !(temperature < 3.4e38f) || !(top_p > 0.f) || !(top_p <= 1.f))
+            return set_error(BQ_ERR_INVALID_ARG, "gemv_topk: need temperature > 0 (finite) and 0 < top_p <= 1");
+    }
+    if (!gemv_rows_supported((int)M, w->fmt, w->N, w->K, k))
+        return set_error(BQ_ERR_SHAPE,
+                         "gemv_topk: needs K a multiple of 1024 and the digit fragments and logits of a CTA in "
+                         "shared memory (K=%lld, N=%lld, M=%lld)",
+                         (long long)w->K, (long long)w->N, (long long)M);
+    const size_t need = gemv_rows_workspace_bytes((int)M, w->fmt, w->N, w->K, k);
+    if (!workspace || ws_bytes < need)
+        return set_error(BQ_ERR_WORKSPACE, "gemv_topk: workspace needs %zu bytes, got %zu", need,
+                         workspace ? ws_bytes : (size_t)0);
+    if (!aligned16(workspace))
+        return set_error(BQ_ERR_ALIGNMENT, "gemv_topk: workspace must be 16-byte aligned");
+    if (take_injected_launch_failure())
+        return set_error(BQ_ERR_CUDA, "%s: injected launch failure (test hook)", "gemv_topk");
+    unsigned int *status = device_status(&st);
+    if (!status)
+        return st;
+    GemvArgs a{x, (int)xt, (int)M, (int)w->fmt, w->N, w->K, w->words,
+               reinterpret_cast<const __half *>(w->scales), nullptr, (int)BQ_F32, workspace, ws_bytes, status,
+               pipeline_wait_ns()};
+    TopkArgs t{k, vals, idx, u, temperature, top_p, tokens};
+    unsigned launches = 0;
+    cudaError_t e = launch_gemv_topk(a, t, stream, &launches);
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "gemv_topk launch: %s", cudaGetErrorString(e));
+    note_launches(launches);
+    return BQ_OK;
+}
+
 size_t bq_gemm_prefill_workspace_bytes(int64_t M, const bq_weight *w)
 {
     if (!w || M < 1 || w->N < 1 || w->K < 128 || w->K % 128)

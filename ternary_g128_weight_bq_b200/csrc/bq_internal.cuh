@@ -68,9 +68,19 @@ size_t gemv_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, unsigned *launches);
 // integer tensor-core path, whole output rows per CTA (gemv_rows.cu): K a multiple of 1024 and
 // the digit fragments of all of K in shared memory
-bool gemv_rows_supported(int M, int fmt, int64_t N, int64_t K);
-size_t gemv_rows_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
+bool gemv_rows_supported(int M, int fmt, int64_t N, int64_t K, int topk_k = 0);
+size_t gemv_rows_workspace_bytes(int M, int fmt, int64_t N, int64_t K, int topk_k = 0);
 cudaError_t launch_gemv_rows(const GemvArgs &a, cudaStream_t s, unsigned *launches);
+// the same kernels selecting the k largest outputs of every token row (and drawing a token)
+struct TopkArgs {
+    int k;                    // 1 .. 32
+    float *vals;              // [M][k]
+    int *idx;                 // [M][k]
+    const float *u;           // [M] or null
+    float temperature, top_p;
+    int *tokens;              // [M] (with u)
+};
+cudaError_t launch_gemv_topk(const GemvArgs &a, const TopkArgs &t, cudaStream_t s, unsigned *launches);
 // Device address and size of the fixed scratch array of bq_gemv_noalloc on the current
 // device (gemv_rows.cu); resolved once per device.
 cudaError_t gemv_static_scratch(void **ptr, size_t *bytes);

@@ -47,6 +47,7 @@
 #include "bq_internal.cuh"
 #include "gemv_mma.cuh"
 #include "sm100_ptx.cuh"
+#include "topk.cuh"
 
 namespace bq {
 namespace {
@@ -69,19 +70,23 @@ template <int FMT> struct RCfg {
 };
 
 struct RLayout {
-    int frag, colf, cfix, red, ring, bars, total, stage_bytes, scale_off;
+    int frag, colf, cfix, red, lg, tks, tko, ring, bars, total, stage_bytes, scale_off;
 };
 
-// Shared-memory layout (host and device compute the same thing).
+// Shared-memory layout (host and device compute the same thing). topk adds the selection scratch
+// and its k output keys, lg_floats the CTA's logits [M][rows] (when they are kept on chip).
 template <int FMT, int CS>
-__host__ __device__ inline RLayout rows_layout(int G, int TB, int S)
+__host__ __device__ inline RLayout rows_layout(int G, int TB, int S, int lg_floats = 0, bool topk = false)
 {
     RLayout L;
     L.frag = 0;                                           // [CS][G][2][32][4] u32
     L.colf = CS * G * 1024;                               // [2 CS][G] f32
     L.cfix = L.colf + 2 * CS * G * 4;                     // [CS][G][8] s32
     L.red = L.cfix + CS * G * 32;                         // [2][8 groups][TB][CS][16 rows][2] f32
-    L.ring = (L.red + 2 * kGroupWarps * TB * CS * 32 * 4 + 1023) / 1024 * 1024;
+    L.lg = L.red + 2 * kGroupWarps * TB * CS * 32 * 4;    // top-k: [M][rows] f32
+    L.tks = (L.lg + 4 * lg_floats + 15) / 16 * 16;        // top-k: selection scratch
+    L.tko = L.tks + (topk ? (int)sizeof(topk::Smem) : 0);        // top-k: k output keys
+    L.ring = (L.tko + (topk ? 8 * topk::kMaxK : 0) + 1023) / 1024 * 1024;
     L.scale_off = TB * RCfg<FMT>::kTileBytes;             // scales [TB][16 rows][8] fp16 after the words
     L.stage_bytes = (L.scale_off + TB * 256 + 1023) / 1024 * 1024;
     L.bars = L.ring + S * L.stage_bytes;
@@ -101,7 +106,7 @@ struct Bars {
 template <int FMT, int CS, typename XT>
 __global__ void __launch_bounds__(256)
 gemv_rows_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint32_t *__restrict__ frag,
-                      float *__restrict__ colf, int *__restrict__ cfix)
+                      float *__restrict__ colf, int *__restrict__ cfix, unsigned int *__restrict__ topk_counter)
 {
     // the GEMV that reads these fragments may set itself up and stream its weights meanwhile
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -109,6 +114,8 @@ gemv_rows_prep_kernel(const XT *__restrict__ x, int M, int64_t K, uint32_t *__re
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int G = (int)(K / 128);
     const int item = (int)((blockIdx.x * 256 + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (topk_counter && blockIdx.x == 0 && threadIdx.x == 0)
+        *topk_counter = 0u;                      // the top-k ticket of the GEMV that follows
     if (item < G * M) {
         if (FMT == BQ_TERNARY_B3_G128)
             build_item_b3<CS, XT>(x, M, K, G, item, lane, frag, colf, cfix);
@@ -227,23 +234,94 @@ __device__ __forceinline__ void slice_tiles(const uint8_t *__restrict__ st, int 
     }
 }
 
+// Top-k mode: instead of y, the k largest logits of every token (keys as in topk.cuh). Each CTA
+// keeps its rows' logits in shared memory, selects their k largest and writes them to cand; the
+// last CTA to finish (a ticket on counter, which the prep kernel zeroes) selects the k largest of
+// all CTAs' candidates, writes vals / idx and, with u given, draws a token per row.
+struct TopkParams {
+    int k, lg_rows;                 // k <= 32; rows of the per-CTA logits buffer
+    float *lg_glob;                 // the logits buffers [grid][M][lg_rows] in the workspace, or null
+                                    // (kept in shared memory)
+    unsigned long long *cand;       // [grid][M][k]
+    unsigned int *counter;
+    float *vals;                    // [M][k]
+    int *idx;                       // [M][k]
+    const float *u;                 // [M] uniform numbers, or null (no draw)
+    float temp, top_p;
+    int *tokens;                    // [M]
+};
+
+// The end of a top-k call, run by the NT consumer threads once their tile-groups are done.
+template <int NT>
+__device__ void topk_tail(const TopkParams &tp, const float *lg, topk::Smem *sm, unsigned long long *out, int M,
+                          int64_t N, int t0, int t1, bool ok)
+{
+    const int tid = threadIdx.x;
+    const int64_t row0 = (int64_t)t0 * 16;
+    const int64_t rows_end = (int64_t)t1 * 16 < N ? (int64_t)t1 * 16 : N;
+    const int nrow = (int)(rows_end - row0);                       // this CTA's rows (>= 1)
+    const int kk = nrow < tp.k ? nrow : tp.k;
+    asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");          // every logit is in lg
+    for (int m = 0; m < M; m++) {
+        const float *lm = lg + m * tp.lg_rows;
+        topk::select<NT>([&](int i) { return topk::key_of(lm[i], (uint32_t)(row0 + i)); }, nrow, kk, sm, out, tid, 1);
+        if (tid < tp.k) {
+            // rows past the CTA's own (fewer than k) and aborted calls leave the lowest key
+            const unsigned long long key = ok && tid < kk ? out[tid] : 0ull;
+            tp.cand[((int64_t)blockIdx.x * M + m) * tp.k + tid] = key;
+        }
+    }
+    // ticket: the last CTA to arrive merges
+    asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+    if (tid == 0) {
+        __threadfence();
+        sm->last = atomicAdd(tp.counter, 1u) == gridDim.x - 1;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+    if (!sm->last)
+        return;
+    __threadfence();
+    const int n = (int)gridDim.x * tp.k;
+    for (int m = 0; m < M; m++) {
+        const unsigned long long *cm = tp.cand;
+        topk::select<NT>([&](int i) {
+            const int c = i / tp.k, j = i % tp.k;
+            return __ldcg(cm + ((int64_t)c * M + m) * tp.k + j);
+        }, n, tp.k, sm, out, tid, 1);
+        if (tid < tp.k) {
+            tp.vals[m * tp.k + tid] = topk::value_of(out[tid]);
+            tp.idx[m * tp.k + tid] = (int)topk::index_of(out[tid]);
+        }
+        if (tp.u && tid < 32) {
+            const int tok = topk::draw(out, tp.k, tp.temp, tp.top_p, tp.u[m], tid);
+            if (tid == 0)
+                tp.tokens[m] = tok;
+        }
+    }
+    if (tid == 0)
+        *tp.counter = 0u;
+}
+
 // WG warp groups of 8 consumer warps (WG = 2 only at one column set, for long streams): warp
 // w takes group w % 8 of every slice and tiles w / 8, w / 8 + WG, ... of the tile-group.
-template <int FMT, int CS, int WG>
+template <int FMT, int CS, int WG, bool TOPK>
 __global__ void __launch_bounds__((WG * kGroupWarps + 1) * 32, CS == 1 && WG == 1 ? 2 : 1)
 gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s, int M,
                  int64_t N, int64_t K, void *__restrict__ y, int yt, int T, int TB, int S,
                  const uint32_t *__restrict__ frag_g, const float *__restrict__ colf_g, const int *__restrict__ cfix_g,
-                 uint32_t one, unsigned int *dev_status, uint64_t wait_ns)
+                 uint32_t one, unsigned int *dev_status, uint64_t wait_ns, const TopkParams tp)
 {
     using SCH = Scheme<FMT, CS>;
     constexpr int kConsumers = WG * kGroupWarps;
     constexpr int kTileBytes = RCfg<FMT>::kTileBytes, kBoxes = RCfg<FMT>::kBoxes;
     const int G = (int)(K / 128), C = (int)(K / 1024);
-    const RLayout L = rows_layout<FMT, CS>(G, TB, S);
+    const RLayout L = rows_layout<FMT, CS>(G, TB, S, TOPK && !tp.lg_glob ? M * tp.lg_rows : 0, TOPK);
     extern __shared__ uint8_t smem_raw[];
     // align by an offset on the shared array itself, so every access stays a shared-memory one
     uint8_t *smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
+    float *const lgp = TOPK ? (tp.lg_glob ? tp.lg_glob + (int64_t)blockIdx.x * M * tp.lg_rows
+                                          : reinterpret_cast<float *>(smem + L.lg))
+                            : nullptr;
     uint32_t *frag_s = reinterpret_cast<uint32_t *>(smem + L.frag);
     float *colf_s = reinterpret_cast<float *>(smem + L.colf);
     int *cfix_s = reinterpret_cast<int *>(smem + L.cfix);
@@ -441,10 +519,17 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
                 const int j = o / (CS * 32), rem = o % (CS * 32);
                 const int tok = 2 * (rem >> 5) + (rem & 1), row = (rem & 31) >> 1;
                 const int64_t n = (int64_t)(tb + j) * 16 + row;
-                if (ok && tok < M && n < N)
+                if (TOPK) {
+                    if (tok < M)
+                        lgp[tok * tp.lg_rows + (tb - t0 + j) * 16 + row] = v;
+                } else if (ok && tok < M && n < N) {
                     store_y<float>(y, yt, (int64_t)tok * N + n, v);
+                }
             }
         }
+        if (TOPK)
+            topk_tail<kConsumers * 32>(tp, lgp, reinterpret_cast<topk::Smem *>(smem + L.tks),
+                      reinterpret_cast<unsigned long long *>(smem + L.tko), M, N, t0, t1, ok);
     }
     if (threadIdx.x == 0) {
         // the bulk copy this thread issued must have landed before the CTA exits
@@ -486,22 +571,28 @@ int sm_count_rows()
 
 struct RPlan {
     int CS, WG, TB, S, grid, T, smem;
+    int lg_rows;                                  // top-k: rows of the per-CTA logits buffer (0: plain GEMV)
+    bool lg_glob;                                 // top-k: logits in the workspace (too large for shared memory)
     size_t frag_bytes, colf_bytes, cfix_bytes;
+    size_t cand_bytes, counter_bytes;             // top-k: candidates [grid][M][k] u64, the ticket counter
+    size_t lg_bytes;                              // top-k with lg_glob: [grid][M][lg_rows] f32
 };
 
 template <int FMT, int CS>
-int rows_total(int G, int TB, int S) { return rows_layout<FMT, CS>(G, TB, S).total; }
+int rows_total(int G, int TB, int S, int lg) { return rows_layout<FMT, CS>(G, TB, S, lg < 0 ? 0 : lg, lg != 0).total; }
 
-int rows_total_rt(int fmt, int CS, int G, int TB, int S)
+// lg: the top-k logits kept in shared memory (> 0), top-k with them in the workspace (< 0), or a
+// plain GEMV (0)
+int rows_total_rt(int fmt, int CS, int G, int TB, int S, int lg)
 {
     if (fmt == BQ_TERNARY_B3_G128)
-        return CS == 1 ? rows_total<BQ_TERNARY_B3_G128, 1>(G, TB, S) : CS == 2 ? rows_total<BQ_TERNARY_B3_G128, 2>(G, TB, S)
-             : CS == 3 ? rows_total<BQ_TERNARY_B3_G128, 3>(G, TB, S) : rows_total<BQ_TERNARY_B3_G128, 4>(G, TB, S);
+        return CS == 1 ? rows_total<BQ_TERNARY_B3_G128, 1>(G, TB, S, lg) : CS == 2 ? rows_total<BQ_TERNARY_B3_G128, 2>(G, TB, S, lg)
+             : CS == 3 ? rows_total<BQ_TERNARY_B3_G128, 3>(G, TB, S, lg) : rows_total<BQ_TERNARY_B3_G128, 4>(G, TB, S, lg);
     if (fmt == BQ_BINARY_G128)
-        return CS == 1 ? rows_total<BQ_BINARY_G128, 1>(G, TB, S) : CS == 2 ? rows_total<BQ_BINARY_G128, 2>(G, TB, S)
-             : CS == 3 ? rows_total<BQ_BINARY_G128, 3>(G, TB, S) : rows_total<BQ_BINARY_G128, 4>(G, TB, S);
-    return CS == 1 ? rows_total<BQ_TERNARY_G128, 1>(G, TB, S) : CS == 2 ? rows_total<BQ_TERNARY_G128, 2>(G, TB, S)
-         : CS == 3 ? rows_total<BQ_TERNARY_G128, 3>(G, TB, S) : rows_total<BQ_TERNARY_G128, 4>(G, TB, S);
+        return CS == 1 ? rows_total<BQ_BINARY_G128, 1>(G, TB, S, lg) : CS == 2 ? rows_total<BQ_BINARY_G128, 2>(G, TB, S, lg)
+             : CS == 3 ? rows_total<BQ_BINARY_G128, 3>(G, TB, S, lg) : rows_total<BQ_BINARY_G128, 4>(G, TB, S, lg);
+    return CS == 1 ? rows_total<BQ_TERNARY_G128, 1>(G, TB, S, lg) : CS == 2 ? rows_total<BQ_TERNARY_G128, 2>(G, TB, S, lg)
+         : CS == 3 ? rows_total<BQ_TERNARY_G128, 3>(G, TB, S, lg) : rows_total<BQ_TERNARY_G128, 4>(G, TB, S, lg);
 }
 
 // Tiles per tile-group: as many as a CTA owns, up to 4 per warp group; two warp groups (16
@@ -510,15 +601,35 @@ int rows_total_rt(int fmt, int CS, int G, int TB, int S)
 // 16; 24 warps, at 80 registers a thread, 5% slower). Stages: as many as fit, preferring (with one warp group) a
 // footprint that lets two CTAs share an SM, so that the next call's CTA can become resident and
 // prefetch while this one runs; 0 stages if even three do not fit.
-RPlan rows_plan(int M, int fmt, int64_t N, int64_t K)
+// Top-k (topk_k > 0) adds the CTA's logits [M][per * 16] and the selection scratch to shared
+// memory, and the candidates and the ticket counter to the workspace.
+static RPlan rows_plan_lg(int M, int fmt, int64_t N, int64_t K, int topk_k, bool lg_glob);
+
+// Top-k keeps the CTA's logits in shared memory when that leaves at least four stages (or as many
+// as without them), else in the workspace, where they stay in L2 (at most 148 x 8 x 1680 x 4
+// bytes at the LM head); the selection then reads them from L2.
+RPlan rows_plan(int M, int fmt, int64_t N, int64_t K, int topk_k)
+{
+    if (topk_k <= 0)
+        return rows_plan_lg(M, fmt, N, K, 0, false);
+    const RPlan on_chip = rows_plan_lg(M, fmt, N, K, topk_k, false);
+    const RPlan in_ws = rows_plan_lg(M, fmt, N, K, topk_k, true);
+    const int want = in_ws.S < 4 ? in_ws.S : 4;
+    return on_chip.S >= 3 && on_chip.S >= want ? on_chip : in_ws;
+}
+
+static RPlan rows_plan_lg(int M, int fmt, int64_t N, int64_t K, int topk_k, bool lg_glob)
 {
     RPlan p{};
+    p.lg_glob = lg_glob;
     p.CS = (M * kColsPerTok + 7) / 8;
     const int G = (int)(K / 128);
     p.T = (int)((N + 15) / 16);
     const int sms = sm_count_rows();
     p.grid = p.T < sms ? p.T : sms;
     const int per = (p.T + p.grid - 1) / p.grid;
+    p.lg_rows = topk_k > 0 ? per * 16 : 0;
+    const int lg = topk_k > 0 ? (lg_glob ? -1 : M * p.lg_rows) : 0;
     p.WG = p.CS == 1 && per >= 2 * kWarpTiles ? 2 : 1;
     // as many tiles per tile-group as a warp group can take, the CTA's tiles spread evenly over
     // its tile-groups (9 tiles: 5 + 4, not 8 + 1), and fewer if three stages do not fit
@@ -528,13 +639,13 @@ RPlan rows_plan(int M, int fmt, int64_t N, int64_t K)
         p.S = 0;
         if (p.WG == 1)
             for (int s = kMaxStages; s >= 3; s--)
-                if (rows_total_rt(fmt, p.CS, G, p.TB, s) <= kSmemPair) {
+                if (rows_total_rt(fmt, p.CS, G, p.TB, s, lg) <= kSmemPair) {
                     p.S = s;
                     break;
                 }
         if (p.S < 4) {
             for (int s = kMaxStages; s >= 3; s--)
-                if (rows_total_rt(fmt, p.CS, G, p.TB, s) <= kSmemLimit) {
+                if (rows_total_rt(fmt, p.CS, G, p.TB, s, lg) <= kSmemLimit) {
                     p.S = s;
                     break;
                 }
@@ -542,16 +653,19 @@ RPlan rows_plan(int M, int fmt, int64_t N, int64_t K)
         if (p.S >= 3)
             break;
     }
-    p.smem = p.S ? rows_total_rt(fmt, p.CS, G, p.TB, p.S) : 0;
+    p.smem = p.S ? rows_total_rt(fmt, p.CS, G, p.TB, p.S, lg) : 0;
     auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
     p.frag_bytes = al((size_t)p.CS * G * 1024);
     p.colf_bytes = al((size_t)2 * p.CS * G * 4);
     p.cfix_bytes = al((size_t)p.CS * G * 32);
+    p.cand_bytes = topk_k > 0 ? al((size_t)p.grid * M * topk_k * 8) : 0;
+    p.counter_bytes = topk_k > 0 ? 256 : 0;
+    p.lg_bytes = topk_k > 0 && lg_glob ? al((size_t)p.grid * M * p.lg_rows * 4) : 0;
     return p;
 }
 
 template <int FMT, int CS, int WG, typename XT>
-cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s)
+cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s, const TopkParams *tk)
 {
     EncodeTiledFn enc = encode_fn_rows();
     if (!enc)
@@ -589,7 +703,7 @@ cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s)
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    auto kern = gemv_rows_kernel<FMT, CS, WG>;
+    auto kern = tk ? gemv_rows_kernel<FMT, CS, WG, true> : gemv_rows_kernel<FMT, CS, WG, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
@@ -597,6 +711,16 @@ cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s)
     uint32_t *frag = reinterpret_cast<uint32_t *>(ws);
     float *colf = reinterpret_cast<float *>(ws + pl.frag_bytes);
     int *cfix = reinterpret_cast<int *>(ws + pl.frag_bytes + pl.colf_bytes);
+    TopkParams tp{};
+    unsigned int *counter = nullptr;
+    if (tk) {
+        tp = *tk;
+        uint8_t *tw = ws + pl.frag_bytes + pl.colf_bytes + pl.cfix_bytes;
+        tp.cand = reinterpret_cast<unsigned long long *>(tw);
+        tp.counter = counter = reinterpret_cast<unsigned int *>(tw + pl.cand_bytes);
+        tp.lg_rows = pl.lg_rows;
+        tp.lg_glob = pl.lg_glob ? reinterpret_cast<float *>(tw + pl.cand_bytes + pl.counter_bytes) : nullptr;
+    }
     // programmatic dependent launches: each kernel may start before its predecessor in the
     // stream has finished, and waits for it (griddepcontrol.wait) before reading x or the
     // fragments, or writing anything
@@ -611,7 +735,7 @@ cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s)
     pcfg.attrs = attr;
     pcfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&pcfg, gemv_rows_prep_kernel<FMT, CS, XT>, static_cast<const XT *>(a.x), a.M, a.K, frag,
-                           colf, cfix);
+                           colf, cfix, counter);
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
@@ -622,17 +746,17 @@ cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, mw, ms, a.M, a.N, a.K, a.y, a.yt, pl.T, pl.TB, pl.S, (const uint32_t *)frag,
-                              (const float *)colf, (const int *)cfix, 1u, a.dev_status, a.wait_ns);
+                              (const float *)colf, (const int *)cfix, 1u, a.dev_status, a.wait_ns, tp);
 }
 
 template <int FMT, typename XT>
-cudaError_t launch_rows_cs(const GemvArgs &a, const RPlan &pl, cudaStream_t s)
+cudaError_t launch_rows_cs(const GemvArgs &a, const RPlan &pl, cudaStream_t s, const TopkParams *tk)
 {
     switch (pl.CS) {
-    case 1: return pl.WG == 2 ? launch_rows_t<FMT, 1, 2, XT>(a, pl, s) : launch_rows_t<FMT, 1, 1, XT>(a, pl, s);
-    case 2: return launch_rows_t<FMT, 2, 1, XT>(a, pl, s);
-    case 3: return launch_rows_t<FMT, 3, 1, XT>(a, pl, s);
-    default: return launch_rows_t<FMT, 4, 1, XT>(a, pl, s);
+    case 1: return pl.WG == 2 ? launch_rows_t<FMT, 1, 2, XT>(a, pl, s, tk) : launch_rows_t<FMT, 1, 1, XT>(a, pl, s, tk);
+    case 2: return launch_rows_t<FMT, 2, 1, XT>(a, pl, s, tk);
+    case 3: return launch_rows_t<FMT, 3, 1, XT>(a, pl, s, tk);
+    default: return launch_rows_t<FMT, 4, 1, XT>(a, pl, s, tk);
     }
 }
 
@@ -640,31 +764,51 @@ cudaError_t launch_rows_cs(const GemvArgs &a, const RPlan &pl, cudaStream_t s)
 
 // K a multiple of 1024 (whole 8-scale slices) and the digit fragments of all of K in shared
 // memory next to at least three stages.
-bool gemv_rows_supported(int M, int fmt, int64_t N, int64_t K)
+bool gemv_rows_supported(int M, int fmt, int64_t N, int64_t K, int topk_k)
 {
     if (M < 1 || M > 8 || K % 1024 != 0 || N < 1)
         return false;
-    return rows_plan(M, fmt, N, K).S >= 3;
+    return rows_plan(M, fmt, N, K, topk_k).S >= 3;
 }
 
-size_t gemv_rows_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
+size_t gemv_rows_workspace_bytes(int M, int fmt, int64_t N, int64_t K, int topk_k)
 {
-    const RPlan p = rows_plan(M, fmt, N, K);
-    return p.frag_bytes + p.colf_bytes + p.cfix_bytes;
+    const RPlan p = rows_plan(M, fmt, N, K, topk_k);
+    return p.frag_bytes + p.colf_bytes + p.cfix_bytes + p.cand_bytes + p.counter_bytes + p.lg_bytes;
+}
+
+// Plain GEMV (tk null) or the top-k GEMV.
+static cudaError_t launch_rows_any(const GemvArgs &a, cudaStream_t s, const TopkParams *tk)
+{
+    const RPlan pl = rows_plan(a.M, a.fmt, a.N, a.K, tk ? tk->k : 0);
+    if (a.fmt == BQ_BINARY_G128)
+        return a.xt == BQ_F16 ? launch_rows_cs<BQ_BINARY_G128, __half>(a, pl, s, tk)
+                              : launch_rows_cs<BQ_BINARY_G128, __nv_bfloat16>(a, pl, s, tk);
+    if (a.fmt == BQ_TERNARY_B3_G128)
+        return a.xt == BQ_F16 ? launch_rows_cs<BQ_TERNARY_B3_G128, __half>(a, pl, s, tk)
+                              : launch_rows_cs<BQ_TERNARY_B3_G128, __nv_bfloat16>(a, pl, s, tk);
+    return a.xt == BQ_F16 ? launch_rows_cs<BQ_TERNARY_G128, __half>(a, pl, s, tk)
+                          : launch_rows_cs<BQ_TERNARY_G128, __nv_bfloat16>(a, pl, s, tk);
 }
 
 cudaError_t launch_gemv_rows(const GemvArgs &a, cudaStream_t s, unsigned *launches)
 {
-    const RPlan pl = rows_plan(a.M, a.fmt, a.N, a.K);
     *launches = 2;                                        // digit prep + the GEMV
-    if (a.fmt == BQ_BINARY_G128)
-        return a.xt == BQ_F16 ? launch_rows_cs<BQ_BINARY_G128, __half>(a, pl, s)
-                              : launch_rows_cs<BQ_BINARY_G128, __nv_bfloat16>(a, pl, s);
-    if (a.fmt == BQ_TERNARY_B3_G128)
-        return a.xt == BQ_F16 ? launch_rows_cs<BQ_TERNARY_B3_G128, __half>(a, pl, s)
-                              : launch_rows_cs<BQ_TERNARY_B3_G128, __nv_bfloat16>(a, pl, s);
-    return a.xt == BQ_F16 ? launch_rows_cs<BQ_TERNARY_G128, __half>(a, pl, s)
-                          : launch_rows_cs<BQ_TERNARY_G128, __nv_bfloat16>(a, pl, s);
+    return launch_rows_any(a, s, nullptr);
+}
+
+cudaError_t launch_gemv_topk(const GemvArgs &a, const TopkArgs &t, cudaStream_t s, unsigned *launches)
+{
+    *launches = 2;                                        // digit prep + the GEMV with its selection
+    TopkParams tp{};
+    tp.k = t.k;
+    tp.vals = t.vals;
+    tp.idx = t.idx;
+    tp.u = t.u;
+    tp.temp = t.temperature;
+    tp.top_p = t.top_p;
+    tp.tokens = t.tokens;
+    return launch_rows_any(a, s, &tp);
 }
 
 // ---------------------------------------------------------------------------------------
