@@ -135,6 +135,9 @@ class Oracle:
         L.bqo_gemv_rows.restype = ctypes.c_int
         L.bqo_embed.argtypes = [ctypes.c_int, P, I64, P, P, I64, I64, P]
         L.bqo_embed.restype = I64
+        L.bqo_mlp_swiglu.argtypes = [ctypes.c_int, P, ctypes.c_int, I64, I64, P, P, P, P, I64, ctypes.c_int,
+                                     P, P, I64, P, P, P]
+        L.bqo_mlp_swiglu.restype = ctypes.c_int
         L.bqo_quantize_g128.argtypes = [ctypes.c_int, P, I64, I64, P, P]
         L.bqo_quantize_g128.restype = ctypes.c_int
         L.bqo_topk.argtypes = [P, I64, I64, ctypes.c_int, P, P]
@@ -216,6 +219,24 @@ class Oracle:
         out = np.zeros((len(i), K), dtype=np.float64)
         bad = self.L.bqo_embed(fmt, _p(i), len(i), _p(w), _p(s), w.shape[0], K, _p(out))
         return out, int(bad)
+
+    def mlp_swiglu(self, x, xt: int, fmt_gu: int, gate, up, fmt_d: int, down):
+        """(a [M, F], y [M, N], bound [M, N]) in fp64 for gate/up/down = (packed, scales) pairs,
+        gate and up [F, K], down [N, F]."""
+        xb = _bits16(x)
+        M, K = xb.shape
+        wg, sg = _weights(fmt_gu, gate[0]), _bits16(gate[1])
+        wu, su = _weights(fmt_gu, up[0]), _bits16(up[1])
+        wd, sd = _weights(fmt_d, down[0]), _bits16(down[1])
+        F, N = wg.shape[0], wd.shape[0]
+        a = np.zeros((M, F), dtype=np.float64)
+        y = np.zeros((M, N), dtype=np.float64)
+        b = np.zeros((M, N), dtype=np.float64)
+        st = self.L.bqo_mlp_swiglu(fmt_gu, _p(xb), xt, M, K, _p(wg), _p(sg), _p(wu), _p(su), F, fmt_d,
+                                   _p(wd), _p(sd), N, _p(a), _p(y), _p(b))
+        if st != OK:
+            raise ValueError(f"mlp status {st}")
+        return a, y, b
 
     def quantize(self, fmt: int, w):
         """Dense fp32 w [N, K] -> (q int8 [N, K], s fp16 bits uint16 [N, K/128]): the

@@ -524,6 +524,43 @@ int64_t bqo_sample_topk(const double *vals, const int64_t *idx, int k, double T,
 }
 
 /* ---------------------------------------------------------------------------------------
+ * SwiGLU MLP of a decode step. [card] "Model overview": the blocks use a SwiGLU MLP. For each
+ * token row m: g = x W_gate^T and u = x W_up^T (the product above, fp64, k ascending),
+ * a = silu(g) * u with silu(z) = z / (1 + e^(-z)), y = a W_down^T (fp64, j ascending). The bound
+ * of y[m, n] is 2e-3 * sum_j |a[m, j] * s_down[n, j / 128]|. a is returned too ([M, F]).
+ * ------------------------------------------------------------------------------------- */
+
+int bqo_mlp_swiglu(int fmt_gu, const uint16_t *x, int xt, int64_t M, int64_t K, const uint32_t *wg,
+                   const uint16_t *sg, const uint32_t *wu, const uint16_t *su, int64_t F, int fmt_d,
+                   const uint32_t *wd, const uint16_t *sd, int64_t N, double *a, double *y, double *bound)
+{
+    if (bqo_row_bytes(fmt_gu, K) < 0 || bqo_row_bytes(fmt_d, F) < 0 || M < 0 || N < 0)
+        return BQO_ERR_SHAPE;
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t f = 0; f < F; f++) {
+            double g = 0.0, u = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                const double xk = x_value(x, xt, m * K + k);
+                g += xk * bqo_weight(fmt_gu, wg, sg, K, f, k);
+                u += xk * bqo_weight(fmt_gu, wu, su, K, f, k);
+            }
+            a[m * F + f] = g / (1.0 + exp(-g)) * u;
+        }
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t j = 0; j < F; j++) {
+                double av = a[m * F + j];
+                acc += av * bqo_weight(fmt_d, wd, sd, F, n, j);
+                mag += fabs(av * bqo_f16_to_f64(sd[n * (F / 128) + j / 128]));
+            }
+            y[m * N + n] = acc;
+            bound[m * N + n] = 2e-3 * mag;
+        }
+    }
+    return BQO_OK;
+}
+
+/* ---------------------------------------------------------------------------------------
  * Dense -> g128 quantiser. The pages name the format but not how q and s are obtained ([card]
  * "Weight representation: Binary g128" points to a whitepaper that is not among them). The
  * reading taken: the least-squares fit of each group of 128 weights w,

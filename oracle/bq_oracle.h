@@ -45,6 +45,9 @@ int bqo_gemv_rows(int fmt, const uint16_t *x, int xt, int64_t M, int64_t K,
 int64_t bqo_embed(int fmt, const int32_t *ids, int64_t T, const uint32_t *words,
                   const uint16_t *scales, int64_t N, int64_t K, double *out);
 uint16_t bqo_mlx_affine_dequant(uint16_t s_f16, int q01);
+int bqo_mlp_swiglu(int fmt_gu, const uint16_t *x, int xt, int64_t M, int64_t K, const uint32_t *wg,
+                   const uint16_t *sg, const uint32_t *wu, const uint16_t *su, int64_t F, int fmt_d,
+                   const uint32_t *wd, const uint16_t *sd, int64_t N, double *a, double *y, double *bound);
 int bqo_quantize_g128(int fmt, const float *w, int64_t N, int64_t K, int8_t *q, uint16_t *s);
 int bqo_topk(const double *y, int64_t M, int64_t N, int k, int64_t *idx, double *vals);
 int64_t bqo_sample_topk(const double *vals, const int64_t *idx, int k, double T, double top_p, double u);

@@ -89,6 +89,13 @@ MUTANTS = {
         "s[n * (K / 128) + g] = bqo_f64_to_f16(sum / 128.0);", "s[n * (K / 128) + g] = bqo_f64_to_f16(sum / 127.0);"),
     "quantize_binary_zero_negative": (
         "qg[k] = wg[k] >= 0.0f ? 1 : -1;\n                    sum +=", "qg[k] = wg[k] > 0.0f ? 1 : -1;\n                    sum +="),
+    "mlp_silu_sign": (
+        "a[m * F + f] = g / (1.0 + exp(-g)) * u;", "a[m * F + f] = g / (1.0 + exp(g)) * u;"),
+    "mlp_gate_up_swapped": (
+        "a[m * F + f] = g / (1.0 + exp(-g)) * u;", "a[m * F + f] = u / (1.0 + exp(-u)) * g;"),
+    "mlp_bound_gate_scale": (
+        "mag += fabs(av * bqo_f16_to_f64(sd[n * (F / 128) + j / 128]));",
+        "mag += fabs(av * bqo_f16_to_f64(sg[(n % F) * (K / 128)]));"),
     "sum_skips_last_k": (
         "for (int64_t k = 0; k < K; k++) {\n                double xv",
         "for (int64_t k = 0; k < K - 1; k++) {\n                double xv"),

@@ -265,6 +265,67 @@ def pin_b3_bits_per_weight(o):
 
 
 # --------------------------------------------------------------------------------------
+# SwiGLU MLP (model card "Model overview")
+# --------------------------------------------------------------------------------------
+
+def _mlp_case(o, seed, M, K, F, N, fmt_gu=None):
+    fmt_gu = T if fmt_gu is None else fmt_gu
+    rng = np.random.default_rng(seed)
+    qg = synth.random_ternary(seed, 2, (F, K)).numpy() if fmt_gu == T else synth.random_signs(seed, 1, (F, K)).numpy()
+    qu = synth.random_ternary(seed, 3, (F, K)).numpy() if fmt_gu == T else synth.random_signs(seed, 4, (F, K)).numpy()
+    qd = synth.random_signs(seed, 5, (N, F)).numpy()
+    sg = (2.0 ** rng.integers(-4, 0, size=(F, K // 128))).astype(np.float16)
+    su = (2.0 ** rng.integers(-4, 0, size=(F, K // 128))).astype(np.float16)
+    sd = (2.0 ** rng.integers(-6, -2, size=(N, F // 128))).astype(np.float16)
+    x = _exact_x(M, K, seed + 1)
+    packs = [o.pack(fmt_gu, qg, sg), o.pack(fmt_gu, qu, su), o.pack(B, qd, sd)]
+    assert all(p[0] == oracle.OK for p in packs)
+    return x, (qg, sg), (qu, su), (qd, sd), [(p[1], p[2]) for p in packs]
+
+
+def pin_mlp_vs_numpy(o):
+    """Dense numpy fp64: W = q * s for the three matrices, g, u, a = g sigma(g) u, y = a Wd^T."""
+    for fmt_gu in (T, B):
+        x, g_, u_, d_, packed = _mlp_case(o, 41, 3, 256, 256, 200, fmt_gu)
+        a, y, b = o.mlp_swiglu(x, oracle.X_F16, fmt_gu, packed[0], packed[1], B, packed[2])
+        xs = x.astype(np.float64)
+        g = xs @ _dense(*g_).T
+        u = xs @ _dense(*u_).T
+        a_ref = g * (1.0 / (1.0 + np.exp(-g))) * u
+        assert np.allclose(a, a_ref, rtol=1e-12, atol=1e-300)
+        y_ref = a_ref @ _dense(*d_).T
+        assert np.allclose(y, y_ref, rtol=1e-9, atol=1e-12 * np.max(np.abs(y_ref)))
+        b_ref = 2e-3 * (np.abs(a_ref) @ np.abs(_dense(*d_)).T)
+        assert np.allclose(b, b_ref, rtol=1e-9)
+
+
+def pin_mlp_silu_identities(o):
+    """silu(z) - silu(-z) = z; silu(z) ~ z for large z and ~ 0 for large -z; zero up codes give
+    a = 0 and y = 0."""
+    K, F, N = 128, 128, 128
+    x = np.zeros((1, K), np.float16)
+    x[0, 0] = 1.0
+    qg = np.ones((F, K), np.int8)
+    qg[1::2] = -1                                    # gate row 2i+1 = -(gate row 2i)
+    sg = np.full((F, 1), 2.0, np.float16)
+    sg[4:6] = 32768.0                                # g = +-32768 for rows 4, 5
+    qu = np.ones((F, K), np.int8)                   # u = s_u = 1
+    su = np.ones((F, 1), np.float16)
+    qd = np.ones((N, F), np.int8)
+    sd = np.ones((N, 1), np.float16)
+    pg, pu, pd = o.pack(T, qg, sg), o.pack(T, qu, su), o.pack(B, qd, sd)
+    a, y, b = o.mlp_swiglu(x, oracle.X_F16, T, pg[1:], pu[1:], B, pd[1:])
+    for i in (0, 2, 6):
+        g = float(sg[i, 0])
+        assert abs((a[0, i] - a[0, i + 1]) - g) <= 1e-15 * g
+    assert abs(a[0, 4] - 32768.0) <= 1e-9 and abs(a[0, 5]) <= 1e-300
+    qz = np.zeros((F, K), np.int8)
+    pz = o.pack(T, qz, su)
+    a0, y0, _ = o.mlp_swiglu(x, oracle.X_F16, T, pg[1:], pz[1:], B, pd[1:])
+    assert np.all(a0 == 0) and np.all(y0 == 0)
+
+
+# --------------------------------------------------------------------------------------
 # Dense -> g128 quantiser (least-squares fit per group; the pages do not give the method)
 # --------------------------------------------------------------------------------------
 
@@ -608,6 +669,8 @@ def test_b3_examples(orc): pin_b3_examples(orc)
 def test_b3_byte_values(orc): pin_b3_byte_values(orc)
 def test_b3_equals_2bit(orc): pin_b3_equals_2bit(orc)
 def test_b3_bits_per_weight(orc): pin_b3_bits_per_weight(orc)
+def test_mlp_vs_numpy(orc): pin_mlp_vs_numpy(orc)
+def test_mlp_silu_identities(orc): pin_mlp_silu_identities(orc)
 def test_quantize_hand(orc): pin_quantize_hand(orc)
 def test_quantize_binary_closed_form(orc): pin_quantize_binary_closed_form(orc)
 def test_quantize_ternary_bruteforce(orc): pin_quantize_ternary_bruteforce(orc)
