@@ -379,6 +379,110 @@ def lm_head_topk_entry(bq, device, stream, peaks, ob, w, x, xd, oracle_timing):
     return ent
 
 
+def mlp_entry(bq, device, stream, peaks, ob):
+    """The SwiGLU MLP of one block at M = 1: gate and up 20480 x 5120 and down 5120 x 20480, binary
+    (the two MLP GEMVs of the full-depth step), as one fused call and as three GEMVs with SwiGLU
+    in torch between them. Weights of 8 blocks rotate (together above L2)."""
+    import numpy as np
+    o = ob.o
+    K, F, N, M = K_HEAD, 20480, K_HEAD, 1
+    copies = 8
+    blocks = []
+    for c in range(copies):
+        mk = lambda rows, cols, tid: bq.BQWeight(bq.BINARY_G128, rows, cols,
+                                                 synth.binary_words(100 * c + tid, rows, cols, device=device),
+                                                 synth.scales(100 * c + tid, rows, cols // 128, device=device))
+        blocks.append((mk(F, K, 1), mk(F, K, 2), mk(N, F, 3)))
+    x = synth.activations(0, M, K)
+    xd = x.to(device)
+    y = torch.empty((M, N), dtype=torch.float32, device=device)
+    ws = torch.empty(bq.mlp_swiglu_workspace_bytes(M, *blocks[0]), dtype=torch.uint8, device=device)
+    g = torch.cuda.CUDAGraph()
+    for b in blocks:
+        bq.mlp_swiglu(xd, *b, out=y, workspace=ws)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(2 * copies):
+            bq.mlp_swiglu(xd, *blocks[i % copies], out=y, workspace=ws)
+    ms = time_single(g.replay, 10, 3, stream) / (2 * copies)
+    del g
+    # separate: gate, up, SwiGLU (torch), down
+    gy = torch.empty((M, F), dtype=torch.float32, device=device)
+    uy = torch.empty((M, F), dtype=torch.float32, device=device)
+    act = torch.empty((M, F), dtype=torch.float32, device=device)
+    g2 = torch.cuda.CUDAGraph()
+    def sep(b):
+        bq.gemv(xd, b[0], out=gy)
+        bq.gemv(xd, b[1], out=uy)
+        torch.mul(torch.nn.functional.silu(gy), uy, out=act)
+        bq.gemv(act, b[2], out=y)
+    for b in blocks:
+        sep(b)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g2, stream=stream):
+        for i in range(2 * copies):
+            sep(blocks[i % copies])
+    ms_sep = time_single(g2.replay, 10, 3, stream) / (2 * copies)
+    del g2
+    bq.mlp_swiglu(xd, *blocks[0], out=y, workspace=ws)
+    torch.cuda.synchronize()
+    # parity: sampled rows of the first block against the oracle
+    b0 = blocks[0]
+    host = lambda w: (w.words.cpu().numpy().view(np.uint32), w.scales.cpu().numpy())
+    rows = np.arange(0, N, 40)
+    _, y_ref, bound = ob.orc.mlp_swiglu(x, o.X_BF16, o.BINARY, host(b0[0]), host(b0[1]), o.BINARY, host(b0[2]))
+    ratio = float(np.max(np.abs(y.cpu().numpy()[:, rows] - y_ref[:, rows]) / bound[:, rows]))
+    nbytes = 2 * gemv_bytes(F, K, M, 1) + gemv_bytes(N, F, M, 1)
+    gbs = nbytes / 1e9 / (ms / 1e3)
+    del blocks, ws
+    return {"workload": "SwiGLU MLP of one block, binary g128, M=1: gate and up 20480x5120 (one GEMV with the "
+                        "SwiGLU epilogue), down 5120x20480 on the fp32 activations",
+            "us": round(ms * 1e3, 2), "GBps": round(gbs, 1), "bound": "hbm",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"],
+            "separate_calls_us": round(ms_sep * 1e3, 2),
+            "timing": f"graphs of back-to-back calls rotating {copies} blocks ({copies * nbytes / 1e6:.0f} MB)",
+            "parity": {"max_err_over_bound": round(ratio, 5), "rows": int(len(rows))}}
+
+
+def quantize_entry(bq, device, stream, peaks, ob, fmt_name):
+    """Dense bf16 weights (N=20480, K=5120, 210 MB, above L2) to the packed format by the
+    least-squares fit of every group of 128; algorithmic bytes = dense read + packed and scales
+    written."""
+    import numpy as np
+    o = ob.o
+    N, K = 20480, K_HEAD
+    fmt = {"binary": bq.BINARY_G128, "ternary": bq.TERNARY_G128, "ternary_b3": bq.TERNARY_B3_G128}[fmt_name]
+    ofmt = {"binary": o.BINARY, "ternary": o.TERNARY, "ternary_b3": o.TERNARY_B3}[fmt_name]
+    wd = (synth.activations(5, N, K, dtype=torch.float32) * 0.02).to(torch.bfloat16).to(device)
+    pw = bq.quantize_g128(wd, fmt)
+    out_bytes = pw.words.numel() * pw.words.element_size() + pw.scales.numel() * 2
+    nbytes = N * K * 2 + out_bytes
+    ms = time_single(lambda: bq.quantize_g128(wd, fmt), 10, 3, stream)
+    gbs = nbytes / 1e9 / (ms / 1e3)
+    # parity: the first 64 rows against the oracle's fit, bit for bit (codes and scales)
+    rows = 64
+    w_host = wd[:rows].float().cpu().numpy()
+    q_ref, s_ref = ob.orc.quantize(o.TERNARY if ofmt == o.TERNARY_B3 else ofmt, w_host)
+    st, packed_ref, _ = ob.orc.pack(ofmt, q_ref, s_ref.view(np.float16))
+    got = pw.words[:rows].cpu().numpy()
+    if ofmt != o.TERNARY_B3:
+        got = got.view(np.uint32)
+    exact = bool(np.array_equal(got, packed_ref) and
+                 np.array_equal(pw.scales[:rows].cpu().view(torch.int16).numpy().view(np.uint16), s_ref))
+
+    def work(lo, hi):
+        ob.orc.quantize(o.TERNARY if ofmt == o.TERNARY_B3 else ofmt, w_host[lo:hi])
+    dt, n = ob.time_items(work, rows, ob.cores)
+    del wd, pw
+    return {"workload": f"dense bf16 -> {fmt_name} g128 quantiser (least-squares fit per group), N=20480, K=5120",
+            "us": round(ms * 1e3, 1), "GBps": round(gbs, 1), "bound": "hbm",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"],
+            "timing": "back-to-back calls on one 210 MB dense matrix (above L2)",
+            "parity": {"bit_exact_rows": rows, "bit_exact": exact},
+            "oracle": {"all_cores": {"GBps": round(n * (K * 2 + out_bytes / N) / 1e9 / dt, 4), "cores": ob.cores,
+                                     "sample": f"{n} rows of the 64-row slice, {dt:.3f} s"}}}
+
+
 def _rotating_gemv_ms(bq, mats, x, y, ws, stream, reps=20):
     """Device ms of one call over a CUDA graph of back-to-back calls that rotate through `mats`
     (weight copies together larger than L2)."""
@@ -551,6 +655,9 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
     # ---- config 5: binary prefill (M=512) and the full-depth decode step
     out.append(prefill_report(bq, device, stream, peaks, ob, "binary", l2))
     out.append(full_depth_step(bq, device, stream, peaks, ob))
+    out.append(mlp_entry(bq, device, stream, peaks, ob))
+    for fmt_name in ("binary", "ternary", "ternary_b3"):
+        out.append(quantize_entry(bq, device, stream, peaks, ob, fmt_name))
     torch.cuda.empty_cache()
     return out
 
@@ -961,7 +1068,7 @@ def run_case(args):
     stream = torch.cuda.Stream(device)
     N, M, K = args.N, args.M, args.K
     with torch.cuda.stream(stream):
-        if args.case in ("gemv", "prefill"):
+        if args.case in ("gemv", "prefill", "topk"):
             if args.fmt == "binary":
                 w = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(0, N, K, device=device),
                                 synth.scales(0, N, K // 128, device=device))
@@ -971,7 +1078,16 @@ def run_case(args):
                 w = pack(q, synth.scales(0, N, K // 128, device=device))
                 del q
             x = synth.activations(0, M, K).to(device)
-            if args.case == "gemv":
+            if args.case == "topk":
+                ws = torch.empty(bq.gemv_topk_workspace_bytes(M, w, 20), dtype=torch.uint8, device=device)
+                u = torch.full((M,), 0.37, dtype=torch.float32, device=device)
+                outs = (torch.empty((M, 20), dtype=torch.float32, device=device),
+                        torch.empty((M, 20), dtype=torch.int32, device=device),
+                        torch.empty((M,), dtype=torch.int32, device=device))
+                fn = lambda: bq.gemv_topk(x, w, k=20, u=u, workspace=ws, out=outs)
+                bits = {"binary": 1, "ternary": 2, "ternary_b3": 26 * 8 / 128}[args.fmt]
+                work = {"GBps": gemv_bytes(N, K, M, bits) / 1e9}
+            elif args.case == "gemv":
                 y = torch.empty((M, N), dtype=torch.float32, device=device)
                 ws = torch.empty(max(bq.gemv_workspace_bytes(M, w), 16), dtype=torch.uint8, device=device)
                 fn = lambda: bq.gemv(x, w, out=y, workspace=ws)
@@ -1007,7 +1123,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="total CPU time budget of --impl reference (split over warm-up and steps)")
-    ap.add_argument("--case", choices=["gemv", "prefill", "embed"],
+    ap.add_argument("--case", choices=["gemv", "prefill", "embed", "topk"],
                     help="time one workload alone (for profiling) instead of the benchmark")
     ap.add_argument("--fmt", choices=["binary", "ternary", "ternary_b3"], default="binary")
     ap.add_argument("--N", type=int, default=248320)

@@ -144,6 +144,25 @@ bq_status bq_pack_ternary_b3_g128(const int8_t *q, const uint16_t *s_in, int64_t
                                   uint8_t *bytes, uint16_t *s_out, cudaStream_t stream);
 
 /*
+ * Dense weights to a packed format: the least-squares fit of every group of 128 weights w,
+ * packed as the pack calls do. The pages give the formats but not how q and s are obtained
+ * (model card section "Weight representation: Binary g128" refers to a whitepaper that is not
+ * among them); this call takes
+ *   binary:  q = +1 where w >= 0, else -1; s = mean |w| (the best scale for those signs);
+ *   ternary (2-bit or base-3 storage): the q in {-1, 0, +1} and s minimising sum (w - s q)^2,
+ *            i.e. q = sign(w) on the j largest |w| (equal |w|: lower position first) with j
+ *            maximising (their sum)^2 / j (the smallest such j; none for a group of zeros),
+ *            and s their mean |w|;
+ * s rounded to fp16 (nearest even). Sums and scores are taken in fp64.
+ *   w       [N][K] dense, wt = BQ_F32, BQ_BF16 or BQ_F16 (infinities or NaNs give undefined codes)
+ *   packed  out: uint32 words [N][K/32] or [N][K/16], or bytes [N][26 K/128] (base-3)
+ *   scales  out: fp16 [N][K/128]
+ * Asynchronous on `stream` (one kernel); all pointers 16-byte aligned.
+ */
+bq_status bq_quantize_g128(const void *w, bq_dtype wt, int64_t N, int64_t K, bq_format fmt,
+                           void *packed, uint16_t *scales, cudaStream_t stream);
+
+/*
  * Inverse of the pack calls: q int8 [N][K] and, if s_out is not NULL, a copy of the
  * scales. SYNCHRONOUS. Returns BQ_ERR_INVALID_CODE if a ternary code 3, or an invalid base-3
  * byte, is found (the q of its codes is written as 0).
@@ -156,7 +175,7 @@ bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStr
  * Model card "prism-ml/Bonsai-27B-mlx-1bit", sections "Weight representation: Binary g128"
  * and "CUDA (NVIDIA GPUs)"; the decode (tg128) workload of section "Cross-platform
  * throughput".
- *   x          [M][K], xt = BQ_F16 or BQ_BF16. A token row that holds an infinity or a NaN
+ *   x          [M][K], xt = BQ_F16, BQ_BF16 or BQ_F32. A token row that holds an infinity or a NaN
  *              gets non-finite outputs (NaN where K is a multiple of 1024, where the kernels
  *              carry x as integer digits per group; +-inf or NaN otherwise).
  *   M          1..8
@@ -233,6 +252,30 @@ bq_status bq_gemv_topk(const void *x, bq_dtype xt, int64_t M, const bq_weight *w
 
 /* Workspace bytes bq_gemv_topk needs (0 if the shape or k is not supported). */
 size_t bq_gemv_topk_workspace_bytes(int64_t M, const bq_weight *w, int k);
+
+/*
+ * SwiGLU MLP of a decode step: y = (silu(x Wg^T) * (x Wu^T)) Wd^T with silu(z) = z / (1 + e^-z).
+ * Model card "prism-ml/Bonsai-27B-mlx-1bit", section "Model overview": the blocks use a SwiGLU
+ * MLP. The gate and up projections run as one GEMV over interleaved 16-row tiles of gate and up,
+ * whose epilogue writes the activations a = silu(g) * u (fp32, in the workspace) instead of g and
+ * u; the down GEMV then reads a as its x. Three kernel launches (the x prep, the gate/up GEMV,
+ * the down GEMV's prep and GEMV: four) chained by programmatic dependent launch.
+ *   x       [M][K], xt = BQ_F16, BQ_BF16 or BQ_F32; M 1..8
+ *   gate, up  the same format, N = F rows, K a multiple of 1024
+ *   down    N rows, K = F (any format)
+ *   y       [M][N], yt = BQ_F32, BQ_BF16 or BQ_F16
+ *   workspace  bq_mlp_swiglu_workspace_bytes(M, gate, up, down) bytes, 16-byte aligned: the x
+ *           fragments of the gate/up GEMV, a (M*F*4 bytes) and the down GEMV's workspace.
+ * Errors: as bq_gemv; BQ_ERR_SHAPE when the shapes do not chain or the gate/up projection does not
+ * fit the tensor-core path.
+ */
+bq_status bq_mlp_swiglu(const void *x, bq_dtype xt, int64_t M, const bq_weight *gate,
+                        const bq_weight *up, const bq_weight *down, void *y, bq_dtype yt,
+                        void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes bq_mlp_swiglu needs (0 if the shapes are not supported). */
+size_t bq_mlp_swiglu_workspace_bytes(int64_t M, const bq_weight *gate, const bq_weight *up,
+                                     const bq_weight *down);
 
 /*
  * Prefill GEMM: the same product for M up to 512 token rows (larger M is accepted),

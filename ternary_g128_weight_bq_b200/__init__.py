@@ -68,12 +68,15 @@ def lib() -> ctypes.CDLL:
             "bq_pack_binary_g128": ([P, P, I64, I64, P, P, P], I),
             "bq_pack_ternary_g128": ([P, P, I64, I64, P, P, P], I),
             "bq_pack_ternary_b3_g128": ([P, P, I64, I64, P, P, P], I),
+            "bq_quantize_g128": ([P, I, I64, I64, I, P, P, P], I),
             "bq_unpack_g128": ([W, P, P, P], I),
             "bq_gemv": ([P, I, I64, W, P, I, P, ctypes.c_size_t, P], I),
             "bq_gemv_workspace_bytes": ([I64, W], ctypes.c_size_t),
             "bq_gemv_noalloc": ([P, I, I64, W, P, I, P], I),
             "bq_gemv_topk": ([P, I, I64, W, I, P, P, P, ctypes.c_float, ctypes.c_float, P, P, ctypes.c_size_t, P], I),
             "bq_gemv_topk_workspace_bytes": ([I64, W, I], ctypes.c_size_t),
+            "bq_mlp_swiglu": ([P, I, I64, W, W, W, P, I, P, ctypes.c_size_t, P], I),
+            "bq_mlp_swiglu_workspace_bytes": ([I64, W, W, W], ctypes.c_size_t),
             "bq_gemm_prefill": ([P, I, I64, W, P, I, P, ctypes.c_size_t, P], I),
             "bq_gemm_prefill_workspace_bytes": ([I64, W], ctypes.c_size_t),
             "bq_embed_gather": ([P, I64, W, P, I, P], I),
@@ -224,6 +227,22 @@ def pack_ternary_b3_g128(q: torch.Tensor, s: torch.Tensor) -> BQWeight:
     return _pack(lib().bq_pack_ternary_b3_g128, TERNARY_B3_G128, q, s)
 
 
+def quantize_g128(w: torch.Tensor, fmt: int) -> BQWeight:
+    """Dense weights [N, K] (fp32, bf16 or fp16) to a packed matrix of format fmt: the
+    least-squares fit of every group of 128 (asynchronous on the current stream)."""
+    _dev(w, "w")
+    if w.dim() != 2 or w.dtype not in _DTYPE:
+        raise ValueError("w must be a 2-D fp32, bf16 or fp16 tensor")
+    N, K = w.shape
+    shape, dtype = _packed_shape(fmt, N, max(K, 128))
+    packed = torch.empty(shape, dtype=dtype, device=w.device)
+    scales = torch.empty((N, max(K // 128, 1)), dtype=torch.float16, device=w.device)
+    with torch.cuda.device(w.device):
+        _check(lib().bq_quantize_g128(w.data_ptr(), _DTYPE[w.dtype], N, K, fmt, packed.data_ptr(),
+                                      scales.data_ptr(), _stream(w.device)))
+    return BQWeight(fmt, N, K, packed, scales)
+
+
 def unpack_g128(w: BQWeight):
     """(q int8 [N, K], scales fp16 [N, K/128]) of a packed matrix (synchronous)."""
     q = torch.empty((w.N, w.K), dtype=torch.int8, device=w.words.device)
@@ -313,6 +332,29 @@ def gemv_topk(x: torch.Tensor, w: BQWeight, k: int = 20, u: torch.Tensor = None,
                                   tokens.data_ptr() if tokens is not None else None, workspace.data_ptr(),
                                   workspace.numel() * workspace.element_size(), _stream(x.device)))
     return (vals, idx) if u is None else (vals, idx, tokens)
+
+
+def mlp_swiglu_workspace_bytes(M: int, gate: BQWeight, up: BQWeight, down: BQWeight) -> int:
+    return int(lib().bq_mlp_swiglu_workspace_bytes(M, gate.c, up.c, down.c))
+
+
+def mlp_swiglu(x: torch.Tensor, gate: BQWeight, up: BQWeight, down: BQWeight, out_dtype=torch.float32,
+               out: torch.Tensor = None, workspace: torch.Tensor = None) -> torch.Tensor:
+    """y = (silu(x @ Wg^T) * (x @ Wu^T)) @ Wd^T for M <= 8 token rows (the gate/up GEMV writes the
+    SwiGLU activations, the down GEMV reads them)."""
+    _operands(x, gate)
+    for name, w in (("up", up), ("down", down)):
+        _same_device(f"{name} words", w.words, x)
+    M = x.shape[0]
+    out = _out(out, (M, down.N), out_dtype, x, down)
+    need = mlp_swiglu_workspace_bytes(M, gate, up, down)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(lib().bq_mlp_swiglu(x.data_ptr(), _DTYPE[x.dtype], M, gate.c, up.c, down.c, out.data_ptr(),
+                                   _DTYPE[out.dtype], workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(), _stream(x.device)))
+    return out
 
 
 def prefill_workspace_bytes(M: int, w: BQWeight) -> int:

@@ -236,6 +236,31 @@ bq_status bq_pack_ternary_b3_g128(const int8_t *q, const uint16_t *s_in, int64_t
     return pack_common(BQ_TERNARY_B3_G128, q, s_in, N, K, bytes, s_out, stream);
 }
 
+bq_status bq_quantize_g128(const void *w, bq_dtype wt, int64_t N, int64_t K, bq_format fmt, void *packed,
+                           uint16_t *scales, cudaStream_t stream)
+{
+    if (!w || !packed || !scales)
+        return set_error(BQ_ERR_INVALID_ARG, "quantize: NULL pointer");
+    if (fmt != BQ_BINARY_G128 && fmt != BQ_TERNARY_G128 && fmt != BQ_TERNARY_B3_G128)
+        return set_error(BQ_ERR_INVALID_ARG, "quantize: unknown format %d", (int)fmt);
+    if (wt != BQ_F32 && wt != BQ_BF16 && wt != BQ_F16)
+        return set_error(BQ_ERR_DTYPE, "quantize: w must be BQ_F32, BQ_BF16 or BQ_F16");
+    if (N < 1 || K < 128 || K % 128 || N > (int64_t(1) << 31) || K > (int64_t(1) << 24))
+        return set_error(BQ_ERR_SHAPE, "quantize: N=%lld K=%lld invalid", (long long)N, (long long)K);
+    if (!aligned16(w) || !aligned16(packed) || !aligned16(scales))
+        return set_error(BQ_ERR_ALIGNMENT, "quantize: w, packed and scales must be 16-byte aligned");
+    if (take_injected_launch_failure())
+        return set_error(BQ_ERR_CUDA, "%s: injected launch failure (test hook)", "quantize");
+    bq_status st;
+    if (!device_status(&st))
+        return st;
+    cudaError_t e = launch_quantize(fmt, w, wt, N, K, packed, scales, stream);
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "quantize launch: %s", cudaGetErrorString(e));
+    note_launches(1);
+    return BQ_OK;
+}
+
 bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStream_t stream)
 {
     bq_status st = validate_weight(w);
@@ -273,12 +298,14 @@ bq_status bq_unpack_g128(const bq_weight *w, int8_t *q, uint16_t *s_out, cudaStr
     return BQ_OK;
 }
 
-static bq_status validate_xy(const char *who, const void *x, bq_dtype xt, const void *y, bq_dtype yt)
+static bq_status validate_xy(const char *who, const void *x, bq_dtype xt, const void *y, bq_dtype yt,
+                             bool x_f32 = false)
 {
     if (!x || !y)
         return set_error(BQ_ERR_INVALID_ARG, "%s: x or y is NULL", who);
-    if (xt != BQ_F16 && xt != BQ_BF16)
-        return set_error(BQ_ERR_DTYPE, "%s: x must be BQ_F16 or BQ_BF16", who);
+    if (xt != BQ_F16 && xt != BQ_BF16 && !(x_f32 && xt == BQ_F32))
+        return set_error(BQ_ERR_DTYPE, x_f32 ? "%s: x must be BQ_F16, BQ_BF16 or BQ_F32" : "%s: x must be BQ_F16 or BQ_BF16",
+                         who);
     if (yt != BQ_F32 && yt != BQ_BF16 && yt != BQ_F16)
         return set_error(BQ_ERR_DTYPE, "%s: y must be BQ_F32, BQ_BF16 or BQ_F16", who);
     if (!aligned16(x) || !aligned16(y))
@@ -299,7 +326,7 @@ bq_status bq_gemv(const void *x, bq_dtype xt, int64_t M, const bq_weight *w, voi
     bq_status st = validate_weight(w);
     if (st != BQ_OK)
         return st;
-    if ((st = validate_xy("gemv", x, xt, y, yt)) != BQ_OK)
+    if ((st = validate_xy("gemv", x, xt, y, yt, true)) != BQ_OK)
         return st;
     if (M < 1 || M > 8)
         return set_error(BQ_ERR_SHAPE, "gemv: M=%lld, need 1 <= M <= 8", (long long)M);
@@ -331,7 +358,7 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
     bq_status st = validate_weight(w);
     if (st != BQ_OK)
         return st;
-    if ((st = validate_xy("gemv_noalloc", x, xt, y, yt)) != BQ_OK)
+    if ((st = validate_xy("gemv_noalloc", x, xt, y, yt, true)) != BQ_OK)
         return st;
     if (M < 1 || M > 8)
         return set_error(BQ_ERR_SHAPE, "gemv_noalloc: M=%lld, need 1 <= M <= 8", (long long)M);
@@ -382,8 +409,8 @@ bq_status bq_gemv_topk(const void *x, bq_dtype xt, int64_t M, const bq_weight *w
         return st;
     if (!x || !vals || !idx)
         return set_error(BQ_ERR_INVALID_ARG, "gemv_topk: x, vals or idx is NULL");
-    if (xt != BQ_F16 && xt != BQ_BF16)
-        return set_error(BQ_ERR_DTYPE, "gemv_topk: x must be BQ_F16 or BQ_BF16");
+    if (xt != BQ_F16 && xt != BQ_BF16 && xt != BQ_F32)
+        return set_error(BQ_ERR_DTYPE, "gemv_topk: x must be BQ_F16, BQ_BF16 or BQ_F32");
     if (!aligned16(x) || (reinterpret_cast<uintptr_t>(vals) & 3u) || (reinterpret_cast<uintptr_t>(idx) & 3u))
         return set_error(BQ_ERR_ALIGNMENT, "gemv_topk: x must be 16-byte aligned, vals and idx 4-byte aligned");
     if (M < 1 || M > 8)
@@ -423,6 +450,85 @@ bq_status bq_gemv_topk(const void *x, bq_dtype xt, int64_t M, const bq_weight *w
     if (e != cudaSuccess)
         return set_error(BQ_ERR_CUDA, "gemv_topk launch: %s", cudaGetErrorString(e));
     note_launches(launches);
+    return BQ_OK;
+}
+
+// the workspace of bq_mlp_swiglu: the gate/up GEMV's x fragments, the fp32 activations a [M][F],
+// the down GEMV's workspace (each part 256-byte aligned)
+static size_t mlp_parts(int64_t M, const bq_weight *gate, const bq_weight *down, size_t *ws1, size_t *abytes)
+{
+    auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
+    *ws1 = al(gemv_glu_workspace_bytes((int)M, gate->fmt, gate->N, gate->K));
+    *abytes = al((size_t)M * (size_t)gate->N * 4);
+    return *ws1 + *abytes + al(gemv_workspace_bytes((int)M, down->fmt, down->N, down->K));
+}
+
+static bq_status validate_mlp(int64_t M, const bq_weight *gate, const bq_weight *up, const bq_weight *down)
+{
+    bq_status st;
+    if ((st = validate_weight(gate)) != BQ_OK || (st = validate_weight(up)) != BQ_OK ||
+        (st = validate_weight(down)) != BQ_OK)
+        return st;
+    if (up->fmt != gate->fmt || up->N != gate->N || up->K != gate->K)
+        return set_error(BQ_ERR_SHAPE, "mlp_swiglu: gate and up must have the same format and shape");
+    if (down->K != gate->N)
+        return set_error(BQ_ERR_SHAPE, "mlp_swiglu: down has K=%lld, gate and up N=%lld", (long long)down->K,
+                         (long long)gate->N);
+    if (M < 1 || M > 8)
+        return set_error(BQ_ERR_SHAPE, "mlp_swiglu: M=%lld, need 1 <= M <= 8", (long long)M);
+    if (!gemv_glu_supported((int)M, gate->fmt, gate->N, gate->K))
+        return set_error(BQ_ERR_SHAPE, "mlp_swiglu: the gate/up projection needs K a multiple of 1024 and its x "
+                                       "fragments in shared memory (K=%lld, M=%lld)", (long long)gate->K, (long long)M);
+    return BQ_OK;
+}
+
+size_t bq_mlp_swiglu_workspace_bytes(int64_t M, const bq_weight *gate, const bq_weight *up, const bq_weight *down)
+{
+    if (!gate || !up || !down || M < 1 || M > 8 || gate->N < 1 || gate->K < 128 || gate->K % 128 || up->N != gate->N ||
+        up->K != gate->K || down->K != gate->N || down->N < 1)
+        return 0;
+    if (!gemv_glu_supported((int)M, gate->fmt, gate->N, gate->K))
+        return 0;
+    size_t a, b;
+    return mlp_parts(M, gate, down, &a, &b);
+}
+
+bq_status bq_mlp_swiglu(const void *x, bq_dtype xt, int64_t M, const bq_weight *gate, const bq_weight *up,
+                        const bq_weight *down, void *y, bq_dtype yt, void *workspace, size_t ws_bytes,
+                        cudaStream_t stream)
+{
+    bq_status st = validate_mlp(M, gate, up, down);
+    if (st != BQ_OK)
+        return st;
+    if ((st = validate_xy("mlp_swiglu", x, xt, y, yt, true)) != BQ_OK)
+        return st;
+    size_t ws1, abytes;
+    const size_t need = mlp_parts(M, gate, down, &ws1, &abytes);
+    if (!workspace || ws_bytes < need)
+        return set_error(BQ_ERR_WORKSPACE, "mlp_swiglu: workspace needs %zu bytes, got %zu", need,
+                         workspace ? ws_bytes : (size_t)0);
+    if (!aligned16(workspace))
+        return set_error(BQ_ERR_ALIGNMENT, "mlp_swiglu: workspace must be 16-byte aligned");
+    if (take_injected_launch_failure())
+        return set_error(BQ_ERR_CUDA, "%s: injected launch failure (test hook)", "mlp_swiglu");
+    unsigned int *status = device_status(&st);
+    if (!status)
+        return st;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *act = reinterpret_cast<float *>(ws + ws1);
+    GemvArgs a1{x, (int)xt, (int)M, (int)gate->fmt, gate->N, gate->K, gate->words,
+                reinterpret_cast<const __half *>(gate->scales), act, (int)BQ_F32, ws, ws1, status, pipeline_wait_ns()};
+    unsigned l1 = 0, l2 = 0;
+    cudaError_t e = launch_gemv_glu(a1, up->words, reinterpret_cast<const __half *>(up->scales), stream, &l1);
+    if (e == cudaSuccess) {
+        GemvArgs a2{act, (int)BQ_F32, (int)M, (int)down->fmt, down->N, down->K, down->words,
+                    reinterpret_cast<const __half *>(down->scales), y, (int)yt, ws + ws1 + abytes,
+                    ws_bytes - ws1 - abytes, status, pipeline_wait_ns()};
+        e = launch_gemv(a2, stream, &l2);
+    }
+    if (e != cudaSuccess)
+        return set_error(BQ_ERR_CUDA, "mlp_swiglu launch: %s", cudaGetErrorString(e));
+    note_launches(l1 + l2);
     return BQ_OK;
 }
 

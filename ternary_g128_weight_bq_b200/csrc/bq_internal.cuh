@@ -81,6 +81,12 @@ struct TopkArgs {
     int *tokens;              // [M] (with u)
 };
 cudaError_t launch_gemv_topk(const GemvArgs &a, const TopkArgs &t, cudaStream_t s, unsigned *launches);
+// the gate/up projection of a SwiGLU MLP: a.words / a.scales the gate rows, up_* the up rows (same
+// format and shape); y[m][n] = silu(gate) * up
+bool gemv_glu_supported(int M, int fmt, int64_t N, int64_t K);
+size_t gemv_glu_workspace_bytes(int M, int fmt, int64_t N, int64_t K);
+cudaError_t launch_gemv_glu(const GemvArgs &a, const uint32_t *up_words, const __half *up_scales, cudaStream_t s,
+                            unsigned *launches);
 // Device address and size of the fixed scratch array of bq_gemv_noalloc on the current
 // device (gemv_rows.cu); resolved once per device.
 cudaError_t gemv_static_scratch(void **ptr, size_t *bytes);
@@ -102,6 +108,10 @@ struct PrefillArgs {
 size_t prefill_workspace_bytes(int64_t M, int fmt, int64_t N, int64_t K);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s, unsigned *launches);
 
+// least-squares fit of every group of 128 dense weights, packed (quantize.cu)
+cudaError_t launch_quantize(int fmt, const void *w, int wt, int64_t N, int64_t K, void *packed, uint16_t *scales,
+                            cudaStream_t s);
+
 cudaError_t launch_embed(int fmt, const int32_t *ids, int64_t T, const uint32_t *words,
                          const __half *scales, int64_t N, int64_t K, void *out, int ot,
                          unsigned int *dev_status, cudaStream_t s);
@@ -119,5 +129,6 @@ __device__ __forceinline__ void store_out(__half *p, float v) { *p = __float2hal
 
 __device__ __forceinline__ float load_x(const __half *p) { return __half2float(*p); }
 __device__ __forceinline__ float load_x(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float load_x(const float *p) { return *p; }
 
 }  // namespace bq

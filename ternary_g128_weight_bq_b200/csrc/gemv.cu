@@ -186,16 +186,23 @@ cudaError_t launch_simt_m(const GemvArgs &a, cudaStream_t s)
 
 }  // namespace
 
+template <int FMT>
+cudaError_t launch_simt_x(const GemvArgs &a, cudaStream_t s)
+{
+    if (a.xt == BQ_F16)
+        return launch_simt_m<FMT, __half>(a, s);
+    if (a.xt == BQ_BF16)
+        return launch_simt_m<FMT, __nv_bfloat16>(a, s);
+    return launch_simt_m<FMT, float>(a, s);
+}
+
 cudaError_t launch_gemv_simt(const GemvArgs &a, cudaStream_t s)
 {
     if (a.fmt == BQ_BINARY_G128)
-        return a.xt == BQ_F16 ? launch_simt_m<BQ_BINARY_G128, __half>(a, s)
-                              : launch_simt_m<BQ_BINARY_G128, __nv_bfloat16>(a, s);
+        return launch_simt_x<BQ_BINARY_G128>(a, s);
     if (a.fmt == BQ_TERNARY_B3_G128)
-        return a.xt == BQ_F16 ? launch_simt_m<BQ_TERNARY_B3_G128, __half>(a, s)
-                              : launch_simt_m<BQ_TERNARY_B3_G128, __nv_bfloat16>(a, s);
-    return a.xt == BQ_F16 ? launch_simt_m<BQ_TERNARY_G128, __half>(a, s)
-                          : launch_simt_m<BQ_TERNARY_G128, __nv_bfloat16>(a, s);
+        return launch_simt_x<BQ_TERNARY_B3_G128>(a, s);
+    return launch_simt_x<BQ_TERNARY_G128>(a, s);
 }
 
 // Workspace of the tensor-core path (the digit fragments of x); the SIMT kernel needs none.

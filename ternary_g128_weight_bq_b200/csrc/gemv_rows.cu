@@ -254,7 +254,7 @@ struct TopkParams {
 // The end of a top-k call, run by the NT consumer threads once their tile-groups are done.
 template <int NT>
 __device__ void topk_tail(const TopkParams &tp, const float *lg, topk::Smem *sm, unsigned long long *out, int M,
-                          int64_t N, int t0, int t1, bool ok)
+                          int64_t N, int t0, int t1, bool ok, unsigned long long *stage, int stage_bytes)
 {
     const int tid = threadIdx.x;
     const int64_t row0 = (int64_t)t0 * 16;
@@ -282,9 +282,21 @@ __device__ void topk_tail(const TopkParams &tp, const float *lg, topk::Smem *sm,
         return;
     __threadfence();
     const int n = (int)gridDim.x * tp.k;
+    // the stage ring is idle now (every copy into it has been consumed): the candidates of a row go
+    // there once, so the selection's passes read shared memory instead of L2
+    const bool staged = n * 8 <= stage_bytes;
     for (int m = 0; m < M; m++) {
         const unsigned long long *cm = tp.cand;
+        if (staged) {
+            for (int i = tid; i < n; i += NT) {
+                const int c = i / tp.k, j = i % tp.k;
+                stage[i] = __ldcg(cm + ((int64_t)c * M + m) * tp.k + j);
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+        }
         topk::select<NT>([&](int i) {
+            if (staged)
+                return stage[i];
             const int c = i / tp.k, j = i % tp.k;
             return __ldcg(cm + ((int64_t)c * M + m) * tp.k + j);
         }, n, tp.k, sm, out, tid, 1);
@@ -302,15 +314,23 @@ __device__ void topk_tail(const TopkParams &tp, const float *lg, topk::Smem *sm,
         *tp.counter = 0u;
 }
 
+// Modes of the row kernel: the plain GEMV, the top-k selection, and the gate/up projection of a
+// SwiGLU MLP (GLU): logical tile 2i is gate rows 16i .. 16i+15 (tmap_w, tmap_s), tile 2i+1 the
+// same rows of up (tmap_w2, tmap_s2); CTAs and tile-groups hold whole pairs, and the epilogue
+// writes y[m][n] = silu(gate) * up with silu(z) = z / (1 + e^-z) (N = the gate rows).
+enum { kModePlain = 0, kModeTopk = 1, kModeGlu = 2 };
+
 // WG warp groups of 8 consumer warps (WG = 2 only at one column set, for long streams): warp
 // w takes group w % 8 of every slice and tiles w / 8, w / 8 + WG, ... of the tile-group.
-template <int FMT, int CS, int WG, bool TOPK>
+template <int FMT, int CS, int WG, int MODE>
 __global__ void __launch_bounds__((WG * kGroupWarps + 1) * 32, CS == 1 && WG == 1 ? 2 : 1)
-gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s, int M,
+gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
+                 const __grid_constant__ CUtensorMap tmap_w2, const __grid_constant__ CUtensorMap tmap_s2, int M,
                  int64_t N, int64_t K, void *__restrict__ y, int yt, int T, int TB, int S,
                  const uint32_t *__restrict__ frag_g, const float *__restrict__ colf_g, const int *__restrict__ cfix_g,
                  uint32_t one, unsigned int *dev_status, uint64_t wait_ns, const TopkParams tp)
 {
+    constexpr bool TOPK = MODE == kModeTopk, GLU = MODE == kModeGlu;
     using SCH = Scheme<FMT, CS>;
     constexpr int kConsumers = WG * kGroupWarps;
     constexpr int kTileBytes = RCfg<FMT>::kTileBytes, kBoxes = RCfg<FMT>::kBoxes;
@@ -332,7 +352,9 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
     unsigned int *err = dev_status + kSlotErrBits;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = (int)gridDim.x;
-    const int t0 = (int)((int64_t)blockIdx.x * T / P), t1 = (int)(((int64_t)blockIdx.x + 1) * T / P);
+    // whole tiles, or (GLU) whole gate/up pairs, per CTA
+    const int t0 = GLU ? 2 * (int)((int64_t)blockIdx.x * (T / 2) / P) : (int)((int64_t)blockIdx.x * T / P);
+    const int t1 = GLU ? 2 * (int)(((int64_t)blockIdx.x + 1) * (T / 2) / P) : (int)(((int64_t)blockIdx.x + 1) * T / P);
     const int ntg = (t1 - t0 + TB - 1) / TB;               // tile-groups of this CTA
 
     if (threadIdx.x == 0) {
@@ -354,6 +376,10 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
         if (lane == 0) {
             ptx::tma_prefetch_desc(&tmap_w);
             ptx::tma_prefetch_desc(&tmap_s);
+            if (GLU) {
+                ptx::tma_prefetch_desc(&tmap_w2);
+                ptx::tma_prefetch_desc(&tmap_s2);
+            }
             int s = 0, it = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -370,12 +396,15 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
                     uint8_t *st = ring + s * L.stage_bytes;
                     ptx::mbar_arrive_expect_tx(&bars->full[s], (uint32_t)(nt * (kTileBytes + 256)));
                     for (int j = 0; j < nt; j++) {
-                        const int32_t row = (tb + j) * 16;
+                        const bool up = GLU && ((tb + j) & 1);
+                        const int32_t row = (GLU ? (tb + j) >> 1 : tb + j) * 16;
+                        const CUtensorMap *mw = up ? &tmap_w2 : &tmap_w;
+                        const CUtensorMap *ms = up ? &tmap_s2 : &tmap_s;
 #pragma unroll
                         for (int h = 0; h < kBoxes; h++)
-                            ptx::tma_load_2d(st + j * kTileBytes + h * RCfg<FMT>::kBoxBytes, &tmap_w, &bars->full[s],
+                            ptx::tma_load_2d(st + j * kTileBytes + h * RCfg<FMT>::kBoxBytes, mw, &bars->full[s],
                                              (c * kBoxes + h) * RCfg<FMT>::kBoxInner, row);
-                        ptx::tma_load_2d(st + L.scale_off + j * 256, &tmap_s, &bars->full[s], c * 8, row);
+                        ptx::tma_load_2d(st + L.scale_off + j * 256, ms, &bars->full[s], c * 8, row);
                     }
                     if (++s == S) {
                         s = 0;
@@ -510,6 +539,24 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
                 }
             }
             asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
+            if (GLU) {
+                // pairs (gate tile 2 jp, up tile 2 jp + 1) of the tile-group
+                const int npo = (nt >> 1) * CS * 32;
+                for (int o = threadIdx.x; o < npo; o += kConsumers * 32) {
+                    const int jp = o / (CS * 32), rem = o % (CS * 32);
+                    float vg = 0.f, vu = 0.f;
+#pragma unroll
+                    for (int ww = 0; ww < kGroupWarps; ww++) {
+                        vg += rb[ww * TB * CS * 32 + (2 * jp) * CS * 32 + rem];
+                        vu += rb[ww * TB * CS * 32 + (2 * jp + 1) * CS * 32 + rem];
+                    }
+                    const int tok = 2 * (rem >> 5) + (rem & 1), row = (rem & 31) >> 1;
+                    const int64_t n = (int64_t)((tb >> 1) + jp) * 16 + row;
+                    if (ok && tok < M && n < N)
+                        store_y<float>(y, yt, (int64_t)tok * N + n, vg / (1.f + expf(-vg)) * vu);
+                }
+                continue;
+            }
             const int nout = nt * CS * 32;
             for (int o = threadIdx.x; o < nout; o += kConsumers * 32) {
                 float v = 0.f;
@@ -529,7 +576,8 @@ gemv_rows_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_consta
         }
         if (TOPK)
             topk_tail<kConsumers * 32>(tp, lgp, reinterpret_cast<topk::Smem *>(smem + L.tks),
-                      reinterpret_cast<unsigned long long *>(smem + L.tko), M, N, t0, t1, ok);
+                                       reinterpret_cast<unsigned long long *>(smem + L.tko), M, N, t0, t1, ok,
+                                       reinterpret_cast<unsigned long long *>(ring), S * L.stage_bytes);
     }
     if (threadIdx.x == 0) {
         // the bulk copy this thread issued must have landed before the CTA exits
@@ -603,7 +651,7 @@ int rows_total_rt(int fmt, int CS, int G, int TB, int S, int lg)
 // prefetch while this one runs; 0 stages if even three do not fit.
 // Top-k (topk_k > 0) adds the CTA's logits [M][per * 16] and the selection scratch to shared
 // memory, and the candidates and the ticket counter to the workspace.
-static RPlan rows_plan_lg(int M, int fmt, int64_t N, int64_t K, int topk_k, bool lg_glob);
+static RPlan rows_plan_lg(int M, int fmt, int64_t N, int64_t K, int topk_k, bool lg_glob, bool glu = false);
 
 // Top-k keeps the CTA's logits in shared memory when that leaves at least four stages (or as many
 // as without them), else in the workspace, where they stay in L2 (at most 148 x 8 x 1680 x 4
@@ -618,24 +666,33 @@ RPlan rows_plan(int M, int fmt, int64_t N, int64_t K, int topk_k)
     return on_chip.S >= 3 && on_chip.S >= want ? on_chip : in_ws;
 }
 
-static RPlan rows_plan_lg(int M, int fmt, int64_t N, int64_t K, int topk_k, bool lg_glob)
+// glu: N gate rows, 2 ceil(N / 16) logical tiles in gate/up pairs; CTAs and tile-groups take
+// whole pairs, so per and TB are even.
+static RPlan rows_plan_lg(int M, int fmt, int64_t N, int64_t K, int topk_k, bool lg_glob, bool glu)
 {
     RPlan p{};
     p.lg_glob = lg_glob;
     p.CS = (M * kColsPerTok + 7) / 8;
     const int G = (int)(K / 128);
-    p.T = (int)((N + 15) / 16);
+    const int units = (int)((N + 15) / 16);               // tiles, or gate/up pairs
+    p.T = glu ? 2 * units : units;
     const int sms = sm_count_rows();
-    p.grid = p.T < sms ? p.T : sms;
-    const int per = (p.T + p.grid - 1) / p.grid;
+    p.grid = units < sms ? units : sms;
+    const int per_units = (units + p.grid - 1) / p.grid;
+    const int per = glu ? 2 * per_units : per_units;
     p.lg_rows = topk_k > 0 ? per * 16 : 0;
     const int lg = topk_k > 0 ? (lg_glob ? -1 : M * p.lg_rows) : 0;
     p.WG = p.CS == 1 && per >= 2 * kWarpTiles ? 2 : 1;
     // as many tiles per tile-group as a warp group can take, the CTA's tiles spread evenly over
     // its tile-groups (9 tiles: 5 + 4, not 8 + 1), and fewer if three stages do not fit
-    for (int tbmax = kWarpTiles * p.WG; tbmax >= 1; tbmax--) {
-        const int ntg = (per + tbmax - 1) / tbmax;
-        p.TB = (per + ntg - 1) / ntg;
+    for (int tbmax = kWarpTiles * p.WG; tbmax >= (glu ? 2 : 1); tbmax -= glu ? 2 : 1) {
+        if (glu) {
+            const int ntg = (per_units + tbmax / 2 - 1) / (tbmax / 2);
+            p.TB = 2 * ((per_units + ntg - 1) / ntg);
+        } else {
+            const int ntg = (per + tbmax - 1) / tbmax;
+            p.TB = (per + ntg - 1) / ntg;
+        }
         p.S = 0;
         if (p.WG == 1)
             for (int s = kMaxStages; s >= 3; s--)
@@ -664,46 +721,68 @@ static RPlan rows_plan_lg(int M, int fmt, int64_t N, int64_t K, int topk_k, bool
     return p;
 }
 
-template <int FMT, int CS, int WG, typename XT>
-cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s, const TopkParams *tk)
+// The up matrix of a GLU launch (same format, shape and layout as a.words / a.scales).
+struct GluUp {
+    const uint32_t *words;
+    const __half *scales;
+};
+
+template <int FMT>
+CUresult encode_weight_maps(EncodeTiledFn enc, const uint32_t *words, const __half *scales, int64_t N, int64_t K,
+                            CUtensorMap *mw, CUtensorMap *ms)
 {
-    EncodeTiledFn enc = encode_fn_rows();
-    if (!enc)
-        return cudaErrorNotSupported;
-    const cuuint64_t G = (cuuint64_t)(a.K / 128);
-    CUtensorMap mw, ms;
+    const cuuint64_t G = (cuuint64_t)(K / 128);
     cuuint32_t est[2] = {1, 1};
     CUresult r;
     if (FMT == BQ_TERNARY_B3_G128) {
         // bytes [N][26 G]; a box is one 208-byte block (8 groups) of 16 rows, unswizzled: at a
         // 208-byte pitch the 8 rows a warp reads fall in distinct banks
         const cuuint64_t rb = (cuuint64_t)b3::kGroupBytes * G;
-        cuuint64_t wdims[2] = {rb, (cuuint64_t)a.N};
+        cuuint64_t wdims[2] = {rb, (cuuint64_t)N};
         cuuint64_t wstr[1] = {rb};
         cuuint32_t wbox[2] = {(cuuint32_t)b3::kBlockBytes, 16};
-        r = enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t *>(a.words), wdims, wstr, wbox, est,
+        r = enc(mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t *>(words), wdims, wstr, wbox, est,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
-        const cuuint64_t wpr = (cuuint64_t)(FMT == BQ_BINARY_G128 ? a.K / 32 : a.K / 16);
-        cuuint64_t wdims[2] = {wpr, (cuuint64_t)a.N};
+        const cuuint64_t wpr = (cuuint64_t)(FMT == BQ_BINARY_G128 ? K / 32 : K / 16);
+        cuuint64_t wdims[2] = {wpr, (cuuint64_t)N};
         cuuint64_t wstr[1] = {wpr * 4};
         cuuint32_t wbox[2] = {32, 16};                   // 128 bytes x 16 rows
-        r = enc(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(a.words), wdims, wstr, wbox, est,
+        r = enc(mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(words), wdims, wstr, wbox, est,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     }
     if (r != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
-    cuuint64_t sdims[2] = {G, (cuuint64_t)a.N};
+        return r;
+    cuuint64_t sdims[2] = {G, (cuuint64_t)N};
     cuuint64_t sstr[1] = {G * 2};
     cuuint32_t sbox[2] = {8, 16};                        // the 8 scales of a 1024-k slice x 16 rows
-    r = enc(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<__half *>(a.scales), sdims, sstr, sbox, est,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS)
+    return enc(ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<__half *>(scales), sdims, sstr, sbox, est,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+template <int FMT, int CS, int WG, typename XT>
+cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s, const TopkParams *tk,
+                          const GluUp *glu)
+{
+    EncodeTiledFn enc = encode_fn_rows();
+    if (!enc)
+        return cudaErrorNotSupported;
+    const cuuint64_t G = (cuuint64_t)(a.K / 128);
+    CUtensorMap mw, ms, mw2, ms2;
+    if (encode_weight_maps<FMT>(enc, a.words, a.scales, a.N, a.K, &mw, &ms) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    auto kern = tk ? gemv_rows_kernel<FMT, CS, WG, true> : gemv_rows_kernel<FMT, CS, WG, false>;
+    if (glu) {
+        if (encode_weight_maps<FMT>(enc, glu->words, glu->scales, a.N, a.K, &mw2, &ms2) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    } else {
+        mw2 = mw;
+        ms2 = ms;
+    }
+    auto kern = tk ? gemv_rows_kernel<FMT, CS, WG, kModeTopk>
+              : glu ? gemv_rows_kernel<FMT, CS, WG, kModeGlu> : gemv_rows_kernel<FMT, CS, WG, kModePlain>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess)
         return e;
@@ -745,18 +824,21 @@ cudaError_t launch_rows_t(const GemvArgs &a, const RPlan &pl, cudaStream_t s, co
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mw, ms, a.M, a.N, a.K, a.y, a.yt, pl.T, pl.TB, pl.S, (const uint32_t *)frag,
-                              (const float *)colf, (const int *)cfix, 1u, a.dev_status, a.wait_ns, tp);
+    return cudaLaunchKernelEx(&cfg, kern, mw, ms, mw2, ms2, a.M, a.N, a.K, a.y, a.yt, pl.T, pl.TB, pl.S,
+                              (const uint32_t *)frag, (const float *)colf, (const int *)cfix, 1u, a.dev_status,
+                              a.wait_ns, tp);
 }
 
 template <int FMT, typename XT>
-cudaError_t launch_rows_cs(const GemvArgs &a, const RPlan &pl, cudaStream_t s, const TopkParams *tk)
+cudaError_t launch_rows_cs(const GemvArgs &a, const RPlan &pl, cudaStream_t s, const TopkParams *tk,
+                           const GluUp *glu)
 {
     switch (pl.CS) {
-    case 1: return pl.WG == 2 ? launch_rows_t<FMT, 1, 2, XT>(a, pl, s, tk) : launch_rows_t<FMT, 1, 1, XT>(a, pl, s, tk);
-    case 2: return launch_rows_t<FMT, 2, 1, XT>(a, pl, s, tk);
-    case 3: return launch_rows_t<FMT, 3, 1, XT>(a, pl, s, tk);
-    default: return launch_rows_t<FMT, 4, 1, XT>(a, pl, s, tk);
+    case 1:
+        return pl.WG == 2 ? launch_rows_t<FMT, 1, 2, XT>(a, pl, s, tk, glu) : launch_rows_t<FMT, 1, 1, XT>(a, pl, s, tk, glu);
+    case 2: return launch_rows_t<FMT, 2, 1, XT>(a, pl, s, tk, glu);
+    case 3: return launch_rows_t<FMT, 3, 1, XT>(a, pl, s, tk, glu);
+    default: return launch_rows_t<FMT, 4, 1, XT>(a, pl, s, tk, glu);
     }
 }
 
@@ -777,18 +859,47 @@ size_t gemv_rows_workspace_bytes(int M, int fmt, int64_t N, int64_t K, int topk_
     return p.frag_bytes + p.colf_bytes + p.cfix_bytes + p.cand_bytes + p.counter_bytes + p.lg_bytes;
 }
 
-// Plain GEMV (tk null) or the top-k GEMV.
-static cudaError_t launch_rows_any(const GemvArgs &a, cudaStream_t s, const TopkParams *tk)
+template <int FMT>
+static cudaError_t launch_rows_x(const GemvArgs &a, const RPlan &pl, cudaStream_t s, const TopkParams *tk,
+                                 const GluUp *glu)
 {
-    const RPlan pl = rows_plan(a.M, a.fmt, a.N, a.K, tk ? tk->k : 0);
+    if (a.xt == BQ_F16)
+        return launch_rows_cs<FMT, __half>(a, pl, s, tk, glu);
+    if (a.xt == BQ_BF16)
+        return launch_rows_cs<FMT, __nv_bfloat16>(a, pl, s, tk, glu);
+    return launch_rows_cs<FMT, float>(a, pl, s, tk, glu);
+}
+
+// Plain GEMV (tk, glu null), the top-k GEMV, or the gate/up projection with SwiGLU.
+static cudaError_t launch_rows_any(const GemvArgs &a, cudaStream_t s, const TopkParams *tk, const GluUp *glu = nullptr)
+{
+    const RPlan pl = glu ? rows_plan_lg(a.M, a.fmt, a.N, a.K, 0, false, true) : rows_plan(a.M, a.fmt, a.N, a.K, tk ? tk->k : 0);
     if (a.fmt == BQ_BINARY_G128)
-        return a.xt == BQ_F16 ? launch_rows_cs<BQ_BINARY_G128, __half>(a, pl, s, tk)
-                              : launch_rows_cs<BQ_BINARY_G128, __nv_bfloat16>(a, pl, s, tk);
+        return launch_rows_x<BQ_BINARY_G128>(a, pl, s, tk, glu);
     if (a.fmt == BQ_TERNARY_B3_G128)
-        return a.xt == BQ_F16 ? launch_rows_cs<BQ_TERNARY_B3_G128, __half>(a, pl, s, tk)
-                              : launch_rows_cs<BQ_TERNARY_B3_G128, __nv_bfloat16>(a, pl, s, tk);
-    return a.xt == BQ_F16 ? launch_rows_cs<BQ_TERNARY_G128, __half>(a, pl, s, tk)
-                          : launch_rows_cs<BQ_TERNARY_G128, __nv_bfloat16>(a, pl, s, tk);
+        return launch_rows_x<BQ_TERNARY_B3_G128>(a, pl, s, tk, glu);
+    return launch_rows_x<BQ_TERNARY_G128>(a, pl, s, tk, glu);
+}
+
+bool gemv_glu_supported(int M, int fmt, int64_t N, int64_t K)
+{
+    if (M < 1 || M > 8 || K % 1024 != 0 || N < 1)
+        return false;
+    return rows_plan_lg(M, fmt, N, K, 0, false, true).S >= 3;
+}
+
+size_t gemv_glu_workspace_bytes(int M, int fmt, int64_t N, int64_t K)
+{
+    const RPlan p = rows_plan_lg(M, fmt, N, K, 0, false, true);
+    return p.frag_bytes + p.colf_bytes + p.cfix_bytes;
+}
+
+cudaError_t launch_gemv_glu(const GemvArgs &a, const uint32_t *up_words, const __half *up_scales, cudaStream_t s,
+                            unsigned *launches)
+{
+    *launches = 2;                                        // digit prep + the gate/up GEMV with SwiGLU
+    const GluUp up{up_words, up_scales};
+    return launch_rows_any(a, s, nullptr, &up);
 }
 
 cudaError_t launch_gemv_rows(const GemvArgs &a, cudaStream_t s, unsigned *launches)

@@ -77,10 +77,18 @@ __device__ void select(KeyAt key_at, int n, int k, Smem *sm, unsigned long long 
             sm->hist[b] = 0u;
         bar<NT>(id);
         const int shift = 56 - plen;
-        for (int i = tid; i < n; i += NT) {
-            const unsigned long long key = key_at(i);
-            if (plen == 0 || (key >> (64 - plen)) == (prefix >> (64 - plen)))
-                atomicAdd(&sm->hist[(key >> shift) & 255u], 1u);
+        // logits crowd into a few bins: the lanes of a warp that hit the same bin add once
+        for (int i0 = tid - lane; i0 < n; i0 += NT) {
+            const int i = i0 + lane;
+            int bin = -1;
+            if (i < n) {
+                const unsigned long long key = key_at(i);
+                if (plen == 0 || (key >> (64 - plen)) == (prefix >> (64 - plen)))
+                    bin = (int)((key >> shift) & 255u);
+            }
+            const unsigned same = __match_any_sync(0xffffffffu, bin);
+            if (bin >= 0 && lane == __ffs(same) - 1)
+                atomicAdd(&sm->hist[bin], (uint32_t)__popc(same));
         }
         bar<NT>(id);
         if (tid < 32) {

@@ -79,8 +79,9 @@ def test_validation_before_any_cuda_call(libbq):
     # misaligned words / x
     assert libbq.bq_gemv(16, 1, 1, W(_weight(words=20)), 16, 2, None, 0, None) == 3
     assert libbq.bq_gemv(18, 1, 1, W(_weight()), 16, 2, None, 0, None) == 3
-    # dtypes
-    assert libbq.bq_gemv(16, 2, 1, W(_weight()), 16, 2, None, 0, None) == 4
+    # dtypes (fp32 x is accepted by the GEMV, not by the prefill)
+    assert libbq.bq_gemv(16, 5, 1, W(_weight()), 16, 2, None, 0, None) == 4
+    assert libbq.bq_gemm_prefill(16, 2, 1, W(_weight()), 16, 2, None, 0, None) == 4
     assert libbq.bq_gemv(16, 1, 1, W(_weight()), 16, 9, None, 0, None) == 4
     # M range
     assert libbq.bq_gemv(16, 1, 0, W(_weight()), 16, 2, None, 0, None) == 2
