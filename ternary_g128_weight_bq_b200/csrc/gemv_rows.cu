@@ -242,7 +242,7 @@ struct TopkParams {
     int k, lg_rows;                 // k <= 32; rows of the per-CTA logits buffer
     float *lg_glob;                 // the logits buffers [grid][M][lg_rows] in the workspace, or null
                                     // (kept in shared memory)
-    unsigned long long *cand;       // [grid][M][k]
+    unsigned long long *cand;       // [grid][M][k], then the k-th key of each [grid][M]
     unsigned int *counter;
     float *vals;                    // [M][k]
     int *idx;                       // [M][k]
@@ -269,6 +269,8 @@ __device__ void topk_tail(const TopkParams &tp, const float *lg, topk::Smem *sm,
             // rows past the CTA's own (fewer than k) and aborted calls leave the lowest key
             const unsigned long long key = ok && tid < kk ? out[tid] : 0ull;
             tp.cand[((int64_t)blockIdx.x * M + m) * tp.k + tid] = key;
+            if (tid == tp.k - 1)        // this CTA's k-th key: the k largest overall are all >= it
+                tp.cand[(int64_t)gridDim.x * M * tp.k + (int64_t)blockIdx.x * M + m] = key;
         }
     }
     // ticket: the last CTA to arrive merges
@@ -276,30 +278,73 @@ __device__ void topk_tail(const TopkParams &tp, const float *lg, topk::Smem *sm,
     if (tid == 0) {
         __threadfence();
         sm->last = atomicAdd(tp.counter, 1u) == gridDim.x - 1;
+        for (int m = 0; m < 8; m++)
+            sm->floor[m] = 0ull;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
     if (!sm->last)
         return;
     __threadfence();
     const int n = (int)gridDim.x * tp.k;
-    // the stage ring is idle now (every copy into it has been consumed): the candidates of a row go
-    // there once, so the selection's passes read shared memory instead of L2
+    // The stage ring is idle now (every copy into it has been consumed): the candidates of a row go
+    // there once. The k largest overall are all at or above the largest of the CTAs' k-th keys, so
+    // only the candidates at or above that floor (usually a few more than k) need ranking.
     const bool staged = n * 8 <= stage_bytes;
     for (int m = 0; m < M; m++) {
         const unsigned long long *cm = tp.cand;
-        if (staged) {
+        const unsigned long long *kth = tp.cand + (int64_t)gridDim.x * M * tp.k;
+        unsigned long long lo = 0ull;
+        for (int c = tid; c < (int)gridDim.x; c += NT) {
+            const unsigned long long v = __ldcg(kth + (int64_t)c * M + m);
+            lo = v > lo ? v : lo;
+        }
+        if (staged)
             for (int i = tid; i < n; i += NT) {
-                const int c = i / tp.k, j = i % tp.k;
+                const int c = i / tp.k, j = i - c * tp.k;
                 stage[i] = __ldcg(cm + ((int64_t)c * M + m) * tp.k + j);
             }
-            asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, lo, d);
+            lo = o > lo ? o : lo;
         }
-        topk::select<NT>([&](int i) {
+        if ((tid & 31) == 0)
+            atomicMax(&sm->floor[m], lo);
+        if (tid == 0)
+            sm->cnt = 0;
+        asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+        lo = sm->floor[m];
+        auto key_at = [&](int i) {
             if (staged)
                 return stage[i];
-            const int c = i / tp.k, j = i % tp.k;
+            const int c = i / tp.k, j = i - c * tp.k;
             return __ldcg(cm + ((int64_t)c * M + m) * tp.k + j);
-        }, n, tp.k, sm, out, tid, 1);
+        };
+        for (int i = tid; i < n; i += NT) {
+            const unsigned long long key = key_at(i);
+            if (key >= lo) {
+                const int slot = atomicAdd(&sm->cnt, 1);
+                if (slot < topk::kGather)
+                    sm->buf[slot] = key;
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+        const int cnt = sm->cnt;
+        if (cnt <= topk::kGather) {
+            // rank = the number of larger keys (keys are unique)
+            if (tid < cnt) {
+                const unsigned long long a = sm->buf[tid];
+                int r = 0;
+                for (int j = 0; j < cnt; j++)
+                    r += sm->buf[j] > a;
+                if (r < tp.k)
+                    out[r] = a;
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+        } else {
+            // many candidates tie near the floor: the radix selection over all of them
+            topk::select<NT>(key_at, n, tp.k, sm, out, tid, 1);
+        }
         if (tid < tp.k) {
             tp.vals[m * tp.k + tid] = topk::value_of(out[tid]);
             tp.idx[m * tp.k + tid] = (int)topk::index_of(out[tid]);
@@ -653,17 +698,16 @@ int rows_total_rt(int fmt, int CS, int G, int TB, int S, int lg)
 // memory, and the candidates and the ticket counter to the workspace.
 static RPlan rows_plan_lg(int M, int fmt, int64_t N, int64_t K, int topk_k, bool lg_glob, bool glu = false);
 
-// Top-k keeps the CTA's logits in shared memory when that leaves at least four stages (or as many
-// as without them), else in the workspace, where they stay in L2 (at most 148 x 8 x 1680 x 4
-// bytes at the LM head); the selection then reads them from L2.
+// Top-k keeps the CTA's logits in shared memory when that costs no pipeline stage, else in the
+// workspace, where they stay in L2 (at most 148 x 8 x 1680 x 4 bytes at the LM head); the
+// selection then reads them from L2.
 RPlan rows_plan(int M, int fmt, int64_t N, int64_t K, int topk_k)
 {
     if (topk_k <= 0)
         return rows_plan_lg(M, fmt, N, K, 0, false);
     const RPlan on_chip = rows_plan_lg(M, fmt, N, K, topk_k, false);
     const RPlan in_ws = rows_plan_lg(M, fmt, N, K, topk_k, true);
-    const int want = in_ws.S < 4 ? in_ws.S : 4;
-    return on_chip.S >= 3 && on_chip.S >= want ? on_chip : in_ws;
+    return on_chip.S >= 3 && on_chip.S >= in_ws.S ? on_chip : in_ws;
 }
 
 // glu: N gate rows, 2 ceil(N / 16) logical tiles in gate/up pairs; CTAs and tile-groups take
@@ -715,7 +759,7 @@ static RPlan rows_plan_lg(int M, int fmt, int64_t N, int64_t K, int topk_k, bool
     p.frag_bytes = al((size_t)p.CS * G * 1024);
     p.colf_bytes = al((size_t)2 * p.CS * G * 4);
     p.cfix_bytes = al((size_t)p.CS * G * 32);
-    p.cand_bytes = topk_k > 0 ? al((size_t)p.grid * M * topk_k * 8) : 0;
+    p.cand_bytes = topk_k > 0 ? al((size_t)p.grid * M * (topk_k + 1) * 8) : 0;
     p.counter_bytes = topk_k > 0 ? 256 : 0;
     p.lg_bytes = topk_k > 0 && lg_glob ? al((size_t)p.grid * M * p.lg_rows * 4) : 0;
     return p;

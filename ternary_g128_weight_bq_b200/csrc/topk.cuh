@@ -12,7 +12,7 @@
 // bits of the keys that share the prefix chosen so far; one warp finds the bin where the count
 // from the top reaches the number of keys still missing and extends the prefix with it. Once the
 // keys at or above the bottom of that bin are at most 64 (usually after one or two passes for
-// logits), they are gathered and one warp ranks them by comparing every pair.
+// logits), they are gathered and ranked, one thread per key counting the larger ones.
 #pragma once
 
 #include <stdint.h>
@@ -32,6 +32,7 @@ struct Smem {
     int gather;                   // 1: gather keys >= prefix now
     int cnt;                      // gathered keys
     int last;                     // this CTA drew the last ticket
+    unsigned long long floor[8];  // the merge's floor per token row: the largest of the CTAs' k-th keys
 };
 
 __device__ __forceinline__ unsigned long long key_of(float v, uint32_t index)
@@ -110,18 +111,31 @@ __device__ void select(KeyAt key_at, int n, int k, Smem *sm, unsigned long long 
             const uint32_t need = (uint32_t)sm->need;
             const bool mine = excl < need && need <= incl;
             if (mine) {
-                uint32_t above = excl;
-                int j = 0;
-                while (above + h[j] < need)
-                    above += h[j++];
-                const uint32_t bin = 255u - 8u * lane - (uint32_t)j;
+                // the bin (of this lane's 8, descending) where the running count reaches need;
+                // unrolled, so h stays in registers
+                uint32_t above = excl, hsel = 0;
+                int jsel = 0;
+                bool found = false;
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    if (!found) {
+                        if (above + h[j] >= need) {
+                            found = true;
+                            jsel = j;
+                            hsel = h[j];
+                        } else {
+                            above += h[j];
+                        }
+                    }
+                }
+                const uint32_t bin = 255u - 8u * lane - (uint32_t)jsel;
                 const int need2 = (int)(need - above);
                 const unsigned long long p2 = prefix | ((unsigned long long)bin << shift);
                 sm->prefix = p2;
                 sm->plen = plen + 8;
                 sm->need = need2;
-                // keys at or above the bottom of this bin: the k - need2 already above, plus h[j]
-                sm->gather = (k - need2) + (int)h[j] <= kGather || plen + 8 == 64;
+                // keys at or above the bottom of this bin: the k - need2 already above, plus its own
+                sm->gather = (k - need2) + (int)hsel <= kGather || plen + 8 == 64;
             }
         }
         bar<NT>(id);
@@ -139,21 +153,16 @@ __device__ void select(KeyAt key_at, int n, int k, Smem *sm, unsigned long long 
         }
     }
     bar<NT>(id);
-    if (tid < 32) {
-        const int cnt = sm->cnt < kGather ? sm->cnt : kGather;
-        const unsigned long long a = lane < cnt ? sm->buf[lane] : 0ull;
-        const unsigned long long b = lane + 32 < cnt ? sm->buf[lane + 32] : 0ull;
-        int ra = 0, rb = 0;
-        for (int j = 0; j < 32; j++) {
-            const unsigned long long xa = __shfl_sync(0xffffffffu, a, j);
-            const unsigned long long xb = __shfl_sync(0xffffffffu, b, j);
-            ra += (xa > a) + (xb > a);
-            rb += (xa > b) + (xb > b);
-        }
-        if (lane < cnt && ra < k)
-            out[ra] = a;
-        if (lane + 32 < cnt && rb < k)
-            out[rb] = b;
+    // rank of each gathered key = the number of larger ones (keys are unique); one thread per key,
+    // every thread reading the same entry at a time (a shared-memory broadcast)
+    const int cnt = sm->cnt < kGather ? sm->cnt : kGather;
+    if (tid < cnt) {
+        const unsigned long long a = sm->buf[tid];
+        int r = 0;
+        for (int j = 0; j < cnt; j++)
+            r += sm->buf[j] > a;
+        if (r < k)
+            out[r] = a;
     }
     bar<NT>(id);
 }
