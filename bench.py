@@ -1097,6 +1097,22 @@ def run_case(args):
                 y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
                 fn = lambda: bq.gemm_prefill(x, w, out=y)
                 work = {"TFLOPs": 2 * M * N * K / 1e12}
+        elif args.case == "quantize":
+            fmt = {"binary": bq.BINARY_G128, "ternary": bq.TERNARY_G128, "ternary_b3": bq.TERNARY_B3_G128}[args.fmt]
+            wd = (synth.activations(5, N, K, dtype=torch.float32) * 0.02).to(torch.bfloat16).to(device)
+            pw = bq.quantize_g128(wd, fmt)
+            fn = lambda: bq.quantize_g128(wd, fmt)
+            work = {"GBps": (N * K * 2 + pw.words.numel() * pw.words.element_size() + pw.scales.numel() * 2) / 1e9}
+        elif args.case == "mlp":
+            mk = lambda rows, cols, tid: bq.BQWeight(bq.BINARY_G128, rows, cols,
+                                                     synth.binary_words(tid, rows, cols, device=device),
+                                                     synth.scales(tid, rows, cols // 128, device=device))
+            gate, up, down = mk(N, K, 1), mk(N, K, 2), mk(K, N, 3)
+            x = synth.activations(0, M, K).to(device)
+            y = torch.empty((M, K), dtype=torch.float32, device=device)
+            ws = torch.empty(bq.mlp_swiglu_workspace_bytes(M, gate, up, down), dtype=torch.uint8, device=device)
+            fn = lambda: bq.mlp_swiglu(x, gate, up, down, out=y, workspace=ws)
+            work = {"GBps": (2 * gemv_bytes(N, K, M, 1) + gemv_bytes(K, N, M, 1)) / 1e9}
         elif args.case == "embed":
             w = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(0, N, K, device=device),
                             synth.scales(0, N, K // 128, device=device))
@@ -1123,7 +1139,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="total CPU time budget of --impl reference (split over warm-up and steps)")
-    ap.add_argument("--case", choices=["gemv", "prefill", "embed", "topk"],
+    ap.add_argument("--case", choices=["gemv", "prefill", "embed", "topk", "quantize", "mlp"],
                     help="time one workload alone (for profiling) instead of the benchmark")
     ap.add_argument("--fmt", choices=["binary", "ternary", "ternary_b3"], default="binary")
     ap.add_argument("--N", type=int, default=248320)

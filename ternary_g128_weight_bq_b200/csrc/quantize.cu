@@ -99,7 +99,7 @@ quantize_kernel(const WT *__restrict__ w, int64_t N, int64_t K, void *__restrict
     for (int r = 0; r < 4; r++)
         v[r] = wload(wg + 32 * r + lane);
 
-    if (FMT == BQ_BINARY_G128) {
+    if constexpr (FMT == BQ_BINARY_G128) {
         uint32_t *words = static_cast<uint32_t *>(packed) + n * (K / 32) + 4 * g;
         double a = 0.0;
 #pragma unroll
@@ -112,86 +112,85 @@ quantize_kernel(const WT *__restrict__ w, int64_t N, int64_t K, void *__restrict
         const double sum = warp_sum(a);
         if (lane == 0)
             scales[n * G + g] = __half_as_ushort(__double2half(sum / 128.0));
-        return;
-    }
-
-    // ternary: sort (|w|, position) descending
-    unsigned long long key[4];
-#pragma unroll
-    for (int r = 0; r < 4; r++)
-        key[r] = ((unsigned long long)(__float_as_uint(v[r]) & 0x7FFFFFFFu) << 32) |
-                 (0xFFFFFFFFu - (uint32_t)(32 * r + lane));
-    sort128_desc(key, lane);
-    // prefix sums of the sorted magnitudes (element 32 r + lane), scores, arg-max
-    double base = 0.0, best = 0.0, best_sum = 0.0;
-    int best_j = 0;
-#pragma unroll
-    for (int r = 0; r < 4; r++) {
-        double x = (double)__uint_as_float((uint32_t)(key[r] >> 32));
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const double o = __shfl_up_sync(0xffffffffu, x, d);
-            if (lane >= d)
-                x += o;
-        }
-        const double prefix = base + x;
-        const int j = 32 * r + lane + 1;
-        const double score = prefix * prefix / j;
-        if (score > best) {                       // j grows with r: the first maximum per lane
-            best = score;
-            best_j = j;
-            best_sum = prefix;
-        }
-        base = __shfl_sync(0xffffffffu, prefix, 31);
-    }
-    // warp arg-max: largest score, then smallest j
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) {
-        const double ob = __shfl_xor_sync(0xffffffffu, best, m);
-        const int oj = __shfl_xor_sync(0xffffffffu, best_j, m);
-        const double os = __shfl_xor_sync(0xffffffffu, best_sum, m);
-        if (ob > best || (ob == best && oj < best_j && ob > 0.0)) {
-            best = ob;
-            best_j = oj;
-            best_sum = os;
-        }
-    }
-    // the support is the best_j largest keys: those >= the key at sorted position best_j - 1
-    unsigned long long thr = ~0ull;
-    if (best_j > 0) {
-        const int e = best_j - 1;
-        const unsigned long long kr = key[e >> 5];
-        thr = __shfl_sync(0xffffffffu, kr, e & 31);
-    }
-    // (every lane took part in the shuffle above; the key of register e >> 5 of lane e & 31)
-#pragma unroll
-    for (int r = 0; r < 4; r++) {
-        const int pos = 32 * r + lane;
-        const unsigned long long mine = ((unsigned long long)(__float_as_uint(v[r]) & 0x7FFFFFFFu) << 32) |
-                                        (0xFFFFFFFFu - (uint32_t)pos);
-        const int q = best_j > 0 && mine >= thr ? (v[r] >= 0.f ? 1 : -1) : 0;
-        codes_s[warp][pos] = (int8_t)(q + 1);
-    }
-    __syncwarp();
-    if (lane == 0)
-        scales[n * G + g] = __half_as_ushort(__double2half(best_j ? best_sum / best_j : 0.0));
-    const int8_t *c = codes_s[warp];
-    if (FMT == BQ_TERNARY_G128) {
-        if (lane < 8) {                            // 8 words of 16 codes
-            uint32_t word = 0;
-#pragma unroll
-            for (int i = 0; i < 16; i++)
-                word |= (uint32_t)c[16 * lane + i] << (2 * i);
-            static_cast<uint32_t *>(packed)[n * (K / 16) + 8 * g + lane] = word;
-        }
     } else {
-        if (lane < b3::kGroupBytes) {
-            const int cnt = b3::count(lane), k0 = b3::first(lane);
-            uint32_t val = 0;
-            for (int p = 0; p < cnt; p++)
-                val = 3u * val + (uint32_t)c[k0 + p];
-            static_cast<uint8_t *>(packed)[n * (b3::kGroupBytes * G) + b3::byte_offset(G, g, lane)] =
-                (uint8_t)b3::encode(val, cnt);
+        // ternary: sort (|w|, position) descending
+        unsigned long long key[4];
+#pragma unroll
+        for (int r = 0; r < 4; r++)
+            key[r] = ((unsigned long long)(__float_as_uint(v[r]) & 0x7FFFFFFFu) << 32) |
+                     (0xFFFFFFFFu - (uint32_t)(32 * r + lane));
+        sort128_desc(key, lane);
+        // prefix sums of the sorted magnitudes (element 32 r + lane), scores, arg-max
+        double base = 0.0, best = 0.0, best_sum = 0.0;
+        int best_j = 0;
+#pragma unroll
+        for (int r = 0; r < 4; r++) {
+            double x = (double)__uint_as_float((uint32_t)(key[r] >> 32));
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const double o = __shfl_up_sync(0xffffffffu, x, d);
+                if (lane >= d)
+                    x += o;
+            }
+            const double prefix = base + x;
+            const int j = 32 * r + lane + 1;
+            const double score = prefix * prefix / j;
+            if (score > best) {                       // j grows with r: the first maximum per lane
+                best = score;
+                best_j = j;
+                best_sum = prefix;
+            }
+            base = __shfl_sync(0xffffffffu, prefix, 31);
+        }
+        // warp arg-max: largest score, then smallest j
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+            const double ob = __shfl_xor_sync(0xffffffffu, best, m);
+            const int oj = __shfl_xor_sync(0xffffffffu, best_j, m);
+            const double os = __shfl_xor_sync(0xffffffffu, best_sum, m);
+            if (ob > best || (ob == best && oj < best_j && ob > 0.0)) {
+                best = ob;
+                best_j = oj;
+                best_sum = os;
+            }
+        }
+        // the support is the best_j largest keys: those >= the key at sorted position best_j - 1
+        unsigned long long thr = ~0ull;
+        if (best_j > 0) {
+            const int e = best_j - 1;
+            const unsigned long long kr = key[e >> 5];
+            thr = __shfl_sync(0xffffffffu, kr, e & 31);
+        }
+        // (every lane took part in the shuffle above; the key of register e >> 5 of lane e & 31)
+#pragma unroll
+        for (int r = 0; r < 4; r++) {
+            const int pos = 32 * r + lane;
+            const unsigned long long mine = ((unsigned long long)(__float_as_uint(v[r]) & 0x7FFFFFFFu) << 32) |
+                                            (0xFFFFFFFFu - (uint32_t)pos);
+            const int q = best_j > 0 && mine >= thr ? (v[r] >= 0.f ? 1 : -1) : 0;
+            codes_s[warp][pos] = (int8_t)(q + 1);
+        }
+        __syncwarp();
+        if (lane == 0)
+            scales[n * G + g] = __half_as_ushort(__double2half(best_j ? best_sum / best_j : 0.0));
+        const int8_t *c = codes_s[warp];
+        if (FMT == BQ_TERNARY_G128) {
+            if (lane < 8) {                            // 8 words of 16 codes
+                uint32_t word = 0;
+#pragma unroll
+                for (int i = 0; i < 16; i++)
+                    word |= (uint32_t)c[16 * lane + i] << (2 * i);
+                static_cast<uint32_t *>(packed)[n * (K / 16) + 8 * g + lane] = word;
+            }
+        } else {
+            if (lane < b3::kGroupBytes) {
+                const int cnt = b3::count(lane), k0 = b3::first(lane);
+                uint32_t val = 0;
+                for (int p = 0; p < cnt; p++)
+                    val = 3u * val + (uint32_t)c[k0 + p];
+                static_cast<uint8_t *>(packed)[n * (b3::kGroupBytes * G) + b3::byte_offset(G, g, lane)] =
+                    (uint8_t)b3::encode(val, cnt);
+            }
         }
     }
 }
