@@ -435,7 +435,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         // this thread's row in tensor memory: lane r (the warp's lane quarter), columns 16 hk ..
         const uint32_t arow_tmem = tmem_d + ((uint32_t)(32 * (warp & 3)) << 16) + BN + kCols * hk;
 
-        constexpr int kAhead = 4;                           // k-blocks of bits loaded ahead
+        constexpr int kAhead = FMT == BQ_TERNARY_B3_G128 ? 8 : 4;   // k-blocks of packed weights loaded ahead
         uint2 wq[kAhead];
         uint16_t sq[kAhead];
         // base-3 rows: 26 G bytes each, an even number, so every 16-bit load below is aligned
