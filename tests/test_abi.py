@@ -176,3 +176,69 @@ def test_fault_injection_from_environment(tmp_path):
     p = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, timeout=120)
     assert p.returncode == 0, p.stderr
     assert p.stdout.strip().splitlines()[-1] == "[True, True, False]"
+
+
+def test_new_calls_validate_before_any_cuda_call(libbq):
+    """The base-3 pack, the quantiser, the top-k GEMV and the SwiGLU MLP reject bad arguments in
+    host validation; sizes of the base-3 storage; the workspace queries of the new calls."""
+    W = ctypes.byref
+    V = ctypes.c_void_p
+    # sizes: 26 bytes per group of 128; words rounded up
+    assert libbq.bq_packed_bytes(2, 3, 256) == 3 * 52
+    assert libbq.bq_packed_words(2, 3, 128) == (3 * 26 + 3) // 4
+    assert libbq.bq_packed_bytes(0, 3, 256) == 3 * 32 and libbq.bq_packed_bytes(1, 3, 256) == 3 * 64
+    assert libbq.bq_packed_bytes(2, 3, 100) == 0
+    # base-3 pack
+    assert libbq.bq_pack_ternary_b3_g128(None, 16, 1, 128, 16, 16, None) == 1
+    assert libbq.bq_pack_ternary_b3_g128(16, 16, 1, 96, 16, 16, None) == 2
+    assert libbq.bq_pack_ternary_b3_g128(17, 16, 1, 128, 16, 16, None) == 3
+    # quantiser: NULL, format, dtype, shape, alignment
+    assert libbq.bq_quantize_g128(None, 2, 4, 256, 0, 16, 16, None) == 1
+    assert libbq.bq_quantize_g128(16, 2, 4, 256, 7, 16, 16, None) == 1
+    assert libbq.bq_quantize_g128(16, 9, 4, 256, 0, 16, 16, None) == 4
+    assert libbq.bq_quantize_g128(16, 2, 4, 200, 0, 16, 16, None) == 2
+    assert libbq.bq_quantize_g128(16, 2, 4, 256, 0, 24, 16, None) == 3
+    # top-k: k range, NULL outputs, sampling arguments, shape the tensor-core path cannot take,
+    # workspace
+    w = bq._Weight(0, 256, 1024, 1 << 20, 1 << 21)
+    big = 1 << 30
+    args = lambda k=20, vals=1 << 22, u=None, T=0.7, p=0.95, tok=None, ws=1 << 24, wsb=big, K_w=w: (
+        1 << 23, 1, 1, W(K_w), k, vals, 1 << 25, u, T, p, tok, ws, wsb, None)
+    for f in (libbq.bq_gemv_topk,):
+        f.argtypes = [V, ctypes.c_int, ctypes.c_int64, ctypes.POINTER(bq._Weight), ctypes.c_int, V, V, V,
+                      ctypes.c_float, ctypes.c_float, V, V, ctypes.c_size_t, V]
+    assert libbq.bq_gemv_topk(*args(k=0)) == 2 and libbq.bq_gemv_topk(*args(k=33)) == 2
+    assert libbq.bq_gemv_topk(*args(vals=None)) == 1
+    assert libbq.bq_gemv_topk(*args(u=1 << 26)) == 1                          # u without tokens
+    assert libbq.bq_gemv_topk(*args(u=1 << 26, tok=1 << 27, T=0.0)) == 1
+    assert libbq.bq_gemv_topk(*args(u=1 << 26, tok=1 << 27, p=1.5)) == 1
+    w640 = bq._Weight(0, 256, 640, 1 << 20, 1 << 21)
+    assert libbq.bq_gemv_topk(*args(K_w=w640)) == 2
+    assert libbq.bq_gemv_topk(*args(ws=1 << 24, wsb=16)) == 9
+    assert libbq.bq_gemv_topk_workspace_bytes(1, W(w), 20) > 0
+    assert libbq.bq_gemv_topk_workspace_bytes(1, W(w640), 20) == 0
+    lm = bq._Weight(0, 248320, 5120, 1 << 20, 1 << 21)
+    assert libbq.bq_gemv_topk_workspace_bytes(8, W(lm), 20) > 148 * 8 * 20 * 8
+    # SwiGLU MLP: shapes must chain, M range
+    g = bq._Weight(0, 512, 1024, 1 << 20, 1 << 21)
+    u2 = bq._Weight(0, 528, 1024, 1 << 20, 1 << 21)
+    d = bq._Weight(0, 256, 512, 1 << 20, 1 << 21)
+    dbad = bq._Weight(0, 256, 640, 1 << 20, 1 << 21)
+    assert libbq.bq_mlp_swiglu(1 << 23, 1, 1, W(g), W(u2), W(d), 1 << 22, 2, 1 << 24, big, None) == 2
+    assert libbq.bq_mlp_swiglu(1 << 23, 1, 1, W(g), W(g), W(dbad), 1 << 22, 2, 1 << 24, big, None) == 2
+    assert libbq.bq_mlp_swiglu(1 << 23, 1, 9, W(g), W(g), W(d), 1 << 22, 2, 1 << 24, big, None) == 2
+    assert libbq.bq_mlp_swiglu(1 << 23, 1, 1, W(g), W(g), W(d), 1 << 22, 2, 1 << 24, 16, None) == 9
+    assert libbq.bq_mlp_swiglu_workspace_bytes(1, W(g), W(g), W(d)) > 0
+    assert libbq.bq_mlp_swiglu_workspace_bytes(1, W(g), W(u2), W(d)) == 0
+    # injected failures reach the new calls after validation, with nothing launched
+    libbq.bq_debug_fail_next_launches(4)
+    try:
+        assert libbq.bq_gemv_topk(*args()) == 6 and b"injected" in libbq.bq_last_error()
+        assert libbq.bq_mlp_swiglu(1 << 23, 1, 1, W(g), W(g), W(d), 1 << 22, 2, 1 << 24, big, None) == 6
+        assert b"injected" in libbq.bq_last_error()
+        assert libbq.bq_quantize_g128(16, 2, 4, 256, 2, 32, 48, None) == 6
+        assert b"injected" in libbq.bq_last_error()
+        assert libbq.bq_pack_ternary_b3_g128(16, 32, 1, 128, 48, 64, None) == 6
+        assert b"injected" in libbq.bq_last_error()
+    finally:
+        libbq.bq_debug_fail_next_launches(0)

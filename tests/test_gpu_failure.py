@@ -76,3 +76,39 @@ def test_injected_launch_failure_then_recovers(orc):
     torch.cuda.synchronize()
     ref, bound = orc.gemv(oracle.BINARY, x, oracle.X_BF16, words, s, K)
     assert_within_bound(y, ref, bound, "gemv after an injected failure")
+
+
+def test_wait_timeout_in_topk_and_mlp_then_recovers(orc):
+    """The same bounded-wait timeout in the top-k GEMV (its CTAs still take their tickets and the
+    last one still merges, so nothing waits forever) and in the SwiGLU MLP's two GEMVs; then
+    normal calls are correct."""
+    m = bq()
+    N, K, F = 20480, 5120, 2048
+    w, words, s = _binary(m, 51, N, K)
+    g, gw, gs = _binary(m, 52, F, K)
+    u, uw, us = _binary(m, 53, F, K)
+    d, dw, ds = _binary(m, 54, 1024, F)
+    x = synth.activations(55, 2, K)
+    xd = x.cuda()
+    m.get_device_error()
+    m.debug_set_wait_limit_ns(1)
+    try:
+        for call in (lambda: m.gemv_topk(xd, w, k=20), lambda: m.mlp_swiglu(xd, g, u, d)):
+            call()
+            torch.cuda.synchronize()
+            with pytest.raises(m.BQError) as e:
+                m.get_device_error()
+            assert e.value.status_name == "BQ_ERR_TIMEOUT"
+            m.get_device_error()
+    finally:
+        m.debug_set_wait_limit_ns(0)
+    vals, idx = m.gemv_topk(xd, w, k=20)
+    y = m.mlp_swiglu(xd, g, u, d)
+    torch.cuda.synchronize()
+    m.get_device_error()
+    yl = m.gemv(xd, w).cpu().numpy()
+    order = np.array([np.lexsort((np.arange(N), -r.astype(np.float64)))[:20] for r in yl])
+    assert np.array_equal(idx.cpu().numpy(), order)
+    _, y_ref, bound = orc.mlp_swiglu(x, oracle.X_BF16, oracle.BINARY, (gw.numpy(), gs), (uw.numpy(), us),
+                                     oracle.BINARY, (dw.numpy(), ds))
+    assert_within_bound(y, y_ref, bound, "mlp after a timeout")
