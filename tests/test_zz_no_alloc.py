@@ -81,5 +81,10 @@ def test_noalloc_rejects_bad_arguments():
     with pytest.raises(m.BQError) as e:
         m.gemv_noalloc(torch.zeros((9, 1024), dtype=torch.bfloat16, device="cuda"), w)
     assert "M=9" in str(e.value)
-    with pytest.raises(m.BQError):
-        m.gemv_noalloc(x.cuda().float(), w)
+    # fp32 x is accepted (it is digitised like fp16/bf16 x); an unknown dtype code is not
+    y32 = m.gemv_noalloc(x.cuda().float(), w)
+    assert torch.equal(y32, m.gemv_noalloc(x.cuda(), w))
+    y = torch.empty((1, w.N), device="cuda")
+    with pytest.raises(m.BQError) as e:
+        m._check(m.lib().bq_gemv_noalloc(x.cuda().data_ptr(), 5, 1, w.c, y.data_ptr(), 2, m._stream()))
+    assert e.value.status_name == "BQ_ERR_DTYPE"
