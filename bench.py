@@ -499,13 +499,15 @@ def _rotating_gemv_ms(bq, mats, x, y, ws, stream, reps=20):
 
 
 def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
-    """One entry per benchmark configuration (BASELINE's five, in order)."""
+    """One entry per workload: the 1024 x 1024 GEMV, the headline GEMVs, the LM head and the gather,
+    the ternary GEMV and prefill, the binary prefill and the full-depth step, with the native
+    ternary, top-k, MLP and quantiser entries beside them."""
     import numpy as np
     l2 = l2_bytes(device)
     out = []
     o = ob.o
 
-    # ---- config 1: binary GEMV, M=1, K=N=1024, x fp16, seed 0 (L2-resident: reported in us)
+    # ---- binary GEMV, M=1, K=N=1024, x fp16, seed 0 (L2-resident: reported in us)
     N, K = 1024, 1024
     w = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(0, N, K, device=device),
                     synth.scales(0, N, K // 128, device=device))
@@ -517,7 +519,7 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
     bq.gemv(xd, w, out=y, workspace=ws)
     words, sc = _host_binary(0, N, K)
     ratio = ob.max_ratio(o.BINARY, x, o.X_F16, words, sc, K, y.cpu().numpy())
-    e = _gemv_entry("config 1: binary g128 GEMV, M=1, K=N=1024, x fp16, seed 0 (all 1024 outputs checked)",
+    e = _gemv_entry("binary g128 GEMV, M=1, K=N=1024, x fp16, seed 0 (all 1024 outputs checked)",
                     N, K, 1, 1, ms, peaks,
                     {"timing": "graph of 50 back-to-back calls on the same weights (147 KB: L2-resident)",
                      "parity": {"max_err_over_bound": round(ratio, 5), "outputs": N}})
@@ -525,7 +527,7 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
     out.append(e)
     del w, y, ws
 
-    # ---- config 2: the headline GEMVs (K=5120, N in {5120, 20480}, M in {1, 4, 8}); the
+    # ---- the headline GEMVs (K=5120, N in {5120, 20480}, M in {1, 4, 8}); the
     # device times are the breakdown's (rotating weight copies); parity on copy 0
     shapes = []
     for j, (N, M) in enumerate(GEMV_SHAPES):
@@ -545,11 +547,11 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
                                        K // 8 + K // 64, 2 * M * K, N <= 5120)
         shapes.append(ent)
         del w, y
-    out.append({"workload": "config 2: binary g128 decode GEMV, K=5120, N in {5120, 20480}, M in {1, 4, 8} "
+    out.append({"workload": "binary g128 decode GEMV, K=5120, N in {5120, 20480}, M in {1, 4, 8} "
                             "(the headline step; one entry per GEMV, each timed alone over rotating copies)",
                 "bound": "hbm", "peak": peaks["hbm_gbs"], "gemvs": shapes})
 
-    # ---- config 3: LM head (M=1, K=5120, N=248320) and the embedding gather of 4096 ids
+    # ---- LM head (M=1, K=5120, N=248320) and the embedding gather of 4096 ids
     N, K = 248320, K_HEAD
     w = bq.BQWeight(bq.BINARY_G128, N, K, synth.binary_words(0, N, K, device=device),
                     synth.scales(0, N, K // 128, device=device))
@@ -561,7 +563,7 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
     rows = 512
     words, sc = _host_binary(0, rows, K, row0=N - rows)
     ratio = ob.max_ratio(o.BINARY, x, o.X_BF16, words, sc, K, y[:, N - rows:].cpu().numpy())
-    e = _gemv_entry("config 3a: LM-head GEMV, binary g128, M=1, K=5120, N=248320", N, K, 1, 1, ms, peaks,
+    e = _gemv_entry("LM-head GEMV, binary g128, M=1, K=5120, N=248320", N, K, 1, 1, ms, peaks,
                     {"timing": "graph of 20 back-to-back calls (179 MB of weights per call, above L2)",
                      "parity": {"max_err_over_bound": round(ratio, 5), "rows": rows}})
     e["oracle"] = ob.gemv_timing(o.BINARY, x, o.X_BF16, *_host_binary(0, 4096, K), K, K // 8 + K // 64,
@@ -598,7 +600,7 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
         ob.orc.embed(o.BINARY, (ids[lo:hi] % R).numpy(), words, sc, K)
     dt, n = ob.time_items(ework, T, ob.cores)
     gbs = eb / 1e9 / (ms / 1e3)
-    out.append({"workload": "config 3b: embedding gather, 4096 ids uniform in [0, 248320), K=5120, bf16 out",
+    out.append({"workload": "embedding gather, 4096 ids uniform in [0, 248320), K=5120, bf16 out",
                 "us": round(ms * 1e3, 2), "GBps": round(gbs, 1), "bound": "hbm",
                 "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"],
                 "timing": f"graph of {2 * nbuf} back-to-back calls, {nbuf} output buffers rotated ({nbuf * T * K * 2 / 1e6:.0f} MB vs {l2 / 1e6:.0f} MB L2)",
@@ -607,7 +609,7 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
                                          "sample": f"{n} ids (rows of a 4096-row slice), {dt:.3f} s"}}})
     del w, y, ws, outs
 
-    # ---- config 4: ternary GEMV (N=20480, K=5120, M=1) and ternary prefill (M=512)
+    # ---- ternary GEMV (N=20480, K=5120, M=1) and ternary prefill (M=512)
     N, K = 20480, K_HEAD
     copies = max(2, math.ceil(2.5 * l2 / gemv_bytes(N, K, 1, 2)))
     tmats = []
@@ -624,7 +626,7 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
     rows = 256
     words, sc = _host_ternary(ob, 0, rows, K)
     ratio = ob.max_ratio(o.TERNARY, x, o.X_BF16, words, sc, K, y[:, :rows].cpu().numpy())
-    e = _gemv_entry("config 4a: ternary g128 GEMV, M=1, K=5120, N=20480", N, K, 1, 2, ms, peaks,
+    e = _gemv_entry("ternary g128 GEMV, M=1, K=5120, N=20480", N, K, 1, 2, ms, peaks,
                     {"timing": f"graph of back-to-back calls rotating {copies} weight copies (above L2)",
                      "parity": {"max_err_over_bound": round(ratio, 5), "rows": rows}})
     e["oracle"] = ob.gemv_timing(o.TERNARY, x, o.X_BF16, *_host_ternary(ob, 0, 2048, K), K,
@@ -657,7 +659,7 @@ def config_reports(bq, device, stream, peaks, ob: "OracleBench", breakdown):
     out.append(prefill_report(bq, device, stream, peaks, ob, "ternary", l2))
     out.append(prefill_report(bq, device, stream, peaks, ob, "ternary_b3", l2))
 
-    # ---- config 5: binary prefill (M=512) and the full-depth decode step
+    # ---- binary prefill (M=512) and the full-depth decode step
     out.append(prefill_report(bq, device, stream, peaks, ob, "binary", l2))
     out.append(full_depth_step(bq, device, stream, peaks, ob))
     out.append(mlp_entry(bq, device, stream, peaks, ob))
@@ -710,7 +712,7 @@ def prefill_report(bq, device, stream, peaks, ob, fmt_name, l2):
         ob.orc.gemv(fmt, x, o.X_BF16, words[lo:hi], sc[lo:hi], K)
     dt, n = ob.time_items(work, rows, ob.cores)
     del sets, ws
-    name = {"binary": "config 5a: binary g128", "ternary": "config 4b: ternary g128",
+    name = {"binary": "binary g128", "ternary": "ternary g128",
             "ternary_b3": "ternary g128 in base-3 storage (1.75 bits/weight)"}[fmt_name]
     return {"workload": f"{name} prefill GEMM, M=512, K=5120, N=20480, x and y bf16",
             "us": round(ms * 1e3, 1), "TFLOPs": round(tf, 1), "bound": "tensor",
@@ -753,7 +755,7 @@ def full_depth_step(bq, device, stream, peaks, ob=None):
                 bq.gemv(xs[w.K], w, out=ys[(w.N, w.K)], workspace=ws)
         ms = time_single(g.replay, 20, 3, stream)
     gbs = total / 1e9 / (ms / 1e3)
-    res = {"workload": "config 5b: full-depth decode step, 64 blocks x {9120x5120, 5120x5120, 40960x5120, "
+    res = {"workload": "full-depth decode step, 64 blocks x {9120x5120, 5120x5120, 40960x5120, "
                        "5120x20480} binary GEMVs at M=1 (24.8e9 weights)",
            "blocks": FULL_DEPTH_BLOCKS, "gemvs": 4 * FULL_DEPTH_BLOCKS, "bytes": total,
            "us": round(ms * 1e3, 1), "tokens_per_s": round(1e3 / ms, 1), "GBps": round(gbs, 1),
