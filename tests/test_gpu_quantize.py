@@ -57,6 +57,8 @@ def test_quantize_special_groups(orc, ofmt, dfmt):
     w[4, :64] = 1.0
     w[4, 64:128] = 0.001                              # two clusters
     w[5, 128:256] = torch.linspace(-1, 1, 128)
+    w[6, :128] = 0.0
+    w[6, :4] = torch.tensor([3.0, -1.0, 1.0, -1.0])     # equal scores at j = 1 and j = 4: j = 1
     check(orc, w, ofmt, dfmt)
 
 

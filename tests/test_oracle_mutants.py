@@ -83,6 +83,8 @@ MUTANTS = {
         "cum += p[i] / kept;", "cum += p[i] / z;"),
     "quantize_zero_group_full_support": (
         "if (score > best) {", "if (score >= best) {"),
+    "quantize_tie_takes_larger_support": (
+        "if (score > best) {", "if (score > best || (score == best && score > 0.0)) {"),
     "quantize_sort_ascending": (
         "return a->a > b->a ? -1 : 1;", "return a->a > b->a ? 1 : -1;"),
     "quantize_binary_scale_127": (

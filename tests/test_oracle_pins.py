@@ -347,6 +347,20 @@ def pin_quantize_hand(o):
     assert sb[0, 0] == _f16(7 / 128) and sb[1, 0] == _f16(2.0) and sb[2, 0] == _f16(0.0)
 
 
+def pin_quantize_score_tie(o):
+    """An exact tie of the score (sum of the j largest |w|)^2 / j between two supports: |w| =
+    3, 1, 1, 1 gives 9 at j = 1 and 36 / 4 = 9 at j = 4 (8 and 25/3 between), all exact in
+    binary64; the smaller support is taken, so s = 3 rather than 1.5."""
+    w = np.zeros((2, 128), np.float32)
+    w[0, :4] = [3, -1, 1, -1]
+    w[1, [5, 40, 77, 120]] = [-1, 1, -3, 1]              # the same magnitudes elsewhere in a group
+    q, s = o.quantize(T, w)
+    assert q[0, :4].tolist() == [1, 0, 0, 0] and np.all(q[0, 4:] == 0) and s[0, 0] == _f16(3.0)
+    expect = np.zeros(128, np.int8)
+    expect[77] = -1
+    assert np.array_equal(q[1], expect) and s[1, 0] == _f16(3.0)
+
+
 def pin_quantize_binary_closed_form(o):
     rng = np.random.default_rng(31)
     w = (rng.normal(size=(6, 640)) * 0.02).astype(np.float32)
@@ -672,6 +686,7 @@ def test_b3_bits_per_weight(orc): pin_b3_bits_per_weight(orc)
 def test_mlp_vs_numpy(orc): pin_mlp_vs_numpy(orc)
 def test_mlp_silu_identities(orc): pin_mlp_silu_identities(orc)
 def test_quantize_hand(orc): pin_quantize_hand(orc)
+def test_quantize_score_tie(orc): pin_quantize_score_tie(orc)
 def test_quantize_binary_closed_form(orc): pin_quantize_binary_closed_form(orc)
 def test_quantize_ternary_bruteforce(orc): pin_quantize_ternary_bruteforce(orc)
 def test_quantize_invariants(orc): pin_quantize_invariants(orc)
