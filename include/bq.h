@@ -81,11 +81,12 @@ typedef enum { BQ_F16 = 0, BQ_BF16 = 1, BQ_F32 = 2 } bq_dtype;
 
 typedef enum { BQ_BINARY_G128 = 0, BQ_TERNARY_G128 = 1, BQ_TERNARY_B3_G128 = 2 } bq_format;
 
-/* Non-owning view of a packed weight matrix (device memory). */
+/* Non-owning view of a packed weight matrix (device memory). Every call rejects a view outside
+ * these limits with BQ_ERR_SHAPE, and every size query returns 0 for one. */
 typedef struct {
     bq_format fmt;
-    int64_t N;                /* output rows, >= 1 */
-    int64_t K;                /* inputs per row, a positive multiple of 128 */
+    int64_t N;                /* output rows, 1 .. 2^31 */
+    int64_t K;                /* inputs per row, a positive multiple of 128, at most 2^24 */
     const uint32_t *words;    /* [N][K/32] (binary), [N][K/16] (ternary), or the bytes
                                  [N][26 K/128] of the base-3 storage */
     const uint16_t *scales;   /* fp16 [N][K/128] */

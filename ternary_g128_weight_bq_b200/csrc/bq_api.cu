@@ -109,6 +109,14 @@ unsigned int *device_status(bq_status *st)
     return g_status_ptr[dev];
 }
 
+// The format and shape limits every call applies (no pointers looked at): what the size queries
+// accept, so that they never plan for a shape the compute calls reject.
+static bool shape_in_range(const bq_weight *w)
+{
+    return w && (w->fmt == BQ_BINARY_G128 || w->fmt == BQ_TERNARY_G128 || w->fmt == BQ_TERNARY_B3_G128) &&
+           w->N >= 1 && w->N <= (int64_t(1) << 31) && w->K >= 128 && w->K <= (int64_t(1) << 24) && w->K % 128 == 0;
+}
+
 static bq_status validate_weight(const bq_weight *w)
 {
     if (!w)
@@ -159,7 +167,7 @@ unsigned long long bq_kernel_launches(void) { return __atomic_load_n(&g_launches
 
 size_t bq_packed_words(bq_format fmt, int64_t N, int64_t K)
 {
-    if (N < 1 || K < 128 || K % 128)
+    if (N < 1 || K < 128 || K % 128 || N > (int64_t(1) << 31) || K > (int64_t(1) << 24))
         return 0;
     if (fmt == BQ_BINARY_G128)
         return (size_t)N * (size_t)(K / 32);
@@ -172,7 +180,7 @@ size_t bq_packed_words(bq_format fmt, int64_t N, int64_t K)
 
 size_t bq_packed_bytes(bq_format fmt, int64_t N, int64_t K)
 {
-    if (N < 1 || K < 128 || K % 128)
+    if (N < 1 || K < 128 || K % 128 || N > (int64_t(1) << 31) || K > (int64_t(1) << 24))
         return 0;
     if (fmt == BQ_TERNARY_B3_G128)
         return (size_t)N * (size_t)(26 * (K / 128));
@@ -315,7 +323,7 @@ static bq_status validate_xy(const char *who, const void *x, bq_dtype xt, const 
 
 size_t bq_gemv_workspace_bytes(int64_t M, const bq_weight *w)
 {
-    if (!w || M < 1 || M > 8 || w->N < 1 || w->K < 128 || w->K % 128)
+    if (!shape_in_range(w) || M < 1 || M > 8)
         return 0;
     return gemv_workspace_bytes((int)M, w->fmt, w->N, w->K);
 }
@@ -393,7 +401,7 @@ bq_status bq_gemv_noalloc(const void *x, bq_dtype xt, int64_t M, const bq_weight
 
 size_t bq_gemv_topk_workspace_bytes(int64_t M, const bq_weight *w, int k)
 {
-    if (!w || M < 1 || M > 8 || w->N < 1 || w->K < 128 || w->K % 128 || k < 1 || k > 32)
+    if (!shape_in_range(w) || M < 1 || M > 8 || k < 1 || k > 32)
         return 0;
     if (!gemv_rows_supported((int)M, w->fmt, w->N, w->K, k))
         return 0;
@@ -484,8 +492,8 @@ static bq_status validate_mlp(int64_t M, const bq_weight *gate, const bq_weight 
 
 size_t bq_mlp_swiglu_workspace_bytes(int64_t M, const bq_weight *gate, const bq_weight *up, const bq_weight *down)
 {
-    if (!gate || !up || !down || M < 1 || M > 8 || gate->N < 1 || gate->K < 128 || gate->K % 128 || up->N != gate->N ||
-        up->K != gate->K || down->K != gate->N || down->N < 1)
+    if (!shape_in_range(gate) || !shape_in_range(up) || !shape_in_range(down) || M < 1 || M > 8 ||
+        up->N != gate->N || up->K != gate->K || down->K != gate->N)
         return 0;
     if (!gemv_glu_supported((int)M, gate->fmt, gate->N, gate->K))
         return 0;
@@ -534,7 +542,7 @@ bq_status bq_mlp_swiglu(const void *x, bq_dtype xt, int64_t M, const bq_weight *
 
 size_t bq_gemm_prefill_workspace_bytes(int64_t M, const bq_weight *w)
 {
-    if (!w || M < 1 || w->N < 1 || w->K < 128 || w->K % 128)
+    if (!shape_in_range(w) || M < 1 || M > (int64_t(1) << 24))
         return 0;
     return prefill_workspace_bytes(M, w->fmt, w->N, w->K);
 }

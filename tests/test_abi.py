@@ -100,6 +100,24 @@ def test_validation_before_any_cuda_call(libbq):
     assert b"T=-1" in msg
 
 
+def test_size_queries_reject_out_of_range_views(libbq):
+    """The size queries apply the calls' limits (format, 1 <= N <= 2^31, 128 <= K <= 2^24, K a
+    multiple of 128) and return 0 outside them, instead of planning for the shape (a view of
+    N = 2^50, K = 2^40 once reached the planner and divided by zero)."""
+    W = ctypes.byref
+    huge = _weight(N=1 << 50, K=1 << 40)
+    for w in (huge, _weight(fmt=3), _weight(N=(1 << 31) + 1), _weight(K=(1 << 24) + 128), _weight(K=100)):
+        assert libbq.bq_gemv_workspace_bytes(1, W(w)) == 0
+        assert libbq.bq_gemv_topk_workspace_bytes(1, W(w), 20) == 0
+        assert libbq.bq_mlp_swiglu_workspace_bytes(1, W(w), W(w), W(w)) == 0
+        assert libbq.bq_gemm_prefill_workspace_bytes(512, W(w)) == 0
+        assert libbq.bq_packed_words(w.fmt, w.N, w.K) == 0
+    ok = _weight(N=20480, K=5120)
+    assert libbq.bq_gemv_workspace_bytes(1, W(ok)) > 0
+    assert libbq.bq_gemm_prefill_workspace_bytes(1 << 25, W(ok)) == 0
+    assert libbq.bq_packed_words(0, 1 << 31, 1 << 24) == (1 << 31) * (1 << 19)
+
+
 def _symbol_size(name: str) -> int:
     out = subprocess.run(["nm", "-S", "-C", bq.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
@@ -113,12 +131,12 @@ def _symbol_size(name: str) -> int:
 def test_noalloc_array_covers_every_supported_shape(libbq):
     """bq_gemv_noalloc serves a shape from the library's fixed array only when the workspace
     bq_gemv would need fits in it. That array must hold every shape the GEMV kernels take on a
-    148-SM B200 (without a GPU the library plans for 148 SMs): every M, both formats, K up to
-    64K, N up to 2^22. The array's size is read from the library's symbol table."""
+    148-SM B200 (without a GPU the library plans for 148 SMs): every M, all three formats, K up
+    to 64K, N up to 2^22. The array's size is read from the library's symbol table."""
     cap = _symbol_size("bq::g_gemv_scratch")
     assert 64 << 10 <= cap <= 4 << 20
     worst = 0
-    for fmt in (bq.BINARY_G128, bq.TERNARY_G128):
+    for fmt in (bq.BINARY_G128, bq.TERNARY_G128, bq.TERNARY_B3_G128):
         for M in range(1, 9):
             for K in (128, 1024, 2048, 4096, 5120, 6144, 8192, 16384, 20480, 65536):
                 for N in (1, 129, 5120, 20480, 248320, 1 << 22):
