@@ -77,9 +77,19 @@ typedef enum {
     BQ_ERR_WORKSPACE = 9      /* workspace pointer null or smaller than required */
 } bq_status;
 
-typedef enum { BQ_F16 = 0, BQ_BF16 = 1, BQ_F32 = 2 } bq_dtype;
+/* The two *_INT_RANGE_ enumerators are not values to pass: they give the enum the range of a
+ * 32-bit int, so that any int a caller passes is a representable value (the library rejects the
+ * ones it does not know with BQ_ERR_INVALID_ARG or BQ_ERR_DTYPE) and reading it is defined
+ * behaviour in C++ as well as in C. */
+typedef enum {
+    BQ_F16 = 0, BQ_BF16 = 1, BQ_F32 = 2,
+    BQ_DTYPE_INT_RANGE_MIN_ = -2147483647 - 1, BQ_DTYPE_INT_RANGE_MAX_ = 2147483647
+} bq_dtype;
 
-typedef enum { BQ_BINARY_G128 = 0, BQ_TERNARY_G128 = 1, BQ_TERNARY_B3_G128 = 2 } bq_format;
+typedef enum {
+    BQ_BINARY_G128 = 0, BQ_TERNARY_G128 = 1, BQ_TERNARY_B3_G128 = 2,
+    BQ_FORMAT_INT_RANGE_MIN_ = -2147483647 - 1, BQ_FORMAT_INT_RANGE_MAX_ = 2147483647
+} bq_format;
 
 /* Non-owning view of a packed weight matrix (device memory). Every call rejects a view outside
  * these limits with BQ_ERR_SHAPE, and every size query returns 0 for one. */
